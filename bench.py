@@ -1,0 +1,340 @@
+#!/usr/bin/env python
+"""Throughput of the HSTU layer hot path on B200.
+
+A step is one forward pass of the long-history HSTU layer (B=8 sequences,
+n ~ U{4096..8192}, d_model=512, 4 heads of 128, bf16) through the C-ABI call
+hstu_layer_fwd: jagged schedule, LayerNorm, f1 + SiLU + split, pointwise
+attention with the rab bias, LayerNorm(A V) * U, f2 + residual.
+
+Prints one JSON line (rank 0).  `value` is tokens/s over all ranks with the
+inputs resident in HBM; `e2e` repeats the measurement through the same call
+with host (pinned) inputs copied in and the output copied out every step;
+`roofline` reports the attention kernel's causal-FLOP rate against the measured
+dense bf16 peak; `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch with torch.distributed.run; every rank runs its own copy of the
+batch (independent sequences: no collective on the data path, weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hstu_sequential_transducer_02_b200 import workload as W  # noqa: E402
+
+CONFIG_ID = 2
+METRIC = "HSTU layer tokens/s and attention TFLOP/s as % of B200 BF16 dense peak (1 GPU)"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--oracle-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count() or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------
+# fp64 oracle on the host cores (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------
+
+def oracle_sequence_time(wl, s: int, max_tokens=None):
+    import oracle.hstu_oracle as O
+    sp = wl.spec
+    a, b = int(wl.seq_offsets[s]), int(wl.seq_offsets[s + 1])
+    if max_tokens is not None:
+        b = min(b, a + max_tokens)
+    t0 = time.perf_counter()
+    O.layer_forward(wl.x[a:b], wl.layers[0], [0, b - a], wl.timestamps[a:b], sp.num_heads, sp.head_dim)
+    return b - a, time.perf_counter() - t0
+
+
+def cpu_baseline(wl, seconds: float):
+    """Oracle layer forward over whole sequences of the workload, in order, until
+    `seconds` of CPU work have been spent (at least one sequence)."""
+    tokens, elapsed, seqs = 0, 0.0, 0
+    for s in range(len(wl.seq_offsets) - 1):
+        n, t = oracle_sequence_time(wl, s)
+        tokens += n
+        elapsed += t
+        seqs += 1
+        if elapsed >= seconds:
+            break
+    return {"value": tokens / elapsed, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, 1 layer forward over the first {seqs} whole sequence(s) "
+                      f"({tokens} tokens, {elapsed:.1f} s) of the long-history workload"}
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    wl = W.make_workload(CONFIG_ID)
+    B = len(wl.seq_offsets) - 1
+    for w in range(args.warmup):
+        oracle_sequence_time(wl, w % B, max_tokens=256)
+    tokens, elapsed = 0, 0.0
+    for k in range(args.steps):
+        n, t = oracle_sequence_time(wl, k % B)
+        tokens += n
+        elapsed += t
+    value = tokens / elapsed
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "long-history HSTU layer, B=8, n~U{4096..8192}, d=512, H=4, dh=128, 1 layer; "
+                               "one whole sequence per step (sequence k mod 8)",
+                   "global_batch": 1, "seq_len": "4096-8192", "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} steps, one whole sequence each ({tokens} tokens)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def read_traffic(kernel: str):
+    """dram bytes per launch of `kernel` from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 2 and parts[0] == kernel and not line.startswith("#"):
+                try:
+                    return float(parts[1])
+                except ValueError:
+                    return None
+    return None
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from hstu_sequential_transducer_02_b200 import binding as hb
+
+    wl = W.make_workload(CONFIG_ID)
+    sp = wl.spec
+    td = torch.bfloat16
+    T = wl.total_tokens
+    layer = hb.Layer(hb.layer_weights_to_device(wl.layers[0], td), sp.d_model, sp.num_heads, sp.head_dim)
+    x = torch.from_numpy(wl.x).to(td).cuda()
+    offs = torch.from_numpy(wl.seq_offsets).cuda()
+    ts = torch.from_numpy(wl.timestamps).cuda()
+    y = torch.empty_like(x)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        layer.forward(x, offs, ts, out=y)
+    torch.cuda.synchronize()
+    barrier()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    hb.trace_enable(True)
+    torch.cuda.synchronize()
+    barrier()
+    for k in range(args.steps):
+        flush.zero_()  # evict L2 between timed steps (outside the timed events)
+        starts[k].record()
+        layer.forward(x, offs, ts, out=y)
+        ends[k].record()
+    torch.cuda.synchronize()
+    barrier()
+    trace = hb.trace_read()
+    hb.trace_enable(False)
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T / (ms_per_step / 1e3)
+
+    # end to end through the same call: pinned host inputs in, output out, every step
+    x_h = torch.from_numpy(wl.x).to(td).pin_memory()
+    offs_h = torch.from_numpy(wl.seq_offsets).pin_memory()
+    ts_h = torch.from_numpy(wl.timestamps).pin_memory()
+    y_h = torch.empty(x_h.shape, dtype=td).pin_memory()
+    x_d, offs_d, ts_d = torch.empty_like(x), torch.empty_like(offs), torch.empty_like(ts)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        e_s[k].record()
+        x_d.copy_(x_h, non_blocking=True)
+        offs_d.copy_(offs_h, non_blocking=True)
+        ts_d.copy_(ts_h, non_blocking=True)
+        layer.forward(x_d, offs_d, ts_d, out=y)
+        y_h.copy_(y, non_blocking=True)
+        e_e[k].record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * T / (e2e_ms / args.steps / 1e3)
+    h2d = x_h.numel() * x_h.element_size() + offs_h.numel() * 4 + ts_h.numel() * 8
+    d2h = y_h.numel() * y_h.element_size()
+
+    # roofline of the attention kernel
+    import oracle.hstu_oracle as O  # work accounting only (pair count of the mask)
+    pairs = O.attention_pairs(wl.seq_offsets)
+    attn_flops = pairs * 2 * (sp.head_dim + sp.head_dim) * sp.num_heads
+    peaks, peak_src = load_peaks()
+    attn_name = "attn_fwd_tc" if "attn_fwd_tc" in trace else "attn_fwd_simt"
+    attn = trace.get(attn_name, {"count": 0, "ms": float("nan")})
+    attn_ms = attn["ms"] / max(attn["count"], 1)
+    achieved = attn_flops / (attn_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    launches = int(sum(v["count"] for v in trace.values()))
+    traffic = read_traffic(attn_name)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "long-history HSTU layer forward: B=8 jagged sequences, n~U{4096..8192} "
+                                   f"(T={T} tokens), d_model=512, 4 heads x 128, 1 layer, causal, seed 20242",
+                       "global_batch": 8 * world, "seq_len": "4096-8192", "parallelism": f"dp{world}",
+                       "l2": "flushed between timed steps (256 MiB write outside the timed events)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": attn_name, "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "flops_per_launch": attn_flops, "ms_per_launch": attn_ms,
+                         "frac_of_datasheet_2250": achieved / DATASHEET_BF16_TFLOPS},
+            "attention_tflops": achieved,
+            "kernels": {k: {"launches": v["count"], "ms_per_launch": v["ms"] / max(v["count"], 1),
+                            "share": v["ms"] / max(sum(u["ms"] for u in trace.values()), 1e-9)}
+                        for k, v in trace.items()},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, args.oracle_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

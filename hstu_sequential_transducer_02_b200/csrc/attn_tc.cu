@@ -1,0 +1,614 @@
+// Pointwise aggregated attention forward on the sm_100a tensor cores.
+//
+//   O_i = (1/N) * sum_{j in mask(i)} SiLU(q_i . k_j + rab_ij) v_j
+//
+// ("Actions Speak Louder than Words" summary, 1.2; "生成式推荐（一）：HSTU",
+// pointwise aggregated attention: no normalisation over the sequence.)
+//
+// One persistent CTA per SM walks the cost-sorted (sequence, head, q tile)
+// work list in snake order.  Per q tile of 128 rows and each kv tile of 128
+// columns that holds an attended pair:
+//   warp 0      TMA: Q once per item, K/V per kv tile into a ring of stages,
+//               plus the tile's timestamps (and their per-half min/max)
+//   warp 1      one thread issues tcgen05.mma: S = Q K^T into one of two TMEM
+//               buffers, then O += P V into the TMEM accumulator
+//   warps 2-9   epilogue: TMEM -> registers, rab bias (position and time
+//               buckets, bit-exact integer rule), SiLU, mask, bf16 P into
+//               shared memory (128-byte swizzle, the MMA's A layout); at the end
+//               of the item O * (1/N) -> bf16 -> global memory
+// No softmax means no running max and no rescaling: O accumulates in TMEM
+// across all kv tiles.  Fully masked kv tiles are never visited.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace hstu {
+namespace {
+using namespace sm100;
+
+constexpr int BM = 128;                    // q rows per tile (UMMA M)
+constexpr int BN = 128;                    // kv columns per tile
+constexpr int kEpiWarps = 8;               // two warps per TMEM lane quarter (one per 64-column half)
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kBoxBytes = 128 * 128;       // one TMA box: 128 rows x 64 bf16
+constexpr uint32_t kTmemCols = 512;
+
+template <int DH>
+struct Cfg {
+  static constexpr int kStages = DH == 128 ? 2 : 3;
+  static constexpr int kBoxes = DH / 64;
+  static constexpr int kTileBytes = BM * DH * 2;
+};
+
+struct TsStage {
+  int64_t ts[BN];       // timestamps of the tile's columns (0 beyond the sequence)
+  int32_t rel[BN];      // ts - tmin[half] (valid when wide[half] == 0)
+  int64_t tmin[2];      // per 64-column half, over the columns inside the sequence
+  int64_t tmax[2];
+  int32_t wide[2];      // 1: the half's time span does not fit the 32-bit path
+  int32_t pad[2];
+};
+
+struct Barriers {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[3], kv_empty[3];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full, p_empty;
+  uint64_t o_full, o_empty;
+  uint64_t done;
+};
+
+struct TcParams {
+  CUtensorMap map_q;
+  CUtensorMap map_k;
+  CUtensorMap map_v;
+  AttnFwdParams p;
+};
+
+template <int DH>
+struct Layout {
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + Cfg<DH>::kTileBytes;
+  static constexpr int kV = kK + Cfg<DH>::kStages * Cfg<DH>::kTileBytes;
+  static constexpr int kP = kV + Cfg<DH>::kStages * Cfg<DH>::kTileBytes;
+  static constexpr int kTs = kP + BM * BN * 2;
+  static constexpr int kThr = kTs + Cfg<DH>::kStages * (int)sizeof(TsStage);
+  static constexpr int kPosB = kThr + kNumBuckets * 8;
+  static constexpr int kTimeB = kPosB + kNumBuckets * 4;
+  static constexpr int kBar = (kTimeB + kNumBuckets * 4 + 15) & ~15;
+  static constexpr int kMisc = kBar + (int)sizeof(Barriers);
+  static constexpr int kEnd = kMisc + 16;
+  static constexpr int kAlloc = kEnd + 1024;  // slack for 1024-byte alignment of the base
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// snake order over the cost-sorted list: wave w visits CTAs forward when w is even
+__device__ __forceinline__ int snake_item(int k, int b, int G) {
+  const int pos = (k & 1) ? (G - 1 - b) : b;
+  return k * G + pos;
+}
+
+__device__ __forceinline__ float silu_tanh(float s) {
+  const float h = 0.5f * s;
+  return fmaf(h, tanh_approx(h), h);
+}
+
+// ---------------------------------------------------------------------------
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_constant__ TcParams prm) {
+  using C = Cfg<DH>;
+  using L = Layout<DH>;
+  constexpr int S = C::kStages;
+  constexpr int DV = DH;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  int64_t* thr = reinterpret_cast<int64_t*>(smem + L::kThr);
+  float* pos_b = reinterpret_cast<float*>(smem + L::kPosB);
+  float* time_b = reinterpret_cast<float*>(smem + L::kTimeB);
+  TsStage* tss = reinterpret_cast<TsStage*>(smem + L::kTs);
+  const uint32_t sQ = smem_u32(smem + L::kQ);
+  const uint32_t sK = smem_u32(smem + L::kK);
+  const uint32_t sV = smem_u32(smem + L::kV);
+  const uint32_t sP = smem_u32(smem + L::kP);
+
+  const AttnFwdParams& p = prm.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long tmo = p.timeout_ns;
+
+  // ---- set-up
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < S; ++s) { mbar_init(&bars->kv_full[s], 1); mbar_init(&bars->kv_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars->s_full[s], 1); mbar_init(&bars->s_empty[s], kEpiWarps); }
+    mbar_init(&bars->p_full, kEpiWarps);
+    mbar_init(&bars->p_empty, 1);
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_empty, kEpiWarps);
+    mbar_init(&bars->done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&prm.map_q);
+    tma_prefetch_desc(&prm.map_k);
+    tma_prefetch_desc(&prm.map_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int c = threadIdx.x; c < kNumBuckets; c += kThreads) {
+    thr[c] = p.thr.v[c];
+    pos_b[c] = p.pos_bias[c];
+    time_b[c] = p.time_bias[c];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_s0 = tmem_base;          // S buffers at columns 0 and 128
+  const uint32_t tmem_o = tmem_base + 2 * BN;  // O accumulator at column 256
+
+  const int count = *p.item_count;
+  const int G = gridDim.x;
+  const int per_head_rab = p.rab_head_stride != 0;
+
+  if (warp == 0) {
+    // =================================================================== producer
+    int kv_it = 0;
+    for (int k = 0;; ++k) {
+      const int idx = snake_item(k, blockIdx.x, G);
+      if (idx >= count || *abort_flag) break;
+      const WorkItem wi = p.items[idx];
+      const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+      const int r0 = wi.qtile * BM;
+      const int r1 = min(si.n, r0 + BM);
+      if (!mbar_wait(&bars->q_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
+        for (int b = 0; b < C::kBoxes; ++b)
+          tma_load_2d(smem + L::kQ + b * kBoxBytes, &prm.map_q, &bars->q_full, wi.head * DH + 64 * b, si.start + r0);
+      }
+      const KvRange kr = kv_tiles_for(r0, r1, si.hist, BN);
+      const int nk = kv_count(kr);
+      for (int jj = 0; jj < nk; ++jj, ++kv_it) {
+        const int c0 = kv_tile_at(kr, jj) * BN;
+        const int st = kv_it % S;
+        if (!mbar_wait(&bars->kv_empty[st], ((kv_it / S) & 1) ^ 1, tmo, abort_flag)) goto fail;
+        // timestamps of the tile and per-half ranges
+        TsStage& ts = tss[st];
+        int64_t t[4];
+        int64_t mn[2] = {INT64_MAX, INT64_MAX}, mx[2] = {INT64_MIN, INT64_MIN};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = lane + 32 * e;
+          const bool ok = c0 + c < si.n;
+          t[e] = ok ? p.timestamps[si.start + c0 + c] : 0;
+          if (ok) {
+            mn[e >> 1] = min(mn[e >> 1], t[e]);
+            mx[e >> 1] = max(mx[e >> 1], t[e]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            mn[h] = min(mn[h], (int64_t)__shfl_xor_sync(0xffffffffu, (long long)mn[h], o));
+            mx[h] = max(mx[h], (int64_t)__shfl_xor_sync(0xffffffffu, (long long)mx[h], o));
+          }
+          if (mn[h] > mx[h]) { mn[h] = 0; mx[h] = 0; }  // no column of this half inside the sequence
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = lane + 32 * e;
+          ts.ts[c] = t[e];
+          const int64_t d = t[e] - mn[e >> 1];
+          ts.rel[c] = (int32_t)(d < 0 ? 0 : (d > 0x3FFFFFFF ? 0x3FFFFFFF : d));
+        }
+        if (lane == 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            ts.tmin[h] = mn[h];
+            ts.tmax[h] = mx[h];
+            ts.wide[h] = (uint64_t)(mx[h] - mn[h]) >= (1ull << 30) ? 1 : 0;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars->kv_full[st], 2 * C::kTileBytes);
+          for (int b = 0; b < C::kBoxes; ++b) {
+            tma_load_2d(smem + L::kK + st * C::kTileBytes + b * kBoxBytes, &prm.map_k, &bars->kv_full[st],
+                        wi.head * DH + 64 * b, si.start + c0);
+            tma_load_2d(smem + L::kV + st * C::kTileBytes + b * kBoxBytes, &prm.map_v, &bars->kv_full[st],
+                        wi.head * DV + 64 * b, si.start + c0);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp == 1) {
+    // =================================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(BM, BN, false, false);
+      constexpr uint32_t idesc_o = make_idesc_bf16(BM, DV, false, true);
+      int kv_it = 0, s_it = 0, p_it = 0;
+      for (int k = 0;; ++k) {
+        const int idx = snake_item(k, blockIdx.x, G);
+        if (idx >= count || *abort_flag) break;
+        const WorkItem wi = p.items[idx];
+        const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+        const int r0 = wi.qtile * BM;
+        const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
+        const int nk = kv_count(kr);
+        if (!mbar_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
+        int prev_stage = 0;
+        for (int jj = 0; jj <= nk; ++jj) {
+          if (jj < nk) {
+            const int st = kv_it % S;
+            const int sb = s_it & 1;
+            if (!mbar_wait(&bars->kv_full[st], (kv_it / S) & 1, tmo, abort_flag)) goto fail;
+            if (!mbar_wait(&bars->s_empty[sb], ((s_it >> 1) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < DH / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
+              const uint64_t a = make_sw128_desc(sQ + off, 16, 1024);
+              const uint64_t b = make_sw128_desc(sK + st * C::kTileBytes + off, 16, 1024);
+              umma_f16_ss(tmem_s0 + sb * BN, a, b, idesc_s, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars->s_full[sb]);
+            if (jj == nk - 1) umma_commit(&bars->q_empty);
+          }
+          if (jj > 0) {
+            // O (+)= P V for the previous kv tile
+            if (!mbar_wait(&bars->p_full, p_it & 1, tmo, abort_flag)) goto fail;
+            if (jj == 1 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < BN / 16; ++ks) {
+              const uint64_t a = make_sw128_desc(sP + (ks >> 2) * kBoxBytes + (ks & 3) * 32, 16, 1024);
+              const uint64_t b = make_sw128_desc(sV + prev_stage * C::kTileBytes + ks * 16 * 128, kBoxBytes, 1024);
+              umma_f16_ss(tmem_o, a, b, idesc_o, (jj > 1 || ks > 0) ? 1u : 0u);
+            }
+            umma_commit(&bars->kv_empty[prev_stage]);
+            umma_commit(&bars->p_empty);
+            ++p_it;
+          }
+          if (jj < nk) {
+            prev_stage = kv_it % S;
+            ++kv_it;
+            ++s_it;
+          }
+        }
+        umma_commit(&bars->o_full);
+      }
+      // all issued MMAs complete before TMEM is released
+      umma_commit(&bars->done);
+      mbar_wait(&bars->done, 0, tmo, nullptr);
+    }
+  } else {
+    // =================================================================== epilogue
+    const int ew = warp - 2;               // 0..7
+    const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+    const int half = ew >> 2;              // 64-column half of S / of O
+    const int r = quarter * 32 + lane;     // row of the tile
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    int s_it = 0, kv_it = 0, p_it = 0;
+    int cur_head = -1;
+    for (int k = 0;; ++k) {
+      const int idx = snake_item(k, blockIdx.x, G);
+      if (idx >= count || *abort_flag) break;
+      const WorkItem wi = p.items[idx];
+      const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+      if (per_head_rab && wi.head != cur_head) {
+        named_bar_sync(1, 32 * kEpiWarps);
+        for (int c = threadIdx.x - 64; c < kNumBuckets; c += 32 * kEpiWarps) {
+          pos_b[c] = p.pos_bias[wi.head * p.rab_head_stride + c];
+          time_b[c] = p.time_bias[wi.head * p.rab_head_stride + c];
+        }
+        named_bar_sync(1, 32 * kEpiWarps);
+        cur_head = wi.head;
+      }
+      const int r0 = wi.qtile * BM;
+      const int i = r0 + r;
+      const bool live = i < si.n;
+      const bool cand = i >= si.hist;
+      const int64_t ti = live ? p.timestamps[si.start + i] : 0;
+      const int posi = token_pos(i, si.hist);
+      const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
+      const int nk = kv_count(kr);
+      for (int jj = 0; jj < nk; ++jj, ++kv_it, ++s_it, ++p_it) {
+        const int c0 = kv_tile_at(kr, jj) * BN;
+        const int sb = s_it & 1;
+        const int st = kv_it % S;
+        if (!mbar_wait(&bars->s_full[sb], (s_it >> 1) & 1, tmo, abort_flag)) goto fail;
+        tc_fence_after();
+        uint32_t raw[2][32];
+        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + half * 64, raw[0]);
+        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + half * 64 + 32, raw[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
+        if (!mbar_wait(&bars->kv_full[st], (kv_it / S) & 1, tmo, abort_flag)) goto fail;
+        const TsStage& ts = tss[st];
+        // ---- classify this row's 64 columns
+        const int cl = c0 + half * 64;   // first column of the half
+        float pv[64];
+        bool any_live = live && (cand ? (cl < si.hist || (i >= cl && i < cl + 64)) : (cl <= i));
+        const bool full = live && (cand ? (cl + 63 < si.hist) : (cl + 63 <= i));
+        int mode = 0;  // 0: zero, 1: constant bias, 2: <= 3 time buckets (32-bit), 3: general
+        float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
+        int32_t th1 = 0x7FFFFFFF, th2 = 0x7FFFFFFF, th3 = 0x7FFFFFFF, ri = 0;
+        if (any_live) {
+          mode = 3;
+          if (full && posi - (cl + 63) >= kNumBuckets - 1) {
+            const int64_t tmn = ts.tmin[half], tmx = ts.tmax[half];
+            uint64_t dlo, dhi;
+            if (ti >= tmx) { dlo = (uint64_t)(ti - tmx); dhi = (uint64_t)(ti - tmn); }
+            else if (ti <= tmn) { dlo = (uint64_t)(tmn - ti); dhi = (uint64_t)(tmx - ti); }
+            else { dlo = 0; dhi = max((uint64_t)(ti - tmn), (uint64_t)(tmx - ti)); }
+            const int tlo = time_bucket_exact(dlo, thr), thi = time_bucket_exact(dhi, thr);
+            const float pb127 = pos_b[kNumBuckets - 1];
+            const int64_t rel_i = ti - tmn;
+            if (tlo == thi) {
+              mode = 1;
+              b0 = pb127 + time_b[tlo];
+            } else if (thi - tlo <= 3 && !ts.wide[half] && rel_i > -(1ll << 30) && rel_i < (1ll << 30)) {
+              mode = 2;
+              ri = (int32_t)rel_i;
+              b0 = pb127 + time_b[tlo];
+              b1 = pb127 + time_b[min(tlo + 1, thi)];
+              b2 = pb127 + time_b[min(tlo + 2, thi)];
+              b3 = pb127 + time_b[min(tlo + 3, thi)];
+              auto th32 = [&](int b) -> int32_t {
+                if (b > thi) return 0x7FFFFFFF;
+                const int64_t v = thr[b];
+                return v > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)v;
+              };
+              th1 = th32(tlo + 1);
+              th2 = th32(tlo + 2);
+              th3 = th32(tlo + 3);
+            }
+          }
+        }
+        // ---- bias, SiLU, mask
+        if (mode == 0) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) pv[e] = 0.f;
+        } else if (mode == 1) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) pv[e] = silu_tanh(__uint_as_float(raw[e >> 5][e & 31]) + b0);
+        } else if (mode == 2) {
+#pragma unroll
+          for (int e4 = 0; e4 < 16; ++e4) {
+            const int4 rel4 = *reinterpret_cast<const int4*>(&ts.rel[half * 64 + e4 * 4]);
+            const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int e = e4 * 4 + u;
+              const int32_t dd = abs(ri - rv[u]);
+              float bias = b0;
+              bias = dd >= th1 ? b1 : bias;
+              bias = dd >= th2 ? b2 : bias;
+              bias = dd >= th3 ? b3 : bias;
+              pv[e] = silu_tanh(__uint_as_float(raw[e >> 5][e & 31]) + bias);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const int j = cl + e;
+            float v = 0.f;
+            if (attended(i, j, si.n, si.hist)) {
+              const int pb = pos_bucket(posi, token_pos(j, si.hist));
+              const int tb = time_bucket_exact(abs_diff_i64(ti, ts.ts[half * 64 + e]), thr);
+              v = silu_tanh(__uint_as_float(raw[e >> 5][e & 31]) + pos_b[pb] + time_b[tb]);
+            }
+            pv[e] = v;
+          }
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+        // ---- P -> shared memory (A operand, K-major, 128-byte swizzle)
+        if (!mbar_wait(&bars->p_empty, (p_it & 1) ^ 1, tmo, abort_flag)) goto fail;
+        const uint32_t prow = sP + half * kBoxBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(prow + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full);
+      }
+      // ---- O readout
+      if (!mbar_wait(&bars->o_full, k & 1, tmo, abort_flag)) goto fail;
+      tc_fence_after();
+      constexpr int kOc = DV / 2;  // columns of O per thread
+      uint32_t oraw[kOc];
+      if constexpr (kOc == 64) {
+        tmem_ld_32x32b_x32(tmem_o + lane_off + half * kOc, *reinterpret_cast<uint32_t(*)[32]>(&oraw[0]));
+        tmem_ld_32x32b_x32(tmem_o + lane_off + half * kOc + 32, *reinterpret_cast<uint32_t(*)[32]>(&oraw[32]));
+      } else {
+        tmem_ld_32x32b_x32(tmem_o + lane_off + half * kOc, *reinterpret_cast<uint32_t(*)[32]>(&oraw[0]));
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_empty);
+      if (live) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(si.start + i) * p.ldo +
+                             (int64_t)wi.head * DV + half * kOc;
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(oraw[8 * c + 0]) * si.inv_n, __uint_as_float(oraw[8 * c + 1]) * si.inv_n);
+          v.y = pack_bf16x2(__uint_as_float(oraw[8 * c + 2]) * si.inv_n, __uint_as_float(oraw[8 * c + 3]) * si.inv_n);
+          v.z = pack_bf16x2(__uint_as_float(oraw[8 * c + 4]) * si.inv_n, __uint_as_float(oraw[8 * c + 5]) * si.inv_n);
+          v.w = pack_bf16x2(__uint_as_float(oraw[8 * c + 6]) * si.inv_n, __uint_as_float(oraw[8 * c + 7]) * si.inv_n);
+          *reinterpret_cast<uint4*>(out + 8 * c) = v;
+        }
+      }
+    }
+  }
+  goto teardown;
+fail:
+  set_status(p.status, HSTU_ERR_TIMEOUT);
+  *abort_flag = 1;
+  if (warp == 0) {
+    // let every copy this warp may have issued land before the CTA exits (bounded)
+    for (int s = 0; s < S; ++s) {
+      mbar_wait(&bars->kv_full[s], 0, 100000000ll, nullptr);
+      mbar_wait(&bars->kv_full[s], 1, 100000000ll, nullptr);
+    }
+    mbar_wait(&bars->q_full, 0, 100000000ll, nullptr);
+    mbar_wait(&bars->q_full, 1, 100000000ll, nullptr);
+  }
+teardown:
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over [rows, cols] with row stride `ld` elements; box 64 columns x 128 rows, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int DH>
+cudaError_t launch_tc(const AttnFwdParams& p, int grid, cudaStream_t st) {
+  TcParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.p = p;
+  const int64_t hd = (int64_t)p.num_heads * DH;
+  if (!make_map(&tp.map_q, p.q, hd, p.total_rows, p.ldq) || !make_map(&tp.map_k, p.k, hd, p.total_rows, p.ldk) ||
+      !make_map(&tp.map_v, p.v, hd, p.total_rows, p.ldv))
+    return cudaErrorInvalidValue;
+  auto kern = attn_fwd_tc_kernel<DH>;
+  const int smem = Layout<DH>::kAlloc;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, st>>>(tp);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// diagnostics
+__global__ void debug_buckets_kernel(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,
+                                     const Thresholds thr_in, const int32_t* pairs, int n, int32_t* out) {
+  __shared__ int64_t thr[kNumBuckets];
+  for (int c = threadIdx.x; c < kNumBuckets; c += blockDim.x) thr[c] = thr_in.v[c];
+  __syncthreads();
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+    const SeqInfo si = load_seq(offs, num_targets, pairs[3 * e]);
+    const int i = pairs[3 * e + 1], j = pairs[3 * e + 2];
+    int pb = -1, tb = -1, att = 0;
+    if (i >= 0 && i < si.n && j >= 0 && j < si.n) {
+      pb = pos_bucket(token_pos(i, si.hist), token_pos(j, si.hist));
+      tb = time_bucket_exact(abs_diff_i64(ts[si.start + i], ts[si.start + j]), thr);
+      att = attended(i, j, si.n, si.hist) ? 1 : 0;
+    }
+    out[3 * e] = pb;
+    out[3 * e + 1] = tb;
+    out[3 * e + 2] = att;
+  }
+}
+
+__global__ void timeout_probe_kernel(long long timeout_ns, int32_t* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the bounded wait must give up
+  if (!mbar_wait(&bar, 0, timeout_ns, nullptr)) {
+    if (threadIdx.x == 0) *status = HSTU_ERR_TIMEOUT;
+  } else if (threadIdx.x == 0) {
+    *status = HSTU_OK;
+  }
+}
+
+}  // namespace
+
+int tc_tile_m() { return BM; }
+
+bool tc_attn_supported(int dtype, int dh) { return dtype == HSTU_DTYPE_BF16 && (dh == 64 || dh == 128); }
+
+int tc_attn_grid(int max_items) {
+  const int s = num_sms();
+  return max_items < 1 ? 1 : (max_items < s ? max_items : s);
+}
+
+cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStream_t st) {
+  if (p.total_rows <= 0) return cudaSuccess;
+  if (dh == 128) return launch_tc<128>(p, grid, st);
+  if (dh == 64) return launch_tc<64>(p, grid, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,
+                                 const Thresholds& thr, const int32_t* pairs, int n, int32_t* out, cudaStream_t st) {
+  const int grid = (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024;
+  debug_buckets_kernel<<<grid, 256, 0, st>>>(offs, num_targets, ts, thr, pairs, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_timeout_probe(long long timeout_ns, int32_t* status, cudaStream_t st) {
+  timeout_probe_kernel<<<1, 32, 0, st>>>(timeout_ns, status);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

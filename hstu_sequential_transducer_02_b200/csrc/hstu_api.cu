@@ -1,0 +1,726 @@
+// The C ABI of libhstu: argument validation, workspace carving and the launch
+// sequence of each call.  Every step of the computation runs in this
+// library's own kernels; nothing here computes on the host except the
+// time-bucket threshold table.
+#include <math.h>
+#include <mutex>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "trace.cuh"
+
+using namespace hstu;
+
+namespace {
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr long long kDefaultTimeoutNs = 2000000000ll;  // a device-side wait gives up after 2 s
+
+// ---------------------------------------------------------------- workspace carving
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base((char*)b) {}
+  template <typename T>
+  T* take(size_t count) {
+    off = (off + 255) & ~(size_t)255;
+    T* p = base ? (T*)(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+  size_t size() const { return (off + 255) & ~(size_t)255; }
+};
+
+size_t elem_size(int dtype) { return dtype == HSTU_DTYPE_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA; }
+
+#define HSTU_TRY(expr)                      \
+  do {                                      \
+    int _s = (expr);                        \
+    if (_s != HSTU_OK) return _s;           \
+  } while (0)
+#define HSTU_CUDA(expr)                     \
+  do {                                      \
+    cudaError_t _e = (expr);                \
+    if (_e != cudaSuccess) return HSTU_ERR_CUDA; \
+  } while (0)
+
+// ---------------------------------------------------------------- thresholds
+int64_t bucket_floor(int64_t dt, double div) {
+  double v = (double)(dt < 1 ? 1 : dt);
+  return (int64_t)floor(log(v) / div);
+}
+
+void build_thresholds(double div, int nb, int64_t* out) {
+  out[0] = 0;
+  for (int b = 1; b < nb; ++b) {
+    if (bucket_floor(INT64_MAX, div) < b) { out[b] = INT64_MAX; continue; }
+    int64_t lo = 1, hi = INT64_MAX;  // f(hi) >= b
+    if (bucket_floor(lo, div) >= b) { out[b] = lo; continue; }
+    while (hi - lo > 1) {
+      int64_t mid = lo + (hi - lo) / 2;
+      if (bucket_floor(mid, div) >= b) hi = mid; else lo = mid;
+    }
+    out[b] = hi;
+  }
+}
+
+std::mutex g_thr_mu;
+double g_thr_div = -1.0;
+Thresholds g_thr;
+
+Thresholds thresholds_for(double div) {
+  std::lock_guard<std::mutex> lk(g_thr_mu);
+  if (div != g_thr_div) {
+    build_thresholds(div, kNumBuckets, g_thr.v);
+    g_thr_div = div;
+  }
+  return g_thr;
+}
+
+// ---------------------------------------------------------------- validation
+int check_attn_desc(const hstu_attn_desc* d) {
+  if (!d) return HSTU_ERR_INVALID_ARG;
+  if (d->num_heads < 1 || d->num_heads > 1024) return HSTU_ERR_INVALID_ARG;
+  if (d->num_pos_buckets != kNumBuckets || d->num_time_buckets != kNumBuckets) return HSTU_ERR_UNSUPPORTED;
+  if (d->dtype != HSTU_DTYPE_F32 && d->dtype != HSTU_DTYPE_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (d->dqk != d->dv) return HSTU_ERR_UNSUPPORTED;
+  if (d->dqk != 32 && d->dqk != 64 && d->dqk != 128) return HSTU_ERR_UNSUPPORTED;
+  if (d->rab_head_stride != 0 && d->rab_head_stride != kNumBuckets) return HSTU_ERR_INVALID_ARG;
+  if (!(d->time_div > 0.0) || !isfinite(d->time_div)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+int check_jagged(const hstu_jagged* jb) {
+  if (!jb) return HSTU_ERR_INVALID_ARG;
+  if (jb->batch < 0 || jb->total_tokens < 0) return HSTU_ERR_INVALID_ARG;
+  if (!jb->seq_offsets || (jb->total_tokens > 0 && !jb->timestamps)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+int check_rows(const void* p, int64_t ld, int64_t min_ld, int dtype) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  if (ld < min_ld) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(p) || ((ld * (int64_t)elem_size(dtype)) % 16) != 0) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+// ---------------------------------------------------------------- attention
+struct AttnWs {
+  int32_t* status;
+  int32_t* count;
+  WorkItem* items;
+  float* dq_accum;
+  int capacity;
+};
+
+bool use_tc(const hstu_attn_desc* d) {
+  return !(d->flags & HSTU_FLAG_FORCE_SIMT) && tc_attn_supported(d->dtype, d->dqk);
+}
+
+int attn_tile(const hstu_attn_desc* d) { return use_tc(d) ? tc_tile_m() : simt_tile_m(); }
+
+AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd) {
+  AttnWs w;
+  w.status = c.take<int32_t>(kStatusBytes / 4);
+  w.count = c.take<int32_t>(64);
+  const int tile = bwd ? simt_tile_m() : attn_tile(d);
+  w.capacity = (int)work_list_capacity(B, T, d->num_heads, tile);
+  w.items = c.take<WorkItem>(w.capacity);
+  w.dq_accum = bwd ? c.take<float>((size_t)T * d->num_heads * d->dqk) : nullptr;
+  return w;
+}
+
+int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                 int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias, void* out,
+                 int64_t ldo, const AttnWs& w, cudaStream_t st) {
+  const int tile = attn_tile(d);
+  {
+    TraceScope tr("sched_fwd", st);
+    HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, d->num_heads,
+                                     tile, tile, 0, w.capacity, w.items, w.count, w.status, st));
+  }
+  AttnFwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.seq_offsets = jb->seq_offsets;
+  p.num_targets = jb->num_targets;
+  p.timestamps = jb->timestamps;
+  p.q = q; p.ldq = ldq; p.k = k; p.ldk = ldk; p.v = v; p.ldv = ldv;
+  p.out = out; p.ldo = ldo;
+  p.pos_bias = pos_bias; p.time_bias = time_bias;
+  p.rab_head_stride = d->rab_head_stride;
+  p.num_heads = d->num_heads;
+  p.total_rows = jb->total_tokens;
+  p.thr = thresholds_for(d->time_div);
+  p.items = w.items;
+  p.item_count = w.count;
+  p.status = w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  if (use_tc(d)) {
+    TraceScope tr("attn_fwd_tc", st);
+    HSTU_CUDA(launch_attn_fwd_tc(p, d->dqk, tc_attn_grid(w.capacity), st));
+  } else {
+    TraceScope tr("attn_fwd_simt", st);
+    int grid = w.capacity < 148 * 4 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 4;
+    HSTU_CUDA(launch_attn_fwd_simt(p, d->dtype, d->dqk, grid, st));
+  }
+  return HSTU_OK;
+}
+
+int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                 int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias,
+                 const void* dout, int64_t lddo, void* dq, int64_t lddq, void* dk, int64_t lddk, void* dv,
+                 int64_t lddv, float* dpos, float* dtime, const AttnWs& w, cudaStream_t st) {
+  const int tile = simt_tile_m();
+  const int H = d->num_heads, dh = d->dqk;
+  {
+    TraceScope tr("sched_bwd", st);
+    HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, H, tile, tile, 1,
+                                     w.capacity, w.items, w.count, w.status, st));
+  }
+  HSTU_CUDA(cudaMemsetAsync(w.dq_accum, 0, sizeof(float) * (size_t)jb->total_tokens * H * dh, st));
+  AttnBwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.seq_offsets = jb->seq_offsets;
+  p.num_targets = jb->num_targets;
+  p.timestamps = jb->timestamps;
+  p.q = q; p.ldq = ldq; p.k = k; p.ldk = ldk; p.v = v; p.ldv = ldv;
+  p.dout = dout; p.lddo = lddo;
+  p.dq_accum = w.dq_accum;
+  p.dk = dk; p.lddk = lddk; p.dv = dv; p.lddv = lddv;
+  p.pos_bias = pos_bias; p.time_bias = time_bias;
+  p.d_pos_bias = dpos; p.d_time_bias = dtime;
+  p.rab_head_stride = d->rab_head_stride;
+  p.num_heads = H;
+  p.total_rows = jb->total_tokens;
+  p.thr = thresholds_for(d->time_div);
+  p.items = w.items;
+  p.item_count = w.count;
+  p.status = w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  int grid = w.capacity < 148 * 2 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 2;
+  {
+    TraceScope tr("attn_bwd_simt", st);
+    HSTU_CUDA(launch_attn_bwd_simt(p, d->dtype, dh, grid, st));
+  }
+  {
+    TraceScope tr("dq_finalize", st);
+    HSTU_CUDA(launch_dq_finalize(w.dq_accum, jb->seq_offsets, jb->batch, H, dh, d->dtype, dq, lddq, 148 * 8, st));
+  }
+  return HSTU_OK;
+}
+
+// ---------------------------------------------------------------- GEMM dispatch
+int gemm(const GemmParams& p, int dtype, int flags, cudaStream_t st, const char* name) {
+  if (!(flags & HSTU_FLAG_FORCE_SIMT) && tc_gemm_supported(p, dtype)) {
+    TraceScope tr(name, st);
+    return cuda_status(launch_gemm_tc(p, st));
+  }
+  TraceScope tr(name, st);
+  return cuda_status(launch_gemm_simt(p, dtype, st));
+}
+
+// ---------------------------------------------------------------- layer
+int check_layer(const hstu_layer_desc* d, const hstu_layer_weights* w) {
+  if (!d || !w) return HSTU_ERR_INVALID_ARG;
+  HSTU_TRY(check_attn_desc(&d->attn));
+  const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
+  if (dm < 8 || dm > 1024 || dm % 8) return HSTU_ERR_UNSUPPORTED;
+  if (hv > 1024 || hv % 8) return HSTU_ERR_UNSUPPORTED;
+  if (!(d->ln_eps >= 0.f)) return HSTU_ERR_INVALID_ARG;
+  const void* ptrs[] = {w->w1, w->b1, w->ln1_gamma, w->ln1_beta, w->ln2_gamma, w->ln2_beta,
+                        w->w2, w->b2, w->pos_bias, w->time_bias};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+struct LayerBufs {
+  void* xhat; float* mu1; float* rs1; void* z; void* uvqk; void* o; float* mu2; float* rs2; void* g;
+};
+
+struct LayerFwdWs {
+  AttnWs attn;
+  LayerBufs b;
+};
+
+LayerFwdWs carve_layer_fwd(Carver& c, const hstu_layer_desc* d, int B, int T, bool need_all) {
+  LayerFwdWs w;
+  w.attn = carve_attn(c, &d->attn, B, T, false);
+  const size_t es = elem_size(d->attn.dtype);
+  const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
+  (void)need_all;
+  w.b.xhat = c.take<char>((size_t)T * dm * es);
+  w.b.mu1 = c.take<float>(T);
+  w.b.rs1 = c.take<float>(T);
+  w.b.z = nullptr;
+  w.b.uvqk = c.take<char>((size_t)T * 4 * hv * es);
+  w.b.o = c.take<char>((size_t)T * hv * es);
+  w.b.mu2 = c.take<float>(T);
+  w.b.rs2 = c.take<float>(T);
+  w.b.g = c.take<char>((size_t)T * hv * es);
+  return w;
+}
+
+int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const hstu_jagged* jb, const void* x,
+                  void* y, const hstu_layer_saved* saved, const LayerFwdWs& ws, cudaStream_t st) {
+  const int dt = d->attn.dtype;
+  const int dm = d->d_model, H = d->attn.num_heads, dh = d->attn.dv, hv = H * dh;
+  const int T = jb->total_tokens;
+  const int32_t* rows = jb->seq_offsets + jb->batch;  // device row count
+  LayerBufs b = ws.b;
+  if (saved) {
+    b.xhat = saved->xhat; b.mu1 = saved->ln1_mean; b.rs1 = saved->ln1_rstd; b.z = saved->z;
+    b.uvqk = saved->uvqk; b.o = saved->attn_out; b.mu2 = saved->ln2_mean; b.rs2 = saved->ln2_rstd;
+  }
+  // (A1) LayerNorm1
+  {
+    TraceScope tr("ln1", st);
+    HSTU_CUDA(launch_layer_norm(x, dm, w->ln1_gamma, w->ln1_beta, d->ln_eps, b.xhat, dm, b.mu1, b.rs1, T, rows, dm,
+                                dt, st));
+  }
+  // (A1) f1 + SiLU, split layout U | V | Q | K
+  GemmParams g1;
+  memset(&g1, 0, sizeof(g1));
+  g1.M = T; g1.N = 4 * hv; g1.K = dm;
+  g1.A = b.xhat; g1.sam = dm; g1.sak = 1;
+  g1.B = w->w1; g1.sbn = dm; g1.sbk = 1;
+  g1.epi = EPI_BIAS_SILU; g1.bias = w->b1;
+  g1.out = b.uvqk; g1.ldo = 4 * hv;
+  g1.out2 = b.z; g1.ldo2 = 4 * hv;
+  g1.rows_dev = rows;
+  HSTU_TRY(gemm(g1, dt, d->attn.flags, st, "gemm_f1_silu"));
+  // (A2-A4) attention
+  const size_t es = elem_size(dt);
+  const char* uvqk = (const char*)b.uvqk;
+  HSTU_TRY(run_attn_fwd(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + 1 * hv * es,
+                        4 * hv, w->pos_bias, w->time_bias, b.o, hv, ws.attn, st));
+  // (A5) LayerNorm2(A V) * U
+  {
+    TraceScope tr("ln2_gate", st);
+    HSTU_CUDA(launch_ln_gate(b.o, hv, b.uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.b.g, hv, b.mu2,
+                             b.rs2, T, rows, hv, dt, st));
+  }
+  // (A6) f2 + residual
+  GemmParams g2;
+  memset(&g2, 0, sizeof(g2));
+  g2.M = T; g2.N = dm; g2.K = hv;
+  g2.A = ws.b.g; g2.sam = hv; g2.sak = 1;
+  g2.B = w->w2; g2.sbn = hv; g2.sbk = 1;
+  g2.epi = EPI_BIAS_RESIDUAL; g2.bias = w->b2;
+  g2.residual = x; g2.ldr = dm;
+  g2.out = y; g2.ldo = dm;
+  g2.rows_dev = rows;
+  HSTU_TRY(gemm(g2, dt, d->attn.flags, st, "gemm_f2_residual"));
+  return HSTU_OK;
+}
+
+// backward workspace: attention bwd scratch + gradients of the intermediates
+struct LayerBwdWs {
+  AttnWs attn;
+  void* g;       // [T, hv] recomputed gate output
+  void* dg;      // [T, hv]
+  void* d_o;     // [T, hv]
+  void* duvqk;   // [T, 4hv]
+  void* dz;      // [T, 4hv]
+  float* dxhat;  // [T, dm] fp32
+};
+
+LayerBwdWs carve_layer_bwd(Carver& c, const hstu_layer_desc* d, int B, int T) {
+  LayerBwdWs w;
+  w.attn = carve_attn(c, &d->attn, B, T, true);
+  const size_t es = elem_size(d->attn.dtype);
+  const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
+  w.g = c.take<char>((size_t)T * hv * es);
+  w.dg = c.take<char>((size_t)T * hv * es);
+  w.d_o = c.take<char>((size_t)T * hv * es);
+  w.duvqk = c.take<char>((size_t)T * 4 * hv * es);
+  w.dz = c.take<char>((size_t)T * 4 * hv * es);
+  w.dxhat = c.take<float>((size_t)T * dm);
+  return w;
+}
+
+int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const hstu_jagged* jb, const void* x,
+                  const hstu_layer_saved* sv, const void* dy, void* dx, const hstu_layer_grads* gr,
+                  const LayerBwdWs& ws, cudaStream_t st) {
+  const int dt = d->attn.dtype;
+  const int dm = d->d_model, H = d->attn.num_heads, dh = d->attn.dv, hv = H * dh;
+  const int T = jb->total_tokens;
+  const int32_t* rows = jb->seq_offsets + jb->batch;
+  const size_t es = elem_size(dt);
+  const int fl = d->attn.flags;
+  void* duvqk = gr->duvqk ? gr->duvqk : ws.duvqk;
+  // recompute g = LN2(o) * U (cheaper to recompute than to keep)
+  HSTU_CUDA(launch_ln_gate(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g, hv,
+                           nullptr, nullptr, T, rows, hv, dt, st));
+  // y = x + g W2^T + b2:  dW2 = dy^T g, db2 = colsum(dy), dg = dy W2
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = dm; p.N = hv; p.K = T;                 // dW2[m=out, n=in] = sum_t dy[t, m] g[t, n]
+  p.A = dy; p.sam = 1; p.sak = dm;
+  p.B = ws.g; p.sbn = 1; p.sbk = hv;
+  p.epi = EPI_STORE_F32; p.out = gr->dw2; p.ldo = hv; p.k_dev = rows;
+  HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw2"));
+  HSTU_CUDA(launch_col_sum(dy, dm, T, rows, dm, dt, gr->db2, st));
+  memset(&p, 0, sizeof(p));
+  p.M = T; p.N = hv; p.K = dm;                 // dg[t, n] = sum_m dy[t, m] W2[m, n]
+  p.A = dy; p.sam = dm; p.sak = 1;
+  p.B = w->w2; p.sbn = 1; p.sbk = hv;
+  p.epi = EPI_STORE; p.out = ws.dg; p.ldo = hv; p.rows_dev = rows;
+  HSTU_TRY(gemm(p, dt, fl, st, "gemm_dg"));
+  // g = (LN2(o) gamma2 + beta2) * U:  dU, d_o, dgamma2, dbeta2
+  HSTU_CUDA(cudaMemsetAsync(gr->dln2_gamma, 0, sizeof(float) * hv, st));
+  HSTU_CUDA(cudaMemsetAsync(gr->dln2_beta, 0, sizeof(float) * hv, st));
+  HSTU_CUDA(launch_ln_gate_bwd(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, sv->ln2_mean, sv->ln2_rstd, ws.dg,
+                               hv, ws.d_o, hv, gr->dln2_gamma, gr->dln2_beta, T, rows, hv, dt, st));
+  HSTU_CUDA(launch_ln_gate_du(sv->attn_out, hv, w->ln2_gamma, w->ln2_beta, sv->ln2_mean, sv->ln2_rstd, ws.dg, hv,
+                              duvqk, 4 * hv, T, rows, hv, dt, st));
+  // attention backward -> dV, dQ, dK columns of duvqk, rab grads
+  const size_t rab_n = (size_t)(d->attn.rab_head_stride ? H : 1) * kNumBuckets;
+  HSTU_CUDA(cudaMemsetAsync(gr->dpos_bias, 0, sizeof(float) * rab_n, st));
+  HSTU_CUDA(cudaMemsetAsync(gr->dtime_bias, 0, sizeof(float) * rab_n, st));
+  const char* uvqk = (const char*)sv->uvqk;
+  char* du = (char*)duvqk;
+  HSTU_TRY(run_attn_bwd(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + hv * es,
+                        4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, du + 2 * hv * es, 4 * hv, du + 3 * hv * es,
+                        4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias, ws.attn, st));
+  // a = SiLU(z): dz = da * SiLU'(z)
+  HSTU_CUDA(launch_silu_bwd(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, st));
+  // z = xhat W1^T + b1: dW1 = dz^T xhat, db1 = colsum(dz), dxhat = dz W1
+  memset(&p, 0, sizeof(p));
+  p.M = 4 * hv; p.N = dm; p.K = T;
+  p.A = ws.dz; p.sam = 1; p.sak = 4 * hv;
+  p.B = sv->xhat; p.sbn = 1; p.sbk = dm;
+  p.epi = EPI_STORE_F32; p.out = gr->dw1; p.ldo = dm; p.k_dev = rows;
+  HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw1"));
+  HSTU_CUDA(launch_col_sum(ws.dz, 4 * hv, T, rows, 4 * hv, dt, gr->db1, st));
+  memset(&p, 0, sizeof(p));
+  p.M = T; p.N = dm; p.K = 4 * hv;
+  p.A = ws.dz; p.sam = 4 * hv; p.sak = 1;
+  p.B = w->w1; p.sbn = 1; p.sbk = dm;
+  p.epi = EPI_STORE_F32; p.out = ws.dxhat; p.ldo = dm; p.rows_dev = rows;
+  HSTU_TRY(gemm(p, dt, fl, st, "gemm_dxhat"));
+  // xhat = LN1(x): dx = dy + LN1 backward
+  HSTU_CUDA(cudaMemsetAsync(gr->dln1_gamma, 0, sizeof(float) * dm, st));
+  HSTU_CUDA(cudaMemsetAsync(gr->dln1_beta, 0, sizeof(float) * dm, st));
+  HSTU_CUDA(launch_ln_bwd(x, dm, w->ln1_gamma, sv->ln1_mean, sv->ln1_rstd, ws.dxhat, dm, dy, dm, dx, dm,
+                          gr->dln1_gamma, gr->dln1_beta, T, rows, dm, dt, st));
+  return HSTU_OK;
+}
+
+}  // namespace
+
+// =============================================================================
+// exported entry points
+// =============================================================================
+extern "C" {
+
+const char* hstu_status_string(int status) {
+  switch (status) {
+    case HSTU_OK: return "ok";
+    case HSTU_ERR_INVALID_ARG: return "invalid argument";
+    case HSTU_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HSTU_ERR_CUDA: return "CUDA error";
+    case HSTU_ERR_TIMEOUT: return "device wait timed out";
+    case HSTU_ERR_WORKSPACE: return "workspace too small";
+    case HSTU_ERR_BAD_OFFSETS: return "invalid sequence offsets or target counts";
+    default: return "unknown status";
+  }
+}
+
+int hstu_version(void) { return kVersion; }
+
+int hstu_build_time_thresholds(double time_div, int32_t num_buckets, int64_t* out) {
+  if (!out || !(time_div > 0.0) || !isfinite(time_div) || num_buckets < 2 || num_buckets > 1024)
+    return HSTU_ERR_INVALID_ARG;
+  build_thresholds(time_div, num_buckets, out);
+  return HSTU_OK;
+}
+
+int hstu_workspace_status(const void* workspace, int32_t* status, void* stream) {
+  if (!workspace || !status) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  HSTU_CUDA(cudaMemcpyAsync(status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  HSTU_CUDA(cudaStreamSynchronize(st));
+  return HSTU_OK;
+}
+
+int hstu_attn_fwd_workspace_size(const hstu_attn_desc* desc, int32_t batch, int32_t total_tokens, size_t* bytes) {
+  HSTU_TRY(check_attn_desc(desc));
+  if (!bytes || batch < 0 || total_tokens < 0) return HSTU_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_attn(c, desc, batch, total_tokens, false);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int hstu_attn_fwd(const hstu_attn_desc* desc, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                  int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias, void* out,
+                  int64_t ldo, void* workspace, size_t workspace_bytes, void* stream) {
+  HSTU_TRY(check_attn_desc(desc));
+  HSTU_TRY(check_jagged(jb));
+  const int hd = desc->num_heads * desc->dqk;
+  HSTU_TRY(check_rows(q, ldq, hd, desc->dtype));
+  HSTU_TRY(check_rows(k, ldk, hd, desc->dtype));
+  HSTU_TRY(check_rows(v, ldv, hd, desc->dtype));
+  HSTU_TRY(check_rows(out, ldo, hd, desc->dtype));
+  if (!pos_bias || !time_bias) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(hstu_attn_fwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(workspace);
+  AttnWs w = carve_attn(c, desc, jb->batch, jb->total_tokens, false);
+  HSTU_CUDA(cudaMemsetAsync(w.status, 0, kStatusBytes, st));
+  return run_attn_fwd(desc, jb, q, ldq, k, ldk, v, ldv, pos_bias, time_bias, out, ldo, w, st);
+}
+
+int hstu_attn_bwd_workspace_size(const hstu_attn_desc* desc, int32_t batch, int32_t total_tokens, size_t* bytes) {
+  HSTU_TRY(check_attn_desc(desc));
+  if (!bytes || batch < 0 || total_tokens < 0) return HSTU_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_attn(c, desc, batch, total_tokens, true);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int hstu_attn_bwd(const hstu_attn_desc* desc, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                  int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias,
+                  const void* dout, int64_t lddo, void* dq, int64_t lddq, void* dk, int64_t lddk, void* dv,
+                  int64_t lddv, float* d_pos_bias, float* d_time_bias, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  HSTU_TRY(check_attn_desc(desc));
+  HSTU_TRY(check_jagged(jb));
+  const int hd = desc->num_heads * desc->dqk;
+  HSTU_TRY(check_rows(q, ldq, hd, desc->dtype));
+  HSTU_TRY(check_rows(k, ldk, hd, desc->dtype));
+  HSTU_TRY(check_rows(v, ldv, hd, desc->dtype));
+  HSTU_TRY(check_rows(dout, lddo, hd, desc->dtype));
+  HSTU_TRY(check_rows(dq, lddq, hd, desc->dtype));
+  HSTU_TRY(check_rows(dk, lddk, hd, desc->dtype));
+  HSTU_TRY(check_rows(dv, lddv, hd, desc->dtype));
+  if (!pos_bias || !time_bias || !d_pos_bias || !d_time_bias) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(hstu_attn_bwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(workspace);
+  AttnWs w = carve_attn(c, desc, jb->batch, jb->total_tokens, true);
+  HSTU_CUDA(cudaMemsetAsync(w.status, 0, kStatusBytes, st));
+  return run_attn_bwd(desc, jb, q, ldq, k, ldk, v, ldv, pos_bias, time_bias, dout, lddo, dq, lddq, dk, lddk, dv,
+                      lddv, d_pos_bias, d_time_bias, w, st);
+}
+
+int hstu_layer_fwd_workspace_size(const hstu_layer_desc* desc, int32_t batch, int32_t total_tokens, size_t* bytes) {
+  if (!desc || !bytes || batch < 0 || total_tokens < 0) return HSTU_ERR_INVALID_ARG;
+  HSTU_TRY(check_attn_desc(&desc->attn));
+  Carver c(nullptr);
+  carve_layer_fwd(c, desc, batch, total_tokens, true);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, const hstu_jagged* jb, const void* x,
+                   void* y, const hstu_layer_saved* saved, void* workspace, size_t workspace_bytes, void* stream) {
+  HSTU_TRY(check_layer(desc, w));
+  HSTU_TRY(check_jagged(jb));
+  const int dm = desc->d_model;
+  const int dt = desc->attn.dtype;
+  HSTU_TRY(check_rows(x, dm, dm, dt));
+  HSTU_TRY(check_rows(y, dm, dm, dt));
+  if (x == y) return HSTU_ERR_INVALID_ARG;
+  if (saved) {
+    const void* ps[] = {saved->xhat, saved->ln1_mean, saved->ln1_rstd, saved->z, saved->uvqk,
+                        saved->attn_out, saved->ln2_mean, saved->ln2_rstd};
+    for (const void* p : ps)
+      if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  }
+  size_t need;
+  HSTU_TRY(hstu_layer_fwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(workspace);
+  LayerFwdWs ws = carve_layer_fwd(c, desc, jb->batch, jb->total_tokens, true);
+  HSTU_CUDA(cudaMemsetAsync(ws.attn.status, 0, kStatusBytes, st));
+  return run_layer_fwd(desc, w, jb, x, y, saved, ws, st);
+}
+
+int hstu_layer_bwd_workspace_size(const hstu_layer_desc* desc, int32_t batch, int32_t total_tokens, size_t* bytes) {
+  if (!desc || !bytes || batch < 0 || total_tokens < 0) return HSTU_ERR_INVALID_ARG;
+  HSTU_TRY(check_attn_desc(&desc->attn));
+  Carver c(nullptr);
+  carve_layer_bwd(c, desc, batch, total_tokens);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int hstu_layer_bwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, const hstu_jagged* jb, const void* x,
+                   const hstu_layer_saved* saved, const void* dy, void* dx, const hstu_layer_grads* g,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  HSTU_TRY(check_layer(desc, w));
+  HSTU_TRY(check_jagged(jb));
+  if (!saved || !g) return HSTU_ERR_INVALID_ARG;
+  const int dm = desc->d_model;
+  const int dt = desc->attn.dtype;
+  HSTU_TRY(check_rows(x, dm, dm, dt));
+  HSTU_TRY(check_rows(dy, dm, dm, dt));
+  HSTU_TRY(check_rows(dx, dm, dm, dt));
+  const void* ps[] = {saved->xhat, saved->ln1_mean, saved->ln1_rstd, saved->z, saved->uvqk, saved->attn_out,
+                      saved->ln2_mean, saved->ln2_rstd, g->dw1, g->db1, g->dln1_gamma, g->dln1_beta,
+                      g->dln2_gamma, g->dln2_beta, g->dw2, g->db2, g->dpos_bias, g->dtime_bias};
+  for (const void* p : ps)
+    if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  if (g->duvqk && !aligned16(g->duvqk)) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(hstu_layer_bwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(workspace);
+  LayerBwdWs ws = carve_layer_bwd(c, desc, jb->batch, jb->total_tokens);
+  HSTU_CUDA(cudaMemsetAsync(ws.attn.status, 0, kStatusBytes, st));
+  return run_layer_bwd(desc, w, jb, x, saved, dy, dx, g, ws, st);
+}
+
+// ---------------------------------------------------------------- M-FALCON
+namespace {
+struct MfalconWs {
+  LayerFwdWs layer;
+  int32_t* offs;
+  int32_t* nt;
+  int64_t* ts;
+  void* x0;
+  void* x1;
+  int32_t* row_map;
+  int cap;
+};
+
+MfalconWs carve_mfalcon(Carver& c, const hstu_layer_desc* d, int U, int hist_total, int bm) {
+  MfalconWs w;
+  w.cap = hist_total + U * bm;
+  w.layer = carve_layer_fwd(c, d, U, w.cap, true);
+  const size_t es = elem_size(d->attn.dtype);
+  w.offs = c.take<int32_t>(U + 1);
+  w.nt = c.take<int32_t>(U > 0 ? U : 1);
+  w.ts = c.take<int64_t>(w.cap);
+  w.x0 = c.take<char>((size_t)w.cap * d->d_model * es);
+  w.x1 = c.take<char>((size_t)w.cap * d->d_model * es);
+  w.row_map = c.take<int32_t>(w.cap);
+  return w;
+}
+}  // namespace
+
+int mfalcon_rank_workspace_size(const hstu_layer_desc* desc, int32_t num_layers, int32_t num_users,
+                                int32_t hist_total, int32_t microbatch, size_t* bytes) {
+  if (!desc || !bytes || num_layers < 1 || num_users < 0 || hist_total < 0 || microbatch < 1)
+    return HSTU_ERR_INVALID_ARG;
+  HSTU_TRY(check_attn_desc(&desc->attn));
+  if ((int64_t)hist_total + (int64_t)num_users * microbatch >= (1ll << 31)) return HSTU_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  carve_mfalcon(c, desc, num_users, hist_total, microbatch);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, int32_t num_layers,
+                 int32_t num_users, int32_t hist_total, int32_t max_candidates, int32_t microbatch,
+                 const int32_t* hist_offsets, const void* hist_x, const int64_t* hist_ts,
+                 const int32_t* cand_offsets, const void* cand_x, const int64_t* cand_ts, void* cand_out,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!layers || num_layers < 1 || max_candidates < 0 || microbatch < 1) return HSTU_ERR_INVALID_ARG;
+  for (int l = 0; l < num_layers; ++l) HSTU_TRY(check_layer(desc, &layers[l]));
+  if (!hist_offsets || !cand_offsets || !cand_ts || !cand_out || !cand_x) return HSTU_ERR_INVALID_ARG;
+  if (hist_total > 0 && (!hist_x || !hist_ts)) return HSTU_ERR_INVALID_ARG;
+  const int dt = desc->attn.dtype;
+  const int dm = desc->d_model;
+  if ((hist_x && !aligned16(hist_x)) || !aligned16(cand_x) || !aligned16(cand_out)) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(mfalcon_rank_workspace_size(desc, num_layers, num_users, hist_total, microbatch, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(workspace);
+  MfalconWs w = carve_mfalcon(c, desc, num_users, hist_total, microbatch);
+  HSTU_CUDA(cudaMemsetAsync(w.layer.attn.status, 0, kStatusBytes, st));
+  const int n_mb = (max_candidates + microbatch - 1) / microbatch;
+  for (int mb = 0; mb < n_mb; ++mb) {
+    HSTU_CUDA(launch_mfalcon_pack(num_users, mb, microbatch, hist_offsets, hist_x, hist_ts, cand_offsets, cand_x,
+                                  cand_ts, dm, dt, w.offs, w.nt, w.ts, w.x0, w.row_map, nullptr, w.cap, st));
+    hstu_jagged jb;
+    jb.batch = num_users;
+    jb.total_tokens = w.cap;
+    jb.seq_offsets = w.offs;
+    jb.num_targets = w.nt;
+    jb.timestamps = w.ts;
+    void* cur = w.x0;
+    void* nxt = w.x1;
+    for (int l = 0; l < num_layers; ++l) {
+      HSTU_TRY(run_layer_fwd(desc, &layers[l], &jb, cur, nxt, nullptr, w.layer, st));
+      void* t = cur; cur = nxt; nxt = t;
+    }
+    HSTU_CUDA(launch_mfalcon_scatter(cur, dm, dt, w.row_map, w.offs + num_users, w.cap, cand_out, st));
+  }
+  return HSTU_OK;
+}
+
+// ---------------------------------------------------------------- Stochastic Length
+int hstu_stochastic_length_workspace_size(int32_t batch, int32_t total_tokens, size_t* bytes) {
+  if (!bytes || batch < 0 || total_tokens < 0) return HSTU_ERR_INVALID_ARG;
+  Carver c(nullptr);
+  c.take<int32_t>(kStatusBytes / 4);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int hstu_stochastic_length(int32_t batch, int32_t total_tokens, const int32_t* seq_offsets, const uint32_t* coins,
+                           const uint32_t* keys, int32_t max_len, uint32_t prob_u32, int32_t* out_offsets,
+                           int32_t* out_index, void* workspace, size_t workspace_bytes, void* stream) {
+  if (batch < 0 || total_tokens < 0 || max_len < 1 || !seq_offsets || !out_offsets) return HSTU_ERR_INVALID_ARG;
+  if (batch > 0 && (!coins || (total_tokens > 0 && (!keys || !out_index)))) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(hstu_stochastic_length_workspace_size(batch, total_tokens, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t* status = (int32_t*)workspace;
+  HSTU_CUDA(cudaMemsetAsync(status, 0, kStatusBytes, st));
+  HSTU_CUDA(launch_sl_select(batch, total_tokens, seq_offsets, coins, keys, max_len, prob_u32, out_offsets, out_index,
+                             nullptr, status, st));
+  return HSTU_OK;
+}
+
+int hstu_gather_rows(const void* src, void* dst, int64_t row_bytes, const int32_t* index, const int32_t* count,
+                     int32_t capacity, void* stream) {
+  if (!src || !dst || !index || !count || capacity < 0 || row_bytes <= 0 || row_bytes % 4) return HSTU_ERR_INVALID_ARG;
+  if (((uintptr_t)src & 3) || ((uintptr_t)dst & 3)) return HSTU_ERR_INVALID_ARG;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  return cuda_status(launch_gather_rows(src, dst, row_bytes, index, count, capacity, (cudaStream_t)stream));
+}
+
+// ---------------------------------------------------------------- diagnostics
+int hstu_debug_rab_buckets(const hstu_attn_desc* desc, const hstu_jagged* jb, const int32_t* pairs,
+                           int32_t num_pairs, int32_t* out, void* stream) {
+  HSTU_TRY(check_attn_desc(desc));
+  HSTU_TRY(check_jagged(jb));
+  if (num_pairs < 0 || (num_pairs > 0 && (!pairs || !out))) return HSTU_ERR_INVALID_ARG;
+  if (num_pairs == 0) return HSTU_OK;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  Thresholds thr = thresholds_for(desc->time_div);
+  return cuda_status(launch_debug_buckets(jb->seq_offsets, jb->num_targets, jb->timestamps, thr, pairs, num_pairs,
+                                          out, (cudaStream_t)stream));
+}
+
+int hstu_debug_timeout_probe(int64_t timeout_ns, int32_t* status_dev, void* stream) {
+  if (!status_dev || timeout_ns < 1 || timeout_ns > 2000000000ll) return HSTU_ERR_INVALID_ARG;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  return cuda_status(launch_timeout_probe(timeout_ns, status_dev, (cudaStream_t)stream));
+}
+
+}  // extern "C"

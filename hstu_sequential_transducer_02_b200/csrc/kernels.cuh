@@ -1,0 +1,154 @@
+// Internal launcher interfaces of libhstu (not part of the C ABI).
+#pragma once
+
+#include "common.cuh"
+
+namespace hstu {
+
+// ---------------------------------------------------------------- scheduler
+size_t work_list_capacity(int B, int T, int H, int tile);
+cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targets, int B, int T, int H,
+                                   int tm, int tk, int mode, int max_items, WorkItem* items,
+                                   int32_t* count, int32_t* status, cudaStream_t stream);
+
+// ---------------------------------------------------------------- attention
+// time-bucket thresholds, passed by value (kernel parameter space)
+struct Thresholds { int64_t v[kNumBuckets]; };
+
+struct AttnFwdParams {
+  const int32_t* seq_offsets;
+  const int32_t* num_targets;
+  const int64_t* timestamps;
+  const void* q; int64_t ldq;
+  const void* k; int64_t ldk;
+  const void* v; int64_t ldv;
+  void* out; int64_t ldo;
+  const float* pos_bias;
+  const float* time_bias;
+  int rab_head_stride;
+  int num_heads;
+  int total_rows;             // capacity T of the [T, .] tensors
+  Thresholds thr;
+  const WorkItem* items;
+  const int32_t* item_count;
+  int32_t* status;
+  long long timeout_ns;        // bound of every device-side wait
+};
+
+struct AttnBwdParams {
+  const int32_t* seq_offsets;
+  const int32_t* num_targets;
+  const int64_t* timestamps;
+  const void* q; int64_t ldq;
+  const void* k; int64_t ldk;
+  const void* v; int64_t ldv;
+  const void* dout; int64_t lddo;
+  float* dq_accum;            // [rows, H, dh] fp32, zeroed by the caller
+  void* dk; int64_t lddk;
+  void* dv; int64_t lddv;
+  const float* pos_bias;
+  const float* time_bias;
+  float* d_pos_bias;
+  float* d_time_bias;
+  int rab_head_stride;
+  int num_heads;
+  int total_rows;
+  Thresholds thr;
+  const WorkItem* items;
+  const int32_t* item_count;
+  int32_t* status;
+  long long timeout_ns;        // bound of every device-side wait
+};
+
+int simt_tile_m();
+cudaError_t launch_attn_fwd_simt(const AttnFwdParams& p, int dtype, int dh, int grid, cudaStream_t st);
+cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, int dtype, int dh, int grid, cudaStream_t st);
+cudaError_t launch_dq_finalize(const float* acc, const int32_t* offs, int B, int H, int dh, int dtype,
+                               void* dq, int64_t lddq, int grid, cudaStream_t st);
+
+// tcgen05 (sm_100a) attention forward, bf16 in/out, dh in {64, 128}
+int tc_tile_m();
+bool tc_attn_supported(int dtype, int dh);
+cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStream_t st);
+int tc_attn_grid(int max_items);
+
+cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,
+                                 const Thresholds& thr, const int32_t* pairs, int n, int32_t* out,
+                                 cudaStream_t st);
+cudaError_t launch_timeout_probe(long long timeout_ns, int32_t* status, cudaStream_t st);
+
+// ---------------------------------------------------------------- GEMM
+// C[m, n] = sum_k A(m, k) B(n, k) with element strides; fp32 accumulation.
+enum GemmEpilogue {
+  EPI_STORE_F32 = 0,       // out_f32[m*ldo + n] = acc  (beta: += when accumulate)
+  EPI_BIAS_SILU = 1,       // z = acc + bias[n]; out[m, n] = SiLU(z) (dtype); out2[m, n] = z if out2
+  EPI_BIAS_RESIDUAL = 2,   // out[m, n] = acc + bias[n] + residual[m, n] (dtype)
+  EPI_STORE = 3,           // out[m, n] = acc (dtype)
+  EPI_SILU_BWD = 4,        // out[m, n] = acc * SiLU'(aux[m, n]) (dtype) — unused by the forward path
+};
+
+struct GemmParams {
+  int M, N, K;
+  const void* A; int64_t sam, sak;
+  const void* B; int64_t sbn, sbk;
+  int epi;
+  const float* bias;
+  const void* residual; int64_t ldr;
+  void* out; int64_t ldo;
+  void* out2; int64_t ldo2;
+  const int32_t* rows_dev;   // if set: rows = min(M, *rows_dev)
+  const int32_t* k_dev;      // if set: reduction length = min(K, *k_dev)
+  int accumulate;            // EPI_STORE_F32: add to the existing value
+};
+
+cudaError_t launch_gemm_simt(const GemmParams& p, int dtype, cudaStream_t st);
+// tcgen05 GEMM: A [M, K] and B [N, K] both K-major (sak = sbk = 1), bf16
+bool tc_gemm_supported(const GemmParams& p, int dtype);
+cudaError_t launch_gemm_tc(const GemmParams& p, cudaStream_t st);
+
+// ---------------------------------------------------------------- row kernels
+cudaError_t launch_layer_norm(const void* x, int64_t ldx, const float* gamma, const float* beta, float eps,
+                              void* out, int64_t ldo, float* mean, float* rstd, int rows_cap,
+                              const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
+cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
+                           const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
+                           int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
+// backward of g = (LN2(o) gamma + beta) * u: writes d_o (dtype) and accumulates the
+// affine gradients (atomics; the caller zeroes them)
+cudaError_t launch_ln_gate_bwd(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
+                               const float* mean, const float* rstd, const void* dg, int64_t lddg,
+                               void* d_o, int64_t ld_do, float* dgamma, float* dbeta,
+                               int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
+// du = dg * (LN2(o) gamma + beta)
+cudaError_t launch_ln_gate_du(const void* o, int64_t ldo_in, const float* gamma, const float* beta,
+                              const float* mean, const float* rstd, const void* dg, int64_t lddg, void* du,
+                              int64_t lddu, int rows_cap, const int32_t* rows_dev, int d, int dtype,
+                              cudaStream_t st);
+// backward of xhat = LN1(x): dx = dres + LNback(dxhat); accumulates dgamma/dbeta
+cudaError_t launch_ln_bwd(const void* x, int64_t ldx, const float* gamma, const float* mean, const float* rstd,
+                          const float* dxhat, int64_t lddxh, const void* dres, int64_t lddres, void* dx,
+                          int64_t lddx, float* dgamma, float* dbeta, int rows_cap, const int32_t* rows_dev,
+                          int d, int dtype, cudaStream_t st);
+// dz = da * SiLU'(z) (dtype), elementwise on [rows, cols]
+cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
+                            const int32_t* rows_dev, int cols, int dtype, cudaStream_t st);
+// column sums of a [rows, cols] dtype matrix into fp32 out (overwrite)
+cudaError_t launch_col_sum(const void* a, int64_t lda, int rows_cap, const int32_t* rows_dev, int cols,
+                           int dtype, float* out, cudaStream_t st);
+
+cudaError_t launch_gather_rows(const void* src, void* dst, int64_t row_bytes, const int32_t* index,
+                               const int32_t* count, int capacity, cudaStream_t st);
+cudaError_t launch_sl_select(int B, int T, const int32_t* offs, const uint32_t* coins, const uint32_t* keys,
+                             int max_len, uint32_t prob, int32_t* out_offsets, int32_t* out_index,
+                             int32_t* scratch_len, int32_t* status, cudaStream_t st);
+// M-FALCON packing of microbatch `mb`: builds offsets/num_targets/ts/x of [hist ; cand chunk] per user,
+// and the row map used to scatter candidate outputs back.
+cudaError_t launch_mfalcon_pack(int U, int mb, int bm, const int32_t* hist_offs, const void* hist_x,
+                                const int64_t* hist_ts, const int32_t* cand_offs, const void* cand_x,
+                                const int64_t* cand_ts, int d, int dtype, int32_t* out_offs,
+                                int32_t* out_nt, int64_t* out_ts, void* out_x, int32_t* cand_row_map,
+                                int32_t* cand_src_rows, int cap_rows, cudaStream_t st);
+cudaError_t launch_mfalcon_scatter(const void* y, int d, int dtype, const int32_t* cand_row_map,
+                                   const int32_t* total_rows, int cap_rows, void* cand_out, cudaStream_t st);
+
+}  // namespace hstu

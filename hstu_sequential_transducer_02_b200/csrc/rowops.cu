@@ -1,0 +1,725 @@
+// Memory-bound row kernels of the HSTU layer: LayerNorm (forward/backward),
+// LayerNorm(A V) (.) U gating and its backward, SiLU backward, column sums,
+// row gathers, Stochastic Length selection and M-FALCON packing.
+//
+// Every row kernel assigns one warp per row and moves 8 elements per lane per
+// access (16-byte vectors for bf16), with warp-shuffle reductions.
+// ("Actions Speak Louder than Words" summary, 2.2: LayerNorm and SiLU fused
+// into the two linear layers; "Meta HSTU", "Что меняется внутри HSTU":
+// normalisation after aggregation, element-wise product with U.)
+#include <cub/block/block_scan.cuh>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hstu {
+namespace {
+
+constexpr int kRowWarps = 8;          // warps (rows) per block
+constexpr int kMaxChunks = 4;         // 8-element chunks per lane: d <= 32*8*4 = 1024
+
+__device__ __forceinline__ void load8(const float* p, float v[8]) {
+  float4 a = *reinterpret_cast<const float4*>(p);
+  float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float v[8]) {
+  uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store8(float* p, const float v[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ int rows_of(int cap, const int32_t* rows_dev) {
+  if (!rows_dev) return cap;
+  int r = *rows_dev;
+  return r < cap ? r : cap;
+}
+
+// ---------------------------------------------------------------- LayerNorm
+template <typename T>
+__global__ void __launch_bounds__(kRowWarps * 32)
+layer_norm_kernel(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma,
+                  const float* __restrict__ beta, float eps, T* __restrict__ out, int64_t ldo,
+                  float* __restrict__ mean_out, float* __restrict__ rstd_out, int rows_cap,
+                  const int32_t* __restrict__ rows_dev, int d) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int nch = d / 8;
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    float v[kMaxChunks][8];
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        load8(x + (int64_t)row * ldx + ch * 8, v[c]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += v[c][e];
+      }
+    }
+    const float mean = warp_sum(s) / d;
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      if (lane + 32 * c < nch) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { float t = v[c][e] - mean; q += t * t; }
+      }
+    }
+    const float rstd = 1.0f / sqrtf(warp_sum(q) / d + eps);
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float o[8];
+        float g[8], b[8];
+        load8(gamma + ch * 8, g);
+        load8(beta + ch * 8, b);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = (v[c][e] - mean) * rstd * g[e] + b[e];
+        store8(out + (int64_t)row * ldo + ch * 8, o);
+      }
+    }
+    if (lane == 0) {
+      if (mean_out) mean_out[row] = mean;
+      if (rstd_out) rstd_out[row] = rstd;
+    }
+  }
+}
+
+// g = LN(o) * u
+template <typename T>
+__global__ void __launch_bounds__(kRowWarps * 32)
+ln_gate_kernel(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
+               const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+               T* __restrict__ out, int64_t ldout, float* __restrict__ mean_out, float* __restrict__ rstd_out,
+               int rows_cap, const int32_t* __restrict__ rows_dev, int d) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int nch = d / 8;
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    float v[kMaxChunks][8];
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        load8(o + (int64_t)row * ldo_in + ch * 8, v[c]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += v[c][e];
+      }
+    }
+    const float mean = warp_sum(s) / d;
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      if (lane + 32 * c < nch) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { float t = v[c][e] - mean; q += t * t; }
+      }
+    }
+    const float rstd = 1.0f / sqrtf(warp_sum(q) / d + eps);
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float g[8], b[8], uu[8], r[8];
+        load8(gamma + ch * 8, g);
+        load8(beta + ch * 8, b);
+        load8(u + (int64_t)row * ldu + ch * 8, uu);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = ((v[c][e] - mean) * rstd * g[e] + b[e]) * uu[e];
+        store8(out + (int64_t)row * ldout + ch * 8, r);
+      }
+    }
+    if (lane == 0) {
+      if (mean_out) mean_out[row] = mean;
+      if (rstd_out) rstd_out[row] = rstd;
+    }
+  }
+}
+
+// per-block column partials of dgamma/dbeta reduced through shared memory,
+// then one atomic per column per block
+__device__ __forceinline__ void flush_affine_grads(float (*pg)[8], float (*pb)[8], int nch, float* dgamma,
+                                                   float* dbeta, float* red /* smem [2][1024] */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 2 * 1024; i += blockDim.x) red[i] = 0.f;
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        atomicAdd(&red[ch * 8 + e], pg[c][e]);
+        atomicAdd(&red[1024 + ch * 8 + e], pb[c][e]);
+      }
+    }
+  }
+  (void)warp;
+  __syncthreads();
+  for (int i = threadIdx.x; i < nch * 8; i += blockDim.x) {
+    if (dgamma) atomicAdd(&dgamma[i], red[i]);
+    if (dbeta) atomicAdd(&dbeta[i], red[1024 + i]);
+  }
+}
+
+// backward of g = (LN(o) gamma + beta) * u for d_o and the affine gradients
+template <typename T>
+__global__ void __launch_bounds__(kRowWarps * 32)
+ln_gate_bwd_kernel(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
+                   const float* __restrict__ gamma, const float* __restrict__ mean_in,
+                   const float* __restrict__ rstd_in, const T* __restrict__ dg, int64_t lddg,
+                   T* __restrict__ d_o, int64_t ld_do, float* __restrict__ dgamma, float* __restrict__ dbeta,
+                   int rows_cap, const int32_t* __restrict__ rows_dev, int d) {
+  __shared__ float red[2 * 1024];
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int nch = d / 8;
+  float pg[kMaxChunks][8], pb[kMaxChunks][8];
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { pg[c][e] = 0.f; pb[c][e] = 0.f; }
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    const float mean = mean_in[row], rstd = rstd_in[row];
+    float xh[kMaxChunks][8], dxh[kMaxChunks][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float ov[8], uu[8], gg[8], g[8];
+        load8(o + (int64_t)row * ldo_in + ch * 8, ov);
+        load8(u + (int64_t)row * ldu + ch * 8, uu);
+        load8(dg + (int64_t)row * lddg + ch * 8, gg);
+        load8(gamma + ch * 8, g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          xh[c][e] = (ov[e] - mean) * rstd;
+          const float don = gg[e] * uu[e];
+          pg[c][e] += don * xh[c][e];
+          pb[c][e] += don;
+          dxh[c][e] = don * g[e];
+          s1 += dxh[c][e];
+          s2 += dxh[c][e] * xh[c][e];
+        }
+      }
+    }
+    s1 = warp_sum(s1) / d;
+    s2 = warp_sum(s2) / d;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float r[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = rstd * (dxh[c][e] - s1 - xh[c][e] * s2);
+        store8(d_o + (int64_t)row * ld_do + ch * 8, r);
+      }
+    }
+  }
+  flush_affine_grads(pg, pb, nch, dgamma, dbeta, red);
+}
+
+// du = dg * LN(o) (separate pass keeps the register footprint of the kernel above small)
+template <typename T>
+__global__ void __launch_bounds__(kRowWarps * 32)
+ln_gate_du_kernel(const T* __restrict__ o, int64_t ldo_in, const float* __restrict__ gamma,
+                  const float* __restrict__ beta, const float* __restrict__ mean_in,
+                  const float* __restrict__ rstd_in, const T* __restrict__ dg, int64_t lddg,
+                  T* __restrict__ du, int64_t lddu, int rows_cap, const int32_t* __restrict__ rows_dev, int d) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int nch = d / 8;
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    const float mean = mean_in[row], rstd = rstd_in[row];
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float ov[8], gg[8], g[8], b[8], r[8];
+        load8(o + (int64_t)row * ldo_in + ch * 8, ov);
+        load8(dg + (int64_t)row * lddg + ch * 8, gg);
+        load8(gamma + ch * 8, g);
+        load8(beta + ch * 8, b);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = gg[e] * ((ov[e] - mean) * rstd * g[e] + b[e]);
+        store8(du + (int64_t)row * lddu + ch * 8, r);
+      }
+    }
+  }
+}
+
+// dx = dres + rstd * (dxh*gamma - mean(dxh*gamma) - xhat * mean(dxh*gamma*xhat)), dxh fp32
+template <typename T>
+__global__ void __launch_bounds__(kRowWarps * 32)
+ln_bwd_kernel(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma,
+              const float* __restrict__ mean_in, const float* __restrict__ rstd_in,
+              const float* __restrict__ dxhat, int64_t lddxh, const T* __restrict__ dres, int64_t lddres,
+              T* __restrict__ dx, int64_t lddx, float* __restrict__ dgamma, float* __restrict__ dbeta,
+              int rows_cap, const int32_t* __restrict__ rows_dev, int d) {
+  __shared__ float red[2 * 1024];
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int nch = d / 8;
+  float pg[kMaxChunks][8], pb[kMaxChunks][8];
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { pg[c][e] = 0.f; pb[c][e] = 0.f; }
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    const float mean = mean_in[row], rstd = rstd_in[row];
+    float xh[kMaxChunks][8], dg[kMaxChunks][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float xv[8], dv8[8], g[8];
+        load8(x + (int64_t)row * ldx + ch * 8, xv);
+        load8(dxhat + (int64_t)row * lddxh + ch * 8, dv8);
+        load8(gamma + ch * 8, g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          xh[c][e] = (xv[e] - mean) * rstd;
+          pg[c][e] += dv8[e] * xh[c][e];
+          pb[c][e] += dv8[e];
+          dg[c][e] = dv8[e] * g[e];
+          s1 += dg[c][e];
+          s2 += dg[c][e] * xh[c][e];
+        }
+      }
+    }
+    s1 = warp_sum(s1) / d;
+    s2 = warp_sum(s2) / d;
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        float r[8], rs[8];
+        load8(dres + (int64_t)row * lddres + ch * 8, rs);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r[e] = rs[e] + rstd * (dg[c][e] - s1 - xh[c][e] * s2);
+        store8(dx + (int64_t)row * lddx + ch * 8, r);
+      }
+    }
+  }
+  flush_affine_grads(pg, pb, nch, dgamma, dbeta, red);
+}
+
+template <typename T>
+__global__ void silu_bwd_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __restrict__ dz,
+                                int64_t ld, int rows_cap, const int32_t* __restrict__ rows_dev, int cols) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int nch = cols / 8;
+  const int64_t total = (int64_t)rows * nch;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = e / nch;
+    const int ch = (int)(e % nch);
+    float a[8], zz[8], r[8];
+    load8(da + row * ld + ch * 8, a);
+    load8(z + row * ld + ch * 8, zz);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = a[i] * silu_grad_f(zz[i]);
+    store8(dz + row * ld + ch * 8, r);
+  }
+}
+
+// column sums: block handles a chunk of rows for 256 columns (one column per thread)
+template <typename T>
+__global__ void col_sum_kernel(const T* __restrict__ a, int64_t lda, int rows_cap,
+                               const int32_t* __restrict__ rows_dev, int cols, float* __restrict__ out) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int col = blockIdx.x * blockDim.x + threadIdx.x;
+  if (col >= cols) return;
+  const int chunk = (rows + gridDim.y - 1) / gridDim.y;
+  const int r0 = blockIdx.y * chunk, r1 = min(rows, r0 + chunk);
+  float s = 0.f;
+  for (int r = r0; r < r1; ++r) s += Elem<T>::to_f(a[(int64_t)r * lda + col]);
+  if (r1 > r0) atomicAdd(&out[col], s);
+}
+
+__global__ void gather_rows_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst, int64_t words,
+                                   const int32_t* __restrict__ index, const int32_t* __restrict__ count,
+                                   int capacity) {
+  const int n = min(*count, capacity);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < (int64_t)n * words;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / words, w = e % words;
+    dst[r * words + w] = src[(int64_t)index[r] * words + w];
+  }
+}
+
+// ---------------------------------------------------------------- Stochastic Length
+constexpr int kSlThreads = 1024;
+
+__global__ void __launch_bounds__(kSlThreads)
+sl_offsets_kernel(int B, int T, const int32_t* __restrict__ offs, const uint32_t* __restrict__ coins, int max_len,
+                  uint32_t prob, int32_t* __restrict__ out_offs, int32_t* __restrict__ status) {
+  using Scan = cub::BlockScan<int, kSlThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int carry;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    if (offs[0] != 0 || offs[B] > T) set_status(status, HSTU_ERR_BAD_OFFSETS);
+  }
+  __syncthreads();
+  for (int base = 0; base < B; base += kSlThreads) {
+    const int s = base + threadIdx.x;
+    int len = 0;
+    if (s < B) {
+      const int n = max(0, offs[s + 1] - offs[s]);
+      len = (n > max_len && coins[s] < prob) ? max_len : n;
+    }
+    int ex, tot;
+    Scan(tmp).ExclusiveSum(len, ex, tot);
+    if (s < B) out_offs[s] = carry + ex;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out_offs[B] = carry;
+}
+
+// one block per sequence: keep the max_len smallest (key, index) pairs in index order
+__global__ void __launch_bounds__(kSlThreads)
+sl_select_kernel(int B, const int32_t* __restrict__ offs, const uint32_t* __restrict__ coins,
+                 const uint32_t* __restrict__ keys, int max_len, uint32_t prob,
+                 const int32_t* __restrict__ out_offs, int32_t* __restrict__ out_index) {
+  using Scan = cub::BlockScan<int, kSlThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int red[32];
+  __shared__ int carry;
+  const int s = blockIdx.x;
+  if (s >= B) return;
+  const int a = offs[s], n = max(0, offs[s + 1] - a);
+  const int dst0 = out_offs[s];
+  const bool sub = n > max_len && coins[s] < prob;
+  if (!sub) {
+    for (int i = threadIdx.x; i < n; i += kSlThreads) out_index[dst0 + i] = a + i;
+    return;
+  }
+  // composite value (key << 32 | local index) is unique; find the max_len-th smallest by
+  // deciding its bits from the top: prefix search over 64 bits
+  uint64_t prefix = 0;
+  int need = max_len;  // rank (1-based) of the threshold among values with the current prefix
+  for (int bit = 63; bit >= 0; --bit) {
+    // count values whose bits above `bit` equal prefix's and whose `bit` is 0
+    const uint64_t hi_mask = bit == 63 ? 0ull : (~0ull << (bit + 1));
+    int cnt = 0;
+    for (int i = threadIdx.x; i < n; i += kSlThreads) {
+      const uint64_t v = ((uint64_t)keys[a + i] << 32) | (uint32_t)i;
+      if ((v & hi_mask) == (prefix & hi_mask) && !((v >> bit) & 1ull)) ++cnt;
+    }
+    // block reduce
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cnt;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      int t = red[threadIdx.x];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (threadIdx.x == 0) red[0] = t;
+    }
+    __syncthreads();
+    const int zeros = red[0];
+    __syncthreads();
+    if (need > zeros) { prefix |= (1ull << bit); need -= zeros; }
+  }
+  // prefix is the max_len-th smallest value: keep v <= prefix, in index order
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += kSlThreads) {
+    const int i = base + threadIdx.x;
+    int keep = 0;
+    if (i < n) keep = ((((uint64_t)keys[a + i] << 32) | (uint32_t)i) <= prefix) ? 1 : 0;
+    int ex, tot;
+    Scan(tmp).ExclusiveSum(keep, ex, tot);
+    if (keep) out_index[dst0 + carry + ex] = a + i;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += tot;
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- M-FALCON packing
+constexpr int kPackThreads = 1024;
+
+// packed sequence u of microbatch mb: [history_u ; candidates_u[mb*bm, mb*bm + c_u)], or empty if c_u = 0
+__global__ void __launch_bounds__(kPackThreads)
+mfalcon_offsets_kernel(int U, int mb, int bm, const int32_t* __restrict__ hist_offs,
+                       const int32_t* __restrict__ cand_offs, int32_t* __restrict__ out_offs,
+                       int32_t* __restrict__ out_nt) {
+  using Scan = cub::BlockScan<int, kPackThreads>;
+  __shared__ typename Scan::TempStorage tmp;
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < U; base += kPackThreads) {
+    const int u = base + threadIdx.x;
+    int len = 0, c = 0;
+    if (u < U) {
+      const int n = hist_offs[u + 1] - hist_offs[u];
+      const int m = cand_offs[u + 1] - cand_offs[u];
+      c = min(bm, max(0, m - mb * bm));
+      len = c > 0 ? n + c : 0;
+    }
+    int ex, tot;
+    Scan(tmp).ExclusiveSum(len, ex, tot);
+    if (u < U) { out_offs[u] = carry + ex; out_nt[u] = c; }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out_offs[U] = carry;
+}
+
+// one warp per packed row: copy the row of X and its timestamp; record where a candidate row goes
+template <typename T>
+__global__ void mfalcon_rows_kernel(int U, int mb, int bm, const int32_t* __restrict__ hist_offs,
+                                    const T* __restrict__ hist_x, const int64_t* __restrict__ hist_ts,
+                                    const int32_t* __restrict__ cand_offs, const T* __restrict__ cand_x,
+                                    const int64_t* __restrict__ cand_ts, int d,
+                                    const int32_t* __restrict__ out_offs, int64_t* __restrict__ out_ts,
+                                    T* __restrict__ out_x, int32_t* __restrict__ row_map, int cap) {
+  const int lane = threadIdx.x & 31;
+  const int total = min(out_offs[U], cap);
+  for (int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < total; r += gridDim.x * (blockDim.x / 32)) {
+    // user of row r: binary search in out_offs
+    int lo = 0, hi = U;  // out_offs[lo] <= r < out_offs[hi]
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (out_offs[mid] <= r) lo = mid; else hi = mid;
+    }
+    const int u = lo;
+    const int l = r - out_offs[u];
+    const int n = hist_offs[u + 1] - hist_offs[u];
+    const T* src;
+    int64_t ts;
+    int dst_row = -1;
+    if (l < n) {
+      src = hist_x + (int64_t)(hist_offs[u] + l) * d;
+      ts = hist_ts[hist_offs[u] + l];
+    } else {
+      const int c = cand_offs[u] + mb * bm + (l - n);
+      src = cand_x + (int64_t)c * d;
+      ts = cand_ts[c];
+      dst_row = c;
+    }
+    for (int e = lane * 8; e < d; e += 32 * 8) {
+      float v[8];
+      load8(src + e, v);
+      store8(out_x + (int64_t)r * d + e, v);
+    }
+    if (lane == 0) { out_ts[r] = ts; row_map[r] = dst_row; }
+  }
+}
+
+template <typename T>
+__global__ void mfalcon_scatter_kernel(const T* __restrict__ y, int d, const int32_t* __restrict__ row_map,
+                                       const int32_t* __restrict__ total_rows, int cap, T* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int total = min(*total_rows, cap);
+  for (int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < total; r += gridDim.x * (blockDim.x / 32)) {
+    const int dst = row_map[r];
+    if (dst < 0) continue;
+    for (int e = lane * 8; e < d; e += 32 * 8) {
+      float v[8];
+      load8(y + (int64_t)r * d + e, v);
+      store8(out + (int64_t)dst * d + e, v);
+    }
+  }
+}
+
+int row_grid(int rows_cap) {
+  int g = (rows_cap + kRowWarps - 1) / kRowWarps;
+  return g < 1 ? 1 : (g > 148 * 16 ? 148 * 16 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_layer_norm(const void* x, int64_t ldx, const float* gamma, const float* beta, float eps,
+                              void* out, int64_t ldo, float* mean, float* rstd, int rows_cap,
+                              const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = row_grid(rows_cap);
+  if (dtype == HSTU_DTYPE_F32)
+    layer_norm_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo,
+                                                           mean, rstd, rows_cap, rows_dev, d);
+  else
+    layer_norm_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>((const __nv_bfloat16*)x, ldx, gamma, beta, eps,
+                                                                   (__nv_bfloat16*)out, ldo, mean, rstd, rows_cap,
+                                                                   rows_dev, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
+                           const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
+                           int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = row_grid(rows_cap);
+  if (dtype == HSTU_DTYPE_F32)
+    ln_gate_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)o, ldo_in, (const float*)u, ldu, gamma, beta,
+                                                        eps, (float*)out, ldout, mean, rstd, rows_cap, rows_dev, d);
+  else
+    ln_gate_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>(
+        (const __nv_bfloat16*)o, ldo_in, (const __nv_bfloat16*)u, ldu, gamma, beta, eps, (__nv_bfloat16*)out,
+        ldout, mean, rstd, rows_cap, rows_dev, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_gate_bwd(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
+                               const float* mean, const float* rstd, const void* dg, int64_t lddg,
+                               void* d_o, int64_t ld_do, float* dgamma, float* dbeta,
+                               int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = row_grid(rows_cap) < 296 ? row_grid(rows_cap) : 296;
+  if (dtype == HSTU_DTYPE_F32)
+    ln_gate_bwd_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)o, ldo_in, (const float*)u, ldu, gamma,
+                                                            mean, rstd, (const float*)dg, lddg, (float*)d_o, ld_do,
+                                                            dgamma, dbeta, rows_cap, rows_dev, d);
+  else
+    ln_gate_bwd_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>(
+        (const __nv_bfloat16*)o, ldo_in, (const __nv_bfloat16*)u, ldu, gamma, mean, rstd,
+        (const __nv_bfloat16*)dg, lddg, (__nv_bfloat16*)d_o, ld_do, dgamma, dbeta, rows_cap, rows_dev, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_gate_du(const void* o, int64_t ldo_in, const float* gamma, const float* beta,
+                              const float* mean, const float* rstd, const void* dg, int64_t lddg, void* du,
+                              int64_t lddu, int rows_cap, const int32_t* rows_dev, int d, int dtype,
+                              cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = row_grid(rows_cap);
+  if (dtype == HSTU_DTYPE_F32)
+    ln_gate_du_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)o, ldo_in, gamma, beta, mean, rstd,
+                                                           (const float*)dg, lddg, (float*)du, lddu, rows_cap,
+                                                           rows_dev, d);
+  else
+    ln_gate_du_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>(
+        (const __nv_bfloat16*)o, ldo_in, gamma, beta, mean, rstd, (const __nv_bfloat16*)dg, lddg,
+        (__nv_bfloat16*)du, lddu, rows_cap, rows_dev, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_bwd(const void* x, int64_t ldx, const float* gamma, const float* mean, const float* rstd,
+                          const float* dxhat, int64_t lddxh, const void* dres, int64_t lddres, void* dx,
+                          int64_t lddx, float* dgamma, float* dbeta, int rows_cap, const int32_t* rows_dev,
+                          int d, int dtype, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = row_grid(rows_cap) < 296 ? row_grid(rows_cap) : 296;
+  if (dtype == HSTU_DTYPE_F32)
+    ln_bwd_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)x, ldx, gamma, mean, rstd, dxhat, lddxh,
+                                                       (const float*)dres, lddres, (float*)dx, lddx, dgamma, dbeta,
+                                                       rows_cap, rows_dev, d);
+  else
+    ln_bwd_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>(
+        (const __nv_bfloat16*)x, ldx, gamma, mean, rstd, dxhat, lddxh, (const __nv_bfloat16*)dres, lddres,
+        (__nv_bfloat16*)dx, lddx, dgamma, dbeta, rows_cap, rows_dev, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
+                            const int32_t* rows_dev, int cols, int dtype, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = 148 * 8;
+  if (dtype == HSTU_DTYPE_F32)
+    silu_bwd_kernel<float><<<g, 256, 0, st>>>((const float*)da, (const float*)z, (float*)dz, ld, rows_cap,
+                                              rows_dev, cols);
+  else
+    silu_bwd_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16*)da, (const __nv_bfloat16*)z,
+                                                      (__nv_bfloat16*)dz, ld, rows_cap, rows_dev, cols);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_col_sum(const void* a, int64_t lda, int rows_cap, const int32_t* rows_dev, int cols,
+                           int dtype, float* out, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * cols, st);
+  if (e != cudaSuccess || rows_cap <= 0) return e;
+  dim3 grid((cols + 255) / 256, 64);
+  if (dtype == HSTU_DTYPE_F32)
+    col_sum_kernel<float><<<grid, 256, 0, st>>>((const float*)a, lda, rows_cap, rows_dev, cols, out);
+  else
+    col_sum_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)a, lda, rows_cap, rows_dev, cols,
+                                                        out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* src, void* dst, int64_t row_bytes, const int32_t* index,
+                               const int32_t* count, int capacity, cudaStream_t st) {
+  if (capacity <= 0) return cudaSuccess;
+  gather_rows_kernel<<<148 * 8, 256, 0, st>>>((const uint32_t*)src, (uint32_t*)dst, row_bytes / 4, index, count,
+                                              capacity);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sl_select(int B, int T, const int32_t* offs, const uint32_t* coins, const uint32_t* keys,
+                             int max_len, uint32_t prob, int32_t* out_offsets, int32_t* out_index,
+                             int32_t* scratch_len, int32_t* status, cudaStream_t st) {
+  (void)scratch_len;
+  sl_offsets_kernel<<<1, kSlThreads, 0, st>>>(B, T, offs, coins, max_len, prob, out_offsets, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || B == 0) return e;
+  sl_select_kernel<<<B, kSlThreads, 0, st>>>(B, offs, coins, keys, max_len, prob, out_offsets, out_index);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mfalcon_pack(int U, int mb, int bm, const int32_t* hist_offs, const void* hist_x,
+                                const int64_t* hist_ts, const int32_t* cand_offs, const void* cand_x,
+                                const int64_t* cand_ts, int d, int dtype, int32_t* out_offs,
+                                int32_t* out_nt, int64_t* out_ts, void* out_x, int32_t* cand_row_map,
+                                int32_t* cand_src_rows, int cap_rows, cudaStream_t st) {
+  (void)cand_src_rows;
+  mfalcon_offsets_kernel<<<1, kPackThreads, 0, st>>>(U, mb, bm, hist_offs, cand_offs, out_offs, out_nt);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int g = 148 * 4;
+  if (dtype == HSTU_DTYPE_F32)
+    mfalcon_rows_kernel<float><<<g, 256, 0, st>>>(U, mb, bm, hist_offs, (const float*)hist_x, hist_ts, cand_offs,
+                                                  (const float*)cand_x, cand_ts, d, out_offs, out_ts, (float*)out_x,
+                                                  cand_row_map, cap_rows);
+  else
+    mfalcon_rows_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+        U, mb, bm, hist_offs, (const __nv_bfloat16*)hist_x, hist_ts, cand_offs, (const __nv_bfloat16*)cand_x,
+        cand_ts, d, out_offs, out_ts, (__nv_bfloat16*)out_x, cand_row_map, cap_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mfalcon_scatter(const void* y, int d, int dtype, const int32_t* cand_row_map,
+                                   const int32_t* total_rows, int cap_rows, void* cand_out, cudaStream_t st) {
+  const int g = 148 * 4;
+  if (dtype == HSTU_DTYPE_F32)
+    mfalcon_scatter_kernel<float><<<g, 256, 0, st>>>((const float*)y, d, cand_row_map, total_rows, cap_rows,
+                                                     (float*)cand_out);
+  else
+    mfalcon_scatter_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16*)y, d, cand_row_map, total_rows,
+                                                             cap_rows, (__nv_bfloat16*)cand_out);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

@@ -1,0 +1,116 @@
+// Jagged-batch scheduler: builds the (sequence, head, q tile) work list of the
+// attention kernels, sorted by cost (number of kv tiles) in descending order so
+// that persistent CTAs that take items in snake order approximate LPT
+// ("Разная длина истории": real lengths, no padding to a common maximum).
+#include <cub/block/block_scan.cuh>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace hstu {
+
+namespace {
+constexpr int kSchedThreads = 1024;
+constexpr int kCostBins = 2048;  // costs >= kCostBins - 1 share the top bin
+
+// cost of one item: kv tiles for a forward q tile, q tiles for a backward kv tile
+__device__ __forceinline__ int item_cost(int mode, int t, int n, int hist, int tm, int tk) {
+  if (mode == 0) {
+    int r0 = t * tm, r1 = min(n, r0 + tm);
+    return kv_count(kv_tiles_for(r0, r1, hist, tk));
+  }
+  // backward: q tiles that hold a row attending to kv tile t (columns [c0, c1))
+  int c0 = t * tk, c1 = min(n, c0 + tk);
+  int qt_end = (n + tm - 1) / tm;
+  if (c0 < hist) return qt_end - c0 / tm;
+  return (c1 - 1) / tm - c0 / tm + 1;
+}
+
+__global__ void __launch_bounds__(kSchedThreads)
+build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restrict__ num_targets,
+                       int B, int T, int H, int tm, int tk, int mode, int max_items,
+                       WorkItem* __restrict__ items, int32_t* __restrict__ count,
+                       int32_t* __restrict__ status) {
+  using Scan = cub::BlockScan<int, kSchedThreads>;
+  __shared__ typename Scan::TempStorage scan_tmp;
+  __shared__ int hist_bins[kCostBins];
+  __shared__ int bad;
+  const int tid = threadIdx.x;
+  if (tid == 0) bad = 0;
+  for (int c = tid; c < kCostBins; c += kSchedThreads) hist_bins[c] = 0;
+  __syncthreads();
+  // validation of the jagged description
+  if (tid == 0 && (offs[0] != 0 || offs[B] > T || offs[B] < 0)) bad = 1;
+  for (int s = tid; s < B; s += kSchedThreads) {
+    int n = offs[s + 1] - offs[s];
+    int nt = num_targets ? num_targets[s] : 0;
+    if (n < 0 || nt < 0 || nt > n) bad = 1;
+  }
+  __syncthreads();
+  if (bad) {
+    if (tid == 0) { *count = 0; set_status(status, HSTU_ERR_BAD_OFFSETS); }
+    return;
+  }
+  // pass 1: histogram of costs
+  for (int s = tid; s < B; s += kSchedThreads) {
+    SeqInfo si = load_seq(offs, num_targets, s);
+    int tiles = mode == 0 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
+    for (int t = 0; t < tiles; ++t) {
+      int c = item_cost(mode, t, si.n, si.hist, tm, tk);
+      if (c <= 0) continue;
+      atomicAdd(&hist_bins[min(c, kCostBins - 1)], H);
+    }
+  }
+  __syncthreads();
+  // exclusive scan in descending cost order: bin c starts after all bins > c
+  constexpr int kPer = kCostBins / kSchedThreads;
+  int local[kPer];
+  int sum = 0;
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    int c = kCostBins - 1 - (tid * kPer + r);
+    local[r] = hist_bins[c];
+    sum += local[r];
+  }
+  int base, total;
+  Scan(scan_tmp).ExclusiveSum(sum, base, total);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    int c = kCostBins - 1 - (tid * kPer + r);
+    hist_bins[c] = base;  // becomes the cursor of bin c
+    base += local[r];
+  }
+  __syncthreads();
+  if (total > max_items) {  // cannot happen for consistent sizes; refuse rather than overflow
+    if (tid == 0) { *count = 0; set_status(status, HSTU_ERR_WORKSPACE); }
+    return;
+  }
+  // pass 2: scatter
+  for (int s = tid; s < B; s += kSchedThreads) {
+    SeqInfo si = load_seq(offs, num_targets, s);
+    int tiles = mode == 0 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
+    for (int t = 0; t < tiles; ++t) {
+      int c = item_cost(mode, t, si.n, si.hist, tm, tk);
+      if (c <= 0) continue;
+      int pos = atomicAdd(&hist_bins[min(c, kCostBins - 1)], H);
+      for (int h = 0; h < H; ++h) items[pos + h] = WorkItem{s, h, t, c};
+    }
+  }
+  if (tid == 0) *count = total;
+}
+}  // namespace
+
+size_t work_list_capacity(int B, int T, int H, int tile) {
+  return ((size_t)T / tile + (size_t)B + 1) * (size_t)H;
+}
+
+cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targets, int B, int T, int H,
+                                   int tm, int tk, int mode, int max_items, WorkItem* items,
+                                   int32_t* count, int32_t* status, cudaStream_t stream) {
+  build_work_list_kernel<<<1, kSchedThreads, 0, stream>>>(offs, num_targets, B, T, H, tm, tk, mode,
+                                                          max_items, items, count, status);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

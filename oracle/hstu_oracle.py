@@ -208,6 +208,30 @@ def attention_forward_pairwise(q, k, v, seq_offsets, timestamps, pos_bias, time_
     return out
 
 
+def attention_rows(q, k, v, seq_offsets, timestamps, pos_bias, time_bias, rows, num_targets=None,
+                   time_div: float = 0.301):
+    """The same O_i for selected (sequence, row, head) triples only, one row at a
+    time, so that very long sequences can be checked on sampled outputs.
+    Returns [len(rows), dv]."""
+    out = np.zeros((len(rows), np.asarray(v).shape[2]))
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    for r, (s, i, h) in enumerate(rows):
+        a, b = int(offs[s]), int(offs[s + 1])
+        n = b - a
+        nt = 0 if num_targets is None else int(num_targets[s])
+        N = max(history_length(n, nt), 1)
+        j = np.arange(n)
+        att = (j <= i) & ((j < n - nt) | (j == i))
+        p = np.minimum(np.arange(n), n - nt)
+        pb = pos_bucket(p[i] - p)
+        tb = time_bucket(np.asarray(timestamps[a:b], np.int64)[i] - np.asarray(timestamps[a:b], np.int64), time_div)
+        rab = np.asarray(_head_table(pos_bias, h), np.float64)[pb] + np.asarray(_head_table(time_bias, h), np.float64)[tb]
+        sc = np.asarray(k[a:b, h], np.float64) @ np.asarray(q[a + i, h], np.float64) + rab
+        w = np.where(att, silu(sc), 0.0) / N
+        out[r] = w @ np.asarray(v[a:b, h], np.float64)
+    return out
+
+
 def attention_backward(q, k, v, dout, seq_offsets, timestamps, pos_bias, time_bias,
                        num_targets=None, time_div: float = 0.301):
     """Gradients of sum(O * dout) with respect to q, k, v and the two rab tables.
@@ -297,6 +321,31 @@ def layer_forward(x, p, seq_offsets, timestamps, num_heads: int, head_dim: int,
     if return_intermediates:
         return y, dict(xh=xh, z=z, a=a, U=U, V=V, Q=Q, K=K, O=O, on=on, g=g)
     return y
+
+
+def layer_forward_rows(x, p, seq_offsets, timestamps, num_heads: int, head_dim: int, rows,
+                       num_targets=None, eps: float = 1e-5, time_div: float = 0.301):
+    """Y for selected (sequence, row) pairs of one layer: the projection of the
+    whole sequence, then attention, LayerNorm, gate and f2 for those rows only.
+    Returns [len(rows), d]."""
+    x = np.asarray(x, np.float64)
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    out = np.zeros((len(rows), x.shape[1]))
+    cache = {}
+    for r, (s, i) in enumerate(rows):
+        a, b = int(offs[s]), int(offs[s + 1])
+        if s not in cache:
+            xh = layer_norm(x[a:b], p.ln1_g, p.ln1_b, eps)
+            act = silu(xh @ np.asarray(p.w1, np.float64).T + np.asarray(p.b1, np.float64))
+            cache[s] = split_uvqk(act, num_heads, head_dim)
+        U, V, Q, K = cache[s]
+        loc = np.array([0, b - a])
+        nt = None if num_targets is None else [num_targets[s]]
+        o = np.concatenate([attention_rows(Q, K, V, loc, timestamps[a:b], p.pos_bias, p.time_bias, [(0, i, h)],
+                                           nt, time_div)[0] for h in range(num_heads)])
+        on = layer_norm(o[None, :], p.ln2_g, p.ln2_b, eps)[0]
+        out[r] = x[a + i] + (on * U[i].reshape(-1)) @ np.asarray(p.w2, np.float64).T + np.asarray(p.b2, np.float64)
+    return out
 
 
 def stack_forward(x, layers: Sequence, seq_offsets, timestamps, num_heads, head_dim,

@@ -1,0 +1,222 @@
+"""GPU parity of the whole layer (hstu_layer_fwd / hstu_layer_bwd), of M-FALCON
+ranking (mfalcon_rank) and of Stochastic Length, on the five configurations'
+seeded workloads, against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.hstu_oracle as O
+from hstu_sequential_transducer_02_b200 import workload as W
+from tests.helpers import assert_close, dev, errors, layer_to_dev, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+
+def _b():
+    from hstu_sequential_transducer_02_b200 import binding
+    return binding
+
+
+def _layers(wl, force_simt=False):
+    b = _b()
+    td = torch_dtype(wl.spec.dtype)
+    s = wl.spec
+    return [b.Layer(layer_to_dev(p, td), s.d_model, s.num_heads, s.head_dim, force_simt=force_simt)
+            for p in wl.layers]
+
+
+def _forward(wl, layers, num_targets=None):
+    td = torch_dtype(wl.spec.dtype)
+    y = dev(wl.x, td)
+    offs, ts = dev(wl.seq_offsets), dev(wl.timestamps)
+    nt = None if num_targets is None else dev(np.asarray(num_targets, np.int32))
+    for ly in layers:
+        y = ly.forward(y, offs, ts, num_targets=nt)
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy()
+
+
+def _ref(wl, num_targets=None):
+    s = wl.spec
+    return O.stack_forward(wl.x, wl.layers, wl.seq_offsets, wl.timestamps, s.num_heads, s.head_dim,
+                           num_targets=num_targets)
+
+
+def test_layer_config0_fp32():
+    wl = W.make_workload(0)
+    assert_close(_forward(wl, _layers(wl)), _ref(wl), "f32", "config 0")
+
+
+def test_layer_config0_fp32_random_affine():
+    wl = W.make_workload(0, random_affine=True, per_head_rab=True)
+    assert_close(_forward(wl, _layers(wl)), _ref(wl), "f32", "config 0 affine")
+
+
+def test_layer_config1_bf16_two_layers():
+    wl = W.make_workload(1)
+    assert_close(_forward(wl, _layers(wl)), _ref(wl), "bf16", "config 1")
+
+
+def test_layer_config1_random_affine_cuda_core_path():
+    wl = W.make_workload(1, random_affine=True, batch=6)
+    assert_close(_forward(wl, _layers(wl, force_simt=True)), _ref(wl), "bf16", "config 1 simt")
+
+
+@pytest.mark.parametrize("scale", [1 / 32, 1 / 16])
+def test_layer_config2_scaled(scale):
+    wl = W.make_workload(2, scale=scale, random_affine=True)
+    assert_close(_forward(wl, _layers(wl)), _ref(wl), "bf16", f"config 2 x{scale}")
+
+
+def test_layer_config2_full_size_sampled_rows():
+    """The full long-history workload (B=8, n in [4096, 8192]) in the launch
+    configuration the benchmark times; sampled rows against the oracle."""
+    wl = W.make_workload(2)
+    y = _forward(wl, _layers(wl))
+    rng = np.random.default_rng(0)
+    lens = wl.lengths
+    rows = []
+    for s in (0, 5):
+        rows += [(s, 0), (s, 127), (s, 128), (s, int(lens[s]) - 1)] + [(s, int(i)) for i in rng.integers(0, lens[s], 4)]
+    s_ = wl.spec
+    ref = O.layer_forward_rows(wl.x, wl.layers[0], wl.seq_offsets, wl.timestamps, s_.num_heads, s_.head_dim, rows)
+    got = np.stack([y[wl.seq_offsets[s] + i] for s, i in rows])
+    assert_close(got, ref, "bf16", "config 2 full sampled")
+    assert np.all(np.isfinite(y))
+
+
+def test_layer_mfalcon_targets_in_layer_call():
+    wl = W.make_workload(1, batch=5, scale=0.5)
+    nt = np.array([3, 0, 17, 1, 40], dtype=np.int32)
+    nt = np.minimum(nt, wl.lengths).astype(np.int32)
+    assert_close(_forward(wl, _layers(wl), nt), _ref(wl, nt), "bf16", "layer with targets")
+
+
+def _mfalcon_gpu(wl, layers, microbatch):
+    b = _b()
+    td = torch_dtype(wl.spec.dtype)
+    e = wl.extras
+    m_max = int(np.max(np.diff(e["cand_offsets"])))
+    out = b.mfalcon_rank(layers, dev(wl.seq_offsets), dev(wl.x, td), dev(wl.timestamps), dev(e["cand_offsets"]),
+                         dev(e["cand_x"], td), dev(e["cand_ts"]), microbatch, m_max)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy()
+
+
+def test_mfalcon_rank_config3_scaled():
+    wl = W.make_workload(3, scale=1 / 16)
+    e = wl.extras
+    bm = int(e["microbatch"])
+    s = wl.spec
+    got = _mfalcon_gpu(wl, _layers(wl), bm)
+    ref = O.mfalcon_rank(wl.layers, wl.seq_offsets, wl.x, wl.timestamps, e["cand_offsets"], e["cand_x"],
+                         e["cand_ts"], bm, s.num_heads, s.head_dim)
+    assert_close(got, ref, "bf16", "mfalcon scaled")
+
+
+def test_mfalcon_microbatch_invariance_on_gpu():
+    """The same candidates scored with b_m = 7, 32 and all-at-once agree."""
+    wl = W.make_workload(3, scale=1 / 32, batch=3)
+    layers = _layers(wl)
+    a = _mfalcon_gpu(wl, layers, 7)
+    bb = _mfalcon_gpu(wl, layers, 32)
+    c = _mfalcon_gpu(wl, layers, 10 ** 4)
+    assert_close(a, bb.astype(np.float64), "bf16", "b_m 7 vs 32")
+    assert_close(a, c.astype(np.float64), "bf16", "b_m 7 vs all")
+
+
+def test_mfalcon_rank_config3_full_size_sampled():
+    """Full ranking workload (16 users x (2048 + 4096), b_m = 512); sampled
+    candidates against the oracle scoring each candidate alone with its history
+    (the M-FALCON invariant makes that the same value)."""
+    wl = W.make_workload(3)
+    e = wl.extras
+    s = wl.spec
+    got = _mfalcon_gpu(wl, _layers(wl), int(e["microbatch"]))
+    rng = np.random.default_rng(4)
+    picks = [(0, 0), (3, 511), (7, 512), (15, 4095)] + [(int(u), int(c)) for u, c in
+                                                        zip(rng.integers(0, 16, 4), rng.integers(0, 4096, 4))]
+    refs, gots = [], []
+    for u, c in picks:
+        ha, hb = wl.seq_offsets[u], wl.seq_offsets[u + 1]
+        ci = e["cand_offsets"][u] + c
+        xs = np.concatenate([wl.x[ha:hb], e["cand_x"][ci:ci + 1]])
+        ts = np.concatenate([wl.timestamps[ha:hb], e["cand_ts"][ci:ci + 1]])
+        y = O.stack_forward(xs, wl.layers, [0, xs.shape[0]], ts, s.num_heads, s.head_dim, num_targets=[1])
+        refs.append(y[-1])
+        gots.append(got[ci])
+    assert_close(np.stack(gots), np.stack(refs), "bf16", "mfalcon full sampled")
+
+
+def test_stochastic_length_bit_exact():
+    b = _b()
+    wl = W.make_workload(4)
+    e = wl.extras
+    offs, idx = b.stochastic_length(dev(wl.seq_offsets), dev(e["sl_coin"].view(np.int32)),
+                                    dev(e["sl_keys"].view(np.int32)), int(e["sl_len"]), int(e["sl_prob_u32"]))
+    torch.cuda.synchronize()
+    g_ref, o_ref = O.stochastic_length_select(wl.seq_offsets, e["sl_coin"], e["sl_keys"], int(e["sl_len"]),
+                                              int(e["sl_prob_u32"]))
+    offs = offs.cpu().numpy()
+    assert np.array_equal(offs, o_ref)
+    assert np.array_equal(idx.cpu().numpy()[:offs[-1]], g_ref)
+
+
+def _sl_workload(wl):
+    """Apply the oracle's SL selection to the host arrays (inputs of both sides)."""
+    e = wl.extras
+    g, offs = O.stochastic_length_select(wl.seq_offsets, e["sl_coin"], e["sl_keys"], int(e["sl_len"]),
+                                         int(e["sl_prob_u32"]))
+    return g, offs
+
+
+def test_training_step_config4_scaled():
+    """8-layer stack forward + backward with Stochastic Length: dU, dV, dQ, dK
+    and the rab gradients of every layer, plus weight gradients, vs the oracle."""
+    b = _b()
+    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
+    s = wl.spec
+    td = torch.bfloat16
+    e = wl.extras
+    # SL on the GPU, gathers on the GPU
+    offs_d, idx_d = b.stochastic_length(dev(wl.seq_offsets), dev(e["sl_coin"].view(np.int32)),
+                                        dev(e["sl_keys"].view(np.int32)), int(e["sl_len"]), int(e["sl_prob_u32"]))
+    g_ref, o_ref = _sl_workload(wl)
+    T2 = int(o_ref[-1])
+    count = offs_d[-1:]
+    x = b.gather_rows(dev(wl.x, td), idx_d, count, torch.empty(T2, s.d_model, dtype=td, device="cuda"))
+    ts = b.gather_rows(dev(wl.timestamps), idx_d, count, torch.empty(T2, dtype=torch.int64, device="cuda"))
+    gy = b.gather_rows(dev(e["grad_out"], td), idx_d, count, torch.empty(T2, s.d_model, dtype=td, device="cuda"))
+    layers = _layers(wl)
+    hv = s.num_heads * s.head_dim
+    saved = [b.Saved.alloc(T2, s.d_model, hv, td, "cuda") for _ in layers]
+    xs = [x]
+    for ly, sv in zip(layers, saved):
+        xs.append(ly.forward(xs[-1], offs_d, ts, saved=sv))
+    dy = gy
+    grads = [None] * len(layers)
+    for li in range(len(layers) - 1, -1, -1):
+        dy, grads[li] = layers[li].backward(xs[li], dy, saved[li], offs_d, ts)
+    torch.cuda.synchronize()
+    # oracle on the same subsampled inputs
+    x_h = wl.x[g_ref]
+    ts_h = wl.timestamps[g_ref]
+    gy_h = e["grad_out"][g_ref]
+    ref = O.stack_backward(x_h, wl.layers, gy_h, o_ref, ts_h, s.num_heads, s.head_dim)
+    for li in range(len(layers) - 1, -1, -1):
+        duvqk = grads[li]["uvqk"].float().cpu().numpy()
+        r = ref[li]
+        T = T2
+        ref_uvqk = np.concatenate([r["dU"].reshape(T, hv), r["dV"].reshape(T, hv), r["dQ"].reshape(T, hv),
+                                   r["dK"].reshape(T, hv)], axis=1)
+        for c, name in enumerate("UVQK"):
+            ma, rel = errors(duvqk[:, c * hv:(c + 1) * hv], ref_uvqk[:, c * hv:(c + 1) * hv])
+            print(f"layer {li} d{name}: max-abs {ma:.3e} rel-fro {rel:.3e}")
+        for c, name in enumerate("UVQK"):
+            assert_close(duvqk[:, c * hv:(c + 1) * hv], ref_uvqk[:, c * hv:(c + 1) * hv], "bf16", f"L{li} d{name}")
+        for gname, rname in [("pos_bias", "dpos_bias"), ("time_bias", "dtime_bias"), ("w1", "dw1"), ("w2", "dw2"),
+                             ("b1", "db1"), ("b2", "db2"), ("ln1_gamma", "dln1_g"), ("ln2_gamma", "dln2_g")]:
+            got = grads[li][gname].cpu().numpy()
+            rr = r[rname]
+            assert np.linalg.norm(got - rr) <= 1e-2 * max(np.linalg.norm(rr), 1e-6), f"L{li} {gname}"
+    assert_close(dy.float().cpu().numpy(), ref[0]["dx"], "bf16", "dx")

@@ -373,3 +373,22 @@ def test_stochastic_length_rule():
     want = [0, 1, 2, 3 + 3, 3 + 5, 3 + 6, 3 + 8, 13, 14, 15, 16] + list(range(20, 30))
     assert list(gather) == want
     assert list(new_offs) == [0, 3, 7, 11, 21]
+
+
+def test_sampled_row_functions_match_dense():
+    d = W.random_attention_inputs(21, [7, 12], 2, 4, "f32", num_targets=[0, 4], per_head_rab=True)
+    dense = O.attention_forward(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], d["pos_bias"],
+                                d["time_bias"], d["num_targets"])
+    rows = [(0, 0, 0), (0, 6, 1), (1, 3, 0), (1, 9, 1), (1, 11, 0)]
+    got = O.attention_rows(d["q"], d["k"], d["v"], d["seq_offsets"], d["timestamps"], d["pos_bias"],
+                           d["time_bias"], rows, d["num_targets"])
+    for r, (s, i, h) in enumerate(rows):
+        assert np.allclose(got[r], dense[d["seq_offsets"][s] + i, h], rtol=1e-12, atol=1e-14)
+    p = _tiny_layer(22, 8, 2, 4)
+    rng = np.random.default_rng(23)
+    x = rng.normal(size=(19, 8))
+    offs = [0, 7, 19]
+    ts = np.concatenate([np.cumsum(rng.integers(1, 900, 7)), np.cumsum(rng.integers(1, 900, 12))]).astype(np.int64)
+    y = O.layer_forward(x, p, offs, ts, 2, 4, num_targets=[0, 3])
+    yr = O.layer_forward_rows(x, p, offs, ts, 2, 4, [(0, 3), (1, 0), (1, 11)], num_targets=[0, 3])
+    assert np.allclose(yr, y[[3, 7, 18]], rtol=1e-12, atol=1e-12)

@@ -724,3 +724,71 @@ int hstu_debug_timeout_probe(int64_t timeout_ns, int32_t* status_dev, void* stre
 }
 
 }  // extern "C"
+
+// =============================================================================
+// Attention forward without caller-provided scratch.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// attention: an embedding application whose device memory is entirely owned by
+// another allocator, or a latency-bound serving loop that forbids any
+// allocation once it has started.  For them this entry point takes its scratch
+// (the status word and the cost-sorted work list) from a fixed array that the
+// library itself places in device memory, instead of from a workspace.
+//
+// The array is a file-scope __device__ variable of kNoAllocScratchBytes bytes;
+// every GPU on which the library is loaded holds it until the process exits.
+// In host code its name only stands for the variable, it is not a device
+// address, so the address is looked up once per device (cudaGetSymbolAddress,
+// with that device current) on the first call made on that device, and passed
+// to the kernels from then on.
+// =============================================================================
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 1u << 20;  // 1 MiB
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HSTU_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HSTU_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HSTU_OK;
+}
+
+}  // namespace
+
+extern "C" int hstu_attn_fwd_noalloc(const hstu_attn_desc* desc, const hstu_jagged* jb, const void* q, int64_t ldq,
+                                     const void* k, int64_t ldk, const void* v, int64_t ldv,
+                                     const float* pos_bias, const float* time_bias, void* out, int64_t ldo,
+                                     void* stream) {
+  HSTU_TRY(check_attn_desc(desc));
+  HSTU_TRY(check_jagged(jb));
+  const int hd = desc->num_heads * desc->dqk;
+  HSTU_TRY(check_rows(q, ldq, hd, desc->dtype));
+  HSTU_TRY(check_rows(k, ldk, hd, desc->dtype));
+  HSTU_TRY(check_rows(v, ldv, hd, desc->dtype));
+  HSTU_TRY(check_rows(out, ldo, hd, desc->dtype));
+  if (!pos_bias || !time_bias) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(hstu_attn_fwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
+  if (need > kNoAllocScratchBytes) return HSTU_ERR_WORKSPACE;  // problem larger than the fixed array
+  void* scratch = nullptr;
+  HSTU_TRY(noalloc_scratch(&scratch));
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(scratch);
+  AttnWs w = carve_attn(c, desc, jb->batch, jb->total_tokens, false);
+  HSTU_CUDA(cudaMemsetAsync(w.status, 0, kStatusBytes, st));  // the previous call's status must not leak
+  return run_attn_fwd(desc, jb, q, ldq, k, ldk, v, ldv, pos_bias, time_bias, out, ldo, w, st);
+}

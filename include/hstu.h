@@ -192,6 +192,33 @@ int hstu_attn_fwd(const hstu_attn_desc* desc, const hstu_jagged* jb,
                   void* out, int64_t ldo,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* hstu_attn_fwd without a workspace argument, for callers that cannot allocate
+ * device memory where they call it (an application whose device memory is
+ * owned entirely by another allocator, or a serving loop that forbids
+ * allocation once it runs).  The pages describe no such variant: it is a
+ * property of this library, not of the method.
+ *
+ * Same arguments, layouts and result as hstu_attn_fwd.  The scratch it needs
+ * (status word and work list) lives in a 1 MiB array that the library keeps in
+ * the device memory of every GPU it is loaded on, for the life of the process;
+ * the call itself allocates nothing.  A problem whose scratch would exceed the
+ * array (hstu_attn_fwd_workspace_size() > 1 MiB, about 65,000 work items:
+ * (total_tokens/128 + batch + 1) * num_heads) is refused with
+ * HSTU_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (current device at the time of the call); make that first call
+ *     before capturing any stream into a graph.
+ *   - All calls share the one array and each call overwrites it.  Calls that
+ *     may run at the same time on the GPU (different streams without ordering
+ *     between them) race on it and give undefined results: order them.
+ *   - Device-side wait timeouts of this call are recorded in the array's status
+ *     word, which is not readable through this interface. */
+int hstu_attn_fwd_noalloc(const hstu_attn_desc* desc, const hstu_jagged* jb,
+                          const void* q, int64_t ldq, const void* k, int64_t ldk,
+                          const void* v, int64_t ldv,
+                          const float* pos_bias, const float* time_bias,
+                          void* out, int64_t ldo, void* stream);
+
 int hstu_attn_bwd_workspace_size(const hstu_attn_desc* desc, int32_t batch,
                                  int32_t total_tokens, size_t* bytes);
 

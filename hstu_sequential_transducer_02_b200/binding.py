@@ -44,7 +44,8 @@ class AttnDesc(ctypes.Structure):
 
 
 class LayerDesc(ctypes.Structure):
-    _fields_ = [("d_model", _c_i32), ("ln_eps", _c_flt), ("attn", AttnDesc)]
+    _fields_ = [("d_model", _c_i32), ("ln_eps", _c_flt), ("io_dtype", _c_i32), ("reserved", _c_i32),
+                ("attn", AttnDesc)]
 
 
 class Jagged(ctypes.Structure):
@@ -170,8 +171,10 @@ def attn_desc(num_heads: int, head_dim: int, dtype: int, per_head_rab: bool = Fa
 
 
 def layer_desc(d_model: int, num_heads: int, head_dim: int, dtype: int, per_head_rab: bool = False,
-               force_simt: bool = False, eps: float = 1e-5, time_div: float = 0.301) -> LayerDesc:
-    return LayerDesc(d_model, eps, attn_desc(num_heads, head_dim, dtype, per_head_rab, force_simt, time_div))
+               force_simt: bool = False, eps: float = 1e-5, time_div: float = 0.301,
+               io_dtype: Optional[int] = None) -> LayerDesc:
+    return LayerDesc(d_model, eps, dtype if io_dtype is None else io_dtype, 0,
+                     attn_desc(num_heads, head_dim, dtype, per_head_rab, force_simt, time_div))
 
 
 def jagged(seq_offsets: torch.Tensor, timestamps: torch.Tensor, total_tokens: int,
@@ -278,12 +281,17 @@ class Layer:
     """One HSTU layer's descriptor and parameters (device tensors)."""
 
     def __init__(self, weights: Dict[str, torch.Tensor], d_model: int, num_heads: int, head_dim: int,
-                 force_simt: bool = False, eps: float = 1e-5, time_div: float = 0.301):
+                 force_simt: bool = False, eps: float = 1e-5, time_div: float = 0.301,
+                 residual_fp32: bool = False):
+        """residual_fp32: X, Y (and dX, dY) are fp32 tensors while weights and
+        activations use the weights' dtype."""
         self.w = weights
         self.dtype = weights["w1"].dtype
+        self.io_dtype = torch.float32 if residual_fp32 else self.dtype
         self.d_model, self.num_heads, self.head_dim = d_model, num_heads, head_dim
         self.desc = layer_desc(d_model, num_heads, head_dim, _dtype_code(weights["w1"]),
-                               weights["pos_bias"].dim() == 2, force_simt, eps, time_div)
+                               weights["pos_bias"].dim() == 2, force_simt, eps, time_div,
+                               io_dtype=DTYPE_F32 if residual_fp32 else None)
         self.cw = layer_weights(weights)
         self._ws = {}
 

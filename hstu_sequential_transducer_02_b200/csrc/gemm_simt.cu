@@ -27,12 +27,17 @@ __device__ __forceinline__ void epilogue_store(const GemmParams& p, int m, int n
     }
     case EPI_BIAS_RESIDUAL: {
       float y = acc + (p.bias ? p.bias[n] : 0.f);
-      if (p.residual) y += Elem<T>::to_f(((const T*)p.residual)[(int64_t)m * p.ldr + n]);
-      ((T*)p.out)[(int64_t)m * p.ldo + n] = Elem<T>::from_f(y);
+      if (p.residual) {
+        if (p.res_f32) y += ((const float*)p.residual)[(int64_t)m * p.ldr + n];
+        else y += Elem<T>::to_f(((const T*)p.residual)[(int64_t)m * p.ldr + n]);
+      }
+      if (p.out_f32) ((float*)p.out)[(int64_t)m * p.ldo + n] = y;
+      else ((T*)p.out)[(int64_t)m * p.ldo + n] = Elem<T>::from_f(y);
       break;
     }
     default:
-      ((T*)p.out)[(int64_t)m * p.ldo + n] = Elem<T>::from_f(acc);
+      if (p.out_f32) ((float*)p.out)[(int64_t)m * p.ldo + n] = acc;
+      else ((T*)p.out)[(int64_t)m * p.ldo + n] = Elem<T>::from_f(acc);
   }
 }
 

@@ -232,6 +232,8 @@ int check_layer(const hstu_layer_desc* d, const hstu_layer_weights* w) {
   if (dm < 8 || dm > 1024 || dm % 8) return HSTU_ERR_UNSUPPORTED;
   if (hv > 1024 || hv % 8) return HSTU_ERR_UNSUPPORTED;
   if (!(d->ln_eps >= 0.f)) return HSTU_ERR_INVALID_ARG;
+  if (d->io_dtype != HSTU_DTYPE_F32 && d->io_dtype != d->attn.dtype) return HSTU_ERR_UNSUPPORTED;
+  if (d->reserved != 0) return HSTU_ERR_INVALID_ARG;
   const void* ptrs[] = {w->w1, w->b1, w->ln1_gamma, w->ln1_beta, w->ln2_gamma, w->ln2_beta,
                         w->w2, w->b2, w->pos_bias, w->time_bias};
   for (const void* p : ptrs)
@@ -280,8 +282,8 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   // (A1) LayerNorm1
   {
     TraceScope tr("ln1", st);
-    HSTU_CUDA(launch_layer_norm(x, dm, w->ln1_gamma, w->ln1_beta, d->ln_eps, b.xhat, dm, b.mu1, b.rs1, T, rows, dm,
-                                dt, st));
+    HSTU_CUDA(launch_layer_norm(x, dm, d->io_dtype, w->ln1_gamma, w->ln1_beta, d->ln_eps, b.xhat, dm, dt, b.mu1,
+                                b.rs1, T, rows, dm, st));
   }
   // (A1) f1 + SiLU, split layout U | V | Q | K
   GemmParams g1;
@@ -293,6 +295,7 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   g1.out = b.uvqk; g1.ldo = 4 * hv;
   g1.out2 = b.z; g1.ldo2 = 4 * hv;
   g1.rows_dev = rows;
+  g1.status = ws.attn.status;
   HSTU_TRY(gemm(g1, dt, d->attn.flags, st, "gemm_f1_silu"));
   // (A2-A4) attention
   const size_t es = elem_size(dt);
@@ -315,6 +318,9 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   g2.residual = x; g2.ldr = dm;
   g2.out = y; g2.ldo = dm;
   g2.rows_dev = rows;
+  g2.res_f32 = d->io_dtype == HSTU_DTYPE_F32;
+  g2.out_f32 = d->io_dtype == HSTU_DTYPE_F32;
+  g2.status = ws.attn.status;
   HSTU_TRY(gemm(g2, dt, d->attn.flags, st, "gemm_f2_residual"));
   return HSTU_OK;
 }
@@ -328,6 +334,7 @@ struct LayerBwdWs {
   void* duvqk;   // [T, 4hv]
   void* dz;      // [T, 4hv]
   float* dxhat;  // [T, dm] fp32
+  void* dyb;     // [T, dm] dy in the activation dtype, zero-padded to a multiple of 64 rows
 };
 
 LayerBwdWs carve_layer_bwd(Carver& c, const hstu_layer_desc* d, int B, int T) {
@@ -341,6 +348,7 @@ LayerBwdWs carve_layer_bwd(Carver& c, const hstu_layer_desc* d, int B, int T) {
   w.duvqk = c.take<char>((size_t)T * 4 * hv * es);
   w.dz = c.take<char>((size_t)T * 4 * hv * es);
   w.dxhat = c.take<float>((size_t)T * dm);
+  w.dyb = c.take<char>((size_t)T * dm * es);
   return w;
 }
 
@@ -348,37 +356,53 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
                   const hstu_layer_saved* sv, const void* dy, void* dx, const hstu_layer_grads* gr,
                   const LayerBwdWs& ws, cudaStream_t st) {
   const int dt = d->attn.dtype;
+  const int io = d->io_dtype;
   const int dm = d->d_model, H = d->attn.num_heads, dh = d->attn.dv, hv = H * dh;
   const int T = jb->total_tokens;
   const int32_t* rows = jb->seq_offsets + jb->batch;
   const size_t es = elem_size(dt);
   const int fl = d->attn.flags;
   void* duvqk = gr->duvqk ? gr->duvqk : ws.duvqk;
-  // recompute g = LN2(o) * U (cheaper to recompute than to keep)
-  HSTU_CUDA(launch_ln_gate(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g, hv,
-                           nullptr, nullptr, T, rows, hv, dt, st));
+  int32_t* status = ws.attn.status;
+  // The weight-gradient products reduce over tokens in 64-row slices: rows from the
+  // device row count up to the next multiple of 64 of every token-major operand are zeroed.
+  {
+    TraceScope tr("bwd_prep", st);
+    HSTU_CUDA(launch_convert_rows(dy, dm, io, ws.dyb, dm, dt, dm, T, rows, 64, st));
+    HSTU_CUDA(launch_zero_tail_rows(sv->xhat, (int64_t)dm * es, (int64_t)dm * es, T, rows, 64, st));
+    // recompute g = LN2(o) * U (cheaper to recompute than to keep)
+    HSTU_CUDA(launch_ln_gate(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g, hv,
+                             nullptr, nullptr, T, rows, hv, dt, st));
+    HSTU_CUDA(launch_zero_tail_rows(ws.g, (int64_t)hv * es, (int64_t)hv * es, T, rows, 64, st));
+  }
   // y = x + g W2^T + b2:  dW2 = dy^T g, db2 = colsum(dy), dg = dy W2
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.M = dm; p.N = hv; p.K = T;                 // dW2[m=out, n=in] = sum_t dy[t, m] g[t, n]
-  p.A = dy; p.sam = 1; p.sak = dm;
+  p.A = ws.dyb; p.sam = 1; p.sak = dm;
   p.B = ws.g; p.sbn = 1; p.sbk = hv;
-  p.epi = EPI_STORE_F32; p.out = gr->dw2; p.ldo = hv; p.k_dev = rows;
+  p.epi = EPI_STORE_F32; p.out = gr->dw2; p.ldo = hv; p.k_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw2"));
-  HSTU_CUDA(launch_col_sum(dy, dm, T, rows, dm, dt, gr->db2, st));
+  {
+    TraceScope tr("colsum_db2", st);
+    HSTU_CUDA(launch_col_sum(dy, dm, T, rows, dm, io, gr->db2, st));
+  }
   memset(&p, 0, sizeof(p));
   p.M = T; p.N = hv; p.K = dm;                 // dg[t, n] = sum_m dy[t, m] W2[m, n]
-  p.A = dy; p.sam = dm; p.sak = 1;
+  p.A = ws.dyb; p.sam = dm; p.sak = 1;
   p.B = w->w2; p.sbn = 1; p.sbk = hv;
-  p.epi = EPI_STORE; p.out = ws.dg; p.ldo = hv; p.rows_dev = rows;
+  p.epi = EPI_STORE; p.out = ws.dg; p.ldo = hv; p.rows_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dg"));
   // g = (LN2(o) gamma2 + beta2) * U:  dU, d_o, dgamma2, dbeta2
-  HSTU_CUDA(cudaMemsetAsync(gr->dln2_gamma, 0, sizeof(float) * hv, st));
-  HSTU_CUDA(cudaMemsetAsync(gr->dln2_beta, 0, sizeof(float) * hv, st));
-  HSTU_CUDA(launch_ln_gate_bwd(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, sv->ln2_mean, sv->ln2_rstd, ws.dg,
-                               hv, ws.d_o, hv, gr->dln2_gamma, gr->dln2_beta, T, rows, hv, dt, st));
-  HSTU_CUDA(launch_ln_gate_du(sv->attn_out, hv, w->ln2_gamma, w->ln2_beta, sv->ln2_mean, sv->ln2_rstd, ws.dg, hv,
-                              duvqk, 4 * hv, T, rows, hv, dt, st));
+  {
+    TraceScope tr("ln2_gate_bwd", st);
+    HSTU_CUDA(cudaMemsetAsync(gr->dln2_gamma, 0, sizeof(float) * hv, st));
+    HSTU_CUDA(cudaMemsetAsync(gr->dln2_beta, 0, sizeof(float) * hv, st));
+    HSTU_CUDA(launch_ln_gate_bwd(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, sv->ln2_mean, sv->ln2_rstd,
+                                 ws.dg, hv, ws.d_o, hv, gr->dln2_gamma, gr->dln2_beta, T, rows, hv, dt, st));
+    HSTU_CUDA(launch_ln_gate_du(sv->attn_out, hv, w->ln2_gamma, w->ln2_beta, sv->ln2_mean, sv->ln2_rstd, ws.dg, hv,
+                                duvqk, 4 * hv, T, rows, hv, dt, st));
+  }
   // attention backward -> dV, dQ, dK columns of duvqk, rab grads
   const size_t rab_n = (size_t)(d->attn.rab_head_stride ? H : 1) * kNumBuckets;
   HSTU_CUDA(cudaMemsetAsync(gr->dpos_bias, 0, sizeof(float) * rab_n, st));
@@ -389,26 +413,36 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
                         4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, du + 2 * hv * es, 4 * hv, du + 3 * hv * es,
                         4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias, ws.attn, st));
   // a = SiLU(z): dz = da * SiLU'(z)
-  HSTU_CUDA(launch_silu_bwd(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, st));
+  {
+    TraceScope tr("silu_bwd", st);
+    HSTU_CUDA(launch_silu_bwd(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, st));
+    HSTU_CUDA(launch_zero_tail_rows(ws.dz, (int64_t)4 * hv * es, (int64_t)4 * hv * es, T, rows, 64, st));
+  }
   // z = xhat W1^T + b1: dW1 = dz^T xhat, db1 = colsum(dz), dxhat = dz W1
   memset(&p, 0, sizeof(p));
   p.M = 4 * hv; p.N = dm; p.K = T;
   p.A = ws.dz; p.sam = 1; p.sak = 4 * hv;
   p.B = sv->xhat; p.sbn = 1; p.sbk = dm;
-  p.epi = EPI_STORE_F32; p.out = gr->dw1; p.ldo = dm; p.k_dev = rows;
+  p.epi = EPI_STORE_F32; p.out = gr->dw1; p.ldo = dm; p.k_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw1"));
-  HSTU_CUDA(launch_col_sum(ws.dz, 4 * hv, T, rows, 4 * hv, dt, gr->db1, st));
+  {
+    TraceScope tr("colsum_db1", st);
+    HSTU_CUDA(launch_col_sum(ws.dz, 4 * hv, T, rows, 4 * hv, dt, gr->db1, st));
+  }
   memset(&p, 0, sizeof(p));
   p.M = T; p.N = dm; p.K = 4 * hv;
   p.A = ws.dz; p.sam = 4 * hv; p.sak = 1;
   p.B = w->w1; p.sbn = 1; p.sbk = dm;
-  p.epi = EPI_STORE_F32; p.out = ws.dxhat; p.ldo = dm; p.rows_dev = rows;
+  p.epi = EPI_STORE_F32; p.out = ws.dxhat; p.ldo = dm; p.rows_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dxhat"));
   // xhat = LN1(x): dx = dy + LN1 backward
-  HSTU_CUDA(cudaMemsetAsync(gr->dln1_gamma, 0, sizeof(float) * dm, st));
-  HSTU_CUDA(cudaMemsetAsync(gr->dln1_beta, 0, sizeof(float) * dm, st));
-  HSTU_CUDA(launch_ln_bwd(x, dm, w->ln1_gamma, sv->ln1_mean, sv->ln1_rstd, ws.dxhat, dm, dy, dm, dx, dm,
-                          gr->dln1_gamma, gr->dln1_beta, T, rows, dm, dt, st));
+  {
+    TraceScope tr("ln1_bwd", st);
+    HSTU_CUDA(cudaMemsetAsync(gr->dln1_gamma, 0, sizeof(float) * dm, st));
+    HSTU_CUDA(cudaMemsetAsync(gr->dln1_beta, 0, sizeof(float) * dm, st));
+    HSTU_CUDA(launch_ln_bwd(x, dm, w->ln1_gamma, sv->ln1_mean, sv->ln1_rstd, ws.dxhat, dm, dy, dm, dx, dm,
+                            gr->dln1_gamma, gr->dln1_beta, T, rows, dm, io, st));
+  }
   return HSTU_OK;
 }
 
@@ -531,9 +565,9 @@ int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
   HSTU_TRY(check_layer(desc, w));
   HSTU_TRY(check_jagged(jb));
   const int dm = desc->d_model;
-  const int dt = desc->attn.dtype;
-  HSTU_TRY(check_rows(x, dm, dm, dt));
-  HSTU_TRY(check_rows(y, dm, dm, dt));
+  const int io = desc->io_dtype;
+  HSTU_TRY(check_rows(x, dm, dm, io));
+  HSTU_TRY(check_rows(y, dm, dm, io));
   if (x == y) return HSTU_ERR_INVALID_ARG;
   if (saved) {
     const void* ps[] = {saved->xhat, saved->ln1_mean, saved->ln1_rstd, saved->z, saved->uvqk,
@@ -568,10 +602,10 @@ int hstu_layer_bwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
   HSTU_TRY(check_jagged(jb));
   if (!saved || !g) return HSTU_ERR_INVALID_ARG;
   const int dm = desc->d_model;
-  const int dt = desc->attn.dtype;
-  HSTU_TRY(check_rows(x, dm, dm, dt));
-  HSTU_TRY(check_rows(dy, dm, dm, dt));
-  HSTU_TRY(check_rows(dx, dm, dm, dt));
+  const int io = desc->io_dtype;
+  HSTU_TRY(check_rows(x, dm, dm, io));
+  HSTU_TRY(check_rows(dy, dm, dm, io));
+  HSTU_TRY(check_rows(dx, dm, dm, io));
   const void* ps[] = {saved->xhat, saved->ln1_mean, saved->ln1_rstd, saved->z, saved->uvqk, saved->attn_out,
                       saved->ln2_mean, saved->ln2_rstd, g->dw1, g->db1, g->dln1_gamma, g->dln1_beta,
                       g->dln2_gamma, g->dln2_beta, g->dw2, g->db2, g->dpos_bias, g->dtime_bias};
@@ -606,7 +640,7 @@ MfalconWs carve_mfalcon(Carver& c, const hstu_layer_desc* d, int U, int hist_tot
   MfalconWs w;
   w.cap = hist_total + U * bm;
   w.layer = carve_layer_fwd(c, d, U, w.cap, true);
-  const size_t es = elem_size(d->attn.dtype);
+  const size_t es = elem_size(d->io_dtype);
   w.offs = c.take<int32_t>(U + 1);
   w.nt = c.take<int32_t>(U > 0 ? U : 1);
   w.ts = c.take<int64_t>(w.cap);
@@ -638,7 +672,7 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
   for (int l = 0; l < num_layers; ++l) HSTU_TRY(check_layer(desc, &layers[l]));
   if (!hist_offsets || !cand_offsets || !cand_ts || !cand_out || !cand_x) return HSTU_ERR_INVALID_ARG;
   if (hist_total > 0 && (!hist_x || !hist_ts)) return HSTU_ERR_INVALID_ARG;
-  const int dt = desc->attn.dtype;
+  const int dt = desc->io_dtype;
   const int dm = desc->d_model;
   if ((hist_x && !aligned16(hist_x)) || !aligned16(cand_x) || !aligned16(cand_out)) return HSTU_ERR_INVALID_ARG;
   size_t need;

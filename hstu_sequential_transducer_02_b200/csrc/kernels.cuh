@@ -99,6 +99,9 @@ struct GemmParams {
   const int32_t* rows_dev;   // if set: rows = min(M, *rows_dev)
   const int32_t* k_dev;      // if set: reduction length = min(K, *k_dev)
   int accumulate;            // EPI_STORE_F32: add to the existing value
+  int out_f32;               // EPI_BIAS_RESIDUAL / EPI_STORE: output is fp32 (else the operand dtype)
+  int res_f32;               // EPI_BIAS_RESIDUAL: residual is fp32 (else the operand dtype)
+  int32_t* status;           // device status word for bounded-wait timeouts (tensor-core path)
 };
 
 cudaError_t launch_gemm_simt(const GemmParams& p, int dtype, cudaStream_t st);
@@ -107,9 +110,10 @@ bool tc_gemm_supported(const GemmParams& p, int dtype);
 cudaError_t launch_gemm_tc(const GemmParams& p, cudaStream_t st);
 
 // ---------------------------------------------------------------- row kernels
-cudaError_t launch_layer_norm(const void* x, int64_t ldx, const float* gamma, const float* beta, float eps,
-                              void* out, int64_t ldo, float* mean, float* rstd, int rows_cap,
-                              const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
+// xhat = LN(x) * gamma + beta; x in x_dtype, xhat in out_dtype
+cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const float* gamma, const float* beta,
+                              float eps, void* out, int64_t ldo, int out_dtype, float* mean, float* rstd,
+                              int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st);
 cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
                            const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
                            int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
@@ -124,11 +128,19 @@ cudaError_t launch_ln_gate_du(const void* o, int64_t ldo_in, const float* gamma,
                               const float* mean, const float* rstd, const void* dg, int64_t lddg, void* du,
                               int64_t lddu, int rows_cap, const int32_t* rows_dev, int d, int dtype,
                               cudaStream_t st);
-// backward of xhat = LN1(x): dx = dres + LNback(dxhat); accumulates dgamma/dbeta
+// backward of xhat = LN1(x): dx = dres + LNback(dxhat); accumulates dgamma/dbeta.
+// x, dres and dx are in io_dtype, dxhat is fp32
 cudaError_t launch_ln_bwd(const void* x, int64_t ldx, const float* gamma, const float* mean, const float* rstd,
                           const float* dxhat, int64_t lddxh, const void* dres, int64_t lddres, void* dx,
                           int64_t lddx, float* dgamma, float* dbeta, int rows_cap, const int32_t* rows_dev,
-                          int d, int dtype, cudaStream_t st);
+                          int d, int io_dtype, cudaStream_t st);
+// dst (bf16 or fp32 per dst_dtype) = src (src_dtype) for rows < *rows_dev, zero for rows in
+// [*rows_dev, min(cap, round_up(*rows_dev, pad_multiple)))
+cudaError_t launch_convert_rows(const void* src, int64_t lds, int src_dtype, void* dst, int64_t ldd, int dst_dtype,
+                                int cols, int rows_cap, const int32_t* rows_dev, int pad_multiple, cudaStream_t st);
+// zero rows [*rows_dev, min(cap, round_up(*rows_dev, multiple))) of a row-major buffer
+cudaError_t launch_zero_tail_rows(void* buf, int64_t ld_bytes, int64_t row_bytes, int rows_cap,
+                                  const int32_t* rows_dev, int multiple, cudaStream_t st);
 // dz = da * SiLU'(z) (dtype), elementwise on [rows, cols]
 cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
                             const int32_t* rows_dev, int cols, int dtype, cudaStream_t st);

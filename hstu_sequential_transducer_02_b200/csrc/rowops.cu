@@ -58,10 +58,10 @@ __device__ __forceinline__ int rows_of(int cap, const int32_t* rows_dev) {
 }
 
 // ---------------------------------------------------------------- LayerNorm
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(kRowWarps * 32)
 layer_norm_kernel(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma,
-                  const float* __restrict__ beta, float eps, T* __restrict__ out, int64_t ldo,
+                  const float* __restrict__ beta, float eps, TO* __restrict__ out, int64_t ldo,
                   float* __restrict__ mean_out, float* __restrict__ rstd_out, int rows_cap,
                   const int32_t* __restrict__ rows_dev, int d) {
   const int rows = rows_of(rows_cap, rows_dev);
@@ -556,6 +556,38 @@ __global__ void mfalcon_scatter_kernel(const T* __restrict__ y, int d, const int
   }
 }
 
+template <typename TS, typename TD>
+__global__ void convert_rows_kernel(const TS* __restrict__ src, int64_t lds, TD* __restrict__ dst, int64_t ldd,
+                                    int cols, int rows_cap, const int32_t* __restrict__ rows_dev, int pad_multiple) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  int pad_end = ((rows + pad_multiple - 1) / pad_multiple) * pad_multiple;
+  pad_end = pad_end < rows_cap ? pad_end : rows_cap;
+  const int nch = cols / 8;
+  const int64_t total = (int64_t)pad_end * nch;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / nch;
+    const int ch = (int)(e % nch);
+    float v[8];
+    if (r < rows) {
+      load8(src + r * lds + ch * 8, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    store8(dst + r * ldd + ch * 8, v);
+  }
+}
+
+__global__ void zero_tail_rows_kernel(uint32_t* __restrict__ buf, int64_t ld_words, int64_t row_words, int rows_cap,
+                                      const int32_t* __restrict__ rows_dev, int multiple) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  int end = ((rows + multiple - 1) / multiple) * multiple;
+  end = end < rows_cap ? end : rows_cap;
+  const int64_t total = (int64_t)(end - rows) * row_words;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x)
+    buf[(rows + e / row_words) * ld_words + e % row_words] = 0u;
+}
+
 int row_grid(int rows_cap) {
   int g = (rows_cap + kRowWarps - 1) / kRowWarps;
   return g < 1 ? 1 : (g > 148 * 16 ? 148 * 16 : g);
@@ -563,18 +595,25 @@ int row_grid(int rows_cap) {
 
 }  // namespace
 
-cudaError_t launch_layer_norm(const void* x, int64_t ldx, const float* gamma, const float* beta, float eps,
-                              void* out, int64_t ldo, float* mean, float* rstd, int rows_cap,
-                              const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
+cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const float* gamma, const float* beta,
+                              float eps, void* out, int64_t ldo, int out_dtype, float* mean, float* rstd,
+                              int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
   if (rows_cap <= 0) return cudaSuccess;
   const int g = row_grid(rows_cap);
-  if (dtype == HSTU_DTYPE_F32)
-    layer_norm_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo,
-                                                           mean, rstd, rows_cap, rows_dev, d);
+  const int t = kRowWarps * 32;
+  using bf = __nv_bfloat16;
+  if (x_dtype == HSTU_DTYPE_F32 && out_dtype == HSTU_DTYPE_F32)
+    layer_norm_kernel<float, float><<<g, t, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean,
+                                                     rstd, rows_cap, rows_dev, d);
+  else if (x_dtype == HSTU_DTYPE_F32)
+    layer_norm_kernel<float, bf><<<g, t, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd,
+                                                  rows_cap, rows_dev, d);
+  else if (out_dtype == HSTU_DTYPE_F32)
+    layer_norm_kernel<bf, float><<<g, t, 0, st>>>((const bf*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean, rstd,
+                                                  rows_cap, rows_dev, d);
   else
-    layer_norm_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>((const __nv_bfloat16*)x, ldx, gamma, beta, eps,
-                                                                   (__nv_bfloat16*)out, ldo, mean, rstd, rows_cap,
-                                                                   rows_dev, d);
+    layer_norm_kernel<bf, bf><<<g, t, 0, st>>>((const bf*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd,
+                                               rows_cap, rows_dev, d);
   return cudaGetLastError();
 }
 
@@ -630,10 +669,10 @@ cudaError_t launch_ln_gate_du(const void* o, int64_t ldo_in, const float* gamma,
 cudaError_t launch_ln_bwd(const void* x, int64_t ldx, const float* gamma, const float* mean, const float* rstd,
                           const float* dxhat, int64_t lddxh, const void* dres, int64_t lddres, void* dx,
                           int64_t lddx, float* dgamma, float* dbeta, int rows_cap, const int32_t* rows_dev,
-                          int d, int dtype, cudaStream_t st) {
+                          int d, int io_dtype, cudaStream_t st) {
   if (rows_cap <= 0) return cudaSuccess;
   const int g = row_grid(rows_cap) < 296 ? row_grid(rows_cap) : 296;
-  if (dtype == HSTU_DTYPE_F32)
+  if (io_dtype == HSTU_DTYPE_F32)
     ln_bwd_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)x, ldx, gamma, mean, rstd, dxhat, lddxh,
                                                        (const float*)dres, lddres, (float*)dx, lddx, dgamma, dbeta,
                                                        rows_cap, rows_dev, d);
@@ -719,6 +758,34 @@ cudaError_t launch_mfalcon_scatter(const void* y, int d, int dtype, const int32_
   else
     mfalcon_scatter_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16*)y, d, cand_row_map, total_rows,
                                                              cap_rows, (__nv_bfloat16*)cand_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_rows(const void* src, int64_t lds, int src_dtype, void* dst, int64_t ldd, int dst_dtype,
+                                int cols, int rows_cap, const int32_t* rows_dev, int pad_multiple, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  using bf = __nv_bfloat16;
+  const int g = 148 * 8;
+  if (src_dtype == HSTU_DTYPE_F32 && dst_dtype == HSTU_DTYPE_F32)
+    convert_rows_kernel<float, float><<<g, 256, 0, st>>>((const float*)src, lds, (float*)dst, ldd, cols, rows_cap,
+                                                         rows_dev, pad_multiple);
+  else if (src_dtype == HSTU_DTYPE_F32)
+    convert_rows_kernel<float, bf><<<g, 256, 0, st>>>((const float*)src, lds, (bf*)dst, ldd, cols, rows_cap, rows_dev,
+                                                      pad_multiple);
+  else if (dst_dtype == HSTU_DTYPE_F32)
+    convert_rows_kernel<bf, float><<<g, 256, 0, st>>>((const bf*)src, lds, (float*)dst, ldd, cols, rows_cap, rows_dev,
+                                                      pad_multiple);
+  else
+    convert_rows_kernel<bf, bf><<<g, 256, 0, st>>>((const bf*)src, lds, (bf*)dst, ldd, cols, rows_cap, rows_dev,
+                                                   pad_multiple);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_tail_rows(void* buf, int64_t ld_bytes, int64_t row_bytes, int rows_cap,
+                                  const int32_t* rows_dev, int multiple, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  zero_tail_rows_kernel<<<64, 256, 0, st>>>((uint32_t*)buf, ld_bytes / 4, row_bytes / 4, rows_cap, rows_dev,
+                                            multiple);
   return cudaGetLastError();
 }
 

@@ -48,7 +48,7 @@
  *     read it with hstu_workspace_status after synchronising.
  *   - `total_tokens` in hstu_jagged is the capacity (rows of every [T, .]
  *     buffer).  The rows actually used are seq_offsets[batch] <= total_tokens,
- *     read on the device; rows beyond it are not written.
+ *     read on the device; output rows beyond it are not written.
  */
 #ifndef HSTU_H_
 #define HSTU_H_
@@ -96,6 +96,10 @@ typedef struct hstu_attn_desc {
 typedef struct hstu_layer_desc {
   int32_t d_model;          /* d; must be a multiple of 8, <= 1024 */
   float   ln_eps;           /* LayerNorm epsilon, 1e-5 */
+  int32_t io_dtype;         /* element type of the residual stream X, Y (and dX, dY):
+                               attn.dtype, or HSTU_DTYPE_F32 to keep the residual
+                               stream in fp32 while activations and weights are bf16 */
+  int32_t reserved;         /* must be 0 */
   hstu_attn_desc attn;      /* H * dv is the width of U, V, Q, K and of A V */
 } hstu_layer_desc;
 
@@ -245,7 +249,7 @@ int hstu_layer_fwd_workspace_size(const hstu_layer_desc* desc, int32_t batch,
                                   int32_t total_tokens, size_t* bytes);
 
 /* Y = X + f2(LayerNorm2(A V) (.) U) with U, V, Q, K = Split(SiLU(f1(LayerNorm1(X)))).
- *   x, y: device [T, d] dtype, contiguous (row stride d); y may not alias x.
+ *   x, y: device [T, d] io_dtype, contiguous (row stride d); y may not alias x.
  *   saved: NULL for inference, else its buffers receive what hstu_layer_bwd needs. */
 int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w,
                    const hstu_jagged* jb, const void* x, void* y,
@@ -256,8 +260,9 @@ int hstu_layer_bwd_workspace_size(const hstu_layer_desc* desc, int32_t batch,
                                   int32_t total_tokens, size_t* bytes);
 
 /* Gradients of sum(Y * dy) for one layer, from the activations hstu_layer_fwd
- * saved.  dx: device [T, d] dtype (may alias dy).  All gradients in `g` are
- * overwritten, rab gradients included. */
+ * saved.  x, dy, dx: device [T, d] io_dtype (dx may alias dy).  All gradients
+ * in `g` are overwritten, rab gradients included.  Rows of the saved xhat beyond
+ * seq_offsets[batch] (up to the next multiple of 64) are set to zero. */
 int hstu_layer_bwd(const hstu_layer_desc* desc, const hstu_layer_weights* w,
                    const hstu_jagged* jb, const void* x, const hstu_layer_saved* saved,
                    const void* dy, void* dx, const hstu_layer_grads* g,
@@ -281,7 +286,7 @@ int mfalcon_rank_workspace_size(const hstu_layer_desc* desc, int32_t num_layers,
  *   hist_ts [hist_total]; cand_x [cand_offsets[U], d], cand_ts [...]: device;
  *   max_candidates: host upper bound on any user's candidate count (sets the
  *   number of microbatches, ceil(max_candidates / microbatch));
- *   cand_out: device [cand_offsets[U], d] dtype. */
+ *   hist_x, cand_x, cand_out are in desc->io_dtype; cand_out: [cand_offsets[U], d]. */
 int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers,
                  int32_t num_layers, int32_t num_users, int32_t hist_total,
                  int32_t max_candidates, int32_t microbatch,

@@ -38,14 +38,19 @@ def errors(got, ref):
     return max_abs, rel
 
 
-def assert_close(got, ref, dtype_name, what=""):
+def assert_close(got, ref, dtype_name, what="", grad=False):
+    """grad=True: the tensor is a gradient, whose magnitude is set by the loss
+    rather than being O(1); its max-abs bound is taken relative to its largest
+    reference magnitude, max(1, max|ref|), because storing a value of magnitude
+    M in the tensor's dtype alone already errs by up to M * 2^-9 (bf16)."""
     if isinstance(got, torch.Tensor):
         got = got.float().cpu().numpy()
     max_abs, rel = errors(got, ref)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    scale = max(1.0, float(np.max(np.abs(ref)))) if (grad and np.size(ref)) else 1.0
     if dtype_name == "f32":
-        assert max_abs <= FP32_MAX_ABS, f"{what}: max-abs {max_abs:.3e} > {FP32_MAX_ABS}"
+        assert max_abs <= FP32_MAX_ABS * scale, f"{what}: max-abs {max_abs:.3e} > {FP32_MAX_ABS * scale:.3e}"
     else:
         assert rel <= BF16_REL_FRO, f"{what}: rel-Frobenius {rel:.3e} > {BF16_REL_FRO}"
-        assert max_abs <= BF16_MAX_ABS, f"{what}: max-abs {max_abs:.3e} > {BF16_MAX_ABS}"
+        assert max_abs <= BF16_MAX_ABS * scale, f"{what}: max-abs {max_abs:.3e} > {BF16_MAX_ABS * scale:.3e}"
     return max_abs, rel

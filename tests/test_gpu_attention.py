@@ -157,7 +157,7 @@ def test_attn_bwd_matches_oracle(dtype_name, dh, mfalcon):
     rq, rk, rv, rpb, rtb = O.attention_backward(d["q"], d["k"], d["v"], d["dout"], d["seq_offsets"],
                                                 d["timestamps"], d["pos_bias"], d["time_bias"], d["num_targets"])
     for got, ref, name in [(dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")]:
-        assert_close(got.float().cpu().numpy().reshape(ref.shape), ref, dtype_name, name)
+        assert_close(got.float().cpu().numpy().reshape(ref.shape), ref, dtype_name, name, grad=True)
     # rab gradients are fp32 sums over many pairs: relative Frobenius bound
     for got, ref, name in [(dpb, rpb, "dpos"), (dtb, rtb, "dtime")]:
         g = got.cpu().numpy()

@@ -170,53 +170,98 @@ def _sl_workload(wl):
     return g, offs
 
 
-def test_training_step_config4_scaled():
-    """8-layer stack forward + backward with Stochastic Length: dU, dV, dQ, dK
-    and the rab gradients of every layer, plus weight gradients, vs the oracle."""
+def _train_step(wl, residual_fp32: bool):
+    """SL on the GPU, forward through the stack saving activations, backward
+    from dY = G.  Returns the GPU's per-layer inputs x_l, upstream gradients
+    dy_l, gradients, and the SL-selected host arrays."""
     b = _b()
-    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
     s = wl.spec
     td = torch.bfloat16
+    io = torch.float32 if residual_fp32 else td
     e = wl.extras
-    # SL on the GPU, gathers on the GPU
     offs_d, idx_d = b.stochastic_length(dev(wl.seq_offsets), dev(e["sl_coin"].view(np.int32)),
                                         dev(e["sl_keys"].view(np.int32)), int(e["sl_len"]), int(e["sl_prob_u32"]))
     g_ref, o_ref = _sl_workload(wl)
     T2 = int(o_ref[-1])
     count = offs_d[-1:]
-    x = b.gather_rows(dev(wl.x, td), idx_d, count, torch.empty(T2, s.d_model, dtype=td, device="cuda"))
+    x = b.gather_rows(dev(wl.x, io), idx_d, count, torch.empty(T2, s.d_model, dtype=io, device="cuda"))
     ts = b.gather_rows(dev(wl.timestamps), idx_d, count, torch.empty(T2, dtype=torch.int64, device="cuda"))
-    gy = b.gather_rows(dev(e["grad_out"], td), idx_d, count, torch.empty(T2, s.d_model, dtype=td, device="cuda"))
-    layers = _layers(wl)
+    gy = b.gather_rows(dev(e["grad_out"], io), idx_d, count, torch.empty(T2, s.d_model, dtype=io, device="cuda"))
+    layers = [b.Layer(layer_to_dev(p, td), s.d_model, s.num_heads, s.head_dim, residual_fp32=residual_fp32)
+              for p in wl.layers]
     hv = s.num_heads * s.head_dim
     saved = [b.Saved.alloc(T2, s.d_model, hv, td, "cuda") for _ in layers]
     xs = [x]
     for ly, sv in zip(layers, saved):
         xs.append(ly.forward(xs[-1], offs_d, ts, saved=sv))
-    dy = gy
+    dys = [None] * len(layers)
     grads = [None] * len(layers)
+    dy = gy
     for li in range(len(layers) - 1, -1, -1):
+        dys[li] = dy
         dy, grads[li] = layers[li].backward(xs[li], dy, saved[li], offs_d, ts)
     torch.cuda.synchronize()
-    # oracle on the same subsampled inputs
-    x_h = wl.x[g_ref]
-    ts_h = wl.timestamps[g_ref]
-    gy_h = e["grad_out"][g_ref]
-    ref = O.stack_backward(x_h, wl.layers, gy_h, o_ref, ts_h, s.num_heads, s.head_dim)
-    for li in range(len(layers) - 1, -1, -1):
-        duvqk = grads[li]["uvqk"].float().cpu().numpy()
-        r = ref[li]
-        T = T2
-        ref_uvqk = np.concatenate([r["dU"].reshape(T, hv), r["dV"].reshape(T, hv), r["dQ"].reshape(T, hv),
-                                   r["dK"].reshape(T, hv)], axis=1)
-        for c, name in enumerate("UVQK"):
-            ma, rel = errors(duvqk[:, c * hv:(c + 1) * hv], ref_uvqk[:, c * hv:(c + 1) * hv])
-            print(f"layer {li} d{name}: max-abs {ma:.3e} rel-fro {rel:.3e}")
-        for c, name in enumerate("UVQK"):
-            assert_close(duvqk[:, c * hv:(c + 1) * hv], ref_uvqk[:, c * hv:(c + 1) * hv], "bf16", f"L{li} d{name}")
-        for gname, rname in [("pos_bias", "dpos_bias"), ("time_bias", "dtime_bias"), ("w1", "dw1"), ("w2", "dw2"),
-                             ("b1", "db1"), ("b2", "db2"), ("ln1_gamma", "dln1_g"), ("ln2_gamma", "dln2_g")]:
-            got = grads[li][gname].cpu().numpy()
-            rr = r[rname]
-            assert np.linalg.norm(got - rr) <= 1e-2 * max(np.linalg.norm(rr), 1e-6), f"L{li} {gname}"
-    assert_close(dy.float().cpu().numpy(), ref[0]["dx"], "bf16", "dx")
+    host = lambda t: t.float().cpu().numpy().astype(np.float64)
+    return dict(xs=[host(t) for t in xs[:-1]], dys=[host(t) for t in dys], dx=host(dy), grads=grads, T=T2, hv=hv,
+                offs=o_ref, ts=wl.timestamps[g_ref], x0=wl.x[g_ref], g0=e["grad_out"][g_ref])
+
+
+def _layer_errors(r, gr, T, hv):
+    duvqk = gr["uvqk"].float().cpu().numpy()
+    ref_uvqk = np.concatenate([r["dU"].reshape(T, hv), r["dV"].reshape(T, hv), r["dQ"].reshape(T, hv),
+                               r["dK"].reshape(T, hv)], axis=1)
+    out = {}
+    for c, name in enumerate("UVQK"):
+        out["d" + name] = (duvqk[:, c * hv:(c + 1) * hv], ref_uvqk[:, c * hv:(c + 1) * hv])
+    for gname, rname in [("pos_bias", "dpos_bias"), ("time_bias", "dtime_bias"), ("w1", "dw1"), ("w2", "dw2"),
+                         ("b1", "db1"), ("b2", "db2"), ("ln1_gamma", "dln1_g"), ("ln1_beta", "dln1_b"),
+                         ("ln2_gamma", "dln2_g"), ("ln2_beta", "dln2_b")]:
+        out[gname] = (gr[gname].cpu().numpy(), r[rname])
+    return out
+
+
+def _check_train(run, wl, chained_rel_bound):
+    """Per layer, teacher-forced: the oracle's gradients of layer l at the GPU's
+    own layer input x_l and upstream gradient dy_l, at the specification's bf16
+    tolerance.  Chained: the oracle's whole-stack gradients from X and G, at
+    `chained_rel_bound` (bf16 operand rounding accumulates through the stack)."""
+    s = wl.spec
+    T, hv = run["T"], run["hv"]
+    chained = O.stack_backward(run["x0"], wl.layers, run["g0"], run["offs"], run["ts"], s.num_heads, s.head_dim)
+    worst = 0.0
+    for li in range(len(wl.layers) - 1, -1, -1):
+        tf = O.layer_backward(run["xs"][li], wl.layers[li], run["dys"][li], run["offs"], run["ts"], s.num_heads,
+                              s.head_dim)
+        for name, (got, ref) in _layer_errors(tf, run["grads"][li], T, hv).items():
+            ma, rel = errors(got, ref)
+            print(f"layer {li} {name}: teacher-forced rel-fro {rel:.3e} max-abs {ma:.3e}")
+            if name in ("dU", "dV", "dQ", "dK"):
+                assert_close(got, ref, "bf16", f"L{li} {name} (teacher-forced)", grad=True)
+            else:
+                assert rel <= 1e-2, f"L{li} {name} (teacher-forced) rel-fro {rel:.3e}"
+        for name, (got, ref) in _layer_errors(chained[li], run["grads"][li], T, hv).items():
+            _, rel = errors(got, ref)
+            worst = max(worst, rel)
+            assert rel <= chained_rel_bound, f"L{li} {name} (chained) rel-fro {rel:.3e}"
+    print(f"chained worst rel-fro {worst:.3e}")
+    tf0 = O.layer_backward(run["xs"][0], wl.layers[0], run["dys"][0], run["offs"], run["ts"], s.num_heads,
+                           s.head_dim)
+    assert_close(run["dx"], tf0["dx"], "bf16", "dx (teacher-forced)", grad=True)
+
+
+def test_training_step_config4_scaled():
+    """8-layer bf16 stack (fp32 residual stream) forward + backward with
+    Stochastic Length: dU, dV, dQ, dK, the rab gradients and the weight
+    gradients of every layer vs the oracle.  The chained bound 1.5e-2 comes from
+    an fp64 simulation in which only the bf16 rounding of the tensor-core
+    operands (xhat, U/V/Q/K, A V, gate) is applied: that alone moves layer 7's
+    gradients by up to 9.1e-3 from the exact stack."""
+    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
+    _check_train(_train_step(wl, residual_fp32=True), wl, chained_rel_bound=1.5e-2)
+
+
+def test_training_step_bf16_residual_two_layers():
+    """The same step with a bf16 residual stream, two layers deep."""
+    wl = W.make_workload(4, batch=5, scale=1 / 8, random_affine=True)
+    wl.layers = wl.layers[:2]
+    _check_train(_train_step(wl, residual_fp32=False), wl, chained_rel_bound=1e-2)

@@ -30,10 +30,11 @@ using namespace sm100;
 
 constexpr int BM = 128;                    // q rows per tile (UMMA M)
 constexpr int BN = 128;                    // kv columns per tile
-constexpr int kEpiWarps = 8;               // two warps per TMEM lane quarter (one per 64-column half)
+constexpr int kEpiWarps = 16;              // four warps per TMEM lane quarter, one per 32-column segment
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kBoxBytes = 128 * 128;       // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
+constexpr int kRecBytes = kTsRecWords * 4;
 
 template <int DH>
 struct Cfg {
@@ -42,14 +43,15 @@ struct Cfg {
   static constexpr int kTileBytes = BM * DH * 2;
 };
 
-struct TsStage {
-  int64_t ts[BN];       // timestamps of the tile's columns (0 beyond the sequence)
-  int32_t rel[BN];      // ts - tmin[half] (valid when wide[half] == 0)
-  int64_t tmin[2];      // per 64-column half, over the columns inside the sequence
-  int64_t tmax[2];
-  int32_t wide[2];      // 1: the half's time span does not fit the 32-bit path
-  int32_t pad[2];
+// Timestamp record of one kv tile, as written by ts_tiles_kernel.
+struct TsRec {
+  int32_t rel[BN];   // t_j - t_first(sequence), clamped to +-(2^30 - 1); 0 beyond the sequence
+  int32_t mn[4];     // per 32-column segment: min / max of rel over the columns inside the sequence
+  int32_t mx[4];
+  int32_t wide;      // 1 if some column's offset left +-2^30 (then the 64-bit path is used)
+  int32_t pad[3];
 };
+static_assert(sizeof(TsRec) == kRecBytes, "record layout");
 
 struct Barriers {
   uint64_t q_full, q_empty;
@@ -65,6 +67,7 @@ struct TcParams {
   CUtensorMap map_k;
   CUtensorMap map_v;
   AttnFwdParams p;
+  float ln2_over_div;   // ln(2) / time_div
 };
 
 template <int DH>
@@ -74,8 +77,9 @@ struct Layout {
   static constexpr int kV = kK + Cfg<DH>::kStages * Cfg<DH>::kTileBytes;
   static constexpr int kP = kV + Cfg<DH>::kStages * Cfg<DH>::kTileBytes;
   static constexpr int kTs = kP + BM * BN * 2;
-  static constexpr int kThr = kTs + Cfg<DH>::kStages * (int)sizeof(TsStage);
-  static constexpr int kPosB = kThr + kNumBuckets * 8;
+  static constexpr int kThr = kTs + Cfg<DH>::kStages * kRecBytes;
+  static constexpr int kThr32 = kThr + kNumBuckets * 8;
+  static constexpr int kPosB = kThr32 + (kNumBuckets + 4) * 4;
   static constexpr int kTimeB = kPosB + kNumBuckets * 4;
   static constexpr int kBar = (kTimeB + kNumBuckets * 4 + 15) & ~15;
   static constexpr int kMisc = kBar + (int)sizeof(Barriers);
@@ -98,6 +102,22 @@ __device__ __forceinline__ float silu_tanh(float s) {
   return fmaf(h, tanh_approx(h), h);
 }
 
+// Exact time bucket of 0 <= d < 2^31 in O(1): an approximate ln(d)/div rounded
+// to the nearest integer is at most one bucket off, and one comparison with
+// each neighbouring integer threshold corrects it (thr32[b] = min(threshold b,
+// INT32_MAX), thr32[128] = INT32_MAX).
+__device__ __forceinline__ int fast_bucket(int32_t d, const int32_t* thr32, float ln2_over_div) {
+  d = d < 1 ? 1 : d;
+  const int sh = d >= (1 << 23) ? 8 : 0;
+  const float f = __int_as_float(0x4B000000 | (d >> sh)) - 8388608.0f;   // exact: (d >> sh) < 2^23
+  const float x = fmaf(__log2f(f) + (float)sh, ln2_over_div, 12582912.0f);
+  int b = __float_as_int(x) - 0x4B400000;                               // nearest integer
+  b = b < 0 ? 0 : (b > kNumBuckets - 1 ? kNumBuckets - 1 : b);
+  if (d < thr32[b]) b -= 1;
+  else if (d >= thr32[b + 1]) b += 1;
+  return b > kNumBuckets - 1 ? kNumBuckets - 1 : b;
+}
+
 // ---------------------------------------------------------------------------
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_constant__ TcParams prm) {
@@ -111,9 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   int64_t* thr = reinterpret_cast<int64_t*>(smem + L::kThr);
+  int32_t* thr32 = reinterpret_cast<int32_t*>(smem + L::kThr32);
   float* pos_b = reinterpret_cast<float*>(smem + L::kPosB);
   float* time_b = reinterpret_cast<float*>(smem + L::kTimeB);
-  TsStage* tss = reinterpret_cast<TsStage*>(smem + L::kTs);
+  TsRec* recs = reinterpret_cast<TsRec*>(smem + L::kTs);
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sK = smem_u32(smem + L::kK);
   const uint32_t sV = smem_u32(smem + L::kV);
@@ -146,10 +167,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  for (int c = threadIdx.x; c < kNumBuckets; c += kThreads) {
-    thr[c] = p.thr.v[c];
-    pos_b[c] = p.pos_bias[c];
-    time_b[c] = p.time_bias[c];
+  for (int c = threadIdx.x; c < kNumBuckets + 4; c += kThreads) {
+    if (c < kNumBuckets) {
+      thr[c] = p.thr.v[c];
+      thr32[c] = p.thr.v[c] > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)p.thr.v[c];
+      pos_b[c] = p.pos_bias[c];
+      time_b[c] = p.time_bias[c];
+    } else {
+      thr32[c] = 0x7FFFFFFF;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -164,75 +190,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
 
   if (warp == 0) {
     // =================================================================== producer
-    int kv_it = 0;
-    for (int k = 0;; ++k) {
-      const int idx = snake_item(k, blockIdx.x, G);
-      if (idx >= count || *abort_flag) break;
-      const WorkItem wi = p.items[idx];
-      const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
-      const int r0 = wi.qtile * BM;
-      const int r1 = min(si.n, r0 + BM);
-      if (!mbar_wait(&bars->q_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
-      if (lane == 0) {
+    if (lane == 0) {
+      int kv_it = 0;
+      for (int k = 0;; ++k) {
+        const int idx = snake_item(k, blockIdx.x, G);
+        if (idx >= count || *abort_flag) break;
+        const WorkItem wi = p.items[idx];
+        const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+        const int r0 = wi.qtile * BM;
+        const int r1 = min(si.n, r0 + BM);
+        const TsRec* grec = reinterpret_cast<const TsRec*>(p.tile_recs) + p.tile_base[wi.seq];
+        if (!mbar_wait(&bars->q_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
         mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
         for (int b = 0; b < C::kBoxes; ++b)
           tma_load_2d(smem + L::kQ + b * kBoxBytes, &prm.map_q, &bars->q_full, wi.head * DH + 64 * b, si.start + r0);
-      }
-      const KvRange kr = kv_tiles_for(r0, r1, si.hist, BN);
-      const int nk = kv_count(kr);
-      for (int jj = 0; jj < nk; ++jj, ++kv_it) {
-        const int c0 = kv_tile_at(kr, jj) * BN;
-        const int st = kv_it % S;
-        if (!mbar_wait(&bars->kv_empty[st], ((kv_it / S) & 1) ^ 1, tmo, abort_flag)) goto fail;
-        // timestamps of the tile and per-half ranges
-        TsStage& ts = tss[st];
-        int64_t t[4];
-        int64_t mn[2] = {INT64_MAX, INT64_MAX}, mx[2] = {INT64_MIN, INT64_MIN};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = lane + 32 * e;
-          const bool ok = c0 + c < si.n;
-          t[e] = ok ? p.timestamps[si.start + c0 + c] : 0;
-          if (ok) {
-            mn[e >> 1] = min(mn[e >> 1], t[e]);
-            mx[e >> 1] = max(mx[e >> 1], t[e]);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            mn[h] = min(mn[h], (int64_t)__shfl_xor_sync(0xffffffffu, (long long)mn[h], o));
-            mx[h] = max(mx[h], (int64_t)__shfl_xor_sync(0xffffffffu, (long long)mx[h], o));
-          }
-          if (mn[h] > mx[h]) { mn[h] = 0; mx[h] = 0; }  // no column of this half inside the sequence
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = lane + 32 * e;
-          ts.ts[c] = t[e];
-          const int64_t d = t[e] - mn[e >> 1];
-          ts.rel[c] = (int32_t)(d < 0 ? 0 : (d > 0x3FFFFFFF ? 0x3FFFFFFF : d));
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            ts.tmin[h] = mn[h];
-            ts.tmax[h] = mx[h];
-            ts.wide[h] = (uint64_t)(mx[h] - mn[h]) >= (1ull << 30) ? 1 : 0;
-          }
-        }
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&bars->kv_full[st], 2 * C::kTileBytes);
+        const KvRange kr = kv_tiles_for(r0, r1, si.hist, BN);
+        const int nk = kv_count(kr);
+        for (int jj = 0; jj < nk; ++jj, ++kv_it) {
+          const int kt = kv_tile_at(kr, jj);
+          const int st = kv_it % S;
+          if (!mbar_wait(&bars->kv_empty[st], ((kv_it / S) & 1) ^ 1, tmo, abort_flag)) goto fail;
+          mbar_arrive_expect_tx(&bars->kv_full[st], 2 * C::kTileBytes + kRecBytes);
+          bulk_load(&recs[st], grec + kt, kRecBytes, &bars->kv_full[st]);
           for (int b = 0; b < C::kBoxes; ++b) {
             tma_load_2d(smem + L::kK + st * C::kTileBytes + b * kBoxBytes, &prm.map_k, &bars->kv_full[st],
-                        wi.head * DH + 64 * b, si.start + c0);
+                        wi.head * DH + 64 * b, si.start + kt * BN);
             tma_load_2d(smem + L::kV + st * C::kTileBytes + b * kBoxBytes, &prm.map_v, &bars->kv_full[st],
-                        wi.head * DV + 64 * b, si.start + c0);
+                        wi.head * DV + 64 * b, si.start + kt * BN);
           }
         }
-        __syncwarp();
       }
     }
   } else if (warp == 1) {
@@ -297,11 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     }
   } else {
     // =================================================================== epilogue
-    const int ew = warp - 2;               // 0..7
+    const int ew = warp - 2;               // 0..15
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-    const int half = ew >> 2;              // 64-column half of S / of O
+    const int seg = ew >> 2;               // 32-column segment of S (and of O)
     const int r = quarter * 32 + lane;     // row of the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float k_lg = prm.ln2_over_div;
     int s_it = 0, kv_it = 0, p_it = 0;
     int cur_head = -1;
     for (int k = 0;; ++k) {
@@ -322,7 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       const int i = r0 + r;
       const bool live = i < si.n;
       const bool cand = i >= si.hist;
-      const int64_t ti = live ? p.timestamps[si.start + i] : 0;
+      const int64_t t_first = si.n > 0 ? p.timestamps[si.start] : 0;
+      const int64_t ti = live ? p.timestamps[si.start + i] : t_first;
+      const int64_t rel64 = ti - t_first;
+      const bool row_narrow = rel64 > -(1ll << 30) && rel64 < (1ll << 30);
+      const int32_t ri = (int32_t)rel64;
       const int posi = token_pos(i, si.hist);
       const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
       const int nk = kv_count(kr);
@@ -332,114 +323,102 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const int st = kv_it % S;
         if (!mbar_wait(&bars->s_full[sb], (s_it >> 1) & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
-        uint32_t raw[2][32];
-        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + half * 64, raw[0]);
-        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + half * 64 + 32, raw[1]);
+        uint32_t raw[32];
+        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
         if (!mbar_wait(&bars->kv_full[st], (kv_it / S) & 1, tmo, abort_flag)) goto fail;
-        const TsStage& ts = tss[st];
-        // ---- classify this row's 64 columns
-        const int cl = c0 + half * 64;   // first column of the half
-        float pv[64];
-        bool any_live = live && (cand ? (cl < si.hist || (i >= cl && i < cl + 64)) : (cl <= i));
-        const bool full = live && (cand ? (cl + 63 < si.hist) : (cl + 63 <= i));
-        int mode = 0;  // 0: zero, 1: constant bias, 2: <= 3 time buckets (32-bit), 3: general
+        const TsRec& rec = recs[st];
+        // ---- classify this row's 32 columns
+        const int cl = c0 + seg * 32;   // first column of the segment
+        const bool narrow = row_narrow && !rec.wide;
+        const bool any_live = live && (cand ? (cl < si.hist || (i >= cl && i < cl + 32)) : (cl <= i));
+        const bool full = live && (cand ? (cl + 31 < si.hist) : (cl + 31 <= i));
+        int mode = any_live ? 3 : 0;  // 0: zero, 1: one time bucket, 2: 2-4 buckets, 3: general
         float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
-        int32_t th1 = 0x7FFFFFFF, th2 = 0x7FFFFFFF, th3 = 0x7FFFFFFF, ri = 0;
-        if (any_live) {
-          mode = 3;
-          if (full && posi - (cl + 63) >= kNumBuckets - 1) {
-            const int64_t tmn = ts.tmin[half], tmx = ts.tmax[half];
-            uint64_t dlo, dhi;
-            if (ti >= tmx) { dlo = (uint64_t)(ti - tmx); dhi = (uint64_t)(ti - tmn); }
-            else if (ti <= tmn) { dlo = (uint64_t)(tmn - ti); dhi = (uint64_t)(tmx - ti); }
-            else { dlo = 0; dhi = max((uint64_t)(ti - tmn), (uint64_t)(tmx - ti)); }
-            const int tlo = time_bucket_exact(dlo, thr), thi = time_bucket_exact(dhi, thr);
-            const float pb127 = pos_b[kNumBuckets - 1];
-            const int64_t rel_i = ti - tmn;
-            if (tlo == thi) {
-              mode = 1;
-              b0 = pb127 + time_b[tlo];
-            } else if (thi - tlo <= 3 && !ts.wide[half] && rel_i > -(1ll << 30) && rel_i < (1ll << 30)) {
-              mode = 2;
-              ri = (int32_t)rel_i;
-              b0 = pb127 + time_b[tlo];
-              b1 = pb127 + time_b[min(tlo + 1, thi)];
-              b2 = pb127 + time_b[min(tlo + 2, thi)];
-              b3 = pb127 + time_b[min(tlo + 3, thi)];
-              auto th32 = [&](int b) -> int32_t {
-                if (b > thi) return 0x7FFFFFFF;
-                const int64_t v = thr[b];
-                return v > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)v;
-              };
-              th1 = th32(tlo + 1);
-              th2 = th32(tlo + 2);
-              th3 = th32(tlo + 3);
-            }
+        int32_t th1 = 0x7FFFFFFF, th2 = 0x7FFFFFFF, th3 = 0x7FFFFFFF;
+        if (full && narrow && posi - (cl + 31) >= kNumBuckets - 1) {
+          const int32_t mn = rec.mn[seg], mx = rec.mx[seg];
+          int32_t dlo, dhi;
+          if (ri >= mx) { dlo = ri - mx; dhi = ri - mn; }
+          else if (ri <= mn) { dlo = mn - ri; dhi = mx - ri; }
+          else { dlo = 0; dhi = max(ri - mn, mx - ri); }
+          const int tlo = fast_bucket(dlo, thr32, k_lg), thi = fast_bucket(dhi, thr32, k_lg);
+          const float pb127 = pos_b[kNumBuckets - 1];
+          b0 = pb127 + time_b[tlo];
+          if (tlo == thi) {
+            mode = 1;
+          } else if (thi - tlo <= 3) {
+            mode = 2;
+            b1 = pb127 + time_b[tlo + 1];
+            th1 = thr32[tlo + 1];
+            if (thi - tlo >= 2) { b2 = pb127 + time_b[tlo + 2]; th2 = thr32[tlo + 2]; }
+            if (thi - tlo >= 3) { b3 = pb127 + time_b[tlo + 3]; th3 = thr32[tlo + 3]; }
           }
         }
         // ---- bias, SiLU, mask
+        float pv[32];
         if (mode == 0) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) pv[e] = 0.f;
+          for (int e = 0; e < 32; ++e) pv[e] = 0.f;
         } else if (mode == 1) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) pv[e] = silu_tanh(__uint_as_float(raw[e >> 5][e & 31]) + b0);
+          for (int e = 0; e < 32; ++e) pv[e] = silu_tanh(__uint_as_float(raw[e]) + b0);
         } else if (mode == 2) {
 #pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) {
-            const int4 rel4 = *reinterpret_cast<const int4*>(&ts.rel[half * 64 + e4 * 4]);
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const int4 rel4 = *reinterpret_cast<const int4*>(&rec.rel[seg * 32 + e4 * 4]);
             const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int e = e4 * 4 + u;
               const int32_t dd = abs(ri - rv[u]);
-              float bias = b0;
-              bias = dd >= th1 ? b1 : bias;
+              float bias = dd >= th1 ? b1 : b0;
               bias = dd >= th2 ? b2 : bias;
               bias = dd >= th3 ? b3 : bias;
-              pv[e] = silu_tanh(__uint_as_float(raw[e >> 5][e & 31]) + bias);
+              pv[e] = silu_tanh(__uint_as_float(raw[e]) + bias);
             }
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
+          for (int e = 0; e < 32; ++e) {
             const int j = cl + e;
             float v = 0.f;
             if (attended(i, j, si.n, si.hist)) {
               const int pb = pos_bucket(posi, token_pos(j, si.hist));
-              const int tb = time_bucket_exact(abs_diff_i64(ti, ts.ts[half * 64 + e]), thr);
-              v = silu_tanh(__uint_as_float(raw[e >> 5][e & 31]) + pos_b[pb] + time_b[tb]);
+              int tb;
+              if (narrow) tb = fast_bucket(abs(ri - rec.rel[seg * 32 + e]), thr32, k_lg);
+              else tb = time_bucket_exact(abs_diff_i64(ti, p.timestamps[si.start + j]), thr);
+              v = silu_tanh(__uint_as_float(raw[e]) + pos_b[pb] + time_b[tb]);
             }
             pv[e] = v;
           }
         }
-        uint32_t pk[32];
+        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
         // ---- P -> shared memory (A operand, K-major, 128-byte swizzle)
         if (!mbar_wait(&bars->p_empty, (p_it & 1) ^ 1, tmo, abort_flag)) goto fail;
-        const uint32_t prow = sP + half * kBoxBytes + r * 128;
+        const uint32_t prow = sP + (seg >> 1) * kBoxBytes + r * 128;
+        const int cbase = (seg & 1) * 4;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(prow + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        for (int c = 0; c < 4; ++c)
+          st_shared_v4(prow + (((cbase + c) ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full);
       }
-      // ---- O readout
+      // ---- O readout: this warp's DV/4 columns
       if (!mbar_wait(&bars->o_full, k & 1, tmo, abort_flag)) goto fail;
       tc_fence_after();
-      constexpr int kOc = DV / 2;  // columns of O per thread
+      constexpr int kOc = DV / 4;
       uint32_t oraw[kOc];
-      if constexpr (kOc == 64) {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + half * kOc, *reinterpret_cast<uint32_t(*)[32]>(&oraw[0]));
-        tmem_ld_32x32b_x32(tmem_o + lane_off + half * kOc + 32, *reinterpret_cast<uint32_t(*)[32]>(&oraw[32]));
+      if constexpr (kOc == 32) {
+        tmem_ld_32x32b_x32(tmem_o + lane_off + seg * kOc, *reinterpret_cast<uint32_t(*)[32]>(&oraw[0]));
       } else {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + half * kOc, *reinterpret_cast<uint32_t(*)[32]>(&oraw[0]));
+        tmem_ld_32x32b_x16(tmem_o + lane_off + seg * kOc, *reinterpret_cast<uint32_t(*)[16]>(&oraw[0]));
       }
       tmem_ld_wait();
       tc_fence_before();
@@ -447,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       if (lane == 0) mbar_arrive(&bars->o_empty);
       if (live) {
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(si.start + i) * p.ldo +
-                             (int64_t)wi.head * DV + half * kOc;
+                             (int64_t)wi.head * DV + seg * kOc;
 #pragma unroll
         for (int c = 0; c < kOc / 8; ++c) {
           uint4 v;
@@ -464,8 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
 fail:
   set_status(p.status, HSTU_ERR_TIMEOUT);
   *abort_flag = 1;
-  if (warp == 0) {
-    // let every copy this warp may have issued land before the CTA exits (bounded)
+  if (warp == 0 && lane == 0) {
+    // let every copy this CTA may have issued land before it exits (bounded)
     for (int s = 0; s < S; ++s) {
       mbar_wait(&bars->kv_full[s], 0, 100000000ll, nullptr);
       mbar_wait(&bars->kv_full[s], 1, 100000000ll, nullptr);
@@ -480,6 +459,47 @@ teardown:
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Timestamp records: one block of 128 threads per kv tile of the batch.
+__global__ void __launch_bounds__(128) ts_tiles_kernel(const int32_t* __restrict__ offs,
+                                                       const int64_t* __restrict__ ts, int B,
+                                                       const int32_t* __restrict__ tile_base,
+                                                       int32_t* __restrict__ recs) {
+  const int t = blockIdx.x;
+  if (t >= tile_base[B]) return;
+  int lo = 0, hi = B;  // sequence s with tile_base[s] <= t < tile_base[s + 1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_base[mid] <= t) lo = mid; else hi = mid;
+  }
+  const int s = lo;
+  const int start = offs[s], n = offs[s + 1] - start;
+  const int c = (t - tile_base[s]) * BN + threadIdx.x;
+  const bool ok = c < n;
+  const int64_t d = ok ? ts[start + c] - ts[start] : 0;
+  const int64_t lim = (1ll << 30) - 1;
+  const int32_t rel = (int32_t)(d < -lim ? -lim : (d > lim ? lim : d));
+  const bool wide = ok && (d < -lim || d > lim);
+  int32_t mn = ok ? rel : 0x7FFFFFFF, mx = ok ? rel : (int32_t)0x80000000;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const int any_wide = __syncthreads_or(wide);
+  int32_t* rec = recs + (int64_t)t * kTsRecWords;
+  rec[threadIdx.x] = rel;
+  if ((threadIdx.x & 31) == 0) {
+    const int w = threadIdx.x >> 5;
+    rec[BN + w] = mn > mx ? 0 : mn;
+    rec[BN + 4 + w] = mn > mx ? 0 : mx;
+  }
+  if (threadIdx.x == 0) {
+    rec[BN + 8] = any_wide ? 1 : 0;
+    rec[BN + 9] = rec[BN + 10] = rec[BN + 11] = 0;
   }
 }
 
@@ -528,10 +548,11 @@ int num_sms() {
 }
 
 template <int DH>
-cudaError_t launch_tc(const AttnFwdParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_tc(const AttnFwdParams& p, int grid, cudaStream_t st, double time_div) {
   TcParams tp;
   memset(&tp, 0, sizeof(tp));
   tp.p = p;
+  tp.ln2_over_div = (float)(0.69314718055994530942 / time_div);
   const int64_t hd = (int64_t)p.num_heads * DH;
   if (!make_map(&tp.map_q, p.q, hd, p.total_rows, p.ldq) || !make_map(&tp.map_k, p.k, hd, p.total_rows, p.ldk) ||
       !make_map(&tp.map_v, p.v, hd, p.total_rows, p.ldv))
@@ -592,11 +613,20 @@ int tc_attn_grid(int max_items) {
   return max_items < 1 ? 1 : (max_items < s ? max_items : s);
 }
 
-cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStream_t st) {
+cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStream_t st, double time_div) {
   if (p.total_rows <= 0) return cudaSuccess;
-  if (dh == 128) return launch_tc<128>(p, grid, st);
-  if (dh == 64) return launch_tc<64>(p, grid, st);
+  if (dh == 128) return launch_tc<128>(p, grid, st, time_div);
+  if (dh == 64) return launch_tc<64>(p, grid, st, time_div);
   return cudaErrorInvalidValue;
+}
+
+size_t ts_tiles_capacity(int B, int T) { return (size_t)T / BN + (size_t)B + 1; }
+
+cudaError_t launch_ts_tiles(const int32_t* offs, const int64_t* ts, int B, const int32_t* tile_base, int tiles_cap,
+                            int32_t* recs, cudaStream_t st) {
+  if (tiles_cap <= 0) return cudaSuccess;
+  ts_tiles_kernel<<<tiles_cap, 128, 0, st>>>(offs, ts, B, tile_base, recs);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,

@@ -116,6 +116,9 @@ struct AttnWs {
   WorkItem* items;
   float* dq_accum;
   int capacity;
+  int32_t* tile_base;   // tensor-core path: [B+1]
+  int32_t* tile_recs;   // tensor-core path: timestamp records
+  int tiles_cap;
 };
 
 bool use_tc(const hstu_attn_desc* d) {
@@ -132,6 +135,14 @@ AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd) {
   w.capacity = (int)work_list_capacity(B, T, d->num_heads, tile);
   w.items = c.take<WorkItem>(w.capacity);
   w.dq_accum = bwd ? c.take<float>((size_t)T * d->num_heads * d->dqk) : nullptr;
+  w.tile_base = nullptr;
+  w.tile_recs = nullptr;
+  w.tiles_cap = 0;
+  if (!bwd && use_tc(d)) {
+    w.tiles_cap = (int)ts_tiles_capacity(B, T);
+    w.tile_base = c.take<int32_t>((size_t)B + 1);
+    w.tile_recs = c.take<int32_t>((size_t)w.tiles_cap * kTsRecWords);
+  }
   return w;
 }
 
@@ -142,7 +153,11 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   {
     TraceScope tr("sched_fwd", st);
     HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, d->num_heads,
-                                     tile, tile, 0, w.capacity, w.items, w.count, w.status, st));
+                                     tile, tile, 0, w.capacity, w.items, w.count, w.status, st, w.tile_base));
+  }
+  if (w.tile_recs) {
+    TraceScope tr("ts_tiles", st);
+    HSTU_CUDA(launch_ts_tiles(jb->seq_offsets, jb->timestamps, jb->batch, w.tile_base, w.tiles_cap, w.tile_recs, st));
   }
   AttnFwdParams p;
   memset(&p, 0, sizeof(p));
@@ -160,9 +175,11 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   p.item_count = w.count;
   p.status = w.status;
   p.timeout_ns = kDefaultTimeoutNs;
+  p.tile_base = w.tile_base;
+  p.tile_recs = w.tile_recs;
   if (use_tc(d)) {
     TraceScope tr("attn_fwd_tc", st);
-    HSTU_CUDA(launch_attn_fwd_tc(p, d->dqk, tc_attn_grid(w.capacity), st));
+    HSTU_CUDA(launch_attn_fwd_tc(p, d->dqk, tc_attn_grid(w.capacity), st, d->time_div));
   } else {
     TraceScope tr("attn_fwd_simt", st);
     int grid = w.capacity < 148 * 4 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 4;

@@ -7,9 +7,20 @@ namespace hstu {
 
 // ---------------------------------------------------------------- scheduler
 size_t work_list_capacity(int B, int T, int H, int tile);
+// Also writes tile_base[s] = index of sequence s's first kv tile of width tk in a
+// tiled per-tile array (tile_base[B] = total tiles) when tile_base is not null.
 cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targets, int B, int T, int H,
                                    int tm, int tk, int mode, int max_items, WorkItem* items,
-                                   int32_t* count, int32_t* status, cudaStream_t stream);
+                                   int32_t* count, int32_t* status, cudaStream_t stream,
+                                   int32_t* tile_base = nullptr);
+
+// Per kv tile of 128 columns: timestamps as int32 offsets from the sequence's
+// first timestamp, with per-32-column min/max and a flag when any offset
+// leaves +-2^30 (record of kTsRecWords int32, 16-byte multiple).
+constexpr int kTsRecWords = 140;   // rel[128] | min[4] | max[4] | wide | pad[3]
+size_t ts_tiles_capacity(int B, int T);
+cudaError_t launch_ts_tiles(const int32_t* offs, const int64_t* ts, int B, const int32_t* tile_base, int tiles_cap,
+                            int32_t* recs, cudaStream_t st);
 
 // ---------------------------------------------------------------- attention
 // time-bucket thresholds, passed by value (kernel parameter space)
@@ -33,6 +44,8 @@ struct AttnFwdParams {
   const int32_t* item_count;
   int32_t* status;
   long long timeout_ns;        // bound of every device-side wait
+  const int32_t* tile_base;    // tensor-core path: first tile record of each sequence
+  const int32_t* tile_recs;    // tensor-core path: timestamp tile records
 };
 
 struct AttnBwdParams {
@@ -69,7 +82,7 @@ cudaError_t launch_dq_finalize(const float* acc, const int32_t* offs, int B, int
 // tcgen05 (sm_100a) attention forward, bf16 in/out, dh in {64, 128}
 int tc_tile_m();
 bool tc_attn_supported(int dtype, int dh);
-cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStream_t st);
+cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStream_t st, double time_div);
 int tc_attn_grid(int max_items);
 
 cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,

@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(kSchedThreads)
 build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restrict__ num_targets,
                        int B, int T, int H, int tm, int tk, int mode, int max_items,
                        WorkItem* __restrict__ items, int32_t* __restrict__ count,
-                       int32_t* __restrict__ status) {
+                       int32_t* __restrict__ status, int32_t* __restrict__ tile_base) {
   using Scan = cub::BlockScan<int, kSchedThreads>;
   __shared__ typename Scan::TempStorage scan_tmp;
   __shared__ int hist_bins[kCostBins];
@@ -48,8 +48,30 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
   }
   __syncthreads();
   if (bad) {
-    if (tid == 0) { *count = 0; set_status(status, HSTU_ERR_BAD_OFFSETS); }
+    if (tid == 0) {
+      *count = 0;
+      set_status(status, HSTU_ERR_BAD_OFFSETS);
+      if (tile_base) tile_base[B] = 0;
+    }
     return;
+  }
+  // first kv tile (of width tk) of every sequence in a tiled per-tile array
+  if (tile_base) {
+    __shared__ int carry;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < B; base += kSchedThreads) {
+      const int s = base + tid;
+      const int v = s < B ? (offs[s + 1] - offs[s] + tk - 1) / tk : 0;
+      int ex, tot;
+      Scan(scan_tmp).ExclusiveSum(v, ex, tot);
+      if (s < B) tile_base[s] = carry + ex;
+      __syncthreads();
+      if (tid == 0) carry += tot;
+      __syncthreads();
+    }
+    if (tid == 0) tile_base[B] = carry;
+    __syncthreads();
   }
   // pass 1: histogram of costs
   for (int s = tid; s < B; s += kSchedThreads) {
@@ -107,9 +129,9 @@ size_t work_list_capacity(int B, int T, int H, int tile) {
 
 cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targets, int B, int T, int H,
                                    int tm, int tk, int mode, int max_items, WorkItem* items,
-                                   int32_t* count, int32_t* status, cudaStream_t stream) {
+                                   int32_t* count, int32_t* status, cudaStream_t stream, int32_t* tile_base) {
   build_work_list_kernel<<<1, kSchedThreads, 0, stream>>>(offs, num_targets, B, T, H, tm, tk, mode,
-                                                          max_items, items, count, status);
+                                                          max_items, items, count, status, tile_base);
   return cudaGetLastError();
 }
 

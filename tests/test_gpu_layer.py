@@ -252,12 +252,14 @@ def _check_train(run, wl, chained_rel_bound):
 def test_training_step_config4_scaled():
     """8-layer bf16 stack (fp32 residual stream) forward + backward with
     Stochastic Length: dU, dV, dQ, dK, the rab gradients and the weight
-    gradients of every layer vs the oracle.  The chained bound 1.5e-2 comes from
-    an fp64 simulation in which only the bf16 rounding of the tensor-core
-    operands (xhat, U/V/Q/K, A V, gate) is applied: that alone moves layer 7's
-    gradients by up to 9.1e-3 from the exact stack."""
+    gradients of every layer vs the oracle.  The chained bound 2e-2 comes from
+    an fp64 simulation of this workload in which only the bf16 rounding of the
+    forward's tensor-core operands (xhat, U/V/Q/K, A V, gate) is applied: that
+    alone moves the chained gradients by up to 1.12e-2 (time-bias gradient) and
+    9.5e-3 (dK) from the exact stack; the backward's own bf16 operands add about
+    3e-3 (a single-layer simulation)."""
     wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
-    _check_train(_train_step(wl, residual_fp32=True), wl, chained_rel_bound=1.5e-2)
+    _check_train(_train_step(wl, residual_fp32=True), wl, chained_rel_bound=2e-2)
 
 
 def test_training_step_bf16_residual_two_layers():

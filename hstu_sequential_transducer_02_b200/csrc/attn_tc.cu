@@ -31,14 +31,16 @@ using namespace sm100;
 constexpr int BM = 128;                    // q rows per tile (UMMA M)
 constexpr int BN = 128;                    // kv columns per tile
 constexpr int kEpiWarps = 16;              // four warps per TMEM lane quarter, one per 32-column segment
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiWarp0 = 3;               // warps 0: K loads, 1: MMA, 2: V loads, 3..18: epilogue
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kBoxBytes = 128 * 128;       // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
 constexpr int kRecBytes = kTsRecWords * 4;
 
 template <int DH>
 struct Cfg {
-  static constexpr int kStages = DH == 128 ? 2 : 3;
+  static constexpr int kKStages = DH == 128 ? 3 : 4;
+  static constexpr int kVStages = DH == 128 ? 2 : 4;
   static constexpr int kBoxes = DH / 64;
   static constexpr int kTileBytes = BM * DH * 2;
 };
@@ -55,9 +57,9 @@ static_assert(sizeof(TsRec) == kRecBytes, "record layout");
 
 struct Barriers {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[3], kv_empty[3];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, p_empty;
+  uint64_t k_full[4], k_empty[4];
+  uint64_t v_full[4], v_empty[4];
+  uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_empty;
   uint64_t done;
 };
@@ -74,10 +76,9 @@ template <int DH>
 struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + Cfg<DH>::kTileBytes;
-  static constexpr int kV = kK + Cfg<DH>::kStages * Cfg<DH>::kTileBytes;
-  static constexpr int kP = kV + Cfg<DH>::kStages * Cfg<DH>::kTileBytes;
-  static constexpr int kTs = kP + BM * BN * 2;
-  static constexpr int kThr = kTs + Cfg<DH>::kStages * kRecBytes;
+  static constexpr int kV = kK + Cfg<DH>::kKStages * Cfg<DH>::kTileBytes;
+  static constexpr int kTs = kV + Cfg<DH>::kVStages * Cfg<DH>::kTileBytes;
+  static constexpr int kThr = kTs + Cfg<DH>::kVStages * kRecBytes;
   static constexpr int kThr32 = kThr + kNumBuckets * 8;
   static constexpr int kPosB = kThr32 + (kNumBuckets + 4) * 4;
   static constexpr int kTimeB = kPosB + kNumBuckets * 4;
@@ -95,11 +96,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 __device__ __forceinline__ int snake_item(int k, int b, int G) {
   const int pos = (k & 1) ? (G - 1 - b) : b;
   return k * G + pos;
-}
-
-__device__ __forceinline__ float silu_tanh(float s) {
-  const float h = 0.5f * s;
-  return fmaf(h, tanh_approx(h), h);
 }
 
 // Exact time bucket of 0 <= d < 2^31 in O(1): an approximate ln(d)/div rounded
@@ -123,7 +119,8 @@ template <int DH>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_constant__ TcParams prm) {
   using C = Cfg<DH>;
   using L = Layout<DH>;
-  constexpr int S = C::kStages;
+  constexpr int SK = C::kKStages;
+  constexpr int SV = C::kVStages;
   constexpr int DV = DH;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -138,7 +135,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sK = smem_u32(smem + L::kK);
   const uint32_t sV = smem_u32(smem + L::kV);
-  const uint32_t sP = smem_u32(smem + L::kP);
 
   const AttnFwdParams& p = prm.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -148,10 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < S; ++s) { mbar_init(&bars->kv_full[s], 1); mbar_init(&bars->kv_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&bars->s_full[s], 1); mbar_init(&bars->s_empty[s], kEpiWarps); }
-    mbar_init(&bars->p_full, kEpiWarps);
-    mbar_init(&bars->p_empty, 1);
+    for (int s = 0; s < SK; ++s) { mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1); }
+    for (int s = 0; s < SV; ++s) { mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars->s_full[s], 1); mbar_init(&bars->p_full[s], kEpiWarps); }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, kEpiWarps);
     mbar_init(&bars->done, 1);
@@ -181,17 +176,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_s0 = tmem_base;          // S buffers at columns 0 and 128
+  const uint32_t tmem_s0 = tmem_base;          // S / P buffers at columns 0 and 128
   const uint32_t tmem_o = tmem_base + 2 * BN;  // O accumulator at column 256
 
   const int count = *p.item_count;
   const int G = gridDim.x;
   const int per_head_rab = p.rab_head_stride != 0;
 
-  if (warp == 0) {
-    // =================================================================== producer
+  if (warp == 0 || warp == 2) {
+    // =================================================================== producers (0: Q and K, 2: V and records)
     if (lane == 0) {
-      int kv_it = 0;
+      const bool kside = warp == 0;
+      int it = 0;
       for (int k = 0;; ++k) {
         const int idx = snake_item(k, blockIdx.x, G);
         if (idx >= count || *abort_flag) break;
@@ -199,24 +195,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
         const int r0 = wi.qtile * BM;
         const int r1 = min(si.n, r0 + BM);
+        if (kside) {
+          if (!mbar_wait(&bars->q_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
+          mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
+          for (int b = 0; b < C::kBoxes; ++b)
+            tma_load_2d(smem + L::kQ + b * kBoxBytes, &prm.map_q, &bars->q_full, wi.head * DH + 64 * b,
+                        si.start + r0);
+        }
         const TsRec* grec = reinterpret_cast<const TsRec*>(p.tile_recs) + p.tile_base[wi.seq];
-        if (!mbar_wait(&bars->q_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
-        mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
-        for (int b = 0; b < C::kBoxes; ++b)
-          tma_load_2d(smem + L::kQ + b * kBoxBytes, &prm.map_q, &bars->q_full, wi.head * DH + 64 * b, si.start + r0);
         const KvRange kr = kv_tiles_for(r0, r1, si.hist, BN);
         const int nk = kv_count(kr);
-        for (int jj = 0; jj < nk; ++jj, ++kv_it) {
+        for (int jj = 0; jj < nk; ++jj, ++it) {
           const int kt = kv_tile_at(kr, jj);
-          const int st = kv_it % S;
-          if (!mbar_wait(&bars->kv_empty[st], ((kv_it / S) & 1) ^ 1, tmo, abort_flag)) goto fail;
-          mbar_arrive_expect_tx(&bars->kv_full[st], 2 * C::kTileBytes + kRecBytes);
-          bulk_load(&recs[st], grec + kt, kRecBytes, &bars->kv_full[st]);
-          for (int b = 0; b < C::kBoxes; ++b) {
-            tma_load_2d(smem + L::kK + st * C::kTileBytes + b * kBoxBytes, &prm.map_k, &bars->kv_full[st],
-                        wi.head * DH + 64 * b, si.start + kt * BN);
-            tma_load_2d(smem + L::kV + st * C::kTileBytes + b * kBoxBytes, &prm.map_v, &bars->kv_full[st],
-                        wi.head * DV + 64 * b, si.start + kt * BN);
+          if (kside) {
+            const int st = it % SK;
+            if (!mbar_wait(&bars->k_empty[st], ((it / SK) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            mbar_arrive_expect_tx(&bars->k_full[st], C::kTileBytes);
+            for (int b = 0; b < C::kBoxes; ++b)
+              tma_load_2d(smem + L::kK + st * C::kTileBytes + b * kBoxBytes, &prm.map_k, &bars->k_full[st],
+                          wi.head * DH + 64 * b, si.start + kt * BN);
+          } else {
+            const int st = it % SV;
+            if (!mbar_wait(&bars->v_empty[st], ((it / SV) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            mbar_arrive_expect_tx(&bars->v_full[st], C::kTileBytes + kRecBytes);
+            bulk_load(&recs[st], grec + kt, kRecBytes, &bars->v_full[st]);
+            for (int b = 0; b < C::kBoxes; ++b)
+              tma_load_2d(smem + L::kV + st * C::kTileBytes + b * kBoxBytes, &prm.map_v, &bars->v_full[st],
+                          wi.head * DV + 64 * b, si.start + kt * BN);
           }
         }
       }
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = make_idesc_bf16(BM, DV, false, true);
-      int kv_it = 0, s_it = 0, p_it = 0;
+      int s_it = 0, p_it = 0;  // global kv-tile counters: S computed, P V consumed
       for (int k = 0;; ++k) {
         const int idx = snake_item(k, blockIdx.x, G);
         if (idx >= count || *abort_flag) break;
@@ -236,13 +241,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
         const int nk = kv_count(kr);
         if (!mbar_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
-        int prev_stage = 0;
         for (int jj = 0; jj <= nk; ++jj) {
           if (jj < nk) {
-            const int st = kv_it % S;
+            // S = Q K^T into buffer s_it & 1 (its P was consumed by an earlier P V: in-order pipe)
+            const int st = s_it % SK;
             const int sb = s_it & 1;
-            if (!mbar_wait(&bars->kv_full[st], (kv_it / S) & 1, tmo, abort_flag)) goto fail;
-            if (!mbar_wait(&bars->s_empty[sb], ((s_it >> 1) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            if (!mbar_wait(&bars->k_full[st], (s_it / SK) & 1, tmo, abort_flag)) goto fail;
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < DH / 16; ++ks) {
@@ -252,27 +256,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
               umma_f16_ss(tmem_s0 + sb * BN, a, b, idesc_s, ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars->s_full[sb]);
+            umma_commit(&bars->k_empty[st]);
             if (jj == nk - 1) umma_commit(&bars->q_empty);
+            ++s_it;
           }
           if (jj > 0) {
-            // O (+)= P V for the previous kv tile
-            if (!mbar_wait(&bars->p_full, p_it & 1, tmo, abort_flag)) goto fail;
+            // O (+)= P V for the previous kv tile, P read from TMEM
+            const int pb = p_it & 1;
+            const int vs = p_it % SV;
+            if (!mbar_wait(&bars->p_full[pb], (p_it >> 1) & 1, tmo, abort_flag)) goto fail;
+            if (!mbar_wait(&bars->v_full[vs], (p_it / SV) & 1, tmo, abort_flag)) goto fail;
             if (jj == 1 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
             tc_fence_after();
+            const uint32_t pa = tmem_s0 + pb * BN;
 #pragma unroll
             for (int ks = 0; ks < BN / 16; ++ks) {
-              const uint64_t a = make_sw128_desc(sP + (ks >> 2) * kBoxBytes + (ks & 3) * 32, 16, 1024);
-              const uint64_t b = make_sw128_desc(sV + prev_stage * C::kTileBytes + ks * 16 * 128, kBoxBytes, 1024);
-              umma_f16_ss(tmem_o, a, b, idesc_o, (jj > 1 || ks > 0) ? 1u : 0u);
+              // kv columns [16ks, 16ks+16) were written by segment ks/2 at columns 32*(ks/2) + 8*(ks%2)
+              const uint64_t b = make_sw128_desc(sV + vs * C::kTileBytes + ks * 16 * 128, kBoxBytes, 1024);
+              umma_f16_ts(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), b, idesc_o, (jj > 1 || ks > 0) ? 1u : 0u);
             }
-            umma_commit(&bars->kv_empty[prev_stage]);
-            umma_commit(&bars->p_empty);
+            umma_commit(&bars->v_empty[vs]);
             ++p_it;
-          }
-          if (jj < nk) {
-            prev_stage = kv_it % S;
-            ++kv_it;
-            ++s_it;
           }
         }
         umma_commit(&bars->o_full);
@@ -283,13 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     }
   } else {
     // =================================================================== epilogue
-    const int ew = warp - 2;               // 0..15
+    const int ew = warp - kEpiWarp0;       // 0..15
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int seg = ew >> 2;               // 32-column segment of S (and of O)
     const int r = quarter * 32 + lane;     // row of the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float k_lg = prm.ln2_over_div;
-    int s_it = 0, kv_it = 0, p_it = 0;
+    int it = 0;  // global kv-tile counter
     int cur_head = -1;
     for (int k = 0;; ++k) {
       const int idx = snake_item(k, blockIdx.x, G);
@@ -298,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
       if (per_head_rab && wi.head != cur_head) {
         named_bar_sync(1, 32 * kEpiWarps);
-        for (int c = threadIdx.x - 64; c < kNumBuckets; c += 32 * kEpiWarps) {
+        for (int c = threadIdx.x - 32 * kEpiWarp0; c < kNumBuckets; c += 32 * kEpiWarps) {
           pos_b[c] = p.pos_bias[wi.head * p.rab_head_stride + c];
           time_b[c] = p.time_bias[wi.head * p.rab_head_stride + c];
         }
@@ -317,27 +321,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       const int posi = token_pos(i, si.hist);
       const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
       const int nk = kv_count(kr);
-      for (int jj = 0; jj < nk; ++jj, ++kv_it, ++s_it, ++p_it) {
+      for (int jj = 0; jj < nk; ++jj, ++it) {
         const int c0 = kv_tile_at(kr, jj) * BN;
-        const int sb = s_it & 1;
-        const int st = kv_it % S;
-        if (!mbar_wait(&bars->s_full[sb], (s_it >> 1) & 1, tmo, abort_flag)) goto fail;
+        const int sb = it & 1;
+        const int vs = it % SV;
+        if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
-        if (!mbar_wait(&bars->kv_full[st], (kv_it / S) & 1, tmo, abort_flag)) goto fail;
-        const TsRec& rec = recs[st];
+        if (!mbar_wait(&bars->v_full[vs], (it / SV) & 1, tmo, abort_flag)) goto fail;
+        const TsRec& rec = recs[vs];
         // ---- classify this row's 32 columns
         const int cl = c0 + seg * 32;   // first column of the segment
         const bool narrow = row_narrow && !rec.wide;
         const bool any_live = live && (cand ? (cl < si.hist || (i >= cl && i < cl + 32)) : (cl <= i));
         const bool full = live && (cand ? (cl + 31 < si.hist) : (cl + 31 <= i));
-        int mode = any_live ? 3 : 0;  // 0: zero, 1: one time bucket, 2: 2-4 buckets, 3: general
-        float b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
+        int mode = any_live ? 3 : 0;  // 0: zero, 1: one time bucket, 2: two, 4: three or four, 3: general
+        float hb0 = 0.f, hb1 = 0.f, hb2 = 0.f, hb3 = 0.f;   // half of the bias values
         int32_t th1 = 0x7FFFFFFF, th2 = 0x7FFFFFFF, th3 = 0x7FFFFFFF;
         if (full && narrow && posi - (cl + 31) >= kNumBuckets - 1) {
           const int32_t mn = rec.mn[seg], mx = rec.mx[seg];
@@ -347,68 +348,86 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
           else { dlo = 0; dhi = max(ri - mn, mx - ri); }
           const int tlo = fast_bucket(dlo, thr32, k_lg), thi = fast_bucket(dhi, thr32, k_lg);
           const float pb127 = pos_b[kNumBuckets - 1];
-          b0 = pb127 + time_b[tlo];
+          hb0 = 0.5f * (pb127 + time_b[tlo]);
           if (tlo == thi) {
             mode = 1;
           } else if (thi - tlo <= 3) {
-            mode = 2;
-            b1 = pb127 + time_b[tlo + 1];
+            mode = thi - tlo == 1 ? 2 : 4;
+            hb1 = 0.5f * (pb127 + time_b[tlo + 1]);
             th1 = thr32[tlo + 1];
-            if (thi - tlo >= 2) { b2 = pb127 + time_b[tlo + 2]; th2 = thr32[tlo + 2]; }
-            if (thi - tlo >= 3) { b3 = pb127 + time_b[tlo + 3]; th3 = thr32[tlo + 3]; }
+            if (thi - tlo >= 2) { hb2 = 0.5f * (pb127 + time_b[tlo + 2]); th2 = thr32[tlo + 2]; }
+            if (thi - tlo >= 3) { hb3 = 0.5f * (pb127 + time_b[tlo + 3]); th3 = thr32[tlo + 3]; }
           }
         }
-        // ---- bias, SiLU, mask
-        float pv[32];
+        // ---- bias, SiLU (as h + h tanh h with h = (s + bias) / 2), mask; packed bf16 pairs
+        uint32_t pk[16];
         if (mode == 0) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pv[e] = 0.f;
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
         } else if (mode == 1) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pv[e] = silu_tanh(__uint_as_float(raw[e]) + b0);
+          for (int e = 0; e < 16; ++e)
+            pk[e] = silu2_bf16(fmaf(__uint_as_float(raw[2 * e]), 0.5f, hb0),
+                               fmaf(__uint_as_float(raw[2 * e + 1]), 0.5f, hb0));
         } else if (mode == 2) {
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const int4 rel4 = *reinterpret_cast<const int4*>(&rec.rel[seg * 32 + e4 * 4]);
             const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+            float h[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              h[u] = fmaf(__uint_as_float(raw[e4 * 4 + u]), 0.5f, abs(ri - rv[u]) >= th1 ? hb1 : hb0);
+            pk[2 * e4] = silu2_bf16(h[0], h[1]);
+            pk[2 * e4 + 1] = silu2_bf16(h[2], h[3]);
+          }
+        } else if (mode == 4) {
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const int4 rel4 = *reinterpret_cast<const int4*>(&rec.rel[seg * 32 + e4 * 4]);
+            const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+            float h[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              const int e = e4 * 4 + u;
               const int32_t dd = abs(ri - rv[u]);
-              float bias = dd >= th1 ? b1 : b0;
-              bias = dd >= th2 ? b2 : bias;
-              bias = dd >= th3 ? b3 : bias;
-              pv[e] = silu_tanh(__uint_as_float(raw[e]) + bias);
+              float hb = dd >= th1 ? hb1 : hb0;
+              hb = dd >= th2 ? hb2 : hb;
+              hb = dd >= th3 ? hb3 : hb;
+              h[u] = fmaf(__uint_as_float(raw[e4 * 4 + u]), 0.5f, hb);
             }
+            pk[2 * e4] = silu2_bf16(h[0], h[1]);
+            pk[2 * e4 + 1] = silu2_bf16(h[2], h[3]);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int j = cl + e;
-            float v = 0.f;
-            if (attended(i, j, si.n, si.hist)) {
-              const int pb = pos_bucket(posi, token_pos(j, si.hist));
-              int tb;
-              if (narrow) tb = fast_bucket(abs(ri - rec.rel[seg * 32 + e]), thr32, k_lg);
-              else tb = time_bucket_exact(abs_diff_i64(ti, p.timestamps[si.start + j]), thr);
-              v = silu_tanh(__uint_as_float(raw[e]) + pos_b[pb] + time_b[tb]);
+          for (int e2 = 0; e2 < 16; ++e2) {
+            float h[2];
+            bool att[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int e = 2 * e2 + u;
+              const int j = cl + e;
+              att[u] = attended(i, j, si.n, si.hist);
+              float bias = 0.f;
+              if (att[u]) {
+                const int pb = pos_bucket(posi, token_pos(j, si.hist));
+                int tb;
+                if (narrow) tb = fast_bucket(abs(ri - rec.rel[seg * 32 + e]), thr32, k_lg);
+                else tb = time_bucket_exact(abs_diff_i64(ti, p.timestamps[si.start + j]), thr);
+                bias = pos_b[pb] + time_b[tb];
+              }
+              h[u] = 0.5f * (__uint_as_float(raw[e]) + bias);
             }
-            pv[e] = v;
+            const uint32_t v = silu2_bf16(h[0], h[1]);
+            pk[e2] = (att[0] ? (v & 0xFFFFu) : 0u) | (att[1] ? (v & 0xFFFF0000u) : 0u);
           }
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
-        // ---- P -> shared memory (A operand, K-major, 128-byte swizzle)
-        if (!mbar_wait(&bars->p_empty, (p_it & 1) ^ 1, tmo, abort_flag)) goto fail;
-        const uint32_t prow = sP + (seg >> 1) * kBoxBytes + r * 128;
-        const int cbase = (seg & 1) * 4;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          st_shared_v4(prow + (((cbase + c) ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
+        // ---- P -> TMEM, over this segment's own S columns (the A operand of P V)
+        tmem_st_32x32b_x16(tmem_s0 + sb * BN + lane_off + seg * 32, pk);
+        tmem_st_wait();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full);
+        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
       }
       // ---- O readout: this warp's DV/4 columns
       if (!mbar_wait(&bars->o_full, k & 1, tmo, abort_flag)) goto fail;
@@ -443,14 +462,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
 fail:
   set_status(p.status, HSTU_ERR_TIMEOUT);
   *abort_flag = 1;
-  if (warp == 0 && lane == 0) {
+  if ((warp == 0 || warp == 2) && lane == 0) {
     // let every copy this CTA may have issued land before it exits (bounded)
-    for (int s = 0; s < S; ++s) {
-      mbar_wait(&bars->kv_full[s], 0, 100000000ll, nullptr);
-      mbar_wait(&bars->kv_full[s], 1, 100000000ll, nullptr);
+    for (int s = 0; s < 4; ++s) {
+      if (warp == 0 && s < SK) {
+        mbar_wait(&bars->k_full[s], 0, 100000000ll, nullptr);
+        mbar_wait(&bars->k_full[s], 1, 100000000ll, nullptr);
+      }
+      if (warp == 2 && s < SV) {
+        mbar_wait(&bars->v_full[s], 0, 100000000ll, nullptr);
+        mbar_wait(&bars->v_full[s], 1, 100000000ll, nullptr);
+      }
     }
-    mbar_wait(&bars->q_full, 0, 100000000ll, nullptr);
-    mbar_wait(&bars->q_full, 1, 100000000ll, nullptr);
+    if (warp == 0) {
+      mbar_wait(&bars->q_full, 0, 100000000ll, nullptr);
+      mbar_wait(&bars->q_full, 1, 100000000ll, nullptr);
+    }
   }
 teardown:
   tc_fence_before();

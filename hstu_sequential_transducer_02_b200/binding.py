@@ -114,9 +114,14 @@ EXPORTED = ["hstu_status_string", "hstu_version", "hstu_build_time_thresholds", 
             "hstu_stochastic_length", "hstu_gather_rows", "hstu_debug_rab_buckets", "hstu_debug_timeout_probe"]
 
 
+_lib_last_cuda_error = _sig("hstu_last_cuda_error", ctypes.c_char_p, [])
+EXPORTED.append("hstu_last_cuda_error")
+
+
 class HstuError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {status_string(code)} ({code})")
+        detail = f" [{_lib_last_cuda_error().decode()}]" if code == ERR_CUDA else ""
+        super().__init__(f"{where}: {status_string(code)} ({code}){detail}")
         self.code = code
 
 

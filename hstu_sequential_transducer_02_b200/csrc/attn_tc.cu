@@ -5,8 +5,9 @@
 // ("Actions Speak Louder than Words" summary, 1.2; "生成式推荐（一）：HSTU",
 // pointwise aggregated attention: no normalisation over the sequence.)
 //
-// One persistent CTA per SM walks the cost-sorted (sequence, head, q tile)
-// work list in snake order.  Per q tile of 128 rows and each kv tile of 128
+// One persistent CTA per SM takes (sequence, head, q tile) work items from a
+// shared cursor over a list in locality order (long sequences first, then head,
+// then q tile), so the CTAs running at the same time share K/V tiles in L2.  Per q tile of 128 rows and each kv tile of 128
 // columns that holds an attended pair:
 //   warp 0      TMA: Q once per item, K/V per kv tile into a ring of stages,
 //               plus the tile's timestamps (and their per-half min/max)
@@ -39,8 +40,8 @@ constexpr int kRecBytes = kTsRecWords * 4;
 
 template <int DH>
 struct Cfg {
-  static constexpr int kKStages = DH == 128 ? 3 : 4;
-  static constexpr int kVStages = DH == 128 ? 2 : 4;
+  static constexpr int kKStages = DH == 128 ? 2 : 4;
+  static constexpr int kVStages = DH == 128 ? 3 : 4;
   static constexpr int kBoxes = DH / 64;
   static constexpr int kTileBytes = BM * DH * 2;
 };
@@ -55,11 +56,19 @@ struct TsRec {
 };
 static_assert(sizeof(TsRec) == kRecBytes, "record layout");
 
+constexpr int kRecStages = 8;              // timestamp records run up to 8 kv tiles ahead
+constexpr int kSBufs = 3;                  // S/P buffers in TMEM: S runs two kv tiles ahead of P V
+
+constexpr int kItemSlots = 4;              // work items fetched ahead by the Q/K producer
+constexpr int kItemReaders = 2 + kEpiWarps;  // V producer, MMA issuer, epilogue warps
+
 struct Barriers {
+  uint64_t it_full[kItemSlots], it_empty[kItemSlots];
   uint64_t q_full, q_empty;
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
-  uint64_t s_full[2], p_full[2];
+  uint64_t r_full[kRecStages], r_empty[kRecStages];
+  uint64_t s_full[3], p_full[3];
   uint64_t o_full, o_empty;
   uint64_t done;
 };
@@ -78,24 +87,19 @@ struct Layout {
   static constexpr int kK = kQ + Cfg<DH>::kTileBytes;
   static constexpr int kV = kK + Cfg<DH>::kKStages * Cfg<DH>::kTileBytes;
   static constexpr int kTs = kV + Cfg<DH>::kVStages * Cfg<DH>::kTileBytes;
-  static constexpr int kThr = kTs + Cfg<DH>::kVStages * kRecBytes;
+  static constexpr int kThr = kTs + kRecStages * kRecBytes;
   static constexpr int kThr32 = kThr + kNumBuckets * 8;
   static constexpr int kPosB = kThr32 + (kNumBuckets + 4) * 4;
   static constexpr int kTimeB = kPosB + kNumBuckets * 4;
   static constexpr int kBar = (kTimeB + kNumBuckets * 4 + 15) & ~15;
   static constexpr int kMisc = kBar + (int)sizeof(Barriers);
-  static constexpr int kEnd = kMisc + 16;
+  static constexpr int kItems = kMisc + 16;
+  static constexpr int kEnd = kItems + 16;
   static constexpr int kAlloc = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// snake order over the cost-sorted list: wave w visits CTAs forward when w is even
-__device__ __forceinline__ int snake_item(int k, int b, int G) {
-  const int pos = (k & 1) ? (G - 1 - b) : b;
-  return k * G + pos;
 }
 
 // Exact time bucket of 0 <= d < 2^31 in O(1): an approximate ln(d)/div rounded
@@ -114,6 +118,19 @@ __device__ __forceinline__ int fast_bucket(int32_t d, const int32_t* thr32, floa
   return b > kNumBuckets - 1 ? kNumBuckets - 1 : b;
 }
 
+// Waits for outstanding tcgen05.ld into `r`; the register operands keep the
+// compiler from reading them earlier.
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_constant__ TcParams prm) {
@@ -127,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   Barriers* bars = reinterpret_cast<Barriers*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::kItems);
   int64_t* thr = reinterpret_cast<int64_t*>(smem + L::kThr);
   int32_t* thr32 = reinterpret_cast<int32_t*>(smem + L::kThr32);
   float* pos_b = reinterpret_cast<float*>(smem + L::kPosB);
@@ -142,11 +160,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
 
   // ---- set-up
   if (threadIdx.x == 0) {
+    for (int s = 0; s < kItemSlots; ++s) { mbar_init(&bars->it_full[s], 1); mbar_init(&bars->it_empty[s], kItemReaders); }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < SK; ++s) { mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1); }
     for (int s = 0; s < SV; ++s) { mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&bars->s_full[s], 1); mbar_init(&bars->p_full[s], kEpiWarps); }
+    for (int s = 0; s < kRecStages; ++s) { mbar_init(&bars->r_full[s], 1); mbar_init(&bars->r_empty[s], kEpiWarps); }
+    for (int s = 0; s < kSBufs; ++s) { mbar_init(&bars->s_full[s], 1); mbar_init(&bars->p_full[s], kEpiWarps); }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, kEpiWarps);
     mbar_init(&bars->done, 1);
@@ -176,21 +196,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t tmem_s0 = tmem_base;          // S / P buffers at columns 0 and 128
-  const uint32_t tmem_o = tmem_base + 2 * BN;  // O accumulator at column 256
+  const uint32_t tmem_s0 = tmem_base;               // S / P buffers at columns 0, 128, 256
+  const uint32_t tmem_o = tmem_base + kSBufs * BN;  // O accumulator at column 384
 
   const int count = *p.item_count;
-  const int G = gridDim.x;
   const int per_head_rab = p.rab_head_stride != 0;
 
   if (warp == 0 || warp == 2) {
-    // =================================================================== producers (0: Q and K, 2: V and records)
+    // =================================================================== producers (0: Q, K and records, 2: V)
     if (lane == 0) {
       const bool kside = warp == 0;
       int it = 0;
       for (int k = 0;; ++k) {
-        const int idx = snake_item(k, blockIdx.x, G);
-        if (idx >= count || *abort_flag) break;
+        // the Q/K producer fetches the next work item; everyone else reads it from the ring
+        const int slot = k % kItemSlots;
+        int idx;
+        if (kside) {
+          if (!mbar_wait(&bars->it_empty[slot], ((k / kItemSlots) & 1) ^ 1, tmo, abort_flag)) goto fail;
+          idx = *abort_flag ? -1 : atomicAdd(p.item_cursor, 1);
+          if (idx >= count) idx = -1;
+          item_ring[slot] = idx;
+          mbar_arrive(&bars->it_full[slot]);
+        } else {
+          if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
+          idx = item_ring[slot];
+          mbar_arrive(&bars->it_empty[slot]);
+        }
+        if (idx < 0) break;
         const WorkItem wi = p.items[idx];
         const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
         const int r0 = wi.qtile * BM;
@@ -208,6 +240,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         for (int jj = 0; jj < nk; ++jj, ++it) {
           const int kt = kv_tile_at(kr, jj);
           if (kside) {
+            const int rs = it % kRecStages;
+            if (!mbar_wait(&bars->r_empty[rs], ((it / kRecStages) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            mbar_arrive_expect_tx(&bars->r_full[rs], kRecBytes);
+            bulk_load(&recs[rs], grec + kt, kRecBytes, &bars->r_full[rs]);
             const int st = it % SK;
             if (!mbar_wait(&bars->k_empty[st], ((it / SK) & 1) ^ 1, tmo, abort_flag)) goto fail;
             mbar_arrive_expect_tx(&bars->k_full[st], C::kTileBytes);
@@ -217,8 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
           } else {
             const int st = it % SV;
             if (!mbar_wait(&bars->v_empty[st], ((it / SV) & 1) ^ 1, tmo, abort_flag)) goto fail;
-            mbar_arrive_expect_tx(&bars->v_full[st], C::kTileBytes + kRecBytes);
-            bulk_load(&recs[st], grec + kt, kRecBytes, &bars->v_full[st]);
+            mbar_arrive_expect_tx(&bars->v_full[st], C::kTileBytes);
             for (int b = 0; b < C::kBoxes; ++b)
               tma_load_2d(smem + L::kV + st * C::kTileBytes + b * kBoxBytes, &prm.map_v, &bars->v_full[st],
                           wi.head * DV + 64 * b, si.start + kt * BN);
@@ -233,51 +268,59 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       constexpr uint32_t idesc_o = make_idesc_bf16(BM, DV, false, true);
       int s_it = 0, p_it = 0;  // global kv-tile counters: S computed, P V consumed
       for (int k = 0;; ++k) {
-        const int idx = snake_item(k, blockIdx.x, G);
-        if (idx >= count || *abort_flag) break;
+        const int slot = k % kItemSlots;
+        if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
+        const int idx = item_ring[slot];
+        mbar_arrive(&bars->it_empty[slot]);
+        if (idx < 0) break;
         const WorkItem wi = p.items[idx];
         const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
         const int r0 = wi.qtile * BM;
         const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
         const int nk = kv_count(kr);
         if (!mbar_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
-        for (int jj = 0; jj <= nk; ++jj) {
-          if (jj < nk) {
-            // S = Q K^T into buffer s_it & 1 (its P was consumed by an earlier P V: in-order pipe)
-            const int st = s_it % SK;
-            const int sb = s_it & 1;
-            if (!mbar_wait(&bars->k_full[st], (s_it / SK) & 1, tmo, abort_flag)) goto fail;
-            tc_fence_after();
+        // S = Q K^T for the item's kv tile s_loc into buffer s_it % kSBufs; the buffer's
+        // previous P was consumed by a P V issued earlier (the tensor pipe runs in order)
+        int s_loc = 0;
+        auto issue_s = [&]() -> bool {
+          const int st = s_it % SK;
+          const int sb = s_it % kSBufs;
+          if (!mbar_wait(&bars->k_full[st], (s_it / SK) & 1, tmo, abort_flag)) return false;
+          tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < DH / 16; ++ks) {
-              const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
-              const uint64_t a = make_sw128_desc(sQ + off, 16, 1024);
-              const uint64_t b = make_sw128_desc(sK + st * C::kTileBytes + off, 16, 1024);
-              umma_f16_ss(tmem_s0 + sb * BN, a, b, idesc_s, ks > 0 ? 1u : 0u);
-            }
-            umma_commit(&bars->s_full[sb]);
-            umma_commit(&bars->k_empty[st]);
-            if (jj == nk - 1) umma_commit(&bars->q_empty);
-            ++s_it;
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
+            const uint64_t a = make_sw128_desc(sQ + off, 16, 1024);
+            const uint64_t b = make_sw128_desc(sK + st * C::kTileBytes + off, 16, 1024);
+            umma_f16_ss(tmem_s0 + sb * BN, a, b, idesc_s, ks > 0 ? 1u : 0u);
           }
-          if (jj > 0) {
-            // O (+)= P V for the previous kv tile, P read from TMEM
-            const int pb = p_it & 1;
-            const int vs = p_it % SV;
-            if (!mbar_wait(&bars->p_full[pb], (p_it >> 1) & 1, tmo, abort_flag)) goto fail;
-            if (!mbar_wait(&bars->v_full[vs], (p_it / SV) & 1, tmo, abort_flag)) goto fail;
-            if (jj == 1 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
-            tc_fence_after();
-            const uint32_t pa = tmem_s0 + pb * BN;
+          umma_commit(&bars->s_full[sb]);
+          umma_commit(&bars->k_empty[st]);
+          if (s_loc == nk - 1) umma_commit(&bars->q_empty);
+          ++s_it;
+          ++s_loc;
+          return true;
+        };
+        while (s_loc < nk && s_loc < kSBufs - 1)
+          if (!issue_s()) goto fail;
+        for (int jj = 0; jj < nk; ++jj) {
+          // O (+)= P V for kv tile jj, P read from TMEM
+          const int pb = p_it % kSBufs;
+          const int vs = p_it % SV;
+          if (!mbar_wait(&bars->p_full[pb], (p_it / kSBufs) & 1, tmo, abort_flag)) goto fail;
+          if (!mbar_wait(&bars->v_full[vs], (p_it / SV) & 1, tmo, abort_flag)) goto fail;
+          if (jj == 0 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
+          tc_fence_after();
+          const uint32_t pa = tmem_s0 + pb * BN;
 #pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks) {
-              // kv columns [16ks, 16ks+16) were written by segment ks/2 at columns 32*(ks/2) + 8*(ks%2)
-              const uint64_t b = make_sw128_desc(sV + vs * C::kTileBytes + ks * 16 * 128, kBoxBytes, 1024);
-              umma_f16_ts(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), b, idesc_o, (jj > 1 || ks > 0) ? 1u : 0u);
-            }
-            umma_commit(&bars->v_empty[vs]);
-            ++p_it;
+          for (int ks = 0; ks < BN / 16; ++ks) {
+            // kv columns [16ks, 16ks+16) were written by segment ks/2 at columns 32*(ks/2) + 8*(ks%2)
+            const uint64_t b = make_sw128_desc(sV + vs * C::kTileBytes + ks * 16 * 128, kBoxBytes, 1024);
+            umma_f16_ts(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), b, idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
           }
+          umma_commit(&bars->v_empty[vs]);
+          ++p_it;
+          if (s_loc < nk && !issue_s()) goto fail;
         }
         umma_commit(&bars->o_full);
       }
@@ -296,8 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     int it = 0;  // global kv-tile counter
     int cur_head = -1;
     for (int k = 0;; ++k) {
-      const int idx = snake_item(k, blockIdx.x, G);
-      if (idx >= count || *abort_flag) break;
+      const int slot = k % kItemSlots;
+      if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
+      const int idx = item_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->it_empty[slot]);
+      if (idx < 0) break;
       const WorkItem wi = p.items[idx];
       const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
       if (per_head_rab && wi.head != cur_head) {
@@ -323,15 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       const int nk = kv_count(kr);
       for (int jj = 0; jj < nk; ++jj, ++it) {
         const int c0 = kv_tile_at(kr, jj) * BN;
-        const int sb = it & 1;
-        const int vs = it % SV;
-        if (!mbar_wait(&bars->s_full[sb], (it >> 1) & 1, tmo, abort_flag)) goto fail;
+        const int sb = it % kSBufs;
+        const int rs = it % kRecStages;
+        if (!mbar_wait(&bars->r_full[rs], (it / kRecStages) & 1, tmo, abort_flag)) goto fail;
+        const TsRec& rec = recs[rs];
+        if (!mbar_wait(&bars->s_full[sb], (it / kSBufs) & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
         uint32_t raw[32];
-        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
-        tmem_ld_wait();
-        if (!mbar_wait(&bars->v_full[vs], (it / SV) & 1, tmo, abort_flag)) goto fail;
-        const TsRec& rec = recs[vs];
+        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);  // waited for after the classification
         // ---- classify this row's 32 columns
         const int cl = c0 + seg * 32;   // first column of the segment
         const bool narrow = row_narrow && !rec.wide;
@@ -359,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
             if (thi - tlo >= 3) { hb3 = 0.5f * (pb127 + time_b[tlo + 3]); th3 = thr32[tlo + 3]; }
           }
         }
+        tmem_ld_wait_regs(raw);
         // ---- bias, SiLU (as h + h tanh h with h = (s + bias) / 2), mask; packed bf16 pairs
         uint32_t pk[16];
         if (mode == 0) {
@@ -427,7 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
+        if (lane == 0) {
+          mbar_arrive(&bars->p_full[sb]);
+          mbar_arrive(&bars->r_empty[rs]);
+        }
       }
       // ---- O readout: this warp's DV/4 columns
       if (!mbar_wait(&bars->o_full, k & 1, tmo, abort_flag)) goto fail;
@@ -468,6 +518,12 @@ fail:
       if (warp == 0 && s < SK) {
         mbar_wait(&bars->k_full[s], 0, 100000000ll, nullptr);
         mbar_wait(&bars->k_full[s], 1, 100000000ll, nullptr);
+      }
+      if (warp == 0) {
+        for (int rr = s; rr < kRecStages; rr += 4) {
+          mbar_wait(&bars->r_full[rr], 0, 100000000ll, nullptr);
+          mbar_wait(&bars->r_full[rr], 1, 100000000ll, nullptr);
+        }
       }
       if (warp == 2 && s < SV) {
         mbar_wait(&bars->v_full[s], 0, 100000000ll, nullptr);

@@ -3,6 +3,7 @@
 // library's own kernels; nothing here computes on the host except the
 // time-bucket threshold table.
 #include <math.h>
+#include <stdio.h>
 #include <mutex>
 #include <string.h>
 
@@ -43,10 +44,17 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CU
     int _s = (expr);                        \
     if (_s != HSTU_OK) return _s;           \
   } while (0)
-#define HSTU_CUDA(expr)                     \
-  do {                                      \
-    cudaError_t _e = (expr);                \
-    if (_e != cudaSuccess) return HSTU_ERR_CUDA; \
+thread_local char g_last_error[256] = "no error";
+
+int record_cuda_error(cudaError_t e, const char* what) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+  return HSTU_ERR_CUDA;
+}
+
+#define HSTU_CUDA(expr)                                         \
+  do {                                                          \
+    cudaError_t _e = (expr);                                    \
+    if (_e != cudaSuccess) return record_cuda_error(_e, #expr); \
   } while (0)
 
 // ---------------------------------------------------------------- thresholds
@@ -151,9 +159,11 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
                  int64_t ldo, const AttnWs& w, cudaStream_t st) {
   const int tile = attn_tile(d);
   {
+    // tensor-core path: locality order, fetched dynamically (count[1] is the cursor)
     TraceScope tr("sched_fwd", st);
     HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, d->num_heads,
-                                     tile, tile, 0, w.capacity, w.items, w.count, w.status, st, w.tile_base));
+                                     tile, tile, use_tc(d) ? 3 : 0, w.capacity, w.items, w.count, w.status, st,
+                                     w.tile_base));
   }
   if (w.tile_recs) {
     TraceScope tr("ts_tiles", st);
@@ -177,6 +187,7 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   p.timeout_ns = kDefaultTimeoutNs;
   p.tile_base = w.tile_base;
   p.tile_recs = w.tile_recs;
+  p.item_cursor = w.count + 1;
   if (use_tc(d)) {
     TraceScope tr("attn_fwd_tc", st);
     HSTU_CUDA(launch_attn_fwd_tc(p, d->dqk, tc_attn_grid(w.capacity), st, d->time_div));
@@ -484,6 +495,8 @@ const char* hstu_status_string(int status) {
 }
 
 int hstu_version(void) { return kVersion; }
+
+const char* hstu_last_cuda_error(void) { return g_last_error; }
 
 int hstu_build_time_thresholds(double time_div, int32_t num_buckets, int64_t* out) {
   if (!out || !(time_div > 0.0) || !isfinite(time_div) || num_buckets < 2 || num_buckets > 1024)

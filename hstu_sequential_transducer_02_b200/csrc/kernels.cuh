@@ -46,6 +46,7 @@ struct AttnFwdParams {
   long long timeout_ns;        // bound of every device-side wait
   const int32_t* tile_base;    // tensor-core path: first tile record of each sequence
   const int32_t* tile_recs;    // tensor-core path: timestamp tile records
+  int32_t* item_cursor;        // tensor-core path: dynamic work-list cursor (zeroed by the scheduler)
 };
 
 struct AttnBwdParams {

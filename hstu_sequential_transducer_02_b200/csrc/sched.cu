@@ -1,7 +1,8 @@
 // Jagged-batch scheduler: builds the (sequence, head, q tile) work list of the
-// attention kernels, sorted by cost (number of kv tiles) in descending order so
-// that persistent CTAs that take items in snake order approximate LPT
-// ("Разная длина истории": real lengths, no padding to a common maximum).
+// attention kernels ("Разная длина истории": real lengths, no padding to a
+// common maximum).  Two orders: by cost (number of kv tiles) in descending order,
+// for persistent CTAs that take items in snake order (an approximation of LPT);
+// and a locality order for CTAs that fetch items dynamically (mode 3).
 #include <cub/block/block_scan.cuh>
 
 #include "common.cuh"
@@ -13,11 +14,18 @@ namespace {
 constexpr int kSchedThreads = 1024;
 constexpr int kCostBins = 2048;  // costs >= kCostBins - 1 share the top bin
 
-// cost of one item: kv tiles for a forward q tile, q tiles for a backward kv tile
+// cost of one item: kv tiles for a forward q tile (mode 0) or for a pair of
+// q tiles of width tk (mode 2, tm = 2 tk), q tiles for a backward kv tile (mode 1)
 __device__ __forceinline__ int item_cost(int mode, int t, int n, int hist, int tm, int tk) {
   if (mode == 0) {
     int r0 = t * tm, r1 = min(n, r0 + tm);
     return kv_count(kv_tiles_for(r0, r1, hist, tk));
+  }
+  if (mode == 2) {
+    const int r0 = t * tm, rb = r0 + tk;
+    int c = kv_count(kv_tiles_for(r0, min(n, rb), hist, tk));
+    if (rb < n) c += kv_count(kv_tiles_for(rb, min(n, r0 + tm), hist, tk));
+    return c;
   }
   // backward: q tiles that hold a row attending to kv tile t (columns [c0, c1))
   int c0 = t * tk, c1 = min(n, c0 + tk);
@@ -73,10 +81,55 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
     if (tid == 0) tile_base[B] = carry;
     __syncthreads();
   }
+  if (mode == 3) {
+    // Locality order for dynamically fetched forward items: sequences by number of
+    // q tiles (descending), then head, then q tile (descending).  CTAs that run at
+    // the same time then share the K/V tiles of a few (sequence, head) pairs.
+    for (int s = tid; s < B; s += kSchedThreads) {
+      const int tiles = (offs[s + 1] - offs[s] + tm - 1) / tm;
+      if (tiles > 0) atomicAdd(&hist_bins[min(tiles, kCostBins - 1)], tiles * H);
+    }
+    __syncthreads();
+    constexpr int kPer3 = kCostBins / kSchedThreads;
+    int loc[kPer3];
+    int sum3 = 0;
+#pragma unroll
+    for (int r = 0; r < kPer3; ++r) {
+      loc[r] = hist_bins[kCostBins - 1 - (tid * kPer3 + r)];
+      sum3 += loc[r];
+    }
+    int base3, total3;
+    Scan(scan_tmp).ExclusiveSum(sum3, base3, total3);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kPer3; ++r) {
+      hist_bins[kCostBins - 1 - (tid * kPer3 + r)] = base3;
+      base3 += loc[r];
+    }
+    __syncthreads();
+    if (total3 > max_items) {
+      if (tid == 0) { *count = 0; set_status(status, HSTU_ERR_WORKSPACE); }
+      return;
+    }
+    for (int s = tid; s < B; s += kSchedThreads) {
+      const SeqInfo si = load_seq(offs, num_targets, s);
+      const int tiles = (si.n + tm - 1) / tm;
+      if (tiles <= 0) continue;
+      const int base_s = atomicAdd(&hist_bins[min(tiles, kCostBins - 1)], tiles * H);
+      for (int h = 0; h < H; ++h)
+        for (int t = 0; t < tiles; ++t)
+          items[base_s + h * tiles + (tiles - 1 - t)] = WorkItem{s, h, t, item_cost(0, t, si.n, si.hist, tm, tk)};
+    }
+    if (tid == 0) {
+      *count = total3;
+      count[1] = 0;  // dynamic fetch cursor
+    }
+    return;
+  }
   // pass 1: histogram of costs
   for (int s = tid; s < B; s += kSchedThreads) {
     SeqInfo si = load_seq(offs, num_targets, s);
-    int tiles = mode == 0 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
+    int tiles = mode != 1 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
     for (int t = 0; t < tiles; ++t) {
       int c = item_cost(mode, t, si.n, si.hist, tm, tk);
       if (c <= 0) continue;
@@ -111,7 +164,7 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
   // pass 2: scatter
   for (int s = tid; s < B; s += kSchedThreads) {
     SeqInfo si = load_seq(offs, num_targets, s);
-    int tiles = mode == 0 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
+    int tiles = mode != 1 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
     for (int t = 0; t < tiles; ++t) {
       int c = item_cost(mode, t, si.n, si.hist, tm, tk);
       if (c <= 0) continue;

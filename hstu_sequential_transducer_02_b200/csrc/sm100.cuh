@@ -53,6 +53,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a waiting thread sleeps (without taking
+// issue slots) until the phase completes or about `hint_ns` have passed.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase of `bar` with the given parity has completed.  Gives
 // up after `timeout_ns` nanoseconds, or as soon as *abort becomes non-zero;
 // returns false then (the caller records HSTU_ERR_TIMEOUT and unwinds).
@@ -60,12 +74,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
-      if (abort && *abort) return false;
-      if ((long long)(global_timer_ns() - t0) > timeout_ns) return false;
-    }
+  const uint32_t hint = timeout_ns < 1000000ll ? (uint32_t)timeout_ns : 1000000u;  // sleep at most 1 ms per try
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
+    if (abort && *abort) return false;
+    if ((long long)(global_timer_ns() - t0) > timeout_ns) return false;
   }
 }
 

@@ -163,6 +163,11 @@ const char* hstu_status_string(int status);
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int hstu_version(void);
 
+/* Description of the last CUDA error that made a call of this thread return
+ * HSTU_ERR_CUDA (the failing runtime call and CUDA's message); thread-local
+ * static storage, never NULL. */
+const char* hstu_last_cuda_error(void);
+
 /* Integer thresholds of the time bucket (host only, no CUDA call):
  * out[0] = 0 and, for b >= 1, out[b] = the smallest dt >= 1 with
  * floor(ln(dt) / time_div) >= b in fp64 (INT64_MAX if none).  Then

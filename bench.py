@@ -130,6 +130,47 @@ def run_reference(args, rank: int):
 
 
 # ----------------------------------------------------------------------------
+# multi-rank plumbing (host logic; covered on CPU with gloo ranks)
+# ----------------------------------------------------------------------------
+
+def rank_workload(rank: int):
+    """The batch of `rank`: one model (the seeded weights of rank 0) and, for
+    rank r > 0, its own draw of sequences, timestamps and inputs from the same
+    recipe with seed offset 1000 r.  Ranks share no data and exchange nothing
+    on the data path, so per-rank work stays fixed as ranks are added."""
+    wl = W.make_workload(CONFIG_ID)
+    if rank == 0:
+        return wl
+    own = W.make_workload(CONFIG_ID, seed=W.SEED_BASE + CONFIG_ID + 1000 * rank)
+    own.layers = wl.layers
+    return own
+
+
+def reduce_over_ranks(local_ms: float, local_tokens: int, world: int, device=None):
+    """(max over ranks of the timed milliseconds, sum over ranks of the tokens).
+    Every rank calls it at the same point with the same collective sequence."""
+    if world == 1:
+        return float(local_ms), int(local_tokens)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    n = torch.tensor([local_tokens], dtype=torch.int64, device=device)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(n.item())
+
+
+def unmasked_pairs(seq_offsets, num_targets=None) -> int:
+    """Attended (i, j) pairs of a jagged batch: N(N+1)/2 causal pairs of the N
+    history tokens plus (N+1) per candidate (history and itself)."""
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    n = np.diff(offs)
+    nt = np.zeros_like(n) if num_targets is None else np.asarray(num_targets, np.int64)
+    N = n - nt
+    return int(np.sum(N * (N + 1) // 2 + nt * (N + 1)))
+
+
+# ----------------------------------------------------------------------------
 # clocks
 # ----------------------------------------------------------------------------
 
@@ -218,7 +259,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     from hstu_sequential_transducer_02_b200 import binding as hb
 
-    wl = W.make_workload(CONFIG_ID)
+    wl = rank_workload(rank)
     sp = wl.spec
     td = torch.bfloat16
     T = wl.total_tokens
@@ -256,13 +297,9 @@ def main():
     hb.trace_enable(False)
     clk = clocks.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms, T_all = reduce_over_ranks(sum(step_ms), T, world, "cuda")
     ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    value = T_all / (ms_per_step / 1e3)
 
     # end to end through the same call: pinned host inputs in, output out, every step
     x_h = torch.from_numpy(wl.x).to(td).pin_memory()
@@ -285,18 +322,13 @@ def main():
         e_e[k].record()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_s, e_e))
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * T / (e2e_ms / args.steps / 1e3)
+    e2e_ms, _ = reduce_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_s, e_e)), T, world, "cuda")
+    e2e_value = T_all / (e2e_ms / args.steps / 1e3)
     h2d = x_h.numel() * x_h.element_size() + offs_h.numel() * 4 + ts_h.numel() * 8
     d2h = y_h.numel() * y_h.element_size()
 
     # roofline of the attention kernel
-    import oracle.hstu_oracle as O  # work accounting only (pair count of the mask)
-    pairs = O.attention_pairs(wl.seq_offsets)
+    pairs = unmasked_pairs(wl.seq_offsets)
     attn_flops = pairs * 2 * (sp.head_dim + sp.head_dim) * sp.num_heads
     peaks, peak_src = load_peaks()
     attn_name = "attn_fwd_tc" if "attn_fwd_tc" in trace else "attn_fwd_simt"

@@ -23,9 +23,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -45,7 +43,7 @@ L2_BYTES = 126 * 1024 * 1024
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
@@ -175,50 +173,187 @@ def unmasked_pairs(seq_offsets, num_targets=None) -> int:
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the clock-event reasons of one GPU every few
+    milliseconds from a host thread (NVML reads only; nothing is changed)."""
 
-    def __init__(self, index: int):
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, index: int, period_s: float = 0.005):
         self.index = index
-        self.proc = None
-        self.path = None
+        self.period = period_s
+        self.rows = []
+        self.thread = None
+        self.stop_flag = False
+
+    def _loop(self, nv, h):
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((sm, mx, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def start(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
-                                         stderr=subprocess.DEVNULL)
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
         except Exception:
-            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._loop, args=(nv, h), daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.rows and time.time() - t0 < 2.0:  # first sample before the timed region
+            time.sleep(0.001)
+        self.rows = []
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.out.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        rows = self.rows
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({n for _, _, rs in rows for n, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "source": "NVML, 5 ms period, timed region only"}
+
+
+KERNEL_SOURCES = {"attn_fwd_tc": ("attn_tc.cu", "sm100.cuh", "common.cuh", "kernels.cuh")}
+
+
+def kernel_digest(kernel: str):
+    """sha256 (first 16 hex digits) of the sources that make up `kernel`."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES.get(kernel, ()):
+        with open(os.path.join(ROOT, "hstu_sequential_transducer_02_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary
+    (`profiles/dram_traffic.txt`: kernel, bytes, source digest), or None when
+    there is none or the kernel's sources changed after the capture."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and parts[0] == kernel and not line.startswith("#"):
+                if parts[2] != kernel_digest(kernel):
+                    return None
+                try:
+                    return float(parts[1])
+                except ValueError:
+                    return None
+    return None
+
+
+# ----------------------------------------------------------------------------
+# multi-rank plumbing (host logic; covered on CPU with gloo ranks)
+# ----------------------------------------------------------------------------
+
+def rank_workload(rank: int):
+    """The batch of `rank`: one model (the seeded weights of rank 0) and, for
+    rank r > 0, its own draw of sequences, timestamps and inputs from the same
+    recipe with seed offset 1000 r.  Ranks share no data and exchange nothing
+    on the data path, so per-rank work stays fixed as ranks are added."""
+    wl = W.make_workload(CONFIG_ID)
+    if rank == 0:
+        return wl
+    own = W.make_workload(CONFIG_ID, seed=W.SEED_BASE + CONFIG_ID + 1000 * rank)
+    own.layers = wl.layers
+    return own
+
+
+def reduce_over_ranks(local_ms: float, local_tokens: int, world: int, device=None):
+    """(max over ranks of the timed milliseconds, sum over ranks of the tokens).
+    Every rank calls it at the same point with the same collective sequence."""
+    if world == 1:
+        return float(local_ms), int(local_tokens)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    n = torch.tensor([local_tokens], dtype=torch.int64, device=device)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(n.item())
+
+
+def unmasked_pairs(seq_offsets, num_targets=None) -> int:
+    """Attended (i, j) pairs of a jagged batch: N(N+1)/2 causal pairs of the N
+    history tokens plus (N+1) per candidate (history and itself)."""
+    offs = np.asarray(seq_offsets, dtype=np.int64)
+    n = np.diff(offs)
+    nt = np.zeros_like(n) if num_targets is None else np.asarray(num_targets, np.int64)
+    N = n - nt
+    return int(np.sum(N * (N + 1) // 2 + nt * (N + 1)))
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event reasons of one GPU every few
+    milliseconds from a host thread (NVML reads only; nothing is changed)."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index = index
+        self.period = period_s
+        self.rows = []
+        self.thread = None
+        self.stop_flag = False
+
+    def _loop(self, nv, h):
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append((sm, mx, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+        except Exception:
+            return
+        self.thread = threading.Thread(target=self._loop, args=(nv, h), daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.rows and time.time() - t0 < 2.0:  # first sample before the timed region
+            time.sleep(0.001)
+        self.rows = []
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        rows = self.rows
+        if not rows:
+            return None
+        reasons = sorted({n for _, _, rs in rows for n, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "source": "NVML, 5 ms period, timed region only"}
 
 
 def read_traffic(kernel: str):

@@ -7,16 +7,22 @@
 //
 // One persistent CTA per SM takes (sequence, head, q tile) work items from a
 // shared cursor over a list in locality order (long sequences first, then head,
-// then q tile), so the CTAs running at the same time share K/V tiles in L2.  Per q tile of 128 rows and each kv tile of 128
-// columns that holds an attended pair:
-//   warp 0      TMA: Q once per item, K/V per kv tile into a ring of stages,
-//               plus the tile's timestamps (and their per-half min/max)
-//   warp 1      one thread issues tcgen05.mma: S = Q K^T into one of two TMEM
-//               buffers, then O += P V into the TMEM accumulator
-//   warps 2-9   epilogue: TMEM -> registers, rab bias (position and time
-//               buckets, bit-exact integer rule), SiLU, mask, bf16 P into
-//               shared memory (128-byte swizzle, the MMA's A layout); at the end
-//               of the item O * (1/N) -> bf16 -> global memory
+// then q tile), so the CTAs running at the same time share K/V tiles in L2.
+// Per q tile of 128 rows and each kv tile of 128 columns that holds an attended
+// pair:
+//   warp 0        TMA: Q once per item, K per kv tile into a ring of stages, and
+//                 the kv tile's timestamp record (int32 offsets, per-segment
+//                 min/max); it also fetches the work items for everyone
+//   warp 2        TMA: V per kv tile into its own ring
+//   warp 1        one thread issues S = Q K^T (tcgen05.mma, operands in shared
+//                 memory) into one of three TMEM buffers
+//   warp 3        one thread issues O += P V with P read from TMEM (the A
+//                 operand) and V from shared memory
+//   warps 4-19    epilogue, one warp per TMEM lane quarter and 32-column
+//                 segment: S -> registers, rab bias (position and time buckets,
+//                 bit-exact integer rule), SiLU, mask, bf16 P written back over
+//                 the S columns; at the end of the item O * (1/N) -> bf16 ->
+//                 global memory
 // No softmax means no running max and no rescaling: O accumulates in TMEM
 // across all kv tiles.  Fully masked kv tiles are never visited.
 #include <mutex>
@@ -32,7 +38,7 @@ using namespace sm100;
 constexpr int BM = 128;                    // q rows per tile (UMMA M)
 constexpr int BN = 128;                    // kv columns per tile
 constexpr int kEpiWarps = 16;              // four warps per TMEM lane quarter, one per 32-column segment
-constexpr int kEpiWarp0 = 3;               // warps 0: K loads, 1: MMA, 2: V loads, 3..18: epilogue
+constexpr int kEpiWarp0 = 4;               // warps 0: Q/K loads, 1: S MMAs, 2: V loads, 3: P V MMAs, 4..19: epilogue
 constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
 constexpr int kBoxBytes = 128 * 128;       // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t kTmemCols = 512;
@@ -60,7 +66,7 @@ constexpr int kRecStages = 8;              // timestamp records run up to 8 kv t
 constexpr int kSBufs = 3;                  // S/P buffers in TMEM: S runs two kv tiles ahead of P V
 
 constexpr int kItemSlots = 4;              // work items fetched ahead by the Q/K producer
-constexpr int kItemReaders = 2 + kEpiWarps;  // V producer, MMA issuer, epilogue warps
+constexpr int kItemReaders = 3 + kEpiWarps;  // V producer, two MMA issuers, epilogue warps
 
 struct Barriers {
   uint64_t it_full[kItemSlots], it_empty[kItemSlots];
@@ -68,9 +74,9 @@ struct Barriers {
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t r_full[kRecStages], r_empty[kRecStages];
-  uint64_t s_full[3], p_full[3];
+  uint64_t s_full[3], p_full[3], pv_done[3];
   uint64_t o_full, o_empty;
-  uint64_t done;
+  uint64_t done, done_pv;
 };
 
 struct TcParams {
@@ -166,10 +172,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     for (int s = 0; s < SK; ++s) { mbar_init(&bars->k_full[s], 1); mbar_init(&bars->k_empty[s], 1); }
     for (int s = 0; s < SV; ++s) { mbar_init(&bars->v_full[s], 1); mbar_init(&bars->v_empty[s], 1); }
     for (int s = 0; s < kRecStages; ++s) { mbar_init(&bars->r_full[s], 1); mbar_init(&bars->r_empty[s], kEpiWarps); }
-    for (int s = 0; s < kSBufs; ++s) { mbar_init(&bars->s_full[s], 1); mbar_init(&bars->p_full[s], kEpiWarps); }
+    for (int s = 0; s < kSBufs; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], kEpiWarps);
+      mbar_init(&bars->pv_done[s], 1);
+    }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_empty, kEpiWarps);
     mbar_init(&bars->done, 1);
+    mbar_init(&bars->done_pv, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -261,12 +272,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         }
       }
     }
-  } else if (warp == 1) {
-    // =================================================================== MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // =================================================================== MMA issuers
+    // Issue is synchronous with the tensor pipe, so S = Q K^T (warp 1) and O += P V
+    // (warp 3) have a thread each: S of a later kv tile only waits until P V has
+    // consumed its TMEM buffer, not until the P V before it has been issued.
     if (lane == 0) {
+      const bool s_side = warp == 1;
       constexpr uint32_t idesc_s = make_idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = make_idesc_bf16(BM, DV, false, true);
-      int s_it = 0, p_it = 0;  // global kv-tile counters: S computed, P V consumed
+      // descriptors of stage 0; every MMA below adds compile-time offsets to these,
+      // so an issuing thread spends few instructions per MMA (it shares its
+      // sub-partition's issue slots with four epilogue warps)
+      const uint64_t dq0 = make_sw128_desc(sQ, 16, 1024);
+      const uint64_t dk0 = make_sw128_desc(sK, 16, 1024);
+      const uint64_t dv0 = make_sw128_desc(sV, kBoxBytes, 1024);
+      int n_it = 0;  // global kv-tile counter of this thread
       for (int k = 0;; ++k) {
         const int slot = k % kItemSlots;
         if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
@@ -278,55 +299,54 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const int r0 = wi.qtile * BM;
         const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
         const int nk = kv_count(kr);
-        if (!mbar_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
-        // S = Q K^T for the item's kv tile s_loc into buffer s_it % kSBufs; the buffer's
-        // previous P was consumed by a P V issued earlier (the tensor pipe runs in order)
-        int s_loc = 0;
-        auto issue_s = [&]() -> bool {
-          const int st = s_it % SK;
-          const int sb = s_it % kSBufs;
-          if (!mbar_wait(&bars->k_full[st], (s_it / SK) & 1, tmo, abort_flag)) return false;
-          tc_fence_after();
+        if (s_side) {
+          if (!mbar_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
+          for (int jj = 0; jj < nk; ++jj, ++n_it) {
+            // S of kv tile n_it into buffer n_it % kSBufs once P V of tile n_it - kSBufs is done
+            const int st = n_it % SK;
+            const int sb = n_it % kSBufs;
+            if (!mbar_wait(&bars->k_full[st], (n_it / SK) & 1, tmo, abort_flag)) goto fail;
+            if (!mbar_wait(&bars->pv_done[sb], ((n_it / kSBufs) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            tc_fence_after();
+            const uint64_t dk = desc_advance(dk0, st * C::kTileBytes);
+            const uint32_t dS = tmem_s0 + sb * BN;
 #pragma unroll
-          for (int ks = 0; ks < DH / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
-            const uint64_t a = make_sw128_desc(sQ + off, 16, 1024);
-            const uint64_t b = make_sw128_desc(sK + st * C::kTileBytes + off, 16, 1024);
-            umma_f16_ss(tmem_s0 + sb * BN, a, b, idesc_s, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < DH / 16; ++ks) {
+              const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
+              umma_f16_ss(dS, desc_advance(dq0, off), desc_advance(dk, off), idesc_s, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars->s_full[sb]);
+            umma_commit(&bars->k_empty[st]);
+            if (jj == nk - 1) umma_commit(&bars->q_empty);
           }
-          umma_commit(&bars->s_full[sb]);
-          umma_commit(&bars->k_empty[st]);
-          if (s_loc == nk - 1) umma_commit(&bars->q_empty);
-          ++s_it;
-          ++s_loc;
-          return true;
-        };
-        while (s_loc < nk && s_loc < kSBufs - 1)
-          if (!issue_s()) goto fail;
-        for (int jj = 0; jj < nk; ++jj) {
-          // O (+)= P V for kv tile jj, P read from TMEM
-          const int pb = p_it % kSBufs;
-          const int vs = p_it % SV;
-          if (!mbar_wait(&bars->p_full[pb], (p_it / kSBufs) & 1, tmo, abort_flag)) goto fail;
-          if (!mbar_wait(&bars->v_full[vs], (p_it / SV) & 1, tmo, abort_flag)) goto fail;
-          if (jj == 0 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
-          tc_fence_after();
-          const uint32_t pa = tmem_s0 + pb * BN;
+        } else {
+          for (int jj = 0; jj < nk; ++jj, ++n_it) {
+            // O (+)= P V for kv tile n_it, P read from TMEM
+            const int pb = n_it % kSBufs;
+            const int vs = n_it % SV;
+            if (!mbar_wait(&bars->p_full[pb], (n_it / kSBufs) & 1, tmo, abort_flag)) goto fail;
+            if (!mbar_wait(&bars->v_full[vs], (n_it / SV) & 1, tmo, abort_flag)) goto fail;
+            if (jj == 0 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
+            tc_fence_after();
+            const uint32_t pa = tmem_s0 + pb * BN;
+            const uint64_t dv = desc_advance(dv0, vs * C::kTileBytes);
+            const uint32_t acc0 = jj > 0 ? 1u : 0u;
 #pragma unroll
-          for (int ks = 0; ks < BN / 16; ++ks) {
-            // kv columns [16ks, 16ks+16) were written by segment ks/2 at columns 32*(ks/2) + 8*(ks%2)
-            const uint64_t b = make_sw128_desc(sV + vs * C::kTileBytes + ks * 16 * 128, kBoxBytes, 1024);
-            umma_f16_ts(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), b, idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < BN / 16; ++ks) {
+              // kv columns [16ks, 16ks+16) were written by segment ks/2 at columns 32*(ks/2) + 8*(ks%2)
+              umma_f16_ts(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), desc_advance(dv, ks * 16 * 128), idesc_o,
+                          ks > 0 ? 1u : acc0);
+            }
+            umma_commit(&bars->v_empty[vs]);
+            umma_commit(&bars->pv_done[pb]);
           }
-          umma_commit(&bars->v_empty[vs]);
-          ++p_it;
-          if (s_loc < nk && !issue_s()) goto fail;
+          umma_commit(&bars->o_full);
         }
-        umma_commit(&bars->o_full);
       }
-      // all issued MMAs complete before TMEM is released
-      umma_commit(&bars->done);
-      mbar_wait(&bars->done, 0, tmo, nullptr);
+      // all MMAs this thread issued complete before TMEM is released
+      uint64_t* dbar = s_side ? &bars->done : &bars->done_pv;
+      umma_commit(dbar);
+      mbar_wait(dbar, 0, tmo, nullptr);
     }
   } else {
     // =================================================================== epilogue
@@ -378,12 +398,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         tc_fence_after();
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);  // waited for after the classification
-        // ---- classify this row's 32 columns
+        // ---- classify this row's 32 columns:
+        //   rank 0: nothing attended; 1: one time bucket (constant bias); 2: two buckets;
+        //   3: three or four buckets (per-element threshold compares); 4: general
+        //   (per-element mask and exact buckets).  Far from the diagonal the position
+        //   bucket is the last one for every column.
         const int cl = c0 + seg * 32;   // first column of the segment
         const bool narrow = row_narrow && !rec.wide;
         const bool any_live = live && (cand ? (cl < si.hist || (i >= cl && i < cl + 32)) : (cl <= i));
         const bool full = live && (cand ? (cl + 31 < si.hist) : (cl + 31 <= i));
-        int mode = any_live ? 3 : 0;  // 0: zero, 1: one time bucket, 2: two, 4: three or four, 3: general
+        int rank = any_live ? 4 : 0;
         float hb0 = 0.f, hb1 = 0.f, hb2 = 0.f, hb3 = 0.f;   // half of the bias values
         int32_t th1 = 0x7FFFFFFF, th2 = 0x7FFFFFFF, th3 = 0x7FFFFFFF;
         if (full && narrow && posi - (cl + 31) >= kNumBuckets - 1) {
@@ -392,31 +416,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
           if (ri >= mx) { dlo = ri - mx; dhi = ri - mn; }
           else if (ri <= mn) { dlo = mn - ri; dhi = mx - ri; }
           else { dlo = 0; dhi = max(ri - mn, mx - ri); }
-          const int tlo = fast_bucket(dlo, thr32, k_lg), thi = fast_bucket(dhi, thr32, k_lg);
+          const int tlo = fast_bucket(dlo, thr32, k_lg);
           const float pb127 = pos_b[kNumBuckets - 1];
           hb0 = 0.5f * (pb127 + time_b[tlo]);
-          if (tlo == thi) {
-            mode = 1;
-          } else if (thi - tlo <= 3) {
-            mode = thi - tlo == 1 ? 2 : 4;
-            hb1 = 0.5f * (pb127 + time_b[tlo + 1]);
-            th1 = thr32[tlo + 1];
-            if (thi - tlo >= 2) { hb2 = 0.5f * (pb127 + time_b[tlo + 2]); th2 = thr32[tlo + 2]; }
-            if (thi - tlo >= 3) { hb3 = 0.5f * (pb127 + time_b[tlo + 3]); th3 = thr32[tlo + 3]; }
+          if (dhi < thr32[tlo + 1]) {
+            rank = 1;
+          } else {
+            const int thi = fast_bucket(dhi, thr32, k_lg);
+            if (thi - tlo <= 3) {
+              rank = thi - tlo == 1 ? 2 : 3;
+              hb1 = 0.5f * (pb127 + time_b[tlo + 1]);
+              th1 = thr32[tlo + 1];
+              if (thi - tlo >= 2) { hb2 = 0.5f * (pb127 + time_b[tlo + 2]); th2 = thr32[tlo + 2]; }
+              if (thi - tlo >= 3) { hb3 = 0.5f * (pb127 + time_b[tlo + 3]); th3 = thr32[tlo + 3]; }
+            }
           }
         }
+        // one path per warp: the highest rank of its rows (a lower rank's row is a
+        // special case of a higher one; rows beyond the sequence are zeroed below)
+        const int wrank = __reduce_max_sync(0xffffffffu, rank);
         tmem_ld_wait_regs(raw);
         // ---- bias, SiLU (as h + h tanh h with h = (s + bias) / 2), mask; packed bf16 pairs
         uint32_t pk[16];
-        if (mode == 0) {
+        if (wrank == 0) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = 0u;
-        } else if (mode == 1) {
+        } else if (wrank == 1) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = silu2_bf16(fmaf(__uint_as_float(raw[2 * e]), 0.5f, hb0),
-                               fmaf(__uint_as_float(raw[2 * e + 1]), 0.5f, hb0));
-        } else if (mode == 2) {
+          for (int e = 0; e < 16; ++e) {
+            float h0, h1;
+            half_plus2(__uint_as_float(raw[2 * e]), __uint_as_float(raw[2 * e + 1]), hb0, h0, h1);
+            pk[e] = silu2_bf16(h0, h1);
+          }
+        } else if (wrank == 2) {
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const int4 rel4 = *reinterpret_cast<const int4*>(&rec.rel[seg * 32 + e4 * 4]);
@@ -428,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
             pk[2 * e4] = silu2_bf16(h[0], h[1]);
             pk[2 * e4 + 1] = silu2_bf16(h[2], h[3]);
           }
-        } else if (mode == 4) {
+        } else if (wrank == 3) {
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const int4 rel4 = *reinterpret_cast<const int4*>(&rec.rel[seg * 32 + e4 * 4]);
@@ -445,7 +477,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
             pk[2 * e4] = silu2_bf16(h[0], h[1]);
             pk[2 * e4 + 1] = silu2_bf16(h[2], h[3]);
           }
+        } else if (__all_sync(0xffffffffu, narrow)) {
+          // general, 32-bit time offsets: per-element mask, position and time bucket,
+          // branch-free in groups of eight so that the bucket chains overlap
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+            float h[8];
+            bool att[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int e = 8 * e8 + u;
+              const int j = cl + e;
+              att[u] = attended(i, j, si.n, si.hist);
+              const int pb = pos_bucket(posi, token_pos(j, si.hist));
+              const int tb = fast_bucket(abs(ri - rec.rel[seg * 32 + e]), thr32, k_lg);
+              h[u] = 0.5f * (__uint_as_float(raw[e]) + (pos_b[pb] + time_b[tb]));
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t v = silu2_bf16(h[2 * q], h[2 * q + 1]);
+              pk[4 * e8 + q] = (att[2 * q] ? (v & 0xFFFFu) : 0u) | (att[2 * q + 1] ? (v & 0xFFFF0000u) : 0u);
+            }
+          }
         } else {
+          // general with 64-bit time differences (a row or column offset beyond +-2^30)
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
             float h[2];
@@ -458,9 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
               float bias = 0.f;
               if (att[u]) {
                 const int pb = pos_bucket(posi, token_pos(j, si.hist));
-                int tb;
-                if (narrow) tb = fast_bucket(abs(ri - rec.rel[seg * 32 + e]), thr32, k_lg);
-                else tb = time_bucket_exact(abs_diff_i64(ti, p.timestamps[si.start + j]), thr);
+                const int tb = time_bucket_exact(abs_diff_i64(ti, p.timestamps[si.start + j]), thr);
                 bias = pos_b[pb] + time_b[tb];
               }
               h[u] = 0.5f * (__uint_as_float(raw[e]) + bias);
@@ -468,6 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
             const uint32_t v = silu2_bf16(h[0], h[1]);
             pk[e2] = (att[0] ? (v & 0xFFFFu) : 0u) | (att[1] ? (v & 0xFFFF0000u) : 0u);
           }
+        }
+        if (rank == 0 && wrank != 4) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
         }
         // ---- P -> TMEM, over this segment's own S columns (the A operand of P V)
         tmem_st_32x32b_x16(tmem_s0 + sb * BN + lane_off + seg * 32, pk);

@@ -10,7 +10,9 @@
 //
 //   warp 0     TMA producer: A and B k-slices (64 deep) into a ring of stages
 //   warp 1     one thread issues tcgen05.mma into one of two TMEM accumulators
-//   warps 2-5  epilogue: TMEM -> registers -> bias / SiLU / residual -> global
+//   warps 2-17 epilogue: TMEM -> registers -> bias / SiLU / residual -> global;
+//              four warps per TMEM lane quarter, each on a quarter of the columns,
+//              so every SM sub-partition has four warps to hide the latencies
 // The two accumulators let the epilogue of one tile overlap the main loop of
 // the next.  ("Actions Speak Louder than Words" summary, 2.2: the linear layers
 // are fused with LayerNorm and SiLU; f1 and f2 are single linear layers.)
@@ -26,7 +28,7 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;                       // one 128-byte swizzle atom of bf16
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 16;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kABytes = BM * BK * 2;         // 16 KB
 
@@ -302,9 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+    const int group = (warp - 2) >> 2;     // quarter of the tile's columns
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    constexpr int kCols = BN / 4;
     int t = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       Unit un;
@@ -316,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const bool row_ok = m < M_eff;
       const bool has_k = un.k1 > un.k0;  // an empty K range never wrote the accumulator
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = group * kCols; c < (group + 1) * kCols; c += 32) {
         __syncwarp();
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_base + ab * BN + lane_off + c, raw);

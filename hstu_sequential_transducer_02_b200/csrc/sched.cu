@@ -13,6 +13,7 @@ namespace hstu {
 namespace {
 constexpr int kSchedThreads = 1024;
 constexpr int kCostBins = 2048;  // costs >= kCostBins - 1 share the top bin
+constexpr int kSeqSmem = 4096;   // sequences whose list offsets fit in shared memory (locality order)
 
 // cost of one item: kv tiles for a forward q tile (mode 0) or for a pair of
 // q tiles of width tk (mode 2, tm = 2 tk), q tiles for a backward kv tile (mode 1)
@@ -111,14 +112,39 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
       if (tid == 0) { *count = 0; set_status(status, HSTU_ERR_WORKSPACE); }
       return;
     }
+    // every sequence's place in the list; the items themselves are then written by
+    // all threads (flat index over sequences in order, H * tiles items each)
+    __shared__ int seq_base[kSeqSmem];
+    const bool flat = tile_base != nullptr && tm == tk && B <= kSeqSmem;
     for (int s = tid; s < B; s += kSchedThreads) {
       const SeqInfo si = load_seq(offs, num_targets, s);
       const int tiles = (si.n + tm - 1) / tm;
       if (tiles <= 0) continue;
       const int base_s = atomicAdd(&hist_bins[min(tiles, kCostBins - 1)], tiles * H);
+      if (flat) {
+        seq_base[s] = base_s;
+        continue;
+      }
       for (int h = 0; h < H; ++h)
         for (int t = 0; t < tiles; ++t)
           items[base_s + h * tiles + (tiles - 1 - t)] = WorkItem{s, h, t, item_cost(0, t, si.n, si.hist, tm, tk)};
+    }
+    if (flat) {
+      __syncthreads();
+      // tile_base[s] (q tiles before sequence s, tm == tk) orders the flat index
+      for (int f = tid; f < total3; f += kSchedThreads) {
+        int lo = 0, hi = B - 1;  // last s with tile_base[s] * H <= f
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if ((int64_t)tile_base[mid] * H <= f) lo = mid; else hi = mid - 1;
+        }
+        const int s = lo;
+        const SeqInfo si = load_seq(offs, num_targets, s);
+        const int tiles = tile_base[s + 1] - tile_base[s];
+        const int local = f - tile_base[s] * H;
+        const int h = local / tiles, t = local - h * tiles;
+        items[seq_base[s] + h * tiles + (tiles - 1 - t)] = WorkItem{s, h, t, item_cost(0, t, si.n, si.hist, tm, tk)};
+      }
     }
     if (tid == 0) {
       *count = total3;

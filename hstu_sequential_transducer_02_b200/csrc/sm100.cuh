@@ -204,6 +204,14 @@ __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The descriptor of an operand `bytes` further on in shared memory: only the
+// 14-bit start-address field changes (no carry out of it for addresses below
+// 256 KB), so the add is done on the low word alone.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)d + (bytes >> 4);
+  return ((d >> 32) << 32) | lo;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D:
 //   D format (1 = f32) in [4,6), A format (1 = bf16) in [7,10), B format in [10,13),
 //   A major in bit 15, B major in bit 16 (0 = K-major, 1 = MN-major),
@@ -229,6 +237,18 @@ __device__ __forceinline__ uint32_t silu2_bf16(float h_lo, float h_hi) {
   asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
   asm("fma.rn.bf16x2 %0, %1, %2, %1;" : "=r"(r) : "r"(h), "r"(t));
   return r;
+}
+
+// (s0, s1) * 0.5 + (c, c) in one packed fp32 instruction
+__device__ __forceinline__ void half_plus2(float s0, float s1, float c, float& h0, float& h1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %4};\n\t"
+      "mov.b64 c, {%5, %5};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(h0), "=f"(h1)
+      : "f"(s0), "f"(s1), "f"(0.5f), "f"(c));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

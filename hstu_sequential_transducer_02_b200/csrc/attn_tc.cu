@@ -112,16 +112,31 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 // to the nearest integer is at most one bucket off, and one comparison with
 // each neighbouring integer threshold corrects it (thr32[b] = min(threshold b,
 // INT32_MAX), thr32[128] = INT32_MAX).
-__device__ __forceinline__ int fast_bucket(int32_t d, const int32_t* thr32, float ln2_over_div) {
-  d = d < 1 ? 1 : d;
-  const int sh = d >= (1 << 23) ? 8 : 0;
-  const float f = __int_as_float(0x4B000000 | (d >> sh)) - 8388608.0f;   // exact: (d >> sh) < 2^23
-  const float x = fmaf(__log2f(f) + (float)sh, ln2_over_div, 12582912.0f);
-  int b = __float_as_int(x) - 0x4B400000;                               // nearest integer
+// Exact time bucket floor(ln(d) / div) of 1 <= d < 2^31 with few shared-memory
+// reads.  y = log2(d) * ln2/div comes from the special-function unit; its error
+// is below 2e-4 (the log2 approximation, float rounding of y < 72, and for
+// d >= 2^23 the eight dropped low bits), so floor(y) is the bucket unless y lies
+// within 2^-9 of an integer.  Only such lanes read one threshold (thr32[b] =
+// smallest d of bucket b, clamped to INT32_MAX; thr32[128] = INT32_MAX) and
+// settle the bucket with an exact integer compare.
+__device__ __forceinline__ int exact_bucket(int32_t d, const int32_t* thr32, float ln2_over_div) {
+  const bool big = d >= (1 << 23);
+  const float f = __int_as_float(0x4B000000 | (big ? d >> 8 : d)) - 8388608.0f;  // exact: < 2^23
+  const float y = (__log2f(f) + (big ? 8.0f : 0.0f)) * ln2_over_div;
+  const float t = (y - 0.5f) + 12582912.0f;                 // round(y - 1/2) = floor(y) off the integers
+  const float fr = y - (t - 12582912.0f);                   // y - floor(y)
+  int b = __float_as_int(t) - 0x4B400000;
   b = b < 0 ? 0 : (b > kNumBuckets - 1 ? kNumBuckets - 1 : b);
-  if (d < thr32[b]) b -= 1;
-  else if (d >= thr32[b + 1]) b += 1;
-  return b > kNumBuckets - 1 ? kNumBuckets - 1 : b;
+  if (fr < 0.001953125f || fr > 0.998046875f) {
+    const bool up = fr > 0.5f;
+    const int32_t th = thr32[up ? b + 1 : b];
+    b += up ? (d >= th ? 1 : 0) : (d < th ? -1 : 0);
+    b = b < 0 ? 0 : (b > kNumBuckets - 1 ? kNumBuckets - 1 : b);
+  }
+  return b;
+}
+__device__ __forceinline__ int fast_bucket(int32_t d, const int32_t* thr32, float ln2_over_div) {
+  return exact_bucket(d < 1 ? 1 : d, thr32, ln2_over_div);
 }
 
 // Waits for outstanding tcgen05.ld into `r`; the register operands keep the
@@ -435,6 +450,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         // one path per warp: the highest rank of its rows (a lower rank's row is a
         // special case of a higher one; rows beyond the sequence are zeroed below)
         const int wrank = __reduce_max_sync(0xffffffffu, rank);
+        // the band serves warps of history rows (rows beyond the sequence are zero)
+        // in segments starting at or after i0 - 128, i0 = the warp's first row
+        const int i0w = r0 + quarter * 32;
+        const bool use_band = wrank == 4 && p.band != nullptr && cl >= i0w - 128 &&
+                              !__any_sync(0xffffffffu, live && cand);
         tmem_ld_wait_regs(raw);
         // ---- bias, SiLU (as h + h tanh h with h = (s + bias) / 2), mask; packed bf16 pairs
         uint32_t pk[16];
@@ -477,26 +497,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
             pk[2 * e4] = silu2_bf16(h[0], h[1]);
             pk[2 * e4 + 1] = silu2_bf16(h[2], h[3]);
           }
+        } else if (use_band) {
+          // near-diagonal segment of history rows: half biases from the band
+          // (bf16 pairs), mask j <= i
+          uint4 bb[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                         make_uint4(0, 0, 0, 0)};
+          if (live) {
+            const uint4* bp = reinterpret_cast<const uint4*>(p.band) + (int64_t)(si.start + i) * kBandChunks +
+                              ((cl - (i0w - 128)) >> 3);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) bb[c] = __ldg(bp + c);
+          }
+          const int lim = live ? i - cl : -1;   // column e of the segment is attended iff e <= lim
+          const uint32_t* bw = reinterpret_cast<const uint32_t*>(bb);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            float h0, h1;
+            half_plus2c(__uint_as_float(raw[2 * q]), __uint_as_float(raw[2 * q + 1]), __uint_as_float(bw[q] << 16),
+                        __uint_as_float(bw[q] & 0xFFFF0000u), h0, h1);
+            const uint32_t v = silu2_bf16(h0, h1);
+            pk[q] = (2 * q <= lim ? (v & 0xFFFFu) : 0u) | (2 * q + 1 <= lim ? (v & 0xFFFF0000u) : 0u);
+          }
         } else if (__all_sync(0xffffffffu, narrow)) {
-          // general, 32-bit time offsets: per-element mask, position and time bucket,
-          // branch-free in groups of eight so that the bucket chains overlap
+          // general, 32-bit time offsets: per-element mask, position and time bucket
+          // (shared-memory reads kept few: the tensor core is reading Q, K and V
+          // from the same shared memory meanwhile)
 #pragma unroll
-          for (int e8 = 0; e8 < 4; ++e8) {
-            float h[8];
-            bool att[8];
+          for (int g4 = 0; g4 < 8; ++g4) {
+            const int4 rel4 = *reinterpret_cast<const int4*>(&rec.rel[seg * 32 + 4 * g4]);
+            const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+            float h[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int e = 8 * e8 + u;
-              const int j = cl + e;
-              att[u] = attended(i, j, si.n, si.hist);
+            for (int u = 0; u < 4; ++u) {
+              const int j = cl + 4 * g4 + u;
+              const int32_t dd = abs(ri - rv[u]);
+              const int tb = exact_bucket(dd < 1 ? 1 : dd, thr32, k_lg);
               const int pb = pos_bucket(posi, token_pos(j, si.hist));
-              const int tb = fast_bucket(abs(ri - rec.rel[seg * 32 + e]), thr32, k_lg);
-              h[u] = 0.5f * (__uint_as_float(raw[e]) + (pos_b[pb] + time_b[tb]));
+              h[u] = 0.5f * (__uint_as_float(raw[4 * g4 + u]) + (pos_b[pb] + time_b[tb]));
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
+              const int j = cl + 4 * g4 + 2 * q;
               const uint32_t v = silu2_bf16(h[2 * q], h[2 * q + 1]);
-              pk[4 * e8 + q] = (att[2 * q] ? (v & 0xFFFFu) : 0u) | (att[2 * q + 1] ? (v & 0xFFFF0000u) : 0u);
+              pk[2 * g4 + q] = (attended(i, j, si.n, si.hist) ? (v & 0xFFFFu) : 0u) |
+                               (attended(i, j + 1, si.n, si.hist) ? (v & 0xFFFF0000u) : 0u);
             }
           }
         } else {
@@ -705,12 +749,94 @@ cudaError_t launch_tc(const AttnFwdParams& p, int grid, cudaStream_t st, double 
   return cudaGetLastError();
 }
 
+// Near-diagonal bias band: for token row i of a sequence and the 160 columns
+// j in [floor32(i) - 128, floor32(i) + 32), half of rab(i, j) as bf16, 0 where
+// (i, j) is not attended.  A warp of 32 rows starting at i0 (a multiple of 32)
+// reaches columns within 127 positions of its rows only in segments starting at
+// i0 - 128 ... i0, which the band covers, so the epilogue reads these biases
+// instead of evaluating both buckets per element there.
+// One block per group of 32 rows (four per 128-row tile of tile_base): the
+// group's 160 column timestamps are staged in shared memory, buckets follow the
+// 32-bit rule of the attention kernel (the 64-bit threshold search beyond it),
+// and the rows leave as 16-byte stores.
+constexpr int kBandCols = kBandChunks * 8;   // 160
+__global__ void __launch_bounds__(256) band_bias_kernel(const int32_t* __restrict__ offs,
+                                                        const int32_t* __restrict__ num_targets,
+                                                        const int64_t* __restrict__ ts, int B,
+                                                        const int32_t* __restrict__ tile_base,
+                                                        const float* __restrict__ pos_bias,
+                                                        const float* __restrict__ time_bias, const Thresholds thr_in,
+                                                        float ln2_over_div, int T,
+                                                        const int32_t* __restrict__ status,
+                                                        uint4* __restrict__ band) {
+  __shared__ int64_t thr[kNumBuckets];
+  __shared__ int32_t thr32[kNumBuckets + 4];
+  __shared__ float pb_s[kNumBuckets], tb_s[kNumBuckets];
+  __shared__ int64_t tcol[kBandCols];
+  __shared__ __align__(16) uint16_t out_s[32][kBandCols];
+  if (*status != 0) return;  // the scheduler found the offsets invalid
+  const int grp = blockIdx.x;
+  if (grp >= 4 * tile_base[B]) return;
+  const int t = grp >> 2;
+  int lo = 0, hi = B;  // sequence s with tile_base[s] <= t < tile_base[s + 1]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (tile_base[mid] <= t) lo = mid; else hi = mid;
+  }
+  const SeqInfo si = load_seq(offs, num_targets, lo);
+  const int i0 = (t - tile_base[lo]) * 128 + 32 * (grp & 3);
+  if (i0 >= si.n || si.start + si.n > T) return;
+  const int jb = i0 - 128;
+  for (int c = threadIdx.x; c < kNumBuckets + 4; c += blockDim.x) {
+    if (c < kNumBuckets) {
+      thr[c] = thr_in.v[c];
+      thr32[c] = thr_in.v[c] > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)thr_in.v[c];
+      pb_s[c] = pos_bias[c];
+      tb_s[c] = time_bias[c];
+    } else {
+      thr32[c] = 0x7FFFFFFF;
+    }
+  }
+  for (int w = threadIdx.x; w < kBandCols; w += blockDim.x) {
+    const int j = jb + w;
+    tcol[w] = (j >= 0 && j < si.n) ? ts[si.start + j] : 0;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 32 * kBandCols; e += blockDim.x) {
+    const int r = e / kBandCols, w = e - r * kBandCols;
+    const int i = i0 + r, j = jb + w;
+    float v = 0.f;
+    if (i < si.n && j >= 0 && attended(i, j, si.n, si.hist)) {
+      const int pb = pos_bucket(token_pos(i, si.hist), token_pos(j, si.hist));
+      const int64_t dt = abs_diff_i64(tcol[128 + r], tcol[w]);   // row i is column 128 + r of the window
+      const int tb = dt < 0x7FFFFFFF ? fast_bucket((int32_t)dt, thr32, ln2_over_div) : time_bucket_exact(dt, thr);
+      v = 0.5f * (pb_s[pb] + tb_s[tb]);
+    }
+    out_s[r][w] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+  __syncthreads();
+  const int rows = si.n - i0 < 32 ? si.n - i0 : 32;
+  for (int e = threadIdx.x; e < rows * kBandChunks; e += blockDim.x) {
+    const int r = e / kBandChunks, c = e - r * kBandChunks;
+    band[(int64_t)(si.start + i0 + r) * kBandChunks + c] = *reinterpret_cast<const uint4*>(&out_s[r][8 * c]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // diagnostics
 __global__ void debug_buckets_kernel(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,
-                                     const Thresholds thr_in, const int32_t* pairs, int n, int32_t* out) {
+                                     const Thresholds thr_in, float ln2_over_div, const int32_t* pairs, int n,
+                                     int32_t* out) {
   __shared__ int64_t thr[kNumBuckets];
-  for (int c = threadIdx.x; c < kNumBuckets; c += blockDim.x) thr[c] = thr_in.v[c];
+  __shared__ int32_t thr32[kNumBuckets + 4];
+  for (int c = threadIdx.x; c < kNumBuckets + 4; c += blockDim.x) {
+    if (c < kNumBuckets) {
+      thr[c] = thr_in.v[c];
+      thr32[c] = thr_in.v[c] > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)thr_in.v[c];
+    } else {
+      thr32[c] = 0x7FFFFFFF;
+    }
+  }
   __syncthreads();
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
     const SeqInfo si = load_seq(offs, num_targets, pairs[3 * e]);
@@ -718,7 +844,10 @@ __global__ void debug_buckets_kernel(const int32_t* offs, const int32_t* num_tar
     int pb = -1, tb = -1, att = 0;
     if (i >= 0 && i < si.n && j >= 0 && j < si.n) {
       pb = pos_bucket(token_pos(i, si.hist), token_pos(j, si.hist));
-      tb = time_bucket_exact(abs_diff_i64(ts[si.start + i], ts[si.start + j]), thr);
+      // the tensor-core kernel's rule: the 32-bit path below 2^31 - 1, else the
+      // 64-bit threshold search
+      const int64_t dt = abs_diff_i64(ts[si.start + i], ts[si.start + j]);
+      tb = dt < 0x7FFFFFFF ? fast_bucket((int32_t)dt, thr32, ln2_over_div) : time_bucket_exact(dt, thr);
       att = attended(i, j, si.n, si.hist) ? 1 : 0;
     }
     out[3 * e] = pb;
@@ -762,6 +891,19 @@ cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStr
 
 size_t ts_tiles_capacity(int B, int T) { return (size_t)T / BN + (size_t)B + 1; }
 
+size_t band_bytes(int T) { return (size_t)T * kBandChunks * 16; }
+
+cudaError_t launch_band_bias(const int32_t* offs, const int32_t* num_targets, const int64_t* ts, int B, int T,
+                             const int32_t* tile_base, int tiles_cap, const float* pos_bias,
+                             const float* time_bias, const Thresholds& thr, double time_div, const int32_t* status,
+                             void* band, cudaStream_t st) {
+  if (T <= 0 || B <= 0 || tiles_cap <= 0) return cudaSuccess;
+  band_bias_kernel<<<4 * tiles_cap, 256, 0, st>>>(offs, num_targets, ts, B, tile_base, pos_bias, time_bias, thr,
+                                                  (float)(0.69314718055994530942 / time_div), T, status,
+                                                  reinterpret_cast<uint4*>(band));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ts_tiles(const int32_t* offs, const int64_t* ts, int B, const int32_t* tile_base, int tiles_cap,
                             int32_t* recs, cudaStream_t st) {
   if (tiles_cap <= 0) return cudaSuccess;
@@ -770,9 +912,11 @@ cudaError_t launch_ts_tiles(const int32_t* offs, const int64_t* ts, int B, const
 }
 
 cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,
-                                 const Thresholds& thr, const int32_t* pairs, int n, int32_t* out, cudaStream_t st) {
+                                 const Thresholds& thr, double time_div, const int32_t* pairs, int n, int32_t* out,
+                                 cudaStream_t st) {
   const int grid = (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024;
-  debug_buckets_kernel<<<grid, 256, 0, st>>>(offs, num_targets, ts, thr, pairs, n, out);
+  debug_buckets_kernel<<<grid, 256, 0, st>>>(offs, num_targets, ts, thr, (float)(0.69314718055994530942 / time_div),
+                                             pairs, n, out);
   return cudaGetLastError();
 }
 

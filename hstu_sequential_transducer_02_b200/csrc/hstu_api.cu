@@ -127,6 +127,7 @@ struct AttnWs {
   int32_t* tile_base;   // tensor-core path: [B+1]
   int32_t* tile_recs;   // tensor-core path: timestamp records
   int tiles_cap;
+  void* band;           // tensor-core path, rab shared by heads: near-diagonal bias band
 };
 
 bool use_tc(const hstu_attn_desc* d) {
@@ -135,7 +136,7 @@ bool use_tc(const hstu_attn_desc* d) {
 
 int attn_tile(const hstu_attn_desc* d) { return use_tc(d) ? tc_tile_m() : simt_tile_m(); }
 
-AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd) {
+AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd, bool with_band = true) {
   AttnWs w;
   w.status = c.take<int32_t>(kStatusBytes / 4);
   w.count = c.take<int32_t>(64);
@@ -146,10 +147,12 @@ AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd) {
   w.tile_base = nullptr;
   w.tile_recs = nullptr;
   w.tiles_cap = 0;
+  w.band = nullptr;
   if (!bwd && use_tc(d)) {
     w.tiles_cap = (int)ts_tiles_capacity(B, T);
     w.tile_base = c.take<int32_t>((size_t)B + 1);
     w.tile_recs = c.take<int32_t>((size_t)w.tiles_cap * kTsRecWords);
+    if (with_band && d->rab_head_stride == 0) w.band = c.take<uint8_t>(band_bytes(T));
   }
   return w;
 }
@@ -168,6 +171,12 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   if (w.tile_recs) {
     TraceScope tr("ts_tiles", st);
     HSTU_CUDA(launch_ts_tiles(jb->seq_offsets, jb->timestamps, jb->batch, w.tile_base, w.tiles_cap, w.tile_recs, st));
+  }
+  if (w.band) {
+    TraceScope tr("band_bias", st);
+    HSTU_CUDA(launch_band_bias(jb->seq_offsets, jb->num_targets, jb->timestamps, jb->batch, jb->total_tokens,
+                               w.tile_base, w.tiles_cap, pos_bias, time_bias, thresholds_for(d->time_div),
+                               d->time_div, w.status, w.band, st));
   }
   AttnFwdParams p;
   memset(&p, 0, sizeof(p));
@@ -188,6 +197,7 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   p.tile_base = w.tile_base;
   p.tile_recs = w.tile_recs;
   p.item_cursor = w.count + 1;
+  p.band = w.band;
   if (use_tc(d)) {
     TraceScope tr("attn_fwd_tc", st);
     HSTU_CUDA(launch_attn_fwd_tc(p, d->dqk, tc_attn_grid(w.capacity), st, d->time_div));
@@ -777,8 +787,8 @@ int hstu_debug_rab_buckets(const hstu_attn_desc* desc, const hstu_jagged* jb, co
   if (num_pairs == 0) return HSTU_OK;
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   Thresholds thr = thresholds_for(desc->time_div);
-  return cuda_status(launch_debug_buckets(jb->seq_offsets, jb->num_targets, jb->timestamps, thr, pairs, num_pairs,
-                                          out, (cudaStream_t)stream));
+  return cuda_status(launch_debug_buckets(jb->seq_offsets, jb->num_targets, jb->timestamps, thr, desc->time_div,
+                                          pairs, num_pairs, out, (cudaStream_t)stream));
 }
 
 int hstu_debug_timeout_probe(int64_t timeout_ns, int32_t* status_dev, void* stream) {
@@ -844,15 +854,15 @@ extern "C" int hstu_attn_fwd_noalloc(const hstu_attn_desc* desc, const hstu_jagg
   HSTU_TRY(check_rows(v, ldv, hd, desc->dtype));
   HSTU_TRY(check_rows(out, ldo, hd, desc->dtype));
   if (!pos_bias || !time_bias) return HSTU_ERR_INVALID_ARG;
-  size_t need;
-  HSTU_TRY(hstu_attn_fwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
-  if (need > kNoAllocScratchBytes) return HSTU_ERR_WORKSPACE;  // problem larger than the fixed array
+  Carver sizer(nullptr);
+  carve_attn(sizer, desc, jb->batch, jb->total_tokens, false, false);  // without the bias band
+  if (sizer.size() > kNoAllocScratchBytes) return HSTU_ERR_WORKSPACE;  // problem larger than the fixed array
   void* scratch = nullptr;
   HSTU_TRY(noalloc_scratch(&scratch));
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
   Carver c(scratch);
-  AttnWs w = carve_attn(c, desc, jb->batch, jb->total_tokens, false);
+  AttnWs w = carve_attn(c, desc, jb->batch, jb->total_tokens, false, false);  // no band: bounded scratch
   HSTU_CUDA(cudaMemsetAsync(w.status, 0, kStatusBytes, st));  // the previous call's status must not leak
   return run_attn_fwd(desc, jb, q, ldq, k, ldk, v, ldv, pos_bias, time_bias, out, ldo, w, st);
 }

@@ -18,13 +18,23 @@ cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targe
 // first timestamp, with per-32-column min/max and a flag when any offset
 // leaves +-2^30 (record of kTsRecWords int32, 16-byte multiple).
 constexpr int kTsRecWords = 140;   // rel[128] | min[4] | max[4] | wide | pad[3]
+constexpr int kBandChunks = 20;    // 8-column bf16 chunks per row of the near-diagonal bias band
 size_t ts_tiles_capacity(int B, int T);
+
 cudaError_t launch_ts_tiles(const int32_t* offs, const int64_t* ts, int B, const int32_t* tile_base, int tiles_cap,
                             int32_t* recs, cudaStream_t st);
+
 
 // ---------------------------------------------------------------- attention
 // time-bucket thresholds, passed by value (kernel parameter space)
 struct Thresholds { int64_t v[kNumBuckets]; };
+
+size_t band_bytes(int T);
+cudaError_t launch_band_bias(const int32_t* offs, const int32_t* num_targets, const int64_t* ts, int B, int T,
+                             const int32_t* tile_base, int tiles_cap, const float* pos_bias,
+                             const float* time_bias, const Thresholds& thr, double time_div, const int32_t* status,
+                             void* band, cudaStream_t st);
+
 
 struct AttnFwdParams {
   const int32_t* seq_offsets;
@@ -47,6 +57,7 @@ struct AttnFwdParams {
   const int32_t* tile_base;    // tensor-core path: first tile record of each sequence
   const int32_t* tile_recs;    // tensor-core path: timestamp tile records
   int32_t* item_cursor;        // tensor-core path: dynamic work-list cursor (zeroed by the scheduler)
+  const void* band;            // tensor-core path: near-diagonal half-bias band (bf16), or null
 };
 
 struct AttnBwdParams {
@@ -87,7 +98,7 @@ cudaError_t launch_attn_fwd_tc(const AttnFwdParams& p, int dh, int grid, cudaStr
 int tc_attn_grid(int max_items);
 
 cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets, const int64_t* ts,
-                                 const Thresholds& thr, const int32_t* pairs, int n, int32_t* out,
+                                 const Thresholds& thr, double time_div, const int32_t* pairs, int n, int32_t* out,
                                  cudaStream_t st);
 cudaError_t launch_timeout_probe(long long timeout_ns, int32_t* status, cudaStream_t st);
 

@@ -251,6 +251,18 @@ __device__ __forceinline__ void half_plus2(float s0, float s1, float c, float& h
       : "f"(s0), "f"(s1), "f"(0.5f), "f"(c));
 }
 
+// (s0, s1) * 0.5 + (c0, c1) in one packed fp32 instruction
+__device__ __forceinline__ void half_plus2c(float s0, float s1, float c0, float c1, float& h0, float& h1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %4};\n\t"
+      "mov.b64 c, {%5, %6};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(h0), "=f"(h1)
+      : "f"(s0), "f"(s1), "f"(0.5f), "f"(c0), "f"(c1));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

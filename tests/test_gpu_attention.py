@@ -112,6 +112,40 @@ def test_rab_bucket_and_mask_dump_bit_exact():
     assert np.array_equal(got, np.array(want, dtype=np.int32))
 
 
+def _oracle_thresholds():
+    """Smallest |dt| of every time bucket, by bisection over the oracle's rule."""
+    thr = []
+    for b in range(128):
+        lo, hi = 0, 2 ** 62
+        while lo < hi:
+            mid = (lo + hi) // 2
+            if int(O.time_bucket(np.int64(mid))) >= b:
+                hi = mid
+            else:
+                lo = mid + 1
+        thr.append(lo)
+    return thr
+
+
+def test_time_bucket_at_every_threshold():
+    """The tensor-core kernel's 32-bit bucket rule (log estimate, exact compare
+    near a boundary) and the 64-bit search, bit-exact against the oracle at
+    every bucket threshold and three steps either side."""
+    b = _b()
+    ds = [0, 1, 2, 3, 2 ** 23 - 1, 2 ** 23, 2 ** 23 + 1, 2 ** 31 - 2, 2 ** 31 - 1, 2 ** 31, 2 ** 40 + 7]
+    for t in _oracle_thresholds():
+        ds += [d for d in range(t - 3, t + 4) if 0 <= d < 2 ** 45]
+    ds = np.array(sorted(set(ds)), dtype=np.int64)
+    base = 1_700_000_000
+    ts = np.concatenate([[base], base + ds]).astype(np.int64)   # row k > 0 is dt = ds[k-1] from row 0
+    n = len(ts)
+    offs = np.array([0, n], dtype=np.int32)
+    pairs = np.array([(0, k, 0) for k in range(1, n)] + [(0, 0, k) for k in range(1, n)], dtype=np.int32)
+    got = b.debug_rab_buckets(dev(offs), dev(ts), dev(pairs.reshape(-1)).reshape(-1, 3)).cpu().numpy()
+    want = O.time_bucket(np.concatenate([ds, ds]))
+    assert np.array_equal(got[:, 1], want.astype(np.int32))
+
+
 def test_bounded_wait_times_out_and_reports():
     b = _b()
     st = torch.full((1,), -1, dtype=torch.int32, device="cuda")

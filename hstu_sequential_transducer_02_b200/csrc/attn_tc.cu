@@ -755,24 +755,29 @@ cudaError_t launch_tc(const AttnFwdParams& p, int grid, cudaStream_t st, double 
 // reaches columns within 127 positions of its rows only in segments starting at
 // i0 - 128 ... i0, which the band covers, so the epilogue reads these biases
 // instead of evaluating both buckets per element there.
-// One block per group of 32 rows (four per 128-row tile of tile_base): the
-// group's 160 column timestamps are staged in shared memory, buckets follow the
-// 32-bit rule of the attention kernel (the 64-bit threshold search beyond it),
-// and the rows leave as 16-byte stores.
+// One block per group of 32 rows (four per 128-row tile of tile_base), one
+// thread per band column: timestamps become 32-bit offsets from the sequence's
+// first one (the 64-bit threshold search serves blocks whose offsets leave
+// +-2^30), buckets follow the 32-bit rule of the attention kernel, and the rows
+// leave as 16-byte stores.
 constexpr int kBandCols = kBandChunks * 8;   // 160
-__global__ void __launch_bounds__(256) band_bias_kernel(const int32_t* __restrict__ offs,
-                                                        const int32_t* __restrict__ num_targets,
-                                                        const int64_t* __restrict__ ts, int B,
-                                                        const int32_t* __restrict__ tile_base,
-                                                        const float* __restrict__ pos_bias,
-                                                        const float* __restrict__ time_bias, const Thresholds thr_in,
-                                                        float ln2_over_div, int T,
-                                                        const int32_t* __restrict__ status,
-                                                        uint4* __restrict__ band) {
+__device__ __noinline__ int band_bucket_wide(int64_t ti, int64_t tj, const int64_t* thr) {
+  return time_bucket_exact(abs_diff_i64(ti, tj), thr);
+}
+__global__ void __launch_bounds__(kBandCols) band_bias_kernel(const int32_t* __restrict__ offs,
+                                                              const int32_t* __restrict__ num_targets,
+                                                              const int64_t* __restrict__ ts, int B,
+                                                              const int32_t* __restrict__ tile_base,
+                                                              const float* __restrict__ pos_bias,
+                                                              const float* __restrict__ time_bias,
+                                                              const Thresholds thr_in, float ln2_over_div, int T,
+                                                              const int32_t* __restrict__ status,
+                                                              uint4* __restrict__ band) {
   __shared__ int64_t thr[kNumBuckets];
   __shared__ int32_t thr32[kNumBuckets + 4];
   __shared__ float pb_s[kNumBuckets], tb_s[kNumBuckets];
-  __shared__ int64_t tcol[kBandCols];
+  __shared__ int32_t rel_s[kBandCols];
+  __shared__ int64_t abs_s[kBandCols];
   __shared__ __align__(16) uint16_t out_s[32][kBandCols];
   if (*status != 0) return;  // the scheduler found the offsets invalid
   const int grp = blockIdx.x;
@@ -786,8 +791,9 @@ __global__ void __launch_bounds__(256) band_bias_kernel(const int32_t* __restric
   const SeqInfo si = load_seq(offs, num_targets, lo);
   const int i0 = (t - tile_base[lo]) * 128 + 32 * (grp & 3);
   if (i0 >= si.n || si.start + si.n > T) return;
-  const int jb = i0 - 128;
-  for (int c = threadIdx.x; c < kNumBuckets + 4; c += blockDim.x) {
+  const int w = threadIdx.x;
+  const int j = i0 - 128 + w;
+  for (int c = w; c < kNumBuckets + 4; c += kBandCols) {
     if (c < kNumBuckets) {
       thr[c] = thr_in.v[c];
       thr32[c] = thr_in.v[c] > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)thr_in.v[c];
@@ -797,26 +803,29 @@ __global__ void __launch_bounds__(256) band_bias_kernel(const int32_t* __restric
       thr32[c] = 0x7FFFFFFF;
     }
   }
-  for (int w = threadIdx.x; w < kBandCols; w += blockDim.x) {
-    const int j = jb + w;
-    tcol[w] = (j >= 0 && j < si.n) ? ts[si.start + j] : 0;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < 32 * kBandCols; e += blockDim.x) {
-    const int r = e / kBandCols, w = e - r * kBandCols;
-    const int i = i0 + r, j = jb + w;
+  const int64_t t_first = ts[si.start];
+  const int64_t tj = (j >= 0 && j < si.n) ? ts[si.start + j] : t_first;
+  const int64_t rel = tj - t_first;
+  const int64_t lim = (1ll << 30) - 1;
+  rel_s[w] = (int32_t)(rel < -lim ? -lim : (rel > lim ? lim : rel));
+  abs_s[w] = tj;
+  const bool wide = __syncthreads_or(rel < -lim || rel > lim) != 0;
+  const int32_t relj = rel_s[w];
+  const int posj = token_pos(j, si.hist);
+  const int rows = si.n - i0 < 32 ? si.n - i0 : 32;
+  for (int r = 0; r < rows; ++r) {
+    const int i = i0 + r;
     float v = 0.f;
-    if (i < si.n && j >= 0 && attended(i, j, si.n, si.hist)) {
-      const int pb = pos_bucket(token_pos(i, si.hist), token_pos(j, si.hist));
-      const int64_t dt = abs_diff_i64(tcol[128 + r], tcol[w]);   // row i is column 128 + r of the window
-      const int tb = dt < 0x7FFFFFFF ? fast_bucket((int32_t)dt, thr32, ln2_over_div) : time_bucket_exact(dt, thr);
+    if (j >= 0 && attended(i, j, si.n, si.hist)) {
+      const int pb = pos_bucket(token_pos(i, si.hist), posj);
+      const int tb = wide ? band_bucket_wide(abs_s[128 + r], tj, thr)     // row i is window column 128 + r
+                          : fast_bucket(abs(rel_s[128 + r] - relj), thr32, ln2_over_div);
       v = 0.5f * (pb_s[pb] + tb_s[tb]);
     }
     out_s[r][w] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
   __syncthreads();
-  const int rows = si.n - i0 < 32 ? si.n - i0 : 32;
-  for (int e = threadIdx.x; e < rows * kBandChunks; e += blockDim.x) {
+  for (int e = w; e < rows * kBandChunks; e += kBandCols) {
     const int r = e / kBandChunks, c = e - r * kBandChunks;
     band[(int64_t)(si.start + i0 + r) * kBandChunks + c] = *reinterpret_cast<const uint4*>(&out_s[r][8 * c]);
   }
@@ -898,7 +907,7 @@ cudaError_t launch_band_bias(const int32_t* offs, const int32_t* num_targets, co
                              const float* time_bias, const Thresholds& thr, double time_div, const int32_t* status,
                              void* band, cudaStream_t st) {
   if (T <= 0 || B <= 0 || tiles_cap <= 0) return cudaSuccess;
-  band_bias_kernel<<<4 * tiles_cap, 256, 0, st>>>(offs, num_targets, ts, B, tile_base, pos_bias, time_bias, thr,
+  band_bias_kernel<<<4 * tiles_cap, kBandCols, 0, st>>>(offs, num_targets, ts, B, tile_base, pos_bias, time_bias, thr,
                                                   (float)(0.69314718055994530942 / time_div), T, status,
                                                   reinterpret_cast<uint4*>(band));
   return cudaGetLastError();

@@ -588,6 +588,196 @@ __global__ void zero_tail_rows_kernel(uint32_t* __restrict__ buf, int64_t ld_wor
     buf[(rows + e / row_words) * ld_words + e % row_words] = 0u;
 }
 
+
+// ---------------------------------------------------------------- LayerNorm, d = 256 * NCH
+// One warp per row as above, but gamma and beta stay in registers for all of the
+// warp's rows and the next row is loaded (as raw 16-byte vectors) while the
+// current one is normalised, so each warp keeps two rows of loads in flight.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ void get(float v[8]) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = *reinterpret_cast<const float4*>(p);
+    b = *reinterpret_cast<const float4*>(p + 4);
+  }
+  __device__ __forceinline__ void get(float v[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+template <int NCH>
+__device__ __forceinline__ void row_stats(const float (&v)[NCH][8], float eps, float& mean, float& rstd) {
+  constexpr float inv_d = 1.0f / (256 * NCH);
+  float sm = 0.f;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sm += v[c][e];
+  mean = warp_sum(sm) * inv_d;
+  float q = 0.f;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { const float t = v[c][e] - mean; q = fmaf(t, t, q); }
+  rstd = 1.0f / sqrtf(warp_sum(q) * inv_d + eps);
+}
+
+template <typename T, typename TO, int NCH>
+__global__ void __launch_bounds__(kRowWarps * 32, 2)
+layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma, const float* __restrict__ beta,
+                float eps, TO* __restrict__ out, int64_t ldo, float* __restrict__ mean_out,
+                float* __restrict__ rstd_out, int rows_cap, const int32_t* __restrict__ rows_dev) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * kRowWarps;
+  float g[NCH][8], b[NCH][8];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    load8(gamma + (lane + 32 * c) * 8, g[c]);
+    load8(beta + (lane + 32 * c) * 8, b[c]);
+  }
+  int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  Raw8<T> cur[NCH];
+  if (row < rows)
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) cur[c].load(x + (int64_t)row * ldx + (lane + 32 * c) * 8);
+  for (; row < rows; row += stride) {
+    Raw8<T> nxt[NCH];
+    if (row + stride < rows)
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) nxt[c].load(x + (int64_t)(row + stride) * ldx + (lane + 32 * c) * 8);
+    float v[NCH][8];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) cur[c].get(v[c]);
+    float mean, rstd;
+    row_stats<NCH>(v, eps, mean, rstd);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      float o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = fmaf((v[c][e] - mean) * rstd, g[c][e], b[c][e]);
+      store8(out + (int64_t)row * ldo + (lane + 32 * c) * 8, o);
+    }
+    if (lane == 0) {
+      if (mean_out) mean_out[row] = mean;
+      if (rstd_out) rstd_out[row] = rstd;
+    }
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) cur[c] = nxt[c];
+  }
+}
+
+// g = LN(o) * u, d = 256 * NCH
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kRowWarps * 32, 2)
+ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
+             const float* __restrict__ gamma, const float* __restrict__ beta, float eps, T* __restrict__ out,
+             int64_t ldout, float* __restrict__ mean_out, float* __restrict__ rstd_out, int rows_cap,
+             const int32_t* __restrict__ rows_dev) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * kRowWarps;
+  float g[NCH][8], b[NCH][8];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    load8(gamma + (lane + 32 * c) * 8, g[c]);
+    load8(beta + (lane + 32 * c) * 8, b[c]);
+  }
+  int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  Raw8<T> co[NCH], cu[NCH];
+  if (row < rows)
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      co[c].load(o + (int64_t)row * ldo_in + (lane + 32 * c) * 8);
+      cu[c].load(u + (int64_t)row * ldu + (lane + 32 * c) * 8);
+    }
+  for (; row < rows; row += stride) {
+    Raw8<T> no[NCH], nu[NCH];
+    if (row + stride < rows)
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        no[c].load(o + (int64_t)(row + stride) * ldo_in + (lane + 32 * c) * 8);
+        nu[c].load(u + (int64_t)(row + stride) * ldu + (lane + 32 * c) * 8);
+      }
+    float v[NCH][8];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) co[c].get(v[c]);
+    float mean, rstd;
+    row_stats<NCH>(v, eps, mean, rstd);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      float uu[8], r[8];
+      cu[c].get(uu);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[e] = fmaf((v[c][e] - mean) * rstd, g[c][e], b[c][e]) * uu[e];
+      store8(out + (int64_t)row * ldout + (lane + 32 * c) * 8, r);
+    }
+    if (lane == 0) {
+      if (mean_out) mean_out[row] = mean;
+      if (rstd_out) rstd_out[row] = rstd;
+    }
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) { co[c] = no[c]; cu[c] = nu[c]; }
+  }
+}
+
+// grid of the register-resident row kernels: a few blocks per SM, each warp
+// walking rows with a grid-sized stride
+int rows_grid(int rows_cap) {
+  const int g = (rows_cap + kRowWarps - 1) / kRowWarps;
+  return g < 1 ? 1 : (g > 148 * 4 ? 148 * 4 : g);
+}
+
+template <typename T, typename TO>
+cudaError_t launch_ln_rows(const T* x, int64_t ldx, const float* gamma, const float* beta, float eps, TO* out,
+                           int64_t ldo, float* mean, float* rstd, int rows_cap, const int32_t* rows_dev, int d,
+                           cudaStream_t st) {
+  const int g = rows_grid(rows_cap), t = kRowWarps * 32;
+  switch (d / 256) {
+    case 1: layer_norm_rows<T, TO, 1><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    case 2: layer_norm_rows<T, TO, 2><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    case 3: layer_norm_rows<T, TO, 3><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    default: layer_norm_rows<T, TO, 4><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_ln_gate_rows(const T* o, int64_t ldo_in, const T* u, int64_t ldu, const float* gamma,
+                                const float* beta, float eps, T* out, int64_t ldout, float* mean, float* rstd,
+                                int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
+  const int g = rows_grid(rows_cap), t = kRowWarps * 32;
+  switch (d / 256) {
+    case 1: ln_gate_rows<T, 1><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    case 2: ln_gate_rows<T, 2><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    case 3: ln_gate_rows<T, 3><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    default: ln_gate_rows<T, 4><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+  }
+  return cudaGetLastError();
+}
+
+bool fast_rows_ok(int d, const void* a, int64_t lda, const void* b, int64_t ldb, const void* c, int64_t ldc,
+                  int esize_ab, int esize_c) {
+  if (d % 256 || d / 256 < 1 || d / 256 > 4) return false;
+  auto al = [](const void* p) { return ((uintptr_t)p & 15) == 0; };
+  if (!al(a) || !al(c) || (b && !al(b))) return false;
+  if ((lda * esize_ab) % 16 || (ldc * esize_c) % 16 || (b && (ldb * esize_ab) % 16)) return false;
+  return true;
+}
+
 int row_grid(int rows_cap) {
   int g = (rows_cap + kRowWarps - 1) / kRowWarps;
   return g < 1 ? 1 : (g > 148 * 16 ? 148 * 16 : g);
@@ -599,9 +789,23 @@ cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const flo
                               float eps, void* out, int64_t ldo, int out_dtype, float* mean, float* rstd,
                               int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
   if (rows_cap <= 0) return cudaSuccess;
+  using bf = __nv_bfloat16;
+  const int xs = x_dtype == HSTU_DTYPE_F32 ? 4 : 2, os = out_dtype == HSTU_DTYPE_F32 ? 4 : 2;
+  if (fast_rows_ok(d, x, ldx, nullptr, 0, out, ldo, xs, os) && gamma && beta) {
+    if (x_dtype == HSTU_DTYPE_F32 && out_dtype == HSTU_DTYPE_F32)
+      return launch_ln_rows<float, float>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean, rstd,
+                                          rows_cap, rows_dev, d, st);
+    if (x_dtype == HSTU_DTYPE_F32)
+      return launch_ln_rows<float, bf>((const float*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd, rows_cap,
+                                       rows_dev, d, st);
+    if (out_dtype == HSTU_DTYPE_F32)
+      return launch_ln_rows<bf, float>((const bf*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean, rstd, rows_cap,
+                                       rows_dev, d, st);
+    return launch_ln_rows<bf, bf>((const bf*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd, rows_cap,
+                                  rows_dev, d, st);
+  }
   const int g = row_grid(rows_cap);
   const int t = kRowWarps * 32;
-  using bf = __nv_bfloat16;
   if (x_dtype == HSTU_DTYPE_F32 && out_dtype == HSTU_DTYPE_F32)
     layer_norm_kernel<float, float><<<g, t, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean,
                                                      rstd, rows_cap, rows_dev, d);
@@ -621,6 +825,15 @@ cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t
                            const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
                            int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
   if (rows_cap <= 0) return cudaSuccess;
+  const int es = dtype == HSTU_DTYPE_F32 ? 4 : 2;
+  if (fast_rows_ok(d, o, ldo_in, u, ldu, out, ldout, es, es) && gamma && beta) {
+    if (dtype == HSTU_DTYPE_F32)
+      return launch_ln_gate_rows<float>((const float*)o, ldo_in, (const float*)u, ldu, gamma, beta, eps, (float*)out,
+                                        ldout, mean, rstd, rows_cap, rows_dev, d, st);
+    return launch_ln_gate_rows<__nv_bfloat16>((const __nv_bfloat16*)o, ldo_in, (const __nv_bfloat16*)u, ldu, gamma,
+                                              beta, eps, (__nv_bfloat16*)out, ldout, mean, rstd, rows_cap, rows_dev,
+                                              d, st);
+  }
   const int g = row_grid(rows_cap);
   if (dtype == HSTU_DTYPE_F32)
     ln_gate_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)o, ldo_in, (const float*)u, ldu, gamma, beta,

@@ -17,6 +17,7 @@ namespace {
 
 constexpr int kVersion = 10000;  // 1.0.0
 constexpr long long kDefaultTimeoutNs = 2000000000ll;  // a device-side wait gives up after 2 s
+constexpr int kMaxDevices = 64;                        // per-device caches (side stream, scratch address)
 
 // ---------------------------------------------------------------- workspace carving
 struct Carver {
@@ -157,9 +158,10 @@ AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd, bo
   return w;
 }
 
-int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
-                 int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias, void* out,
-                 int64_t ldo, const AttnWs& w, cudaStream_t st) {
+// The attention's preparation (work list, timestamp tile records, bias band)
+// depends only on the offsets, timestamps and bias tables, not on Q, K, V.
+int run_attn_prep(const hstu_attn_desc* d, const hstu_jagged* jb, const float* pos_bias, const float* time_bias,
+                  const AttnWs& w, cudaStream_t st) {
   const int tile = attn_tile(d);
   {
     // tensor-core path: locality order, fetched dynamically (count[1] is the cursor)
@@ -178,6 +180,12 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
                                w.tile_base, w.tiles_cap, pos_bias, time_bias, thresholds_for(d->time_div),
                                d->time_div, w.status, w.band, st));
   }
+  return HSTU_OK;
+}
+
+int run_attn_main(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                  int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias, void* out,
+                  int64_t ldo, const AttnWs& w, cudaStream_t st) {
   AttnFwdParams p;
   memset(&p, 0, sizeof(p));
   p.seq_offsets = jb->seq_offsets;
@@ -206,6 +214,39 @@ int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
     int grid = w.capacity < 148 * 4 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 4;
     HSTU_CUDA(launch_attn_fwd_simt(p, d->dtype, d->dqk, grid, st));
   }
+  return HSTU_OK;
+}
+
+int run_attn_fwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                 int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias, void* out,
+                 int64_t ldo, const AttnWs& w, cudaStream_t st) {
+  HSTU_TRY(run_attn_prep(d, jb, pos_bias, time_bias, w, st));
+  return run_attn_main(d, jb, q, ldq, k, ldk, v, ldv, pos_bias, time_bias, out, ldo, w, st);
+}
+
+// ---------------------------------------------------------------- side stream
+// One non-blocking stream per device on which the layer forward runs the
+// attention preparation while LayerNorm1 and f1 run on the caller's stream;
+// fork and join through events.  Record-and-wait pairs are made under a mutex;
+// a join that waits for a later record (another caller's) still implies this
+// caller's work, which precedes it on the same in-order stream.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[kMaxDevices];
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
+  SideStream& ss = g_side[dev];
+  if (!ss.s) {
+    HSTU_CUDA(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
+    HSTU_CUDA(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
+    HSTU_CUDA(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+  }
+  *out = &ss;
   return HSTU_OK;
 }
 
@@ -317,6 +358,16 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
     b.xhat = saved->xhat; b.mu1 = saved->ln1_mean; b.rs1 = saved->ln1_rstd; b.z = saved->z;
     b.uvqk = saved->uvqk; b.o = saved->attn_out; b.mu2 = saved->ln2_mean; b.rs2 = saved->ln2_rstd;
   }
+  // attention preparation on the side stream, overlapping LayerNorm1 and f1
+  SideStream* side = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    HSTU_TRY(side_stream(&side));
+    HSTU_CUDA(cudaEventRecord(side->fork, st));
+    HSTU_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    HSTU_TRY(run_attn_prep(&d->attn, jb, w->pos_bias, w->time_bias, ws.attn, side->s));
+    HSTU_CUDA(cudaEventRecord(side->join, side->s));
+  }
   // (A1) LayerNorm1
   {
     TraceScope tr("ln1", st);
@@ -338,8 +389,9 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   // (A2-A4) attention
   const size_t es = elem_size(dt);
   const char* uvqk = (const char*)b.uvqk;
-  HSTU_TRY(run_attn_fwd(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + 1 * hv * es,
-                        4 * hv, w->pos_bias, w->time_bias, b.o, hv, ws.attn, st));
+  HSTU_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  HSTU_TRY(run_attn_main(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + 1 * hv * es,
+                         4 * hv, w->pos_bias, w->time_bias, b.o, hv, ws.attn, st));
   // (A5) LayerNorm2(A V) * U
   {
     TraceScope tr("ln2_gate", st);
@@ -821,7 +873,6 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 1u << 20;  // 1 MiB
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 

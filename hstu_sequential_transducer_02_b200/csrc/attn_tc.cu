@@ -403,6 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       const int posi = token_pos(i, si.hist);
       const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
       const int nk = kv_count(kr);
+      // this row's last one-bucket segment: distances in [c_lo, c_hi) share the
+      // bias 2 * c_hb (empty until the first one); far from the diagonal the bucket
+      // rarely changes from one kv tile to the next
+      int32_t c_lo = 0x7FFFFFFF, c_hi = 0;
+      float c_hb = 0.f;
       for (int jj = 0; jj < nk; ++jj, ++it) {
         const int c0 = kv_tile_at(kr, jj) * BN;
         const int sb = it % kSBufs;
@@ -431,11 +436,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
           if (ri >= mx) { dlo = ri - mx; dhi = ri - mn; }
           else if (ri <= mn) { dlo = mn - ri; dhi = mx - ri; }
           else { dlo = 0; dhi = max(ri - mn, mx - ri); }
+          if (dlo >= c_lo && dhi < c_hi) {
+            rank = 1;
+            hb0 = c_hb;
+          } else {
           const int tlo = fast_bucket(dlo, thr32, k_lg);
           const float pb127 = pos_b[kNumBuckets - 1];
           hb0 = 0.5f * (pb127 + time_b[tlo]);
           if (dhi < thr32[tlo + 1]) {
             rank = 1;
+            c_lo = thr32[tlo];
+            c_hi = thr32[tlo + 1];
+            c_hb = hb0;
           } else {
             const int thi = fast_bucket(dhi, thr32, k_lg);
             if (thi - tlo <= 3) {
@@ -445,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
               if (thi - tlo >= 2) { hb2 = 0.5f * (pb127 + time_b[tlo + 2]); th2 = thr32[tlo + 2]; }
               if (thi - tlo >= 3) { hb3 = 0.5f * (pb127 + time_b[tlo + 3]); th3 = thr32[tlo + 3]; }
             }
+          }
           }
         }
         // one path per warp: the highest rank of its rows (a lower rank's row is a

@@ -48,6 +48,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the M-FALCON and training-step measurements")
     return ap.parse_args()
 
 
@@ -372,6 +373,121 @@ def read_traffic(kernel: str):
     return None
 
 
+
+# ----------------------------------------------------------------------------
+# further rows of the path, measured on their own workloads (1 GPU)
+# ----------------------------------------------------------------------------
+
+def _trace_attention(trace, name, flops):
+    a = trace.get(name)
+    if not a or not a["count"]:
+        return None
+    ms = a["ms"] / a["count"]
+    return {"kernel": name, "launches": a["count"], "ms_per_launch": ms,
+            "tflops": flops / a["count"] / (ms / 1e3) / 1e12 if flops else None}  # flops: all traced launches
+
+
+def measure_mfalcon(hb, steps: int):
+    """M-FALCON ranking (16 users, n = 2048 history, m = 4096 candidates in
+    microbatches of b_m = 512, d_model = 256, 2 heads of 128, 1 layer):
+    candidates scored per second through mfalcon_rank."""
+    import torch
+    wl = W.make_workload(3)
+    sp, e = wl.spec, wl.extras
+    td = torch.bfloat16
+    layer = hb.Layer(hb.layer_weights_to_device(wl.layers[0], td), sp.d_model, sp.num_heads, sp.head_dim)
+    bm = int(e["microbatch"])
+    m_max = int(np.max(np.diff(e["cand_offsets"])))
+    args = (torch.from_numpy(wl.seq_offsets).cuda(), torch.from_numpy(wl.x).to(td).cuda(),
+            torch.from_numpy(wl.timestamps).cuda(), torch.from_numpy(e["cand_offsets"]).cuda(),
+            torch.from_numpy(e["cand_x"]).to(td).cuda(), torch.from_numpy(e["cand_ts"]).cuda())
+    out = hb.mfalcon_rank([layer], *args, bm, m_max)
+    for _ in range(2):
+        hb.mfalcon_rank([layer], *args, bm, m_max, out=out)
+    torch.cuda.synchronize()
+    hb.trace_enable(True)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        hb.mfalcon_rank([layer], *args, bm, m_max, out=out)
+    t1.record()
+    torch.cuda.synchronize()
+    trace = hb.trace_read()
+    hb.trace_enable(False)
+    ms = t0.elapsed_time(t1) / steps
+    U = len(wl.seq_offsets) - 1
+    n = int(np.diff(wl.seq_offsets)[0])
+    cands = int(e["cand_offsets"][-1])
+    mbs = (m_max + bm - 1) // bm
+    pairs = U * mbs * (n * (n + 1) // 2) + cands * (n + 1)   # history recomputed per microbatch
+    flops = pairs * 2 * 2 * sp.head_dim * sp.num_heads
+    return {"workload": f"M-FALCON: {U} users, n={n} history, m={cands // U} candidates, b_m={bm}, "
+                        f"d_model={sp.d_model}, {sp.num_heads} heads x {sp.head_dim}, 1 layer",
+            "candidates_per_s": cands / (ms / 1e3), "ms_per_call": ms, "calls": steps,
+            "attention": _trace_attention(trace, "attn_fwd_tc", flops * steps)}
+
+
+def measure_training(hb, steps: int):
+    """Training step of the 8-layer stack (64 sequences, power-law lengths in
+    [64, 4096] cut by Stochastic Length to 1024 with p = 0.8, d_model = 512, 8
+    heads of 64, fp32 residual stream): SL, forward with saved activations,
+    backward from dY = G; tokens (after SL) per second."""
+    import torch
+    wl = W.make_workload(4)
+    sp, e = wl.spec, wl.extras
+    td, io = torch.bfloat16, torch.float32
+    layers = [hb.Layer(hb.layer_weights_to_device(p_, td), sp.d_model, sp.num_heads, sp.head_dim,
+                       residual_fp32=True) for p_ in wl.layers]
+    offs_in = torch.from_numpy(wl.seq_offsets).cuda()
+    coins = torch.from_numpy(e["sl_coin"].view(np.int32)).cuda()
+    keys = torch.from_numpy(e["sl_keys"].view(np.int32)).cuda()
+    x_all = torch.from_numpy(wl.x).to(io).cuda()
+    ts_all = torch.from_numpy(wl.timestamps).cuda()
+    g_all = torch.from_numpy(e["grad_out"]).to(io).cuda()
+    hv = sp.num_heads * sp.head_dim
+    T_cap = wl.total_tokens
+    x = torch.empty(T_cap, sp.d_model, dtype=io, device="cuda")
+    ts = torch.empty(T_cap, dtype=torch.int64, device="cuda")
+    gy = torch.empty_like(x)
+    saved = [hb.Saved.alloc(T_cap, sp.d_model, hv, td, "cuda") for _ in layers]
+    acts = [torch.empty_like(x) for _ in layers]
+
+    def step():
+        offs, idx = hb.stochastic_length(offs_in, coins, keys, int(e["sl_len"]), int(e["sl_prob_u32"]))
+        cnt = offs[-1:]
+        hb.gather_rows(x_all, idx, cnt, x)
+        hb.gather_rows(ts_all, idx, cnt, ts)
+        hb.gather_rows(g_all, idx, cnt, gy)
+        h = x
+        for ly, sv, a in zip(layers, saved, acts):
+            h = ly.forward(h, offs, ts, saved=sv, out=a)
+        dy = gy
+        ins = [x] + acts[:-1]
+        for li in range(len(layers) - 1, -1, -1):
+            dy, _ = layers[li].backward(ins[li], dy, saved[li], offs, ts)
+        return offs
+
+    offs = step()
+    torch.cuda.synchronize()
+    T2 = int(offs[-1].item())
+    hb.trace_enable(True)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    trace = hb.trace_read()
+    hb.trace_enable(False)
+    ms = t0.elapsed_time(t1) / steps
+    tot = sum(v["ms"] for v in trace.values()) or 1e-9
+    top = sorted(trace.items(), key=lambda kv: -kv[1]["ms"])[:6]
+    return {"workload": f"training step: 8 layers, B=64, power-law n in [64,4096], SL to 1024 (p=0.8) -> "
+                        f"T={T2} tokens, d_model={sp.d_model}, {sp.num_heads} heads x {sp.head_dim}, "
+                        "fp32 residual stream, forward + backward",
+            "tokens_per_s": T2 / (ms / 1e3), "ms_per_step": ms, "steps": steps,
+            "top_kernels": {k: {"share": v["ms"] / tot, "ms_per_step": v["ms"] / steps} for k, v in top}}
+
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
@@ -496,6 +612,9 @@ def main():
             "gpu_launches": launches,
             "clocks": clk,
         }
+        if world == 1 and not args.no_extra:
+            line["mfalcon"] = measure_mfalcon(hb, 5)
+            line["training"] = measure_training(hb, 3)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.oracle_seconds)
         print(json.dumps(line), flush=True)

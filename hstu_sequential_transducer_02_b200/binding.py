@@ -219,12 +219,12 @@ def attn_fwd(q, k, v, seq_offsets, timestamps, pos_bias, time_bias, num_heads: i
 
 
 def attn_bwd(q, k, v, dout, seq_offsets, timestamps, pos_bias, time_bias, num_heads: int, num_targets=None,
-             time_div: float = 0.301, stream=None):
+             time_div: float = 0.301, stream=None, force_simt: bool = False):
     """Returns dq, dk, dv ([T, H*dh], dtype of q) and the rab gradients (float, table shape)."""
     T = q.shape[0]
     dh = q.shape[1] // num_heads
     dt = _dtype_code(q)
-    d = attn_desc(num_heads, dh, dt, pos_bias.dim() == 2, False, time_div)
+    d = attn_desc(num_heads, dh, dt, pos_bias.dim() == 2, force_simt, time_div)
     jb = jagged(seq_offsets, timestamps, T, num_targets)
     nbytes = _c_size()
     _check(_lib_attn_bwd_ws(ctypes.byref(d), jb.batch, T, ctypes.byref(nbytes)), "hstu_attn_bwd_workspace_size")

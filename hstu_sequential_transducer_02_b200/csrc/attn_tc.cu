@@ -112,33 +112,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
 // to the nearest integer is at most one bucket off, and one comparison with
 // each neighbouring integer threshold corrects it (thr32[b] = min(threshold b,
 // INT32_MAX), thr32[128] = INT32_MAX).
-// Exact time bucket floor(ln(d) / div) of 1 <= d < 2^31 with few shared-memory
-// reads.  y = log2(d) * ln2/div comes from the special-function unit; its error
-// is below 2e-4 (the log2 approximation, float rounding of y < 72, and for
-// d >= 2^23 the eight dropped low bits), so floor(y) is the bucket unless y lies
-// within 2^-9 of an integer.  Only such lanes read one threshold (thr32[b] =
-// smallest d of bucket b, clamped to INT32_MAX; thr32[128] = INT32_MAX) and
-// settle the bucket with an exact integer compare.
-__device__ __forceinline__ int exact_bucket(int32_t d, const int32_t* thr32, float ln2_over_div) {
-  const bool big = d >= (1 << 23);
-  const float f = __int_as_float(0x4B000000 | (big ? d >> 8 : d)) - 8388608.0f;  // exact: < 2^23
-  const float y = (__log2f(f) + (big ? 8.0f : 0.0f)) * ln2_over_div;
-  const float t = (y - 0.5f) + 12582912.0f;                 // round(y - 1/2) = floor(y) off the integers
-  const float fr = y - (t - 12582912.0f);                   // y - floor(y)
-  int b = __float_as_int(t) - 0x4B400000;
-  b = b < 0 ? 0 : (b > kNumBuckets - 1 ? kNumBuckets - 1 : b);
-  if (fr < 0.001953125f || fr > 0.998046875f) {
-    const bool up = fr > 0.5f;
-    const int32_t th = thr32[up ? b + 1 : b];
-    b += up ? (d >= th ? 1 : 0) : (d < th ? -1 : 0);
-    b = b < 0 ? 0 : (b > kNumBuckets - 1 ? kNumBuckets - 1 : b);
-  }
-  return b;
-}
-__device__ __forceinline__ int fast_bucket(int32_t d, const int32_t* thr32, float ln2_over_div) {
-  return exact_bucket(d < 1 ? 1 : d, thr32, ln2_over_div);
-}
-
 // Waits for outstanding tcgen05.ld into `r`; the register operands keep the
 // compiler from reading them earlier.
 __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {

@@ -137,11 +137,17 @@ bool use_tc(const hstu_attn_desc* d) {
 
 int attn_tile(const hstu_attn_desc* d) { return use_tc(d) ? tc_tile_m() : simt_tile_m(); }
 
+bool use_tc_bwd(const hstu_attn_desc* d) {
+  return !(d->flags & HSTU_FLAG_FORCE_SIMT) && tc_attn_bwd_supported(d->dtype, d->dqk) && d->dqk == d->dv;
+}
+
+int attn_bwd_tile(const hstu_attn_desc* d) { return use_tc_bwd(d) ? tc_bwd_tile() : simt_tile_m(); }
+
 AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd, bool with_band = true) {
   AttnWs w;
   w.status = c.take<int32_t>(kStatusBytes / 4);
   w.count = c.take<int32_t>(64);
-  const int tile = bwd ? simt_tile_m() : attn_tile(d);
+  const int tile = bwd ? attn_bwd_tile(d) : attn_tile(d);
   w.capacity = (int)work_list_capacity(B, T, d->num_heads, tile);
   w.items = c.take<WorkItem>(w.capacity);
   w.dq_accum = bwd ? c.take<float>((size_t)T * d->num_heads * d->dqk) : nullptr;
@@ -254,7 +260,7 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
                  int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias,
                  const void* dout, int64_t lddo, void* dq, int64_t lddq, void* dk, int64_t lddk, void* dv,
                  int64_t lddv, float* dpos, float* dtime, const AttnWs& w, cudaStream_t st) {
-  const int tile = simt_tile_m();
+  const int tile = attn_bwd_tile(d);
   const int H = d->num_heads, dh = d->dqk;
   {
     TraceScope tr("sched_bwd", st);
@@ -281,9 +287,13 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   p.item_count = w.count;
   p.status = w.status;
   p.timeout_ns = kDefaultTimeoutNs;
-  int grid = w.capacity < 148 * 2 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 2;
-  {
+  if (use_tc_bwd(d)) {
+    TraceScope tr("attn_bwd_tc", st);
+    const int grid = w.capacity < 148 ? (w.capacity > 0 ? w.capacity : 1) : 148;
+    HSTU_CUDA(launch_attn_bwd_tc(p, grid, st, d->time_div));
+  } else {
     TraceScope tr("attn_bwd_simt", st);
+    const int grid = w.capacity < 148 * 2 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 2;
     HSTU_CUDA(launch_attn_bwd_simt(p, d->dtype, dh, grid, st));
   }
   {

@@ -88,6 +88,10 @@ struct AttnBwdParams {
 int simt_tile_m();
 cudaError_t launch_attn_fwd_simt(const AttnFwdParams& p, int dtype, int dh, int grid, cudaStream_t st);
 cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, int dtype, int dh, int grid, cudaStream_t st);
+// tcgen05 (sm_100a) attention backward, bf16, dh = 64
+bool tc_attn_bwd_supported(int dtype, int dh);
+int tc_bwd_tile();
+cudaError_t launch_attn_bwd_tc(const AttnBwdParams& p, int grid, cudaStream_t st, double time_div);
 cudaError_t launch_dq_finalize(const float* acc, const int32_t* offs, int B, int H, int dh, int dtype,
                                void* dq, int64_t lddq, int grid, cudaStream_t st);
 

@@ -358,9 +358,17 @@ __global__ void col_sum_kernel(const T* __restrict__ a, int64_t lda, int rows_ca
   if (col >= cols) return;
   const int chunk = (rows + gridDim.y - 1) / gridDim.y;
   const int r0 = blockIdx.y * chunk, r1 = min(rows, r0 + chunk);
-  float s = 0.f;
-  for (int r = r0; r < r1; ++r) s += Elem<T>::to_f(a[(int64_t)r * lda + col]);
-  if (r1 > r0) atomicAdd(&out[col], s);
+  // four independent partial sums keep several loads in flight per thread
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  int r = r0;
+  for (; r + 3 < r1; r += 4) {
+    s0 += Elem<T>::to_f(a[(int64_t)r * lda + col]);
+    s1 += Elem<T>::to_f(a[(int64_t)(r + 1) * lda + col]);
+    s2 += Elem<T>::to_f(a[(int64_t)(r + 2) * lda + col]);
+    s3 += Elem<T>::to_f(a[(int64_t)(r + 3) * lda + col]);
+  }
+  for (; r < r1; ++r) s0 += Elem<T>::to_f(a[(int64_t)r * lda + col]);
+  if (r1 > r0) atomicAdd(&out[col], (s0 + s1) + (s2 + s3));
 }
 
 __global__ void gather_rows_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst, int64_t words,
@@ -913,7 +921,9 @@ cudaError_t launch_col_sum(const void* a, int64_t lda, int rows_cap, const int32
                            int dtype, float* out, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * cols, st);
   if (e != cudaSuccess || rows_cap <= 0) return e;
-  dim3 grid((cols + 255) / 256, 64);
+  // about 64 rows per thread
+  const int chunks = rows_cap / 64 < 1 ? 1 : (rows_cap / 64 > 4096 ? 4096 : rows_cap / 64);
+  dim3 grid((cols + 255) / 256, chunks);
   if (dtype == HSTU_DTYPE_F32)
     col_sum_kernel<float><<<grid, 256, 0, st>>>((const float*)a, lda, rows_cap, rows_dev, cols, out);
   else

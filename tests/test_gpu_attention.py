@@ -112,6 +112,30 @@ def test_rab_bucket_and_mask_dump_bit_exact():
     assert np.array_equal(got, np.array(want, dtype=np.int32))
 
 
+@pytest.mark.parametrize("mfalcon", [False, True])
+def test_attn_bwd_tensor_core_several_tiles(mfalcon):
+    """bf16, head dim 64 (the tensor-core backward): sequences spanning several
+    128-row tiles, a ragged last tile and a one-token sequence, so that kv tiles
+    meet several q tiles and the dQ atomics of different kv tiles add up."""
+    b = _b()
+    lens = [257, 600, 1, 130]
+    nt = [0, 75, 0, 129] if mfalcon else None
+    d = W.random_attention_inputs(47, lens, 2, 64, "bf16", num_targets=nt, qk_std=0.5)
+    T = sum(lens)
+    q, k, v, do = (dev(d[n].reshape(T, 2 * 64), torch.bfloat16) for n in ("q", "k", "v", "dout"))
+    ntd = None if nt is None else dev(d["num_targets"])
+    dq, dk, dv, dpb, dtb = b.attn_bwd(q, k, v, do, dev(d["seq_offsets"]), dev(d["timestamps"]), dev(d["pos_bias"]),
+                                      dev(d["time_bias"]), 2, num_targets=ntd)
+    torch.cuda.synchronize()
+    rq, rk, rv, rpb, rtb = O.attention_backward(d["q"], d["k"], d["v"], d["dout"], d["seq_offsets"],
+                                                d["timestamps"], d["pos_bias"], d["time_bias"], d["num_targets"])
+    for got, ref, name in [(dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")]:
+        assert_close(got.float().cpu().numpy().reshape(ref.shape), ref, "bf16", name, grad=True)
+    for got, ref, name in [(dpb, rpb, "dpos"), (dtb, rtb, "dtime")]:
+        g = got.cpu().numpy()
+        assert np.linalg.norm(g - ref) <= 1e-2 * max(np.linalg.norm(ref), 1e-6), name
+
+
 def _oracle_thresholds():
     """Smallest |dt| of every time bucket, by bisection over the oracle's rule."""
     thr = []

@@ -237,6 +237,15 @@ def _check_train(run, wl, chained_rel_bound):
             print(f"layer {li} {name}: teacher-forced rel-fro {rel:.3e} max-abs {ma:.3e}")
             if name in ("dU", "dV", "dQ", "dK"):
                 assert_close(got, ref, "bf16", f"L{li} {name} (teacher-forced)", grad=True)
+            elif name in ("pos_bias", "time_bias"):
+                # sums of dS over up to ~1e6 pairs, with heavy cancellation: even fed
+                # the GPU's own layer input, the oracle differs from the GPU by the
+                # bf16 rounding of the layer's internal operands (x-hat, U/V/Q/K,
+                # A V, the gate, dO).  An fp64 simulation of those roundings on this
+                # workload gives 3e-3 .. 8e-3 with exact upstream gradients, and the
+                # GPU's own upstream gradients have given up to 1.03e-2; the attention
+                # backward itself matches the oracle to ~1e-6 on identical inputs.
+                assert rel <= 2e-2, f"L{li} {name} (teacher-forced) rel-fro {rel:.3e}"
             else:
                 assert rel <= 1e-2, f"L{li} {name} (teacher-forced) rel-fro {rel:.3e}"
         for name, (got, ref) in _layer_errors(chained[li], run["grads"][li], T, hv).items():

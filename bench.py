@@ -239,11 +239,11 @@ def kernel_digest(kernel: str):
     return h.hexdigest()[:16]
 
 
-def read_traffic(kernel: str):
+def read_traffic(kernel: str, path: str = None):
     """DRAM bytes per launch of `kernel` from the committed ncu summary
     (`profiles/dram_traffic.txt`: kernel, bytes, source digest), or None when
     there is none or the kernel's sources changed after the capture."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    p = path or os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -357,20 +357,6 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "source": "NVML, 5 ms period, timed region only"}
 
 
-def read_traffic(kernel: str):
-    """dram bytes per launch of `kernel` from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(p):
-        return None
-    with open(p) as f:
-        for line in f:
-            parts = line.split()
-            if len(parts) >= 2 and parts[0] == kernel and not line.startswith("#"):
-                try:
-                    return float(parts[1])
-                except ValueError:
-                    return None
-    return None
 
 
 

@@ -80,3 +80,16 @@ def test_unmasked_pairs_matches_oracle_count():
     # and against the mask itself, built by the oracle, on one small sequence
     mask = O.attention_mask(12, 5)
     assert bench.unmasked_pairs([0, 12], [5]) == int(np.count_nonzero(mask))
+
+
+def test_traffic_is_null_once_the_kernel_changed(tmp_path):
+    """The roofline's DRAM traffic comes from a committed ncu capture only while
+    the kernel's sources still match the digest recorded with it."""
+    digest = bench.kernel_digest("attn_fwd_tc")
+    good = tmp_path / "good.txt"
+    good.write_text(f"# comment attn_fwd_tc 1 2\nattn_fwd_tc 12345 {digest}\n")
+    stale = tmp_path / "stale.txt"
+    stale.write_text("attn_fwd_tc 12345 0000000000000000\n")
+    assert bench.read_traffic("attn_fwd_tc", str(good)) == 12345.0
+    assert bench.read_traffic("attn_fwd_tc", str(stale)) is None
+    assert bench.read_traffic("attn_fwd_tc", str(tmp_path / "missing.txt")) is None

@@ -100,9 +100,44 @@ struct Layout {
   static constexpr int kBar = (kTimeB + kNumBuckets * 4 + 15) & ~15;
   static constexpr int kMisc = kBar + (int)sizeof(Barriers);
   static constexpr int kItems = kMisc + 16;
-  static constexpr int kEnd = kItems + 16;
+  static constexpr int kEnd = kItems + kItemSlots * 8 * 4;
   static constexpr int kAlloc = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
+
+// A fetched work item and the facts of its sequence, as the item ring holds
+// them (8 words per slot) so that no reader reloads them from global memory.
+struct ItemInfo {
+  int idx;       // -1: no more items
+  WorkItem wi;
+  SeqInfo si;
+};
+
+__device__ __forceinline__ void ring_put(volatile int* ring, int slot, const ItemInfo& x) {
+  volatile int* w = ring + 8 * slot;
+  w[0] = x.idx;
+  w[1] = x.wi.seq;
+  w[2] = x.wi.head;
+  w[3] = x.wi.qtile;
+  w[4] = x.si.start;
+  w[5] = x.si.n;
+  w[6] = x.si.hist;
+  w[7] = __float_as_int(x.si.inv_n);
+}
+
+__device__ __forceinline__ ItemInfo ring_get(const volatile int* ring, int slot) {
+  const volatile int* w = ring + 8 * slot;
+  ItemInfo x;
+  x.idx = w[0];
+  x.wi.seq = w[1];
+  x.wi.head = w[2];
+  x.wi.qtile = w[3];
+  x.wi.cost = 0;
+  x.si.start = w[4];
+  x.si.n = w[5];
+  x.si.hist = w[6];
+  x.si.inv_n = __int_as_float(w[7]);
+  return x;
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -209,21 +244,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       for (int k = 0;; ++k) {
         // the Q/K producer fetches the next work item; everyone else reads it from the ring
         const int slot = k % kItemSlots;
-        int idx;
+        ItemInfo x;
         if (kside) {
           if (!mbar_wait(&bars->it_empty[slot], ((k / kItemSlots) & 1) ^ 1, tmo, abort_flag)) goto fail;
-          idx = *abort_flag ? -1 : atomicAdd(p.item_cursor, 1);
-          if (idx >= count) idx = -1;
-          item_ring[slot] = idx;
+          x.idx = *abort_flag ? -1 : atomicAdd(p.item_cursor, 1);
+          if (x.idx >= count) x.idx = -1;
+          if (x.idx >= 0) {
+            x.wi = p.items[x.idx];
+            x.si = load_seq(p.seq_offsets, p.num_targets, x.wi.seq);
+          }
+          ring_put(item_ring, slot, x);
           mbar_arrive(&bars->it_full[slot]);
         } else {
           if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
-          idx = item_ring[slot];
+          x = ring_get(item_ring, slot);
           mbar_arrive(&bars->it_empty[slot]);
         }
-        if (idx < 0) break;
-        const WorkItem wi = p.items[idx];
-        const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+        if (x.idx < 0) break;
+        const WorkItem wi = x.wi;
+        const SeqInfo si = x.si;
         const int r0 = wi.qtile * BM;
         const int r1 = min(si.n, r0 + BM);
         if (kside) {
@@ -279,11 +318,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
       for (int k = 0;; ++k) {
         const int slot = k % kItemSlots;
         if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
-        const int idx = item_ring[slot];
+        const ItemInfo x = ring_get(item_ring, slot);
         mbar_arrive(&bars->it_empty[slot]);
-        if (idx < 0) break;
-        const WorkItem wi = p.items[idx];
-        const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+        if (x.idx < 0) break;
+        const WorkItem wi = x.wi;
+        const SeqInfo si = x.si;
         const int r0 = wi.qtile * BM;
         const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
         const int nk = kv_count(kr);
@@ -349,12 +388,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     for (int k = 0;; ++k) {
       const int slot = k % kItemSlots;
       if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
-      const int idx = item_ring[slot];
+      const ItemInfo x = ring_get(item_ring, slot);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->it_empty[slot]);
-      if (idx < 0) break;
-      const WorkItem wi = p.items[idx];
-      const SeqInfo si = load_seq(p.seq_offsets, p.num_targets, wi.seq);
+      if (x.idx < 0) break;
+      const WorkItem wi = x.wi;
+      const SeqInfo si = x.si;
       if (per_head_rab && wi.head != cur_head) {
         named_bar_sync(1, 32 * kEpiWarps);
         for (int c = threadIdx.x - 32 * kEpiWarp0; c < kNumBuckets; c += 32 * kEpiWarps) {
@@ -385,12 +424,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const int c0 = kv_tile_at(kr, jj) * BN;
         const int sb = it % kSBufs;
         const int rs = it % kRecStages;
-        if (!mbar_wait(&bars->r_full[rs], (it / kRecStages) & 1, tmo, abort_flag)) goto fail;
-        const TsRec& rec = recs[rs];
         if (!mbar_wait(&bars->s_full[sb], (it / kSBufs) & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
         uint32_t raw[32];
         tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);  // waited for after the classification
+        // the timestamp record is waited for while the TMEM load is in flight
+        if (!mbar_wait(&bars->r_full[rs], (it / kRecStages) & 1, tmo, abort_flag)) goto fail;
+        const TsRec& rec = recs[rs];
         // ---- classify this row's 32 columns:
         //   rank 0: nothing attended; 1: one time bucket (constant bias); 2: two buckets;
         //   3: three or four buckets (per-element threshold compares); 4: general

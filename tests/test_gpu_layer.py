@@ -261,14 +261,15 @@ def _check_train(run, wl, chained_rel_bound):
 def test_training_step_config4_scaled():
     """8-layer bf16 stack (fp32 residual stream) forward + backward with
     Stochastic Length: dU, dV, dQ, dK, the rab gradients and the weight
-    gradients of every layer vs the oracle.  The chained bound 2e-2 comes from
-    an fp64 simulation of this workload in which only the bf16 rounding of the
-    forward's tensor-core operands (xhat, U/V/Q/K, A V, gate) is applied: that
-    alone moves the chained gradients by up to 1.12e-2 (time-bias gradient) and
-    9.5e-3 (dK) from the exact stack; the backward's own bf16 operands add about
-    3e-3 (a single-layer simulation)."""
+    gradients of every layer vs the oracle.  The chained bound 3e-2 comes from
+    an fp64 simulation of this workload that rounds to bf16 wherever the GPU
+    stores a bf16 value or feeds one to a tensor core (forward: x-hat, U/V/Q/K,
+    P with the bf16-pair SiLU, A V, the gate; backward: dY, dg, dO, dU, P and dS
+    as MMA operands, dQ/dK/dV, dz): it moves the chained gradients by up to
+    1.79e-2 (time-bias gradient, first layer) and 1.76e-2 (dK); the GPU, which
+    also sums in fp32 with atomics, has given up to 2.16e-2."""
     wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
-    _check_train(_train_step(wl, residual_fp32=True), wl, chained_rel_bound=2e-2)
+    _check_train(_train_step(wl, residual_fp32=True), wl, chained_rel_bound=3e-2)
 
 
 def test_training_step_bf16_residual_two_layers():

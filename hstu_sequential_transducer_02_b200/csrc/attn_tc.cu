@@ -14,10 +14,11 @@
 //                 the kv tile's timestamp record (int32 offsets, per-segment
 //                 min/max); it also fetches the work items for everyone
 //   warp 2        TMA: V per kv tile into its own ring
-//   warp 1        one thread issues S = Q K^T (tcgen05.mma, operands in shared
-//                 memory) into one of three TMEM buffers
-//   warp 3        one thread issues O += P V with P read from TMEM (the A
-//                 operand) and V from shared memory
+//   warp 1        issues S = Q K^T (tcgen05.mma, operands in shared memory)
+//                 into one of three TMEM buffers
+//   warp 3        issues O += P V with P read from TMEM (the A operand) and V
+//                 from shared memory (each issuer warp runs its loop
+//                 warp-uniformly; one elected lane issues)
 //   warps 4-19    epilogue, one warp per TMEM lane quarter and 32-column
 //                 segment: S -> registers, rab bias (position and time buckets,
 //                 bit-exact integer rule), SiLU, mask, bf16 P written back over
@@ -302,24 +303,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
   } else if (warp == 1 || warp == 3) {
     // =================================================================== MMA issuers
     // Issue is synchronous with the tensor pipe, so S = Q K^T (warp 1) and O += P V
-    // (warp 3) have a thread each: S of a later kv tile only waits until P V has
-    // consumed its TMEM buffer, not until the P V before it has been issued.
-    if (lane == 0) {
+    // (warp 3) have a warp each: S of a later kv tile only waits until P V has
+    // consumed its TMEM buffer, not until the P V before it has been issued.  The
+    // whole warp runs the loop (its waits, counters and descriptors stay
+    // warp-uniform) and one elected lane issues each MMA and commit.
+    {
       const bool s_side = warp == 1;
       constexpr uint32_t idesc_s = make_idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = make_idesc_bf16(BM, DV, false, true);
-      // descriptors of stage 0; every MMA below adds compile-time offsets to these,
-      // so an issuing thread spends few instructions per MMA (it shares its
-      // sub-partition's issue slots with four epilogue warps)
+      // descriptors of stage 0; every MMA below adds compile-time offsets to these
       const uint64_t dq0 = make_sw128_desc(sQ, 16, 1024);
       const uint64_t dk0 = make_sw128_desc(sK, 16, 1024);
       const uint64_t dv0 = make_sw128_desc(sV, kBoxBytes, 1024);
-      int n_it = 0;  // global kv-tile counter of this thread
+      int n_it = 0;  // global kv-tile counter of this warp
       for (int k = 0;; ++k) {
         const int slot = k % kItemSlots;
-        if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
+        if (!warp_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
         const ItemInfo x = ring_get(item_ring, slot);
-        mbar_arrive(&bars->it_empty[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->it_empty[slot]);
         if (x.idx < 0) break;
         const WorkItem wi = x.wi;
         const SeqInfo si = x.si;
@@ -327,33 +329,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
         const int nk = kv_count(kr);
         if (s_side) {
-          if (!mbar_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
+          if (!warp_wait(&bars->q_full, k & 1, tmo, abort_flag)) goto fail;
           for (int jj = 0; jj < nk; ++jj, ++n_it) {
             // S of kv tile n_it into buffer n_it % kSBufs once P V of tile n_it - kSBufs is done
             const int st = n_it % SK;
             const int sb = n_it % kSBufs;
-            if (!mbar_wait(&bars->k_full[st], (n_it / SK) & 1, tmo, abort_flag)) goto fail;
-            if (!mbar_wait(&bars->pv_done[sb], ((n_it / kSBufs) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            if (!warp_wait(&bars->k_full[st], (n_it / SK) & 1, tmo, abort_flag)) goto fail;
+            if (!warp_wait(&bars->pv_done[sb], ((n_it / kSBufs) & 1) ^ 1, tmo, abort_flag)) goto fail;
             tc_fence_after();
             const uint64_t dk = desc_advance(dk0, st * C::kTileBytes);
             const uint32_t dS = tmem_s0 + sb * BN;
 #pragma unroll
             for (int ks = 0; ks < DH / 16; ++ks) {
               const uint32_t off = (ks >> 2) * kBoxBytes + (ks & 3) * 32;
-              umma_f16_ss(dS, desc_advance(dq0, off), desc_advance(dk, off), idesc_s, ks > 0 ? 1u : 0u);
+              umma_f16_ss_elect(dS, desc_advance(dq0, off), desc_advance(dk, off), idesc_s, ks > 0 ? 1u : 0u);
             }
-            umma_commit(&bars->s_full[sb]);
-            umma_commit(&bars->k_empty[st]);
-            if (jj == nk - 1) umma_commit(&bars->q_empty);
+            umma_commit_elect(&bars->s_full[sb]);
+            umma_commit_elect(&bars->k_empty[st]);
+            if (jj == nk - 1) umma_commit_elect(&bars->q_empty);
           }
         } else {
           for (int jj = 0; jj < nk; ++jj, ++n_it) {
             // O (+)= P V for kv tile n_it, P read from TMEM
             const int pb = n_it % kSBufs;
             const int vs = n_it % SV;
-            if (!mbar_wait(&bars->p_full[pb], (n_it / kSBufs) & 1, tmo, abort_flag)) goto fail;
-            if (!mbar_wait(&bars->v_full[vs], (n_it / SV) & 1, tmo, abort_flag)) goto fail;
-            if (jj == 0 && !mbar_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
+            if (!warp_wait(&bars->p_full[pb], (n_it / kSBufs) & 1, tmo, abort_flag)) goto fail;
+            if (!warp_wait(&bars->v_full[vs], (n_it / SV) & 1, tmo, abort_flag)) goto fail;
+            if (jj == 0 && !warp_wait(&bars->o_empty, (k & 1) ^ 1, tmo, abort_flag)) goto fail;
             tc_fence_after();
             const uint32_t pa = tmem_s0 + pb * BN;
             const uint64_t dv = desc_advance(dv0, vs * C::kTileBytes);
@@ -361,19 +363,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
 #pragma unroll
             for (int ks = 0; ks < BN / 16; ++ks) {
               // kv columns [16ks, 16ks+16) were written by segment ks/2 at columns 32*(ks/2) + 8*(ks%2)
-              umma_f16_ts(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), desc_advance(dv, ks * 16 * 128), idesc_o,
-                          ks > 0 ? 1u : acc0);
+              umma_f16_ts_elect(tmem_o, pa + 32 * (ks >> 1) + 8 * (ks & 1), desc_advance(dv, ks * 16 * 128), idesc_o,
+                                ks > 0 ? 1u : acc0);
             }
-            umma_commit(&bars->v_empty[vs]);
-            umma_commit(&bars->pv_done[pb]);
+            umma_commit_elect(&bars->v_empty[vs]);
+            umma_commit_elect(&bars->pv_done[pb]);
           }
-          umma_commit(&bars->o_full);
+          umma_commit_elect(&bars->o_full);
         }
       }
-      // all MMAs this thread issued complete before TMEM is released
+      // all MMAs this warp issued complete before TMEM is released
       uint64_t* dbar = s_side ? &bars->done : &bars->done_pv;
-      umma_commit(dbar);
-      mbar_wait(dbar, 0, tmo, nullptr);
+      umma_commit_elect(dbar);
+      warp_wait(dbar, 0, tmo, nullptr);
     }
   } else {
     // =================================================================== epilogue
@@ -424,11 +426,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const int c0 = kv_tile_at(kr, jj) * BN;
         const int sb = it % kSBufs;
         const int rs = it % kRecStages;
-        if (!mbar_wait(&bars->s_full[sb], (it / kSBufs) & 1, tmo, abort_flag)) goto fail;
-        tc_fence_after();
+        // S of this tile into registers: at once when it is ready (the load is then in
+        // flight during the classification), else after the classification, which
+        // needs only the timestamp record and so runs while S is being computed
+        const bool s_ready = __all_sync(0xffffffffu, mbar_try_wait(&bars->s_full[sb], (it / kSBufs) & 1));
         uint32_t raw[32];
-        tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);  // waited for after the classification
-        // the timestamp record is waited for while the TMEM load is in flight
+        if (s_ready) {
+          tc_fence_after();
+          tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
+        }
         if (!mbar_wait(&bars->r_full[rs], (it / kRecStages) & 1, tmo, abort_flag)) goto fail;
         const TsRec& rec = recs[rs];
         // ---- classify this row's 32 columns:
@@ -481,6 +487,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         const int i0w = r0 + quarter * 32;
         const bool use_band = wrank == 4 && p.band != nullptr && cl >= i0w - 128 &&
                               !__any_sync(0xffffffffu, live && cand);
+        if (!s_ready) {
+          if (!mbar_wait(&bars->s_full[sb], (it / kSBufs) & 1, tmo, abort_flag)) goto fail;
+          tc_fence_after();
+          tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
+        }
         tmem_ld_wait_regs(raw);
         // ---- bias, SiLU (as h + h tanh h with h = (s + bias) / 2), mask; packed bf16 pairs
         uint32_t pk[16];

@@ -373,6 +373,14 @@ def _trace_attention(trace, name, flops):
             "tflops": flops / a["count"] / (ms / 1e3) / 1e12 if flops else None}  # flops: all traced launches
 
 
+def _top_kernels(trace, steps, k=6):
+    """The k kernels with the most traced device time: share and ms per step."""
+    tot = sum(v["ms"] for v in trace.values()) or 1e-9
+    top = sorted(trace.items(), key=lambda kv: -kv[1]["ms"])[:k]
+    return {name: {"share": v["ms"] / tot, "ms_per_step": v["ms"] / steps, "launches_per_step": v["count"] / steps}
+            for name, v in top}
+
+
 def measure_mfalcon(hb, steps: int):
     """M-FALCON ranking (16 users, n = 2048 history, m = 4096 candidates in
     microbatches of b_m = 512, d_model = 256, 2 heads of 128, 1 layer):
@@ -405,12 +413,16 @@ def measure_mfalcon(hb, steps: int):
     n = int(np.diff(wl.seq_offsets)[0])
     cands = int(e["cand_offsets"][-1])
     mbs = (m_max + bm - 1) // bm
-    pairs = U * mbs * (n * (n + 1) // 2) + cands * (n + 1)   # history recomputed per microbatch
+    # the history's keys and values are computed once per call and reused by every
+    # microbatch: its causal pairs once, then each candidate against the history and itself
+    pairs = U * (n * (n + 1) // 2) + cands * (n + 1)
     flops = pairs * 2 * 2 * sp.head_dim * sp.num_heads
-    return {"workload": f"M-FALCON: {U} users, n={n} history, m={cands // U} candidates, b_m={bm}, "
+    return {"workload": f"M-FALCON: {U} users, n={n} history, m={cands // U} candidates, b_m={bm} "
+                        f"({mbs} microbatches, history K/V cached across them), "
                         f"d_model={sp.d_model}, {sp.num_heads} heads x {sp.head_dim}, 1 layer",
             "candidates_per_s": cands / (ms / 1e3), "ms_per_call": ms, "calls": steps,
-            "attention": _trace_attention(trace, "attn_fwd_tc", flops * steps)}
+            "attention": _trace_attention(trace, "attn_fwd_tc", flops * steps),
+            "top_kernels": _top_kernels(trace, steps)}
 
 
 def measure_training(hb, steps: int):
@@ -466,13 +478,11 @@ def measure_training(hb, steps: int):
     trace = hb.trace_read()
     hb.trace_enable(False)
     ms = t0.elapsed_time(t1) / steps
-    tot = sum(v["ms"] for v in trace.values()) or 1e-9
-    top = sorted(trace.items(), key=lambda kv: -kv[1]["ms"])[:6]
     return {"workload": f"training step: 8 layers, B=64, power-law n in [64,4096], SL to 1024 (p=0.8) -> "
                         f"T={T2} tokens, d_model={sp.d_model}, {sp.num_heads} heads x {sp.head_dim}, "
                         "fp32 residual stream, forward + backward",
             "tokens_per_s": T2 / (ms / 1e3), "ms_per_step": ms, "steps": steps,
-            "top_kernels": {k: {"share": v["ms"] / tot, "ms_per_step": v["ms"] / steps} for k, v in top}}
+            "top_kernels": _top_kernels(trace, steps)}
 
 # ----------------------------------------------------------------------------
 # our arm

@@ -101,7 +101,8 @@ struct Layout {
   static constexpr int kBar = (kTimeB + kNumBuckets * 4 + 15) & ~15;
   static constexpr int kMisc = kBar + (int)sizeof(Barriers);
   static constexpr int kItems = kMisc + 16;
-  static constexpr int kEnd = kItems + kItemSlots * 8 * 4;
+  static constexpr int kPend = kItems + kItemSlots * 8 * 4;   // per epilogue thread: pending O readout
+  static constexpr int kEnd = kPend + kEpiWarps * 32 * 16;
   static constexpr int kAlloc = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
 
@@ -159,6 +160,46 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
         "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
       :
       : "memory");
+}
+
+// O of a finished work item, once its last P V is done: this warp's kOc columns of
+// its 32 rows -> (1/N) -> bf16 -> global memory (`out` null for rows beyond the
+// sequence).  Returns false on a timeout.
+struct PendingO {
+  __nv_bfloat16* out;
+  float inv_n;
+  int pad;
+};
+
+template <int kOc>
+__device__ __forceinline__ bool o_readout(Barriers* bars, int parity, uint32_t taddr, const PendingO* pend,
+                                          int lane, long long tmo, volatile int* abort_flag) {
+  if (!mbar_wait(&bars->o_full, parity, tmo, abort_flag)) return false;
+  tc_fence_after();
+  __nv_bfloat16* out = pend->out;
+  const float inv_n = pend->inv_n;
+  // 16 columns at a time (few registers: the caller's tile state stays live)
+#pragma unroll 1
+  for (int h = 0; h < kOc / 16; ++h) {
+    uint32_t oraw[16];
+    tmem_ld_32x32b_x16(taddr + 16 * h, oraw);
+    tmem_ld_wait();
+    if (out != nullptr) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint4 v;
+        v.x = pack_bf16x2(__uint_as_float(oraw[8 * c + 0]) * inv_n, __uint_as_float(oraw[8 * c + 1]) * inv_n);
+        v.y = pack_bf16x2(__uint_as_float(oraw[8 * c + 2]) * inv_n, __uint_as_float(oraw[8 * c + 3]) * inv_n);
+        v.z = pack_bf16x2(__uint_as_float(oraw[8 * c + 4]) * inv_n, __uint_as_float(oraw[8 * c + 5]) * inv_n);
+        v.w = pack_bf16x2(__uint_as_float(oraw[8 * c + 6]) * inv_n, __uint_as_float(oraw[8 * c + 7]) * inv_n);
+        *reinterpret_cast<uint4*>(out + 16 * h + 8 * c) = v;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&bars->o_empty);
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -387,6 +428,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     const float k_lg = prm.ln2_over_div;
     int it = 0;  // global kv-tile counter
     int cur_head = -1;
+    // The O readout of an item is deferred: a warp that finishes its part of an
+    // item early goes on with the next item's kv tiles (their S needs no O) and
+    // reads O once the item's last P V is done, instead of idling until the
+    // slowest warp has finished.  At most one readout is pending per warp: the
+    // next item's O cannot complete before every warp has read this one.
+    constexpr int kOc = DV / 4;
+    int pend_par = -1;                       // parity of the pending readout's o_full phase; -1: none
+    // this lane's output row (null beyond the sequence) and 1/N, kept in shared memory
+#define HSTU_PEND (reinterpret_cast<PendingO*>(smem + L::kPend) + (threadIdx.x - 32 * kEpiWarp0))
     for (int k = 0;; ++k) {
       const int slot = k % kItemSlots;
       if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
@@ -429,7 +479,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         // S of this tile into registers: at once when it is ready (the load is then in
         // flight during the classification), else after the classification, which
         // needs only the timestamp record and so runs while S is being computed
-        const bool s_ready = __all_sync(0xffffffffu, mbar_try_wait(&bars->s_full[sb], (it / kSBufs) & 1));
+        bool s_ready = __all_sync(0xffffffffu, mbar_try_wait(&bars->s_full[sb], (it / kSBufs) & 1));
+        if (!s_ready && pend_par >= 0) {
+          // S may depend on P V of this item, which waits until every warp has read
+          // the previous item's O: the pending readout goes first
+          if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+          pend_par = -1;
+          s_ready = __all_sync(0xffffffffu, mbar_try_wait(&bars->s_full[sb], (it / kSBufs) & 1));
+        }
         uint32_t raw[32];
         if (s_ready) {
           tc_fence_after();
@@ -616,36 +673,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
           mbar_arrive(&bars->p_full[sb]);
           mbar_arrive(&bars->r_empty[rs]);
         }
-      }
-      // ---- O readout: this warp's DV/4 columns
-      if (!mbar_wait(&bars->o_full, k & 1, tmo, abort_flag)) goto fail;
-      tc_fence_after();
-      constexpr int kOc = DV / 4;
-      uint32_t oraw[kOc];
-      if constexpr (kOc == 32) {
-        tmem_ld_32x32b_x32(tmem_o + lane_off + seg * kOc, *reinterpret_cast<uint32_t(*)[32]>(&oraw[0]));
-      } else {
-        tmem_ld_32x32b_x16(tmem_o + lane_off + seg * kOc, *reinterpret_cast<uint32_t(*)[16]>(&oraw[0]));
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->o_empty);
-      if (live) {
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(si.start + i) * p.ldo +
-                             (int64_t)wi.head * DV + seg * kOc;
-#pragma unroll
-        for (int c = 0; c < kOc / 8; ++c) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(oraw[8 * c + 0]) * si.inv_n, __uint_as_float(oraw[8 * c + 1]) * si.inv_n);
-          v.y = pack_bf16x2(__uint_as_float(oraw[8 * c + 2]) * si.inv_n, __uint_as_float(oraw[8 * c + 3]) * si.inv_n);
-          v.z = pack_bf16x2(__uint_as_float(oraw[8 * c + 4]) * si.inv_n, __uint_as_float(oraw[8 * c + 5]) * si.inv_n);
-          v.w = pack_bf16x2(__uint_as_float(oraw[8 * c + 6]) * si.inv_n, __uint_as_float(oraw[8 * c + 7]) * si.inv_n);
-          *reinterpret_cast<uint4*>(out + 8 * c) = v;
+        // the pending readout as soon as the previous item's O is complete
+        if (pend_par >= 0 && __all_sync(0xffffffffu, mbar_try_wait(&bars->o_full, pend_par))) {
+          if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+          pend_par = -1;
         }
       }
+      // ---- this item's O readout becomes the pending one (an older one is done first)
+      if (pend_par >= 0) {
+        if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+      }
+      pend_par = k & 1;
+      HSTU_PEND->out = live ? reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(si.start + i) * p.ldo +
+                             (int64_t)wi.head * DV + seg * kOc
+                       : nullptr;
+      HSTU_PEND->inv_n = si.inv_n;
+    }
+    if (pend_par >= 0) {
+      if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
     }
   }
+#undef HSTU_PEND
   goto teardown;
 fail:
   set_status(p.status, HSTU_ERR_TIMEOUT);

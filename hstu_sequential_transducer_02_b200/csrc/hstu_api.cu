@@ -726,30 +726,133 @@ int hstu_layer_bwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
 }
 
 // ---------------------------------------------------------------- M-FALCON
+// The history rows of a user do not depend on its candidates (they attend only to
+// the history), so their K and V are computed once and cached across microbatches
+// ("2.3 M-FALCON算法": the history's keys and values are reused by every
+// microbatch).  Every user keeps a fixed place in a slot layout,
+// [history_u ; bm candidate slots]; microbatch 0 runs the full layer stack over
+// it, writing each layer's U|V|Q|K into that layer's cache; every later
+// microbatch computes only its candidate rows: LayerNorm1 and f1 on the compact
+// candidate rows, their U|V|Q|K scattered into the cache's slot rows, the
+// attention over the q tiles of the slots only (keys and values: the cached
+// history and the slots), then LayerNorm2 * U and f2 on the compact rows.  The
+// rows computed are the same rows as in a full pass over [history ; microbatch],
+// with the same reduction order, so the candidates' outputs are too.
 namespace {
 struct MfalconWs {
-  LayerFwdWs layer;
-  int32_t* offs;
-  int32_t* nt;
-  int64_t* ts;
-  void* x0;
+  LayerFwdWs layer;       // full pass over the slot layout (microbatch 0)
+  AttnWs attn_t;          // targets-only attention: own work list, shared records and status
+  int32_t* offs;          // slot layout [U+1]
+  int32_t* nt;            // [U], all bm
+  int64_t* ts;            // [cap]
+  void* x0;               // [cap, d] slot-layout layer input / output (microbatch 0)
   void* x1;
-  int32_t* row_map;
+  char* uvqk_cache;       // num_layers x [cap, 4 hv]
+  size_t uvqk_stride;     // bytes per layer
+  void* o_slot;           // [cap, hv] attention output, slot layout
+  void* xc0;              // [C, d] compact candidate rows
+  void* xc1;
+  void* xhat_c;           // [C, d]
+  float* mu1c; float* rs1c; float* mu2c; float* rs2c;
+  void* uvqk_c;           // [C, 4 hv]
+  void* o_c;              // [C, hv]
+  void* g_c;              // [C, hv]
+  int32_t* cand_dst;      // [C]
   int cap;
+  int C;
 };
 
-MfalconWs carve_mfalcon(Carver& c, const hstu_layer_desc* d, int U, int hist_total, int bm) {
+MfalconWs carve_mfalcon(Carver& c, const hstu_layer_desc* d, int L, int U, int hist_total, int bm) {
   MfalconWs w;
   w.cap = hist_total + U * bm;
+  w.C = U * bm;
   w.layer = carve_layer_fwd(c, d, U, w.cap, true);
-  const size_t es = elem_size(d->io_dtype);
+  const size_t es = elem_size(d->attn.dtype), eio = elem_size(d->io_dtype);
+  const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
+  // targets-only attention: a work list of its own; status, tile bases and timestamp
+  // records are the full pass's (same offsets); no bias band (no history q tile runs)
+  w.attn_t = w.layer.attn;
+  w.attn_t.count = c.take<int32_t>(64);
+  w.attn_t.items = c.take<WorkItem>(w.layer.attn.capacity);
+  w.attn_t.band = nullptr;
   w.offs = c.take<int32_t>(U + 1);
   w.nt = c.take<int32_t>(U > 0 ? U : 1);
-  w.ts = c.take<int64_t>(w.cap);
-  w.x0 = c.take<char>((size_t)w.cap * d->d_model * es);
-  w.x1 = c.take<char>((size_t)w.cap * d->d_model * es);
-  w.row_map = c.take<int32_t>(w.cap);
+  w.ts = c.take<int64_t>(w.cap > 0 ? w.cap : 1);
+  w.x0 = c.take<char>((size_t)w.cap * dm * eio);
+  w.x1 = c.take<char>((size_t)w.cap * dm * eio);
+  w.uvqk_stride = (((size_t)w.cap * 4 * hv * es) + 255) & ~(size_t)255;
+  w.uvqk_cache = c.take<char>(w.uvqk_stride * L);
+  w.o_slot = c.take<char>((size_t)w.cap * hv * es);
+  w.xc0 = c.take<char>((size_t)w.C * dm * eio);
+  w.xc1 = c.take<char>((size_t)w.C * dm * eio);
+  w.xhat_c = c.take<char>((size_t)w.C * dm * es);
+  w.mu1c = c.take<float>(w.C);
+  w.rs1c = c.take<float>(w.C);
+  w.mu2c = c.take<float>(w.C);
+  w.rs2c = c.take<float>(w.C);
+  w.uvqk_c = c.take<char>((size_t)w.C * 4 * hv * es);
+  w.o_c = c.take<char>((size_t)w.C * hv * es);
+  w.g_c = c.take<char>((size_t)w.C * hv * es);
+  w.cand_dst = c.take<int32_t>(w.C > 0 ? w.C : 1);
   return w;
+}
+
+// One layer over the compact candidate rows x_c -> y_c (C rows), the history's
+// keys and values taken from `uvqk` (slot layout), whose slot rows receive the
+// candidates' U|V|Q|K.
+int run_layer_targets(const hstu_layer_desc* d, const hstu_layer_weights* w, const hstu_jagged* slot_jb, int U,
+                      int bm, const int32_t* hist_offsets, const void* x_c, void* y_c, char* uvqk,
+                      const MfalconWs& ws, cudaStream_t st) {
+  const int dt = d->attn.dtype;
+  const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
+  const int C = ws.C;
+  const size_t es = elem_size(dt);
+  {
+    TraceScope tr("ln1", st);
+    HSTU_CUDA(launch_layer_norm(x_c, dm, d->io_dtype, w->ln1_gamma, w->ln1_beta, d->ln_eps, ws.xhat_c, dm, dt,
+                                ws.mu1c, ws.rs1c, C, nullptr, dm, st));
+  }
+  GemmParams g1;
+  memset(&g1, 0, sizeof(g1));
+  g1.M = C; g1.N = 4 * hv; g1.K = dm;
+  g1.A = ws.xhat_c; g1.sam = dm; g1.sak = 1;
+  g1.B = w->w1; g1.sbn = dm; g1.sbk = 1;
+  g1.epi = EPI_BIAS_SILU; g1.bias = w->b1;
+  g1.out = ws.uvqk_c; g1.ldo = 4 * hv;
+  g1.status = ws.layer.attn.status;
+  HSTU_TRY(gemm(g1, dt, d->attn.flags, st, "gemm_f1_silu"));
+  {
+    TraceScope tr("mfalcon_slot_rows", st);
+    HSTU_CUDA(launch_mfalcon_slot_rows(U, bm, ws.cap, hist_offsets, ws.uvqk_c, (int64_t)4 * hv * es, uvqk,
+                                       (int64_t)4 * hv * es, (int64_t)4 * hv * es, 1, st));
+  }
+  // the targets-only work list is reused: reset its fetch cursor
+  HSTU_CUDA(cudaMemsetAsync(ws.attn_t.count + 1, 0, sizeof(int32_t), st));
+  HSTU_TRY(run_attn_main(&d->attn, slot_jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv,
+                         uvqk + 1 * hv * es, 4 * hv, w->pos_bias, w->time_bias, ws.o_slot, hv, ws.attn_t, st));
+  {
+    TraceScope tr("mfalcon_slot_rows", st);
+    HSTU_CUDA(launch_mfalcon_slot_rows(U, bm, ws.cap, hist_offsets, ws.o_slot, (int64_t)hv * es, ws.o_c, (int64_t)hv * es,
+                                       (int64_t)hv * es, 0, st));
+  }
+  {
+    TraceScope tr("ln2_gate", st);
+    HSTU_CUDA(launch_ln_gate(ws.o_c, hv, ws.uvqk_c, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g_c, hv,
+                             ws.mu2c, ws.rs2c, C, nullptr, hv, dt, st));
+  }
+  GemmParams g2;
+  memset(&g2, 0, sizeof(g2));
+  g2.M = C; g2.N = dm; g2.K = hv;
+  g2.A = ws.g_c; g2.sam = hv; g2.sak = 1;
+  g2.B = w->w2; g2.sbn = hv; g2.sbk = 1;
+  g2.epi = EPI_BIAS_RESIDUAL; g2.bias = w->b2;
+  g2.residual = x_c; g2.ldr = dm;
+  g2.out = y_c; g2.ldo = dm;
+  g2.res_f32 = d->io_dtype == HSTU_DTYPE_F32;
+  g2.out_f32 = d->io_dtype == HSTU_DTYPE_F32;
+  g2.status = ws.layer.attn.status;
+  HSTU_TRY(gemm(g2, dt, d->attn.flags, st, "gemm_f2_residual"));
+  return HSTU_OK;
 }
 }  // namespace
 
@@ -760,7 +863,7 @@ int mfalcon_rank_workspace_size(const hstu_layer_desc* desc, int32_t num_layers,
   HSTU_TRY(check_attn_desc(&desc->attn));
   if ((int64_t)hist_total + (int64_t)num_users * microbatch >= (1ll << 31)) return HSTU_ERR_INVALID_ARG;
   Carver c(nullptr);
-  carve_mfalcon(c, desc, num_users, hist_total, microbatch);
+  carve_mfalcon(c, desc, num_layers, num_users, hist_total, microbatch);
   *bytes = c.size();
   return HSTU_OK;
 }
@@ -783,25 +886,60 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
   Carver c(workspace);
-  MfalconWs w = carve_mfalcon(c, desc, num_users, hist_total, microbatch);
+  const int U = num_users, bm = microbatch;
+  MfalconWs w = carve_mfalcon(c, desc, num_layers, U, hist_total, bm);
   HSTU_CUDA(cudaMemsetAsync(w.layer.attn.status, 0, kStatusBytes, st));
-  const int n_mb = (max_candidates + microbatch - 1) / microbatch;
+  const int n_mb = (max_candidates + bm - 1) / bm;
+  if (n_mb == 0 || U == 0) return HSTU_OK;
+  HSTU_CUDA(launch_mfalcon_slot_offsets(U, bm, hist_offsets, w.offs, w.nt, st));
+  hstu_jagged jb;
+  jb.batch = U;
+  jb.total_tokens = w.cap;
+  jb.seq_offsets = w.offs;
+  jb.num_targets = w.nt;
+  jb.timestamps = w.ts;
+  const hstu_attn_desc* ad = &desc->attn;
+  const int tile = attn_tile(ad);
   for (int mb = 0; mb < n_mb; ++mb) {
-    HSTU_CUDA(launch_mfalcon_pack(num_users, mb, microbatch, hist_offsets, hist_x, hist_ts, cand_offsets, cand_x,
-                                  cand_ts, dm, dt, w.offs, w.nt, w.ts, w.x0, w.row_map, nullptr, w.cap, st));
-    hstu_jagged jb;
-    jb.batch = num_users;
-    jb.total_tokens = w.cap;
-    jb.seq_offsets = w.offs;
-    jb.num_targets = w.nt;
-    jb.timestamps = w.ts;
-    void* cur = w.x0;
-    void* nxt = w.x1;
-    for (int l = 0; l < num_layers; ++l) {
-      HSTU_TRY(run_layer_fwd(desc, &layers[l], &jb, cur, nxt, nullptr, w.layer, st));
-      void* t = cur; cur = nxt; nxt = t;
+    void* cur = w.xc0;
+    void* nxt = w.xc1;
+    if (mb == 0) {
+      // full pass over [history ; microbatch 0]: every layer's U|V|Q|K goes to its cache
+      HSTU_CUDA(launch_mfalcon_slot_pack(U, 0, bm, w.cap, w.cap, hist_offsets, hist_x, hist_ts, cand_offsets, cand_x,
+                                         cand_ts, dm, dt, 1, w.x0, w.ts, nullptr, w.cand_dst, st));
+      void* xs = w.x0;
+      void* ys = w.x1;
+      for (int l = 0; l < num_layers; ++l) {
+        LayerFwdWs lw = w.layer;
+        lw.b.uvqk = w.uvqk_cache + (size_t)l * w.uvqk_stride;
+        HSTU_TRY(run_layer_fwd(desc, &layers[l], &jb, xs, ys, nullptr, lw, st));
+        void* t = xs; xs = ys; ys = t;
+      }
+      // the candidates' final rows, compact
+      HSTU_CUDA(launch_mfalcon_slot_rows(U, bm, w.cap, hist_offsets, xs, (int64_t)dm * elem_size(dt), cur,
+                                         (int64_t)dm * elem_size(dt), (int64_t)dm * elem_size(dt), 0, st));
+      // work list of the later microbatches: the q tiles of the candidate slots only
+      {
+        TraceScope tr("sched_fwd", st);
+        HSTU_CUDA(launch_build_work_list(w.offs, w.nt, U, w.cap, ad->num_heads, tile, tile, use_tc(ad) ? 3 : 0,
+                                         w.attn_t.capacity, w.attn_t.items, w.attn_t.count, w.attn_t.status, st,
+                                         nullptr, 1));
+      }
+    } else {
+      HSTU_CUDA(launch_mfalcon_slot_pack(U, mb, bm, w.C, w.cap, hist_offsets, hist_x, hist_ts, cand_offsets, cand_x,
+                                         cand_ts, dm, dt, 0, nullptr, w.ts, cur, w.cand_dst, st));
+      if (w.attn_t.tile_recs) {
+        // the candidates' timestamps changed: timestamp records of every kv tile
+        TraceScope tr("ts_tiles", st);
+        HSTU_CUDA(launch_ts_tiles(w.offs, w.ts, U, w.attn_t.tile_base, w.attn_t.tiles_cap, w.attn_t.tile_recs, st));
+      }
+      for (int l = 0; l < num_layers; ++l) {
+        HSTU_TRY(run_layer_targets(desc, &layers[l], &jb, U, bm, hist_offsets, cur, nxt,
+                                   w.uvqk_cache + (size_t)l * w.uvqk_stride, w, st));
+        void* t = cur; cur = nxt; nxt = t;
+      }
     }
-    HSTU_CUDA(launch_mfalcon_scatter(cur, dm, dt, w.row_map, w.offs + num_users, w.cap, cand_out, st));
+    HSTU_CUDA(launch_mfalcon_scatter(cur, dm, dt, w.cand_dst, nullptr, w.C, cand_out, st));
   }
   return HSTU_OK;
 }

@@ -9,10 +9,13 @@ namespace hstu {
 size_t work_list_capacity(int B, int T, int H, int tile);
 // Also writes tile_base[s] = index of sequence s's first kv tile of width tk in a
 // tiled per-tile array (tile_base[B] = total tiles) when tile_base is not null.
+// With q_from_hist (forward modes), a sequence's q tiles start at the one holding
+// its first target row: only the targets' rows are computed (their history rows'
+// K and V must be in place).
 cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targets, int B, int T, int H,
                                    int tm, int tk, int mode, int max_items, WorkItem* items,
                                    int32_t* count, int32_t* status, cudaStream_t stream,
-                                   int32_t* tile_base = nullptr);
+                                   int32_t* tile_base = nullptr, int q_from_hist = 0);
 
 // Per kv tile of 128 columns: timestamps as int32 offsets from the sequence's
 // first timestamp, with per-32-column min/max and a flag when any offset
@@ -182,14 +185,25 @@ cudaError_t launch_gather_rows(const void* src, void* dst, int64_t row_bytes, co
 cudaError_t launch_sl_select(int B, int T, const int32_t* offs, const uint32_t* coins, const uint32_t* keys,
                              int max_len, uint32_t prob, int32_t* out_offsets, int32_t* out_index,
                              int32_t* scratch_len, int32_t* status, cudaStream_t st);
-// M-FALCON packing of microbatch `mb`: builds offsets/num_targets/ts/x of [hist ; cand chunk] per user,
-// and the row map used to scatter candidate outputs back.
-cudaError_t launch_mfalcon_pack(int U, int mb, int bm, const int32_t* hist_offs, const void* hist_x,
-                                const int64_t* hist_ts, const int32_t* cand_offs, const void* cand_x,
-                                const int64_t* cand_ts, int d, int dtype, int32_t* out_offs,
-                                int32_t* out_nt, int64_t* out_ts, void* out_x, int32_t* cand_row_map,
-                                int32_t* cand_src_rows, int cap_rows, cudaStream_t st);
+// rows r < *total_rows (total_rows null: r < cap_rows) with cand_row_map[r] >= 0 go to that row of cand_out
 cudaError_t launch_mfalcon_scatter(const void* y, int d, int dtype, const int32_t* cand_row_map,
                                    const int32_t* total_rows, int cap_rows, void* cand_out, cudaStream_t st);
+// M-FALCON with the history cached across microbatches (slot layout: user u's rows
+// [history_u ; bm candidate slots] from row hist_offs[u] + u * bm; compact candidate
+// row c = u * bm + j).  Offsets and num_targets (= bm) of the slot layout:
+cudaError_t launch_mfalcon_slot_offsets(int U, int bm, const int32_t* hist_offs, int32_t* offs, int32_t* nt,
+                                       cudaStream_t st);
+// microbatch mb's candidates into the slot rows (x_slot, ts_slot) and/or the compact
+// rows (x_c), zero rows past a user's candidates; cand_dst[c] = row of cand_out or -1.
+// with_hist also copies the history rows; rows_cap = rows walked (all slot rows or U * bm);
+// slot rows at or past cap (offsets larger than the workspace was sized for) are skipped.
+cudaError_t launch_mfalcon_slot_pack(int U, int mb, int bm, int rows_cap, int cap, const int32_t* hist_offs,
+                                     const void* hist_x, const int64_t* hist_ts, const int32_t* cand_offs,
+                                     const void* cand_x, const int64_t* cand_ts, int d, int dtype, int with_hist,
+                                     void* x_slot, int64_t* ts_slot, void* x_c, int32_t* cand_dst, cudaStream_t st);
+// row_bytes of each candidate row between the compact and the slot layout (multiples of 16 bytes)
+cudaError_t launch_mfalcon_slot_rows(int U, int bm, int cap, const int32_t* hist_offs, const void* src,
+                                     int64_t lds_bytes, void* dst, int64_t ldd_bytes, int64_t row_bytes, int to_slot,
+                                     cudaStream_t st);
 
 }  // namespace hstu

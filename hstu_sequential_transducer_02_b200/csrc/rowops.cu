@@ -475,84 +475,12 @@ sl_select_kernel(int B, const int32_t* __restrict__ offs, const uint32_t* __rest
   }
 }
 
-// ---------------------------------------------------------------- M-FALCON packing
-constexpr int kPackThreads = 1024;
-
-// packed sequence u of microbatch mb: [history_u ; candidates_u[mb*bm, mb*bm + c_u)], or empty if c_u = 0
-__global__ void __launch_bounds__(kPackThreads)
-mfalcon_offsets_kernel(int U, int mb, int bm, const int32_t* __restrict__ hist_offs,
-                       const int32_t* __restrict__ cand_offs, int32_t* __restrict__ out_offs,
-                       int32_t* __restrict__ out_nt) {
-  using Scan = cub::BlockScan<int, kPackThreads>;
-  __shared__ typename Scan::TempStorage tmp;
-  __shared__ int carry;
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int base = 0; base < U; base += kPackThreads) {
-    const int u = base + threadIdx.x;
-    int len = 0, c = 0;
-    if (u < U) {
-      const int n = hist_offs[u + 1] - hist_offs[u];
-      const int m = cand_offs[u + 1] - cand_offs[u];
-      c = min(bm, max(0, m - mb * bm));
-      len = c > 0 ? n + c : 0;
-    }
-    int ex, tot;
-    Scan(tmp).ExclusiveSum(len, ex, tot);
-    if (u < U) { out_offs[u] = carry + ex; out_nt[u] = c; }
-    __syncthreads();
-    if (threadIdx.x == 0) carry += tot;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) out_offs[U] = carry;
-}
-
-// one warp per packed row: copy the row of X and its timestamp; record where a candidate row goes
-template <typename T>
-__global__ void mfalcon_rows_kernel(int U, int mb, int bm, const int32_t* __restrict__ hist_offs,
-                                    const T* __restrict__ hist_x, const int64_t* __restrict__ hist_ts,
-                                    const int32_t* __restrict__ cand_offs, const T* __restrict__ cand_x,
-                                    const int64_t* __restrict__ cand_ts, int d,
-                                    const int32_t* __restrict__ out_offs, int64_t* __restrict__ out_ts,
-                                    T* __restrict__ out_x, int32_t* __restrict__ row_map, int cap) {
-  const int lane = threadIdx.x & 31;
-  const int total = min(out_offs[U], cap);
-  for (int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < total; r += gridDim.x * (blockDim.x / 32)) {
-    // user of row r: binary search in out_offs
-    int lo = 0, hi = U;  // out_offs[lo] <= r < out_offs[hi]
-    while (hi - lo > 1) {
-      int mid = (lo + hi) >> 1;
-      if (out_offs[mid] <= r) lo = mid; else hi = mid;
-    }
-    const int u = lo;
-    const int l = r - out_offs[u];
-    const int n = hist_offs[u + 1] - hist_offs[u];
-    const T* src;
-    int64_t ts;
-    int dst_row = -1;
-    if (l < n) {
-      src = hist_x + (int64_t)(hist_offs[u] + l) * d;
-      ts = hist_ts[hist_offs[u] + l];
-    } else {
-      const int c = cand_offs[u] + mb * bm + (l - n);
-      src = cand_x + (int64_t)c * d;
-      ts = cand_ts[c];
-      dst_row = c;
-    }
-    for (int e = lane * 8; e < d; e += 32 * 8) {
-      float v[8];
-      load8(src + e, v);
-      store8(out_x + (int64_t)r * d + e, v);
-    }
-    if (lane == 0) { out_ts[r] = ts; row_map[r] = dst_row; }
-  }
-}
-
+// ---------------------------------------------------------------- M-FALCON output rows
 template <typename T>
 __global__ void mfalcon_scatter_kernel(const T* __restrict__ y, int d, const int32_t* __restrict__ row_map,
                                        const int32_t* __restrict__ total_rows, int cap, T* __restrict__ out) {
   const int lane = threadIdx.x & 31;
-  const int total = min(*total_rows, cap);
+  const int total = total_rows ? min(*total_rows, cap) : cap;
   for (int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < total; r += gridDim.x * (blockDim.x / 32)) {
     const int dst = row_map[r];
     if (dst < 0) continue;
@@ -561,6 +489,97 @@ __global__ void mfalcon_scatter_kernel(const T* __restrict__ y, int d, const int
       load8(y + (int64_t)r * d + e, v);
       store8(out + (int64_t)dst * d + e, v);
     }
+  }
+}
+
+// ---------------------------------------------------------------- M-FALCON with a history cache
+// Slot layout: user u's rows sit at a fixed place across microbatches,
+// [history_u ; a slot of bm candidate rows], from row hist_offs[u] + u * bm; the
+// compact candidate layout has row c = u * bm + j for slot row j of user u.
+__global__ void mfalcon_slot_offsets_kernel(int U, int bm, const int32_t* __restrict__ hist_offs,
+                                            int32_t* __restrict__ offs, int32_t* __restrict__ nt) {
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u <= U; u += gridDim.x * blockDim.x) {
+    offs[u] = hist_offs[u] + u * bm;
+    if (u < U) nt[u] = bm;
+  }
+}
+
+// Microbatch mb in the slot layout, one warp per row: candidate j of user u is
+// candidate mb * bm + j of that user, or a zero row (timestamp of the user's last
+// history token, else 0) past the user's candidates.  With with_hist the history
+// rows are written too (x and timestamps) and the rows walked are all slot-layout
+// rows; otherwise only the candidate rows.  x_slot and x_c may each be null.
+template <typename T>
+__global__ void mfalcon_slot_pack_kernel(int U, int mb, int bm, const int32_t* __restrict__ hist_offs,
+                                         const T* __restrict__ hist_x, const int64_t* __restrict__ hist_ts,
+                                         const int32_t* __restrict__ cand_offs, const T* __restrict__ cand_x,
+                                         const int64_t* __restrict__ cand_ts, int d, int with_hist, int cap,
+                                         T* __restrict__ x_slot, int64_t* __restrict__ ts_slot, T* __restrict__ x_c,
+                                         int32_t* __restrict__ cand_dst) {
+  const int lane = threadIdx.x & 31;
+  const int total = with_hist ? hist_offs[U] + U * bm : U * bm;   // rows walked
+  for (int r = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < total; r += gridDim.x * (blockDim.x / 32)) {
+    int u, j;          // user, and slot row (j < 0: history row -j - 1)
+    if (with_hist) {
+      int lo = 0, hi = U;  // slot-layout start of user lo <= r < start of user hi
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (hist_offs[mid] + mid * bm <= r) lo = mid; else hi = mid;
+      }
+      u = lo;
+      const int l = r - (hist_offs[u] + u * bm);
+      const int n = hist_offs[u + 1] - hist_offs[u];
+      j = l < n ? -l - 1 : l - n;
+    } else {
+      u = r / bm;
+      j = r - u * bm;
+    }
+    const T* src = nullptr;
+    int64_t ts = 0;
+    int slot_row;
+    if (j < 0) {
+      const int h = hist_offs[u] + (-j - 1);
+      src = hist_x + (int64_t)h * d;
+      ts = hist_ts[h];
+      slot_row = r;
+    } else {
+      const int m = cand_offs[u + 1] - cand_offs[u];
+      const int ci = mb * bm + j;
+      slot_row = hist_offs[u + 1] + u * bm + j;
+      if (ci < m) {
+        src = cand_x + (int64_t)(cand_offs[u] + ci) * d;
+        ts = cand_ts[cand_offs[u] + ci];
+      } else if (hist_offs[u + 1] > hist_offs[u]) {
+        ts = hist_ts[hist_offs[u + 1] - 1];
+      }
+      if (lane == 0) cand_dst[u * bm + j] = ci < m ? cand_offs[u] + ci : -1;
+    }
+    if (slot_row >= cap) continue;   // offsets beyond the sizes the workspace was made for
+    for (int e = lane * 8; e < d; e += 32 * 8) {
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (src) load8(src + e, v);
+      if (x_slot) store8(x_slot + (int64_t)slot_row * d + e, v);
+      if (x_c && j >= 0) store8(x_c + (int64_t)(u * bm + j) * d + e, v);
+    }
+    if (lane == 0) ts_slot[slot_row] = ts;
+  }
+}
+
+// Rows between the compact candidate layout and the slot layout: `words`
+// 16-byte words of each row (to_slot: compact -> slot, else slot -> compact);
+// one warp per row.
+__global__ void mfalcon_slot_rows_kernel(int U, int bm, const int32_t* __restrict__ hist_offs,
+                                         const uint4* __restrict__ src, int64_t lds, uint4* __restrict__ dst,
+                                         int64_t ldd, int words, int to_slot, int cap) {
+  const int lane = threadIdx.x & 31;
+  const int rows = U * bm;
+  for (int c = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); c < rows; c += gridDim.x * (blockDim.x / 32)) {
+    const int u = c / bm, j = c - u * bm;
+    const int64_t slot_row = hist_offs[u + 1] + (int64_t)u * bm + j;
+    if (slot_row >= cap) continue;   // offsets beyond the sizes the workspace was made for
+    const uint4* s_row = src + (to_slot ? (int64_t)c * lds : slot_row * lds);
+    uint4* d_row = dst + (to_slot ? slot_row * ldd : (int64_t)c * ldd);
+    for (int w = lane; w < words; w += 32) d_row[w] = s_row[w];
   }
 }
 
@@ -951,24 +970,35 @@ cudaError_t launch_sl_select(int B, int T, const int32_t* offs, const uint32_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_mfalcon_pack(int U, int mb, int bm, const int32_t* hist_offs, const void* hist_x,
-                                const int64_t* hist_ts, const int32_t* cand_offs, const void* cand_x,
-                                const int64_t* cand_ts, int d, int dtype, int32_t* out_offs,
-                                int32_t* out_nt, int64_t* out_ts, void* out_x, int32_t* cand_row_map,
-                                int32_t* cand_src_rows, int cap_rows, cudaStream_t st) {
-  (void)cand_src_rows;
-  mfalcon_offsets_kernel<<<1, kPackThreads, 0, st>>>(U, mb, bm, hist_offs, cand_offs, out_offs, out_nt);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int g = 148 * 4;
+cudaError_t launch_mfalcon_slot_offsets(int U, int bm, const int32_t* hist_offs, int32_t* offs, int32_t* nt,
+                                       cudaStream_t st) {
+  mfalcon_slot_offsets_kernel<<<(U + 256) / 256, 256, 0, st>>>(U, bm, hist_offs, offs, nt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mfalcon_slot_pack(int U, int mb, int bm, int rows_cap, int cap, const int32_t* hist_offs,
+                                     const void* hist_x, const int64_t* hist_ts, const int32_t* cand_offs,
+                                     const void* cand_x, const int64_t* cand_ts, int d, int dtype, int with_hist,
+                                     void* x_slot, int64_t* ts_slot, void* x_c, int32_t* cand_dst, cudaStream_t st) {
+  if (rows_cap <= 0) return cudaSuccess;
+  const int g = min(148 * 8, (rows_cap + 7) / 8);
   if (dtype == HSTU_DTYPE_F32)
-    mfalcon_rows_kernel<float><<<g, 256, 0, st>>>(U, mb, bm, hist_offs, (const float*)hist_x, hist_ts, cand_offs,
-                                                  (const float*)cand_x, cand_ts, d, out_offs, out_ts, (float*)out_x,
-                                                  cand_row_map, cap_rows);
+    mfalcon_slot_pack_kernel<float><<<g, 256, 0, st>>>(U, mb, bm, hist_offs, (const float*)hist_x, hist_ts, cand_offs,
+                                                       (const float*)cand_x, cand_ts, d, with_hist, cap, (float*)x_slot,
+                                                       ts_slot, (float*)x_c, cand_dst);
   else
-    mfalcon_rows_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+    mfalcon_slot_pack_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
         U, mb, bm, hist_offs, (const __nv_bfloat16*)hist_x, hist_ts, cand_offs, (const __nv_bfloat16*)cand_x,
-        cand_ts, d, out_offs, out_ts, (__nv_bfloat16*)out_x, cand_row_map, cap_rows);
+        cand_ts, d, with_hist, cap, (__nv_bfloat16*)x_slot, ts_slot, (__nv_bfloat16*)x_c, cand_dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mfalcon_slot_rows(int U, int bm, int cap, const int32_t* hist_offs, const void* src,
+                                     int64_t lds_bytes, void* dst, int64_t ldd_bytes, int64_t row_bytes, int to_slot,
+                                     cudaStream_t st) {
+  if ((int64_t)U * bm == 0) return cudaSuccess;
+  mfalcon_slot_rows_kernel<<<148 * 8, 256, 0, st>>>(U, bm, hist_offs, (const uint4*)src, lds_bytes / 16, (uint4*)dst,
+                                                    ldd_bytes / 16, (int)(row_bytes / 16), to_slot, cap);
   return cudaGetLastError();
 }
 

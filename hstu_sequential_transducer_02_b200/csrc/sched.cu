@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(kSchedThreads)
 build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restrict__ num_targets,
                        int B, int T, int H, int tm, int tk, int mode, int max_items,
                        WorkItem* __restrict__ items, int32_t* __restrict__ count,
-                       int32_t* __restrict__ status, int32_t* __restrict__ tile_base) {
+                       int32_t* __restrict__ status, int32_t* __restrict__ tile_base, int q_from_hist) {
   using Scan = cub::BlockScan<int, kSchedThreads>;
   __shared__ typename Scan::TempStorage scan_tmp;
   __shared__ int hist_bins[kCostBins];
@@ -86,8 +86,11 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
     // Locality order for dynamically fetched forward items: sequences by number of
     // q tiles (descending), then head, then q tile (descending).  CTAs that run at
     // the same time then share the K/V tiles of a few (sequence, head) pairs.
+    // (with q_from_hist, only the q tiles from the one holding the first target row on)
     for (int s = tid; s < B; s += kSchedThreads) {
-      const int tiles = (offs[s + 1] - offs[s] + tm - 1) / tm;
+      const int n = offs[s + 1] - offs[s];
+      const int t0 = q_from_hist ? (n - (num_targets ? num_targets[s] : 0)) / tm : 0;
+      const int tiles = (n + tm - 1) / tm - t0;
       if (tiles > 0) atomicAdd(&hist_bins[min(tiles, kCostBins - 1)], tiles * H);
     }
     __syncthreads();
@@ -115,10 +118,11 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
     // every sequence's place in the list; the items themselves are then written by
     // all threads (flat index over sequences in order, H * tiles items each)
     __shared__ int seq_base[kSeqSmem];
-    const bool flat = tile_base != nullptr && tm == tk && B <= kSeqSmem;
+    const bool flat = tile_base != nullptr && tm == tk && B <= kSeqSmem && !q_from_hist;
     for (int s = tid; s < B; s += kSchedThreads) {
       const SeqInfo si = load_seq(offs, num_targets, s);
-      const int tiles = (si.n + tm - 1) / tm;
+      const int t0 = q_from_hist ? si.hist / tm : 0;
+      const int tiles = (si.n + tm - 1) / tm - t0;
       if (tiles <= 0) continue;
       const int base_s = atomicAdd(&hist_bins[min(tiles, kCostBins - 1)], tiles * H);
       if (flat) {
@@ -127,7 +131,8 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
       }
       for (int h = 0; h < H; ++h)
         for (int t = 0; t < tiles; ++t)
-          items[base_s + h * tiles + (tiles - 1 - t)] = WorkItem{s, h, t, item_cost(0, t, si.n, si.hist, tm, tk)};
+          items[base_s + h * tiles + (tiles - 1 - t)] =
+              WorkItem{s, h, t0 + t, item_cost(0, t0 + t, si.n, si.hist, tm, tk)};
     }
     if (flat) {
       __syncthreads();
@@ -156,7 +161,8 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
   for (int s = tid; s < B; s += kSchedThreads) {
     SeqInfo si = load_seq(offs, num_targets, s);
     int tiles = mode != 1 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
-    for (int t = 0; t < tiles; ++t) {
+    const int t0 = (q_from_hist && mode != 1) ? si.hist / tm : 0;
+    for (int t = t0; t < tiles; ++t) {
       int c = item_cost(mode, t, si.n, si.hist, tm, tk);
       if (c <= 0) continue;
       atomicAdd(&hist_bins[min(c, kCostBins - 1)], H);
@@ -191,7 +197,8 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
   for (int s = tid; s < B; s += kSchedThreads) {
     SeqInfo si = load_seq(offs, num_targets, s);
     int tiles = mode != 1 ? (si.n + tm - 1) / tm : (si.n + tk - 1) / tk;
-    for (int t = 0; t < tiles; ++t) {
+    const int t0 = (q_from_hist && mode != 1) ? si.hist / tm : 0;
+    for (int t = t0; t < tiles; ++t) {
       int c = item_cost(mode, t, si.n, si.hist, tm, tk);
       if (c <= 0) continue;
       int pos = atomicAdd(&hist_bins[min(c, kCostBins - 1)], H);
@@ -208,9 +215,10 @@ size_t work_list_capacity(int B, int T, int H, int tile) {
 
 cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targets, int B, int T, int H,
                                    int tm, int tk, int mode, int max_items, WorkItem* items,
-                                   int32_t* count, int32_t* status, cudaStream_t stream, int32_t* tile_base) {
+                                   int32_t* count, int32_t* status, cudaStream_t stream, int32_t* tile_base,
+                                   int q_from_hist) {
   build_work_list_kernel<<<1, kSchedThreads, 0, stream>>>(offs, num_targets, B, T, H, tm, tk, mode,
-                                                          max_items, items, count, status, tile_base);
+                                                          max_items, items, count, status, tile_base, q_from_hist);
   return cudaGetLastError();
 }
 

@@ -291,7 +291,17 @@ int mfalcon_rank_workspace_size(const hstu_layer_desc* desc, int32_t num_layers,
  *   hist_ts [hist_total]; cand_x [cand_offsets[U], d], cand_ts [...]: device;
  *   max_candidates: host upper bound on any user's candidate count (sets the
  *   number of microbatches, ceil(max_candidates / microbatch));
- *   hist_x, cand_x, cand_out are in desc->io_dtype; cand_out: [cand_offsets[U], d]. */
+ *   hist_x, cand_x, cand_out are in desc->io_dtype; cand_out: [cand_offsets[U], d].
+ * The history rows do not depend on the candidates, so every layer's keys and
+ * values of the history are computed once, with microbatch 0, and kept in the
+ * workspace (one U|V|Q|K cache per layer, "the history's KV cache is reused
+ * across microbatches"); every later microbatch computes only its candidates'
+ * rows.  Each user keeps b_m candidate slots in every microbatch: slots past the
+ * user's candidates are computed on zero rows and not written out.
+ * Errors: HSTU_ERR_INVALID_ARG (null or misaligned pointers, bad counts),
+ * HSTU_ERR_WORKSPACE (workspace too small or not 256-byte aligned),
+ * HSTU_ERR_CUDA; errors found on the device go to the status word at the start
+ * of the workspace (hstu_workspace_status). */
 int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers,
                  int32_t num_layers, int32_t num_users, int32_t hist_total,
                  int32_t max_candidates, int32_t microbatch,

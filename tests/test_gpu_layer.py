@@ -125,6 +125,47 @@ def test_mfalcon_microbatch_invariance_on_gpu():
     assert_close(a, c.astype(np.float64), "bf16", "b_m 7 vs all")
 
 
+def _mfalcon_ragged(hist_lens, counts, num_layers, microbatch):
+    """Users with the given history lengths and the first counts[u] of their
+    candidates, through num_layers copies of the layer, against the oracle."""
+    b = _b()
+    wl = W.make_workload(3, scale=1 / 32, batch=len(hist_lens), lengths=hist_lens)
+    e = wl.extras
+    s = wl.spec
+    co = e["cand_offsets"]
+    assert min(np.diff(co)) >= max(counts)
+    sel = np.concatenate([np.arange(co[u], co[u] + counts[u]) for u in range(len(counts))]).astype(np.int64)
+    cand_offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    cand_x, cand_ts = e["cand_x"][sel], e["cand_ts"][sel]
+    td = torch_dtype(s.dtype)
+    got = b.mfalcon_rank(_layers(wl) * num_layers, dev(wl.seq_offsets), dev(wl.x, td), dev(wl.timestamps),
+                         dev(cand_offsets), dev(cand_x, td), dev(cand_ts), microbatch, max(counts))
+    torch.cuda.synchronize()
+    got = got.float().cpu().numpy()
+    ref = O.mfalcon_rank([wl.layers[0]] * num_layers, wl.seq_offsets, wl.x, wl.timestamps, cand_offsets, cand_x,
+                         cand_ts, microbatch, s.num_heads, s.head_dim)
+    assert got.shape == ref.shape
+    return got, ref
+
+
+def test_mfalcon_history_cache_ragged_users_two_layers():
+    """A user without candidates and candidate counts that leave partial
+    microbatches (b_m = 7), through two layers: every microbatch after the first
+    reuses the history keys and values cached for both layers; histories that
+    end inside a q tile (37, 130) recompute that tile's history rows."""
+    got, ref = _mfalcon_ragged([64, 9, 37, 64, 130], [5, 9, 0, 23, 12], 2, 7)
+    assert_close(got, ref, "bf16", "mfalcon cached history, ragged users, 2 layers")
+
+
+def test_mfalcon_user_without_history():
+    """A user with no history: its candidates attend only to themselves (N = 1).
+    One layer: with a single attended term the bf16 SiLU's rounding is not
+    averaged over a history, and a second layer amplifies it past the max-abs
+    bound for one of these candidates (a precision limit of the bf16 P)."""
+    got, ref = _mfalcon_ragged([64, 0, 37], [5, 9, 3], 1, 7)
+    assert_close(got, ref, "bf16", "mfalcon user without history")
+
+
 def test_mfalcon_rank_config3_full_size_sampled():
     """Full ranking workload (16 users x (2048 + 4096), b_m = 512); sampled
     candidates against the oracle scoring each candidate alone with its history

@@ -294,6 +294,27 @@ def make_workload(cid: int, *, seed: Optional[int] = None, scale: float = 1.0,
     return Workload(spec, offsets, ts, x, layers, extras=extras)
 
 
+def interleave_item_action(wl: "Workload", seed: int = 7, delay_mean: float = 60.0) -> "Workload":
+    """Ranking input with every item followed by the user's reaction to it (the
+    ranking setting of the pages: the input alternates objects and the reactions
+    that followed them).  Token k of each sequence of `wl` becomes the item at
+    position 2k; its reaction, at 2k + 1, gets an N(0,1) embedding (rounded like
+    the item embeddings) and the item's timestamp plus a floored Exp(delay_mean)
+    delay.  Layers and weights are wl's."""
+    rng = np.random.default_rng(seed)
+    lens = wl.lengths
+    d = wl.x.shape[1]
+    offs2 = offsets_from_lengths(2 * lens)
+    T2 = int(offs2[-1])
+    x = np.empty((T2, d), dtype=np.float32)
+    ts = np.empty(T2, dtype=np.int64)
+    x[0::2] = wl.x
+    x[1::2] = sample_x(rng, wl.total_tokens, d, wl.spec.dtype)
+    ts[0::2] = wl.timestamps
+    ts[1::2] = wl.timestamps + np.floor(rng.exponential(delay_mean, size=wl.total_tokens)).astype(np.int64)
+    return Workload(wl.spec, offs2.astype(np.int32), ts, x, wl.layers)
+
+
 def random_attention_inputs(seed: int, lengths, num_heads: int, head_dim: int, dtype: str,
                             num_targets=None, per_head_rab: bool = False, qk_std: float = 0.25,
                             gap_mean: float = GAP_MEAN_S):

@@ -189,6 +189,31 @@ def test_mfalcon_rank_config3_full_size_sampled():
     assert_close(np.stack(gots), np.stack(refs), "bf16", "mfalcon full sampled")
 
 
+def test_interleaved_item_action_ranking_mask():
+    """Ranking over items interleaved with the reactions that followed them:
+    the item at position 2k is scored from its row, and the mask must hide its
+    own reaction (2k + 1) and every later event.  On the interleaved sequence
+    that is the causal mask with the diagonal: parity with the oracle on every
+    row, and an item's row is bit-identical when its reaction and everything
+    after it change."""
+    wl = W.interleave_item_action(W.make_workload(1, batch=4, scale=0.25))
+    layers = _layers(wl)
+    y = _forward(wl, layers)
+    assert_close(y, _ref(wl), "bf16", "interleaved items and reactions")
+    rng = np.random.default_rng(11)
+    x2 = wl.x.copy()
+    cut = []
+    for s_ in range(len(wl.seq_offsets) - 1):
+        a, z = int(wl.seq_offsets[s_]), int(wl.seq_offsets[s_ + 1])
+        k = int(rng.integers(0, (z - a) // 2))
+        cut.append((a, a + 2 * k))                       # item row a + 2k; its reaction a + 2k + 1
+        x2[a + 2 * k + 1:z] = W.round_to_bf16(rng.standard_normal((z - a - 2 * k - 1, x2.shape[1])).astype(np.float32))
+    wl2 = W.Workload(wl.spec, wl.seq_offsets, wl.timestamps, x2, wl.layers)
+    y2 = _forward(wl2, layers)
+    for a, item in cut:
+        assert np.array_equal(y[a:item + 1], y2[a:item + 1]), "an item's row saw its own reaction or a later event"
+
+
 def test_stochastic_length_bit_exact():
     b = _b()
     wl = W.make_workload(4)

@@ -392,3 +392,25 @@ def test_sampled_row_functions_match_dense():
     y = O.layer_forward(x, p, offs, ts, 2, 4, num_targets=[0, 3])
     yr = O.layer_forward_rows(x, p, offs, ts, 2, 4, [(0, 3), (1, 0), (1, 11)], num_targets=[0, 3])
     assert np.allclose(yr, y[[3, 7, 18]], rtol=1e-12, atol=1e-12)
+
+
+def test_interleaved_ranking_mask_hides_the_reaction():
+    """Ranking over items interleaved with their reactions: the causal mask with
+    the diagonal hides an item's own reaction (the next position) and every
+    later event, so the oracle's item row does not move when they change, and
+    it does move when an earlier reaction changes."""
+    wl = W.interleave_item_action(W.make_workload(0, batch=2))
+    s_ = wl.spec
+    y = O.stack_forward(wl.x, wl.layers, wl.seq_offsets, wl.timestamps, s_.num_heads, s_.head_dim)
+    a, z = int(wl.seq_offsets[0]), int(wl.seq_offsets[1])
+    k = (z - a) // 4
+    item = a + 2 * k
+    rng = np.random.default_rng(3)
+    x2 = wl.x.copy()
+    x2[item + 1:z] = rng.standard_normal((z - item - 1, x2.shape[1]))   # a shift alone would cancel in LayerNorm
+    y2 = O.stack_forward(x2, wl.layers, wl.seq_offsets, wl.timestamps, s_.num_heads, s_.head_dim)
+    assert np.array_equal(y[a:item + 1], y2[a:item + 1])
+    x3 = wl.x.copy()
+    x3[item - 1] = rng.standard_normal(x3.shape[1])   # the previous item's reaction
+    y3 = O.stack_forward(x3, wl.layers, wl.seq_offsets, wl.timestamps, s_.num_heads, s_.head_dim)
+    assert not np.allclose(y[item], y3[item])

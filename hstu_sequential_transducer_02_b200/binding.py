@@ -92,6 +92,11 @@ _lib_layer_fwd_ws = _sig("hstu_layer_fwd_workspace_size", _c_int, [_P(LayerDesc)
 _lib_layer_fwd = _sig("hstu_layer_fwd", _c_int,
                       [_P(LayerDesc), _P(LayerWeights), _P(Jagged), _c_vp, _c_vp, _P(LayerSaved), _c_vp, _c_size,
                        _c_vp])
+_lib_layer_fwd_host_ws = _sig("hstu_layer_fwd_host_workspace_size", _c_int,
+                              [_P(LayerDesc), _c_i32, _c_i32, _c_i32, _P(_c_size)])
+_lib_layer_fwd_host = _sig("hstu_layer_fwd_host", _c_int,
+                           [_P(LayerDesc), _P(LayerWeights), _c_i32, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i32,
+                            _c_vp, _c_size, _c_vp])
 _lib_layer_bwd_ws = _sig("hstu_layer_bwd_workspace_size", _c_int, [_P(LayerDesc), _c_i32, _c_i32, _P(_c_size)])
 _lib_layer_bwd = _sig("hstu_layer_bwd", _c_int,
                       [_P(LayerDesc), _P(LayerWeights), _P(Jagged), _c_vp, _P(LayerSaved), _c_vp, _c_vp,
@@ -109,7 +114,8 @@ _lib_dbg_timeout = _sig("hstu_debug_timeout_probe", _c_int, [_c_i64, _c_vp, _c_v
 
 EXPORTED = ["hstu_status_string", "hstu_version", "hstu_build_time_thresholds", "hstu_workspace_status",
             "hstu_attn_fwd_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd_workspace_size", "hstu_attn_bwd",
-            "hstu_layer_fwd_workspace_size", "hstu_layer_fwd", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
+            "hstu_layer_fwd_workspace_size", "hstu_layer_fwd", "hstu_layer_fwd_host_workspace_size",
+            "hstu_layer_fwd_host", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
             "mfalcon_rank_workspace_size", "mfalcon_rank", "hstu_stochastic_length_workspace_size",
             "hstu_stochastic_length", "hstu_gather_rows", "hstu_debug_rab_buckets", "hstu_debug_timeout_probe"]
 
@@ -323,6 +329,31 @@ class Layer:
         _check(_lib_layer_fwd(ctypes.byref(self.desc), ctypes.byref(self.cw), ctypes.byref(jb), _ptr(x), _ptr(y),
                               ctypes.byref(sv) if sv is not None else None, _ptr(ws), ws.numel(), _stream(stream)),
                "hstu_layer_fwd")
+        return y
+
+    def forward_host(self, x, seq_offsets, timestamps, num_chunks: int, num_targets=None, out=None, device=None,
+                     stream=None):
+        """The forward from and to host memory (hstu_layer_fwd_host): x, out [T, d]
+        and timestamps on the host (page-locked for the copies to overlap the
+        computation), seq_offsets / num_targets host int32 tensors."""
+        for t in (x, seq_offsets, timestamps) + ((num_targets,) if num_targets is not None else ()):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError("forward_host takes contiguous host tensors")
+        B = seq_offsets.numel() - 1
+        T = int(seq_offsets[-1])
+        dev = torch.device("cuda") if device is None else device
+        nbytes = _c_size()
+        _check(_lib_layer_fwd_host_ws(ctypes.byref(self.desc), B, T, num_chunks, ctypes.byref(nbytes)),
+               "hstu_layer_fwd_host_workspace_size")
+        ws = self._ws.get("fwd_host")
+        if ws is None or ws.numel() < nbytes.value or ws.device != dev:
+            ws = _workspace(nbytes.value, dev)
+            self._ws["fwd_host"] = ws
+        y = torch.empty_like(x) if out is None else out
+        _check(_lib_layer_fwd_host(ctypes.byref(self.desc), ctypes.byref(self.cw), B, _ptr(seq_offsets),
+                                   _ptr(num_targets) if num_targets is not None else None, _ptr(timestamps),
+                                   _ptr(x), _ptr(y), num_chunks, _ptr(ws), ws.numel(), _stream(stream)),
+               "hstu_layer_fwd_host")
         return y
 
     def backward(self, x, dy, saved: Saved, seq_offsets, timestamps, num_targets=None, grads=None, dx=None,

@@ -2,6 +2,7 @@
 // sequence of each call.  Every step of the computation runs in this
 // library's own kernels; nothing here computes on the host except the
 // time-bucket threshold table.
+#include <algorithm>
 #include <math.h>
 #include <stdio.h>
 #include <mutex>
@@ -686,6 +687,151 @@ int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
   LayerFwdWs ws = carve_layer_fwd(c, desc, jb->batch, jb->total_tokens, true);
   HSTU_CUDA(cudaMemsetAsync(ws.attn.status, 0, kStatusBytes, st));
   return run_layer_fwd(desc, w, jb, x, y, saved, ws, st);
+}
+
+// ---------------------------------------------------------------- layer forward from host memory
+namespace {
+constexpr int kMaxChunks = 64;
+
+// Per device: one copy stream each way and the events that chain a call's
+// chunks; a call enqueues under the mutex, so calls do not share events while
+// they are being recorded.
+struct CopyStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in[kMaxChunks] = {}, out[kMaxChunks] = {};
+};
+std::mutex g_copy_mu;
+CopyStreams g_copy[kMaxDevices];
+
+int copy_streams(CopyStreams** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
+  CopyStreams& cs = g_copy[dev];
+  if (!cs.h2d) {
+    HSTU_CUDA(cudaStreamCreateWithFlags(&cs.h2d, cudaStreamNonBlocking));
+    HSTU_CUDA(cudaStreamCreateWithFlags(&cs.d2h, cudaStreamNonBlocking));
+    HSTU_CUDA(cudaEventCreateWithFlags(&cs.start, cudaEventDisableTiming));
+    HSTU_CUDA(cudaEventCreateWithFlags(&cs.done, cudaEventDisableTiming));
+    for (int i = 0; i < kMaxChunks; ++i) {
+      HSTU_CUDA(cudaEventCreateWithFlags(&cs.in[i], cudaEventDisableTiming));
+      HSTU_CUDA(cudaEventCreateWithFlags(&cs.out[i], cudaEventDisableTiming));
+    }
+  }
+  *out = &cs;
+  return HSTU_OK;
+}
+
+struct HostFwdWs {
+  LayerFwdWs layer;
+  void* x;            // [T, d] io_dtype
+  void* y;            // [T, d]
+  int64_t* ts;        // [T]
+  int32_t* offs;      // [B+1] as given
+  int32_t* nt;        // [B]
+  int32_t* chunk_offs;  // kMaxChunks x [B+1], rebased per chunk
+};
+
+HostFwdWs carve_host_fwd(Carver& c, const hstu_layer_desc* d, int B, int T) {
+  HostFwdWs w;
+  w.layer = carve_layer_fwd(c, d, B, T, true);
+  const size_t eio = elem_size(d->io_dtype);
+  w.x = c.take<char>((size_t)T * d->d_model * eio);
+  w.y = c.take<char>((size_t)T * d->d_model * eio);
+  w.ts = c.take<int64_t>(T > 0 ? T : 1);
+  w.offs = c.take<int32_t>((size_t)B + 1);
+  w.nt = c.take<int32_t>(B > 0 ? B : 1);
+  w.chunk_offs = c.take<int32_t>((size_t)kMaxChunks * (B + 1));
+  return w;
+}
+}  // namespace
+
+int hstu_layer_fwd_host_workspace_size(const hstu_layer_desc* desc, int32_t batch, int32_t total_tokens,
+                                       int32_t num_chunks, size_t* bytes) {
+  if (!desc || !bytes || batch < 0 || total_tokens < 0 || num_chunks < 1) return HSTU_ERR_INVALID_ARG;
+  HSTU_TRY(check_attn_desc(&desc->attn));
+  Carver c(nullptr);
+  carve_host_fwd(c, desc, batch, total_tokens);
+  *bytes = c.size();
+  return HSTU_OK;
+}
+
+int hstu_layer_fwd_host(const hstu_layer_desc* desc, const hstu_layer_weights* w, int32_t batch,
+                        const int32_t* seq_offsets, const int32_t* num_targets, const int64_t* timestamps,
+                        const void* x, void* y, int32_t num_chunks, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  HSTU_TRY(check_layer(desc, w));
+  if (batch < 0 || num_chunks < 1 || !seq_offsets || !x || !y) return HSTU_ERR_INVALID_ARG;
+  if (seq_offsets[0] != 0) return HSTU_ERR_INVALID_ARG;
+  for (int s = 0; s < batch; ++s)
+    if (seq_offsets[s + 1] < seq_offsets[s]) return HSTU_ERR_INVALID_ARG;
+  const int T = seq_offsets[batch];
+  if (T > 0 && !timestamps) return HSTU_ERR_INVALID_ARG;
+  size_t need;
+  HSTU_TRY(hstu_layer_fwd_host_workspace_size(desc, batch, T, num_chunks, &need));
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carver c(workspace);
+  HostFwdWs ws = carve_host_fwd(c, desc, batch, T);
+  HSTU_CUDA(cudaMemsetAsync(ws.layer.attn.status, 0, kStatusBytes, st));
+  if (batch == 0 || T == 0) return HSTU_OK;
+  const int dm = desc->d_model;
+  const size_t row_bytes = (size_t)dm * elem_size(desc->io_dtype);
+  // chunks of consecutive sequences with about T / nc tokens each
+  const int nc = std::min(std::min(num_chunks, batch), kMaxChunks);
+  int bounds[kMaxChunks + 1];
+  bounds[0] = 0;
+  for (int ch = 1, s = 0; ch < nc; ++ch) {
+    const int64_t target = (int64_t)T * ch / nc;
+    while (s < batch - (nc - ch) && seq_offsets[s + 1] <= target) ++s;
+    if (s < bounds[ch - 1] + 1) s = bounds[ch - 1] + 1;
+    bounds[ch] = s;
+  }
+  bounds[nc] = batch;
+  std::lock_guard<std::mutex> lk(g_copy_mu);
+  CopyStreams* cs = nullptr;
+  HSTU_TRY(copy_streams(&cs));
+  // the copies may overwrite the workspace only after the stream's earlier work
+  HSTU_CUDA(cudaEventRecord(cs->start, st));
+  HSTU_CUDA(cudaStreamWaitEvent(cs->h2d, cs->start, 0));
+  HSTU_CUDA(cudaStreamWaitEvent(cs->d2h, cs->start, 0));
+  HSTU_CUDA(cudaMemcpyAsync(ws.offs, seq_offsets, sizeof(int32_t) * (batch + 1), cudaMemcpyHostToDevice, cs->h2d));
+  if (num_targets)
+    HSTU_CUDA(cudaMemcpyAsync(ws.nt, num_targets, sizeof(int32_t) * batch, cudaMemcpyHostToDevice, cs->h2d));
+  for (int ch = 0; ch < nc; ++ch) {
+    const int r0 = seq_offsets[bounds[ch]], r1 = seq_offsets[bounds[ch + 1]];
+    if (r1 > r0) {
+      HSTU_CUDA(cudaMemcpyAsync((char*)ws.x + r0 * row_bytes, (const char*)x + r0 * row_bytes,
+                                (size_t)(r1 - r0) * row_bytes, cudaMemcpyHostToDevice, cs->h2d));
+      HSTU_CUDA(cudaMemcpyAsync(ws.ts + r0, timestamps + r0, sizeof(int64_t) * (r1 - r0), cudaMemcpyHostToDevice,
+                                cs->h2d));
+    }
+    HSTU_CUDA(cudaEventRecord(cs->in[ch], cs->h2d));
+  }
+  for (int ch = 0; ch < nc; ++ch) {
+    const int s0 = bounds[ch], nb = bounds[ch + 1] - s0;
+    const int r0 = seq_offsets[s0], r1 = seq_offsets[s0 + nb];
+    HSTU_CUDA(cudaStreamWaitEvent(st, cs->in[ch], 0));
+    int32_t* co = ws.chunk_offs + (size_t)ch * (batch + 1);
+    HSTU_CUDA(launch_rebase_offsets(ws.offs, s0, nb, co, st));
+    hstu_jagged jb;
+    jb.batch = nb;
+    jb.total_tokens = r1 - r0;
+    jb.seq_offsets = co;
+    jb.num_targets = num_targets ? ws.nt + s0 : nullptr;
+    jb.timestamps = ws.ts + r0;
+    HSTU_TRY(run_layer_fwd(desc, w, &jb, (const char*)ws.x + r0 * row_bytes, (char*)ws.y + r0 * row_bytes, nullptr,
+                           ws.layer, st));
+    HSTU_CUDA(cudaEventRecord(cs->out[ch], st));
+    HSTU_CUDA(cudaStreamWaitEvent(cs->d2h, cs->out[ch], 0));
+    if (r1 > r0)
+      HSTU_CUDA(cudaMemcpyAsync((char*)y + r0 * row_bytes, (const char*)ws.y + r0 * row_bytes,
+                                (size_t)(r1 - r0) * row_bytes, cudaMemcpyDeviceToHost, cs->d2h));
+  }
+  HSTU_CUDA(cudaEventRecord(cs->done, cs->d2h));
+  HSTU_CUDA(cudaStreamWaitEvent(st, cs->done, 0));
+  return HSTU_OK;
 }
 
 int hstu_layer_bwd_workspace_size(const hstu_layer_desc* desc, int32_t batch, int32_t total_tokens, size_t* bytes) {

@@ -185,6 +185,8 @@ cudaError_t launch_gather_rows(const void* src, void* dst, int64_t row_bytes, co
 cudaError_t launch_sl_select(int B, int T, const int32_t* offs, const uint32_t* coins, const uint32_t* keys,
                              int max_len, uint32_t prob, int32_t* out_offsets, int32_t* out_index,
                              int32_t* scratch_len, int32_t* status, cudaStream_t st);
+// out[i] = offs[s0 + i] - offs[s0] for i in [0, nb]
+cudaError_t launch_rebase_offsets(const int32_t* offs, int s0, int nb, int32_t* out, cudaStream_t st);
 // rows r < *total_rows (total_rows null: r < cap_rows) with cand_row_map[r] >= 0 go to that row of cand_out
 cudaError_t launch_mfalcon_scatter(const void* y, int d, int dtype, const int32_t* cand_row_map,
                                    const int32_t* total_rows, int cap_rows, void* cand_out, cudaStream_t st);

@@ -583,6 +583,12 @@ __global__ void mfalcon_slot_rows_kernel(int U, int bm, const int32_t* __restric
   }
 }
 
+// offsets of sequences [s0, s0 + nb] rebased to start at row 0
+__global__ void rebase_offsets_kernel(const int32_t* __restrict__ offs, int s0, int nb, int32_t* __restrict__ out) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= nb; i += gridDim.x * blockDim.x)
+    out[i] = offs[s0 + i] - offs[s0];
+}
+
 template <typename TS, typename TD>
 __global__ void convert_rows_kernel(const TS* __restrict__ src, int64_t lds, TD* __restrict__ dst, int64_t ldd,
                                     int cols, int rows_cap, const int32_t* __restrict__ rows_dev, int pad_multiple) {
@@ -967,6 +973,11 @@ cudaError_t launch_sl_select(int B, int T, const int32_t* offs, const uint32_t* 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || B == 0) return e;
   sl_select_kernel<<<B, kSlThreads, 0, st>>>(B, offs, coins, keys, max_len, prob, out_offsets, out_index);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rebase_offsets(const int32_t* offs, int s0, int nb, int32_t* out, cudaStream_t st) {
+  rebase_offsets_kernel<<<(nb + 256) / 256, 256, 0, st>>>(offs, s0, nb, out);
   return cudaGetLastError();
 }
 

@@ -261,6 +261,32 @@ int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w,
                    const hstu_layer_saved* saved,
                    void* workspace, size_t workspace_bytes, void* stream);
 
+/* The layer forward from and to HOST memory: the sequences are split into
+ * `num_chunks` groups of consecutive sequences with about equal token counts;
+ * chunk c's X rows and timestamps are copied in while chunk c-1 is computed
+ * and chunk c-2's Y rows are copied out (one copy stream each way), so that on
+ * a full-duplex link the call takes about as long as the larger of the two
+ * transfers.  Every row is computed exactly as hstu_layer_fwd computes it on
+ * the whole batch (rows of different sequences do not interact), so Y is
+ * bit-identical to that call's.
+ *   seq_offsets [batch+1], num_targets [batch] (or NULL), timestamps [T]:
+ *     HOST arrays, read during the call (T = seq_offsets[batch]);
+ *   x [T, d], y [T, d]: HOST, io_dtype, contiguous; page-locked memory
+ *     (cudaHostAlloc / cudaHostRegister) is needed for the copies to overlap
+ *     the computation, pageable memory works but serialises them;
+ *   num_chunks: 1 .. 64 (clamped to batch);
+ *   workspace: device, hstu_layer_fwd_host_workspace_size bytes, 256-aligned.
+ * The call returns once everything is enqueued; `stream` is complete when Y is
+ * in host memory.  Errors: HSTU_ERR_INVALID_ARG (null pointers, batch < 0,
+ * offsets not starting at 0 or decreasing, num_chunks < 1), HSTU_ERR_WORKSPACE,
+ * HSTU_ERR_CUDA; device-side errors go to the workspace status word. */
+int hstu_layer_fwd_host_workspace_size(const hstu_layer_desc* desc, int32_t batch,
+                                       int32_t total_tokens, int32_t num_chunks, size_t* bytes);
+int hstu_layer_fwd_host(const hstu_layer_desc* desc, const hstu_layer_weights* w, int32_t batch,
+                        const int32_t* seq_offsets, const int32_t* num_targets,
+                        const int64_t* timestamps, const void* x, void* y, int32_t num_chunks,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 int hstu_layer_bwd_workspace_size(const hstu_layer_desc* desc, int32_t batch,
                                   int32_t total_tokens, size_t* bytes);
 

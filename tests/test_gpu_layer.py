@@ -85,6 +85,34 @@ def test_layer_config2_full_size_sampled_rows():
     assert np.all(np.isfinite(y))
 
 
+def test_layer_forward_from_host_memory_bit_identical():
+    """hstu_layer_fwd_host (chunks of sequences whose copies overlap the
+    computation) gives Y bit for bit equal to hstu_layer_fwd on the whole device
+    batch: for 1, 3, 8 and 64 chunks from page-locked memory, from pageable
+    memory, and with M-FALCON targets."""
+    wl = W.make_workload(1, batch=9, scale=0.5)
+    ly = _layers(wl)[0]
+    td = torch_dtype(wl.spec.dtype)
+    x_d, offs_d, ts_d = dev(wl.x, td), dev(wl.seq_offsets), dev(wl.timestamps)
+    y_ref = ly.forward(x_d, offs_d, ts_d).cpu()
+    x_h = torch.from_numpy(wl.x).to(td).pin_memory()
+    offs_h = torch.from_numpy(wl.seq_offsets.astype(np.int32))
+    ts_h = torch.from_numpy(wl.timestamps).pin_memory()
+    for nc in (1, 3, 8, 64):
+        y_h = torch.empty_like(x_h).pin_memory()
+        ly.forward_host(x_h, offs_h, ts_h, nc, out=y_h)
+        torch.cuda.synchronize()
+        assert torch.equal(y_h, y_ref), f"{nc} chunks"
+    y_p = ly.forward_host(torch.from_numpy(wl.x).to(td), offs_h, torch.from_numpy(wl.timestamps), 2)
+    torch.cuda.synchronize()
+    assert torch.equal(y_p, y_ref), "pageable memory"
+    nt = np.minimum([3, 0, 17, 1, 40, 2, 0, 5, 9], wl.lengths).astype(np.int32)
+    y_ref_t = ly.forward(x_d, offs_d, ts_d, num_targets=dev(nt)).cpu()
+    y_t = ly.forward_host(x_h, offs_h, ts_h, 4, num_targets=torch.from_numpy(nt))
+    torch.cuda.synchronize()
+    assert torch.equal(y_t, y_ref_t), "targets"
+
+
 def test_layer_mfalcon_targets_in_layer_call():
     wl = W.make_workload(1, batch=5, scale=0.5)
     nt = np.array([3, 0, 17, 1, 40], dtype=np.int32)

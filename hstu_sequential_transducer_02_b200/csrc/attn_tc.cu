@@ -162,15 +162,16 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
       : "memory");
 }
 
-// O of a finished work item, once its last P V is done: this warp's kOc columns of
-// its 32 rows -> (1/N) -> bf16 -> global memory (`out` null for rows beyond the
-// sequence).  Returns false on a timeout.
+// A deferred O readout of one epilogue thread: its output row (null for rows
+// beyond the sequence) and 1/N.  Kept in shared memory, not in registers.
 struct PendingO {
   __nv_bfloat16* out;
   float inv_n;
   int pad;
 };
 
+// O of a finished work item, once its last P V is done: this warp's kOc columns of
+// its 32 rows -> (1/N) -> bf16 -> global memory.  Returns false on a timeout.
 template <int kOc>
 __device__ __forceinline__ bool o_readout(Barriers* bars, int parity, uint32_t taddr, const PendingO* pend,
                                           int lane, long long tmo, volatile int* abort_flag) {
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
     constexpr int kOc = DV / 4;
     int pend_par = -1;                       // parity of the pending readout's o_full phase; -1: none
     // this lane's output row (null beyond the sequence) and 1/N, kept in shared memory
-#define HSTU_PEND (reinterpret_cast<PendingO*>(smem + L::kPend) + (threadIdx.x - 32 * kEpiWarp0))
+const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + (threadIdx.x - 32 * kEpiWarp0); };
     for (int k = 0;; ++k) {
       const int slot = k % kItemSlots;
       if (!mbar_wait(&bars->it_full[slot], (k / kItemSlots) & 1, tmo, abort_flag)) goto fail;
@@ -483,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         if (!s_ready && pend_par >= 0) {
           // S may depend on P V of this item, which waits until every warp has read
           // the previous item's O: the pending readout goes first
-          if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+          if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, pend(), lane, tmo, abort_flag)) goto fail;
           pend_par = -1;
           s_ready = __all_sync(0xffffffffu, mbar_try_wait(&bars->s_full[sb], (it / kSBufs) & 1));
         }
@@ -675,25 +676,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_tc_kernel(const __grid_c
         }
         // the pending readout as soon as the previous item's O is complete
         if (pend_par >= 0 && __all_sync(0xffffffffu, mbar_try_wait(&bars->o_full, pend_par))) {
-          if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+          if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, pend(), lane, tmo, abort_flag)) goto fail;
           pend_par = -1;
         }
       }
       // ---- this item's O readout becomes the pending one (an older one is done first)
       if (pend_par >= 0) {
-        if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+        if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, pend(), lane, tmo, abort_flag)) goto fail;
       }
       pend_par = k & 1;
-      HSTU_PEND->out = live ? reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(si.start + i) * p.ldo +
+      pend()->out = live ? reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)(si.start + i) * p.ldo +
                              (int64_t)wi.head * DV + seg * kOc
                        : nullptr;
-      HSTU_PEND->inv_n = si.inv_n;
+      pend()->inv_n = si.inv_n;
     }
     if (pend_par >= 0) {
-      if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, HSTU_PEND, lane, tmo, abort_flag)) goto fail;
+      if (!o_readout<kOc>(bars, pend_par, tmem_o + lane_off + seg * kOc, pend(), lane, tmo, abort_flag)) goto fail;
     }
   }
-#undef HSTU_PEND
   goto teardown;
 fail:
   set_status(p.status, HSTU_ERR_TIMEOUT);

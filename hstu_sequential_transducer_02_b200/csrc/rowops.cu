@@ -506,7 +506,7 @@ __global__ void mfalcon_slot_offsets_kernel(int U, int bm, const int32_t* __rest
 
 // Microbatch mb in the slot layout, one warp per row: candidate j of user u is
 // candidate mb * bm + j of that user, or a zero row (timestamp of the user's last
-// history token, else 0) past the user's candidates.  With with_hist the history
+// history token, else of its last candidate, else 0) past the user's candidates.  With with_hist the history
 // rows are written too (x and timestamps) and the rows walked are all slot-layout
 // rows; otherwise only the candidate rows.  x_slot and x_c may each be null.
 template <typename T>
@@ -551,6 +551,8 @@ __global__ void mfalcon_slot_pack_kernel(int U, int mb, int bm, const int32_t* _
         ts = cand_ts[cand_offs[u] + ci];
       } else if (hist_offs[u + 1] > hist_offs[u]) {
         ts = hist_ts[hist_offs[u + 1] - 1];
+      } else if (m > 0) {
+        ts = cand_ts[cand_offs[u + 1] - 1];   // no history: keep the sequence's offsets small
       }
       if (lane == 0) cand_dst[u * bm + j] = ci < m ? cand_offs[u] + ci : -1;
     }

@@ -303,9 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         // far segment: history rows at least 127 positions past every kv row of the
         // warp, so the position bucket is the last one; with one time bucket per
         // lane the bias is constant and dS is summed in registers
-        bool fast = false;
+        // (`two`: the same with at most two time buckets per lane, told apart by one
+        // threshold compare per element, each summed in registers)
+        bool fast = false, two = false;
         int tlo = 0;
-        float hb = 0.f;
+        float hb = 0.f, hb1 = 0.f;
+        int32_t th1 = 0x7FFFFFFF;
         if (wnarrow && i0 + 31 < si.hist && i0 - (j0w + 31) >= kNumBuckets - 1) {
           const int32_t mn = __reduce_min_sync(0xffffffffu, relc), mx = __reduce_max_sync(0xffffffffu, relc);
           int32_t dlo, dhi;
@@ -313,13 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           else if (rj <= mn) { dlo = mn - rj; dhi = mx - rj; }
           else { dlo = 0; dhi = max(rj - mn, mx - rj); }
           tlo = fast_bucket(dlo, thr32, k_lg);
-          fast = __all_sync(0xffffffffu, dhi < thr32[tlo + 1]);
+          th1 = thr32[tlo + 1];
+          fast = __all_sync(0xffffffffu, dhi < th1);
+          two = !fast && __all_sync(0xffffffffu, dhi < thr32[tlo + 2]);   // tlo < 127 here
           hb = pos_b[kNumBuckets - 1] + time_b[tlo];
+          if (two) hb1 = pos_b[kNumBuckets - 1] + time_b[tlo + 1];
         }
         if (!mbar_wait(&bars->sp_full, qi & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
         int cur_tb = -1;
-        float acc_t = 0.f, acc_fast = 0.f;
+        float acc_t = 0.f, acc_fast = 0.f, acc_two = 0.f;
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
           const int cb = 32 * seg + 16 * hh;   // first q column of this half inside the tile
@@ -336,6 +342,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
               pv[e] = jlive ? f * si.inv_n : 0.f;
               dsv[e] = jlive ? __uint_as_float(dr[e]) * g * si.inv_n : 0.f;
               acc_fast += dsv[e];
+            }
+          } else if (two) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int32_t dd = abs(__shfl_sync(0xffffffffu, relc, 16 * hh + e) - rj);
+              const bool up = dd >= th1;   // bucket tlo + 1, else tlo
+              float f, g;
+              silu_and_grad(__uint_as_float(sr[e]) + (up ? hb1 : hb), f, g);
+              pv[e] = jlive ? f * si.inv_n : 0.f;
+              dsv[e] = jlive ? __uint_as_float(dr[e]) * g * si.inv_n : 0.f;
+              acc_fast += up ? 0.f : dsv[e];
+              acc_two += up ? dsv[e] : 0.f;
             }
           } else {
 #pragma unroll
@@ -385,6 +403,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         if (fast) {
           if (jlive) atomicAdd(&gtime[tlo], acc_fast);
           far_pos += acc_fast;   // position bucket 127, added once per item
+        } else if (two) {
+          if (jlive) {
+            if (acc_fast != 0.f) atomicAdd(&gtime[tlo], acc_fast);
+            if (acc_two != 0.f) atomicAdd(&gtime[tlo + 1], acc_two);
+          }
+          far_pos += acc_fast + acc_two;
         } else if (acc_t != 0.f) {
           atomicAdd(&gtime[cur_tb], acc_t);
         }

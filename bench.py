@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--oracle-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the M-FALCON and training-step measurements")
+    ap.add_argument("--profile-attn-bwd", action="store_true",
+                    help="for profilers: run the training workload's attention backward (1 + 3 launches) and exit")
     return ap.parse_args()
 
 
@@ -489,6 +491,36 @@ def measure_training(hb, steps: int):
 # our arm
 # ----------------------------------------------------------------------------
 
+def profile_attn_bwd():
+    """The attention backward alone on the training workload's shapes (the
+    sequence lengths Stochastic Length leaves, 8 heads of 64, bf16): one launch,
+    then three timed ones; prints their mean time.  A target for profilers."""
+    import torch
+    from hstu_sequential_transducer_02_b200 import binding as hb
+    wl = W.make_workload(4)
+    e = wl.extras
+    offs, _ = hb.stochastic_length(torch.from_numpy(wl.seq_offsets).cuda(),
+                                   torch.from_numpy(e["sl_coin"].view(np.int32)).cuda(),
+                                   torch.from_numpy(e["sl_keys"].view(np.int32)).cuda(), int(e["sl_len"]),
+                                   int(e["sl_prob_u32"]))
+    lens = np.diff(offs.cpu().numpy())
+    H, dh = wl.spec.num_heads, wl.spec.head_dim
+    d = W.random_attention_inputs(3, lens, H, dh, "bf16", qk_std=0.5)
+    T = int(sum(lens))
+    q, k, v, do = (torch.from_numpy(d[n].reshape(T, H * dh)).to(torch.bfloat16).cuda() for n in ("q", "k", "v", "dout"))
+    args = (torch.from_numpy(d["seq_offsets"]).cuda(), torch.from_numpy(d["timestamps"]).cuda(),
+            torch.from_numpy(d["pos_bias"]).cuda(), torch.from_numpy(d["time_bias"]).cuda(), H)
+    hb.attn_bwd(q, k, v, do, *args)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        hb.attn_bwd(q, k, v, do, *args)
+    e1.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"attn_bwd_ms": e0.elapsed_time(e1) / 3, "tokens": T, "heads": H, "head_dim": dh}))
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -496,6 +528,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.profile_attn_bwd:
+        profile_attn_bwd()
         return
     import torch
     import torch.distributed as dist

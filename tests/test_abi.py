@@ -109,3 +109,31 @@ def test_null_arguments_rejected_before_any_launch():
                            None) == b.ERR_WORKSPACE
     assert b._lib_dbg_timeout(0, None, None) == b.ERR_INVALID_ARG
     assert b._lib_gather(p, p, 6, p, p, 1, None) == b.ERR_INVALID_ARG
+
+
+def test_host_memory_forward_argument_checks():
+    """hstu_layer_fwd_host validates its host offsets and sizes before it
+    touches the GPU: offsets must start at 0 and not decrease, x and y must be
+    given, num_chunks >= 1, and the workspace must be large enough."""
+    b = _lib()
+    ld = b.layer_desc(64, 2, 32, b.DTYPE_BF16)
+    n = ctypes.c_size_t()
+    assert b._lib_layer_fwd_host_ws(ctypes.byref(ld), 3, 100, 4, ctypes.byref(n)) == b.OK
+    assert n.value > 0 and n.value % 256 == 0
+    assert b._lib_layer_fwd_host_ws(ctypes.byref(ld), 3, 100, 0, ctypes.byref(n)) == b.ERR_INVALID_ARG
+    p = ctypes.c_void_p(1 << 20)     # never dereferenced: every call below fails its host checks
+    w = b.LayerWeights(*([p] * 10))
+    ts = (ctypes.c_int64 * 100)()
+    x = (ctypes.c_uint16 * 6400)()
+    y = (ctypes.c_uint16 * 6400)()
+
+    def call(offs, xx=x, chunks=2, ws_bytes=1 << 40):
+        o = (ctypes.c_int32 * len(offs))(*offs)
+        return b._lib_layer_fwd_host(ctypes.byref(ld), ctypes.byref(w), len(offs) - 1, o, None, ts, xx, y, chunks,
+                                     p, ws_bytes, None)
+
+    assert call([1, 40, 100]) == b.ERR_INVALID_ARG            # does not start at 0
+    assert call([0, 60, 40]) == b.ERR_INVALID_ARG             # decreasing
+    assert call([0, 40, 100], xx=None) == b.ERR_INVALID_ARG
+    assert call([0, 40, 100], chunks=0) == b.ERR_INVALID_ARG
+    assert call([0, 40, 100], ws_bytes=256) == b.ERR_WORKSPACE

@@ -249,9 +249,11 @@ int side_stream(SideStream** out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
   SideStream& ss = g_side[dev];
   if (!ss.s) {
-    HSTU_CUDA(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));
-    HSTU_CUDA(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
-    HSTU_CUDA(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+    SideStream n;   // becomes the device's only once every handle exists
+    HSTU_CUDA(cudaStreamCreateWithFlags(&n.s, cudaStreamNonBlocking));
+    HSTU_CUDA(cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming));
+    HSTU_CUDA(cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming));
+    ss = n;
   }
   *out = &ss;
   return HSTU_OK;
@@ -709,14 +711,17 @@ int copy_streams(CopyStreams** out) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
   CopyStreams& cs = g_copy[dev];
   if (!cs.h2d) {
-    HSTU_CUDA(cudaStreamCreateWithFlags(&cs.h2d, cudaStreamNonBlocking));
-    HSTU_CUDA(cudaStreamCreateWithFlags(&cs.d2h, cudaStreamNonBlocking));
-    HSTU_CUDA(cudaEventCreateWithFlags(&cs.start, cudaEventDisableTiming));
-    HSTU_CUDA(cudaEventCreateWithFlags(&cs.done, cudaEventDisableTiming));
+    // created into a copy that becomes the device's only once every handle exists
+    CopyStreams n;
+    HSTU_CUDA(cudaStreamCreateWithFlags(&n.h2d, cudaStreamNonBlocking));
+    HSTU_CUDA(cudaStreamCreateWithFlags(&n.d2h, cudaStreamNonBlocking));
+    HSTU_CUDA(cudaEventCreateWithFlags(&n.start, cudaEventDisableTiming));
+    HSTU_CUDA(cudaEventCreateWithFlags(&n.done, cudaEventDisableTiming));
     for (int i = 0; i < kMaxChunks; ++i) {
-      HSTU_CUDA(cudaEventCreateWithFlags(&cs.in[i], cudaEventDisableTiming));
-      HSTU_CUDA(cudaEventCreateWithFlags(&cs.out[i], cudaEventDisableTiming));
+      HSTU_CUDA(cudaEventCreateWithFlags(&n.in[i], cudaEventDisableTiming));
+      HSTU_CUDA(cudaEventCreateWithFlags(&n.out[i], cudaEventDisableTiming));
     }
+    cs = n;
   }
   *out = &cs;
   return HSTU_OK;

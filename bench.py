@@ -263,109 +263,18 @@ def read_traffic(kernel: str, path: str = None):
 
 
 # ----------------------------------------------------------------------------
-# multi-rank plumbing (host logic; covered on CPU with gloo ranks)
-# ----------------------------------------------------------------------------
-
-def rank_workload(rank: int):
-    """The batch of `rank`: one model (the seeded weights of rank 0) and, for
-    rank r > 0, its own draw of sequences, timestamps and inputs from the same
-    recipe with seed offset 1000 r.  Ranks share no data and exchange nothing
-    on the data path, so per-rank work stays fixed as ranks are added."""
-    wl = W.make_workload(CONFIG_ID)
-    if rank == 0:
-        return wl
-    own = W.make_workload(CONFIG_ID, seed=W.SEED_BASE + CONFIG_ID + 1000 * rank)
-    own.layers = wl.layers
-    return own
-
-
-def reduce_over_ranks(local_ms: float, local_tokens: int, world: int, device=None):
-    """(max over ranks of the timed milliseconds, sum over ranks of the tokens).
-    Every rank calls it at the same point with the same collective sequence."""
-    if world == 1:
-        return float(local_ms), int(local_tokens)
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    n = torch.tensor([local_tokens], dtype=torch.int64, device=device)
-    dist.all_reduce(n, op=dist.ReduceOp.SUM)
-    return float(t.item()), int(n.item())
-
-
-def unmasked_pairs(seq_offsets, num_targets=None) -> int:
-    """Attended (i, j) pairs of a jagged batch: N(N+1)/2 causal pairs of the N
-    history tokens plus (N+1) per candidate (history and itself)."""
-    offs = np.asarray(seq_offsets, dtype=np.int64)
-    n = np.diff(offs)
-    nt = np.zeros_like(n) if num_targets is None else np.asarray(num_targets, np.int64)
-    N = n - nt
-    return int(np.sum(N * (N + 1) // 2 + nt * (N + 1)))
-
-
-# ----------------------------------------------------------------------------
-# clocks
-# ----------------------------------------------------------------------------
-
-class ClockSampler:
-    """Samples the SM clock and the clock-event reasons of one GPU every few
-    milliseconds from a host thread (NVML reads only; nothing is changed)."""
-
-    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
-               "sw_power_cap": 0x4}
-
-    def __init__(self, index: int, period_s: float = 0.005):
-        self.index = index
-        self.period = period_s
-        self.rows = []
-        self.thread = None
-        self.stop_flag = False
-
-    def _loop(self, nv, h):
-        while not self.stop_flag:
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.rows.append((sm, mx, rs))
-            except Exception:
-                pass
-            time.sleep(self.period)
-
-    def start(self):
-        import threading
-        try:
-            import pynvml as nv
-            nv.nvmlInit()
-            h = nv.nvmlDeviceGetHandleByIndex(self.index)
-        except Exception:
-            return
-        self.thread = threading.Thread(target=self._loop, args=(nv, h), daemon=True)
-        self.thread.start()
-        t0 = time.time()
-        while not self.rows and time.time() - t0 < 2.0:  # first sample before the timed region
-            time.sleep(0.001)
-        self.rows = []
-
-    def stop(self):
-        if self.thread is None:
-            return None
-        self.stop_flag = True
-        self.thread.join(timeout=2)
-        rows = self.rows
-        if not rows:
-            return None
-        reasons = sorted({n for _, _, rs in rows for n, bit in self.REASONS.items() if rs & bit})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows), "source": "NVML, 5 ms period, timed region only"}
-
-
-
-
-
-# ----------------------------------------------------------------------------
 # further rows of the path, measured on their own workloads (1 GPU)
 # ----------------------------------------------------------------------------
+
+def mfalcon_pairs(hist_lens, cand_counts) -> int:
+    """Attended pairs of one mfalcon_rank call with the history's keys and values
+    cached across microbatches: each user's history causally once, then every
+    candidate against its user's history and itself (the same pairs as one
+    M-FALCON pass over [history ; all candidates])."""
+    n = np.asarray(hist_lens, dtype=np.int64)
+    m = np.asarray(cand_counts, dtype=np.int64)
+    return int(np.sum(n * (n + 1) // 2 + m * (n + 1)))
+
 
 def _trace_attention(trace, name, flops):
     a = trace.get(name)
@@ -416,9 +325,7 @@ def measure_mfalcon(hb, steps: int):
     n = int(np.diff(wl.seq_offsets)[0])
     cands = int(e["cand_offsets"][-1])
     mbs = (m_max + bm - 1) // bm
-    # the history's keys and values are computed once per call and reused by every
-    # microbatch: its causal pairs once, then each candidate against the history and itself
-    pairs = U * (n * (n + 1) // 2) + cands * (n + 1)
+    pairs = mfalcon_pairs(np.diff(wl.seq_offsets), np.diff(e["cand_offsets"]))
     flops = pairs * 2 * 2 * sp.head_dim * sp.num_heads
     return {"workload": f"M-FALCON: {U} users, n={n} history, m={cands // U} candidates, b_m={bm} "
                         f"({mbs} microbatches, history K/V cached across them), "

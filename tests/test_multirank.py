@@ -93,3 +93,12 @@ def test_traffic_is_null_once_the_kernel_changed(tmp_path):
     assert bench.read_traffic("attn_fwd_tc", str(good)) == 12345.0
     assert bench.read_traffic("attn_fwd_tc", str(stale)) is None
     assert bench.read_traffic("attn_fwd_tc", str(tmp_path / "missing.txt")) is None
+
+
+def test_mfalcon_pairs_match_one_pass_over_all_candidates():
+    """The ranking row's FLOP count: with the history cached, a call attends the
+    pairs of one M-FALCON pass over [history ; all candidates] per user."""
+    hist = np.array([2048, 0, 37, 130], dtype=np.int64)
+    cands = np.array([4096, 9, 0, 12], dtype=np.int64)
+    offs = np.concatenate([[0], np.cumsum(hist + cands)])
+    assert bench.mfalcon_pairs(hist, cands) == O.attention_pairs(offs, cands)

@@ -102,3 +102,59 @@ def test_mfalcon_pairs_match_one_pass_over_all_candidates():
     cands = np.array([4096, 9, 0, 12], dtype=np.int64)
     offs = np.concatenate([[0], np.cumsum(hist + cands)])
     assert bench.mfalcon_pairs(hist, cands) == O.attention_pairs(offs, cands)
+
+
+def _dp_rank_main(rank, world, port, results):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from hstu_sequential_transducer_02_b200.data_parallel import GradAllReduce, PARAM_GRADS
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        shapes = {"w1": (16, 4), "b1": (16,), "ln1_gamma": (4,), "ln1_beta": (4,), "ln2_gamma": (8,),
+                  "ln2_beta": (8,), "w2": (4, 8), "b2": (4,), "pos_bias": (128,), "time_bias": (128,)}
+        layers = []
+        for l in range(3):
+            g = {n: torch.full(shapes[n], float((rank + 1) * (l + 1))) + torch.arange(
+                int(np.prod(shapes[n])), dtype=torch.float32).reshape(shapes[n]) for n in PARAM_GRADS}
+            g["uvqk"] = torch.full((5, 2), float(rank))      # per-token gradient: not reduced
+            layers.append(g)
+        red = GradAllReduce()
+        for g in reversed(layers):                             # the backward finishes the last layer first
+            red.layer_done(g)
+        red.wait()
+        results[rank] = {(l, n): layers[l][n].clone().numpy() for l in range(3) for n in list(PARAM_GRADS) + ["uvqk"]}
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_gradient_sum_gloo_world2():
+    """Every rank ends with the sum over ranks of each parameter gradient, in
+    its own tensors and shapes; the per-token activation gradient is left alone."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_dp_rank_main, args=(world, _free_port(), results), nprocs=world, join=True,
+                           start_method="spawn")
+        got = dict(results)
+    for rank in range(world):
+        for (l, n), v in got[rank].items():
+            if n == "uvqk":
+                assert np.all(v == rank)
+                continue
+            ar = np.arange(v.size, dtype=np.float32).reshape(v.shape)
+            want = sum(float((r + 1) * (l + 1)) + ar for r in range(world))
+            assert np.array_equal(v, want), (rank, l, n)
+
+
+def test_data_parallel_single_rank_is_a_no_op():
+    import torch
+    from hstu_sequential_transducer_02_b200.data_parallel import GradAllReduce, PARAM_GRADS
+    g = {n: torch.ones(3) for n in PARAM_GRADS}
+    red = GradAllReduce()
+    red.layer_done(g)
+    red.wait()
+    assert all(torch.equal(g[n], torch.ones(3)) for n in PARAM_GRADS)

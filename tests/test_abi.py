@@ -137,3 +137,30 @@ def test_host_memory_forward_argument_checks():
     assert call([0, 40, 100], xx=None) == b.ERR_INVALID_ARG
     assert call([0, 40, 100], chunks=0) == b.ERR_INVALID_ARG
     assert call([0, 40, 100], ws_bytes=256) == b.ERR_WORKSPACE
+
+
+def test_ranking_and_sl_argument_checks():
+    """mfalcon_rank and hstu_stochastic_length refuse bad arguments on the host,
+    before any launch: no layers, microbatch < 1, null or misaligned buffers,
+    a workspace too small; SL with max_len < 1 or missing arrays."""
+    b = _lib()
+    ld = b.layer_desc(64, 2, 32, b.DTYPE_BF16)
+    p = ctypes.c_void_p(1 << 20)      # never dereferenced: every call below fails its host checks
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    w = b.LayerWeights(*([p] * 10))
+    arr = (b.LayerWeights * 1)(w)
+
+    def mf(layers=arr, L=1, bm=8, cand_x=p, cand_out=p, ws_bytes=1 << 40):
+        return b._lib_mf(ctypes.byref(ld), layers, L, 2, 100, 16, bm, p, p, p, p, cand_x, p, cand_out, p, ws_bytes,
+                         None)
+
+    assert mf(layers=None) == b.ERR_INVALID_ARG
+    assert mf(L=0) == b.ERR_INVALID_ARG
+    assert mf(bm=0) == b.ERR_INVALID_ARG
+    assert mf(cand_x=None) == b.ERR_INVALID_ARG
+    assert mf(cand_out=odd) == b.ERR_INVALID_ARG
+    assert mf(ws_bytes=256) == b.ERR_WORKSPACE
+    assert b._lib_sl(4, 100, p, p, p, 0, 0, p, p, p, 1 << 20, None) == b.ERR_INVALID_ARG
+    assert b._lib_sl(4, 100, None, p, p, 8, 0, p, p, p, 1 << 20, None) == b.ERR_INVALID_ARG
+    assert b._lib_sl(4, 100, p, None, p, 8, 0, p, p, p, 1 << 20, None) == b.ERR_INVALID_ARG
+    assert b._lib_sl(4, 100, p, p, p, 8, 0, p, p, p, 16, None) == b.ERR_WORKSPACE

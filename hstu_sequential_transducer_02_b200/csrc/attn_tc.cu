@@ -551,7 +551,9 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
           tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
         }
         tmem_ld_wait_regs(raw);
-        // ---- bias, SiLU (as h + h tanh h with h = (s + bias) / 2), mask; packed bf16 pairs
+        // ---- bias, SiLU, mask; packed bf16 pairs.  With h = (s + bias) / 2: far from the
+        // diagonal (rows with at least 128 attended columns) SiLU = h + h tanh h; near it
+        // and on candidate rows, whose outputs may rest on a few terms, the exact form
         uint32_t pk[16];
         if (wrank == 0) {
 #pragma unroll
@@ -610,7 +612,7 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
             float h0, h1;
             half_plus2c(__uint_as_float(raw[2 * q]), __uint_as_float(raw[2 * q + 1]), __uint_as_float(bw[q] << 16),
                         __uint_as_float(bw[q] & 0xFFFF0000u), h0, h1);
-            const uint32_t v = silu2_bf16(h0, h1);
+            const uint32_t v = silu2_exact_bf16(h0, h1);
             pk[q] = (2 * q <= lim ? (v & 0xFFFFu) : 0u) | (2 * q + 1 <= lim ? (v & 0xFFFF0000u) : 0u);
           }
         } else if (__all_sync(0xffffffffu, narrow)) {
@@ -633,7 +635,7 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
               const int j = cl + 4 * g4 + 2 * q;
-              const uint32_t v = silu2_bf16(h[2 * q], h[2 * q + 1]);
+              const uint32_t v = silu2_exact_bf16(h[2 * q], h[2 * q + 1]);
               pk[2 * g4 + q] = (attended(i, j, si.n, si.hist) ? (v & 0xFFFFu) : 0u) |
                                (attended(i, j + 1, si.n, si.hist) ? (v & 0xFFFF0000u) : 0u);
             }
@@ -657,7 +659,7 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
               }
               h[u] = 0.5f * (__uint_as_float(raw[e]) + bias);
             }
-            const uint32_t v = silu2_bf16(h[0], h[1]);
+            const uint32_t v = silu2_exact_bf16(h[0], h[1]);
             pk[e2] = (att[0] ? (v & 0xFFFFu) : 0u) | (att[1] ? (v & 0xFFFF0000u) : 0u);
           }
         }

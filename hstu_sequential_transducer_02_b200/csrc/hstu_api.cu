@@ -3,6 +3,7 @@
 // library's own kernels; nothing here computes on the host except the
 // time-bucket threshold table.
 #include <algorithm>
+#include <cuda.h>
 #include <math.h>
 #include <stdio.h>
 #include <mutex>
@@ -371,15 +372,22 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
     b.xhat = saved->xhat; b.mu1 = saved->ln1_mean; b.rs1 = saved->ln1_rstd; b.z = saved->z;
     b.uvqk = saved->uvqk; b.o = saved->attn_out; b.mu2 = saved->ln2_mean; b.rs2 = saved->ln2_rstd;
   }
-  // attention preparation on the side stream, overlapping LayerNorm1 and f1
+  // attention preparation on the side stream, overlapping LayerNorm1 and f1.  The
+  // side stream is shared by every caller on the device, so a stream that is being
+  // captured into a graph keeps the preparation on itself: the shared stream must
+  // not join one caller's capture while other callers enqueue work on it.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  HSTU_CUDA(cudaStreamIsCapturing(st, &cap));
   SideStream* side = nullptr;
-  {
+  if (cap == cudaStreamCaptureStatusNone) {
     std::lock_guard<std::mutex> lk(g_side_mu);
     HSTU_TRY(side_stream(&side));
     HSTU_CUDA(cudaEventRecord(side->fork, st));
     HSTU_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
     HSTU_TRY(run_attn_prep(&d->attn, jb, w->pos_bias, w->time_bias, ws.attn, side->s));
     HSTU_CUDA(cudaEventRecord(side->join, side->s));
+  } else {
+    HSTU_TRY(run_attn_prep(&d->attn, jb, w->pos_bias, w->time_bias, ws.attn, st));
   }
   // (A1) LayerNorm1
   {
@@ -402,7 +410,7 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   // (A2-A4) attention
   const size_t es = elem_size(dt);
   const char* uvqk = (const char*)b.uvqk;
-  HSTU_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  if (side) HSTU_CUDA(cudaStreamWaitEvent(st, side->join, 0));
   HSTU_TRY(run_attn_main(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + 1 * hv * es,
                          4 * hv, w->pos_bias, w->time_bias, b.o, hv, ws.attn, st));
   // (A5) LayerNorm2(A V) * U
@@ -1041,7 +1049,11 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
   MfalconWs w = carve_mfalcon(c, desc, num_layers, U, hist_total, bm);
   HSTU_CUDA(cudaMemsetAsync(w.layer.attn.status, 0, kStatusBytes, st));
   const int n_mb = (max_candidates + bm - 1) / bm;
-  if (n_mb == 0 || U == 0) return HSTU_OK;
+  if (U == 0) return HSTU_OK;
+  if (n_mb == 0) {
+    HSTU_CUDA(launch_mfalcon_check_counts(U, 0, cand_offsets, w.layer.attn.status, st));
+    return HSTU_OK;
+  }
   HSTU_CUDA(launch_mfalcon_slot_offsets(U, bm, hist_offsets, w.offs, w.nt, st));
   hstu_jagged jb;
   jb.batch = U;
@@ -1092,6 +1104,8 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
     }
     HSTU_CUDA(launch_mfalcon_scatter(cur, dm, dt, w.cand_dst, nullptr, w.C, cand_out, st));
   }
+  // a user with more candidates than the n_mb microbatches hold had some left unscored
+  HSTU_CUDA(launch_mfalcon_check_counts(U, n_mb * bm, cand_offsets, w.layer.attn.status, st));
   return HSTU_OK;
 }
 
@@ -1174,17 +1188,52 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};   // id of the context the address belongs to
 
-// Device address of the scratch array on the current device (looked up once).
+// The driver's context calls, taken through the runtime's entry-point query so
+// that the library has no link-time dependency on the driver library.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device, looked up once per
+// device and context: the address is only valid in the context it was looked up
+// in, so a call from another context of the device (a non-primary context, or
+// the primary context again after cudaDeviceReset) looks it up afresh.  Context
+// ids are never reused within a process.
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return HSTU_ERR_UNSUPPORTED;
+  unsigned long long id = current_context_id();   // 0: no context current yet
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_noalloc_ptr[dev] || id == 0 || g_noalloc_ctx[dev] != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HSTU_ERR_CUDA;
+    if (id == 0) id = current_context_id();   // the lookup made the device's primary context current
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = id;
   }
   *out = g_noalloc_ptr[dev];
   return HSTU_OK;

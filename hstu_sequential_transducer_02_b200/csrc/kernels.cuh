@@ -203,6 +203,10 @@ cudaError_t launch_mfalcon_slot_pack(int U, int mb, int bm, int rows_cap, int ca
                                      const void* hist_x, const int64_t* hist_ts, const int32_t* cand_offs,
                                      const void* cand_x, const int64_t* cand_ts, int d, int dtype, int with_hist,
                                      void* x_slot, int64_t* ts_slot, void* x_c, int32_t* cand_dst, cudaStream_t st);
+// HSTU_ERR_BAD_OFFSETS into the status word when a user has a negative candidate
+// count or more than `limit` candidates
+cudaError_t launch_mfalcon_check_counts(int U, int limit, const int32_t* cand_offs, int32_t* status,
+                                        cudaStream_t st);
 // row_bytes of each candidate row between the compact and the slot layout (multiples of 16 bytes)
 cudaError_t launch_mfalcon_slot_rows(int U, int bm, int cap, const int32_t* hist_offs, const void* src,
                                      int64_t lds_bytes, void* dst, int64_t ldd_bytes, int64_t row_bytes, int to_slot,

@@ -989,6 +989,25 @@ cudaError_t launch_mfalcon_slot_offsets(int U, int bm, const int32_t* hist_offs,
   return cudaGetLastError();
 }
 
+// A user whose candidate count is negative or exceeds the n_mb * bm slots of the
+// microbatches the caller asked for: the status word records it (candidates past
+// the last microbatch were not scored).  Runs after the scoring, so the status
+// word stays clear while the layers run.
+__global__ void mfalcon_check_counts_kernel(int U, int limit, const int32_t* __restrict__ cand_offs,
+                                            int32_t* __restrict__ status) {
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < U; u += gridDim.x * blockDim.x) {
+    const int m = cand_offs[u + 1] - cand_offs[u];
+    if (m < 0 || m > limit) set_status(status, HSTU_ERR_BAD_OFFSETS);
+  }
+}
+
+cudaError_t launch_mfalcon_check_counts(int U, int limit, const int32_t* cand_offs, int32_t* status,
+                                        cudaStream_t st) {
+  if (U <= 0) return cudaSuccess;
+  mfalcon_check_counts_kernel<<<(U + 255) / 256, 256, 0, st>>>(U, limit, cand_offs, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mfalcon_slot_pack(int U, int mb, int bm, int rows_cap, int cap, const int32_t* hist_offs,
                                      const void* hist_x, const int64_t* hist_ts, const int32_t* cand_offs,
                                      const void* cand_x, const int64_t* cand_ts, int d, int dtype, int with_hist,

@@ -272,13 +272,36 @@ __device__ __forceinline__ float tanh_approx(float x) {
 }
 
 // SiLU of two values, returned as packed bf16x2 (low half = first value):
-// with h = s/2, SiLU(s) = h + h * tanh(h); tanh and the fused multiply-add run on
-// bf16 pairs (one special-function op for two elements).
+// with h = s/2, SiLU(s) = h + h * tanh(h).  tanh and the multiply-add run in
+// fp32 (the add as one packed fp32x2 FMA) and only the result is rounded to
+// bf16, so P carries one rounding; tanh on bf16 pairs would round h and tanh(h)
+// as well and lose the small values of strongly negative s to cancellation.
 __device__ __forceinline__ uint32_t silu2_bf16(float h_lo, float h_hi) {
-  uint32_t h, t, r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(h_hi), "f"(h_lo));
-  asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(h));
-  asm("fma.rn.bf16x2 %0, %1, %2, %1;" : "=r"(r) : "r"(h), "r"(t));
+  const float t_lo = tanh_approx(h_lo), t_hi = tanh_approx(h_hi);
+  float r_lo, r_hi;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "fma.rn.f32x2 d, a, b, a;\n\t"
+      "mov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r_lo), "=f"(r_hi)
+      : "f"(h_lo), "f"(h_hi), "f"(t_lo), "f"(t_hi));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(r_hi), "f"(r_lo));
+  return r;
+}
+
+// The same SiLU of s = 2h from sigma(s) = 1 / (1 + e^-s), accurate to a few fp32
+// ulps for every s, at two special-function ops per element.  The tanh form errs
+// by about 2^-11 |h| in absolute terms, which is large relative to SiLU(s) for
+// strongly negative s; this form serves the rows whose output can rest on a few
+// such terms (near the diagonal, and candidates, whose own column is one term).
+__device__ __forceinline__ uint32_t silu2_exact_bf16(float h_lo, float h_hi) {
+  const float s_lo = h_lo + h_lo, s_hi = h_hi + h_hi;
+  const float r_lo = __fdividef(s_lo, 1.0f + __expf(-s_lo));
+  const float r_hi = __fdividef(s_hi, 1.0f + __expf(-s_hi));
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(r_hi), "f"(r_lo));
   return r;
 }
 

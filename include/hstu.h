@@ -208,15 +208,22 @@ int hstu_attn_fwd(const hstu_attn_desc* desc, const hstu_jagged* jb,
  * property of this library, not of the method.
  *
  * Same arguments, layouts and result as hstu_attn_fwd.  The scratch it needs
- * (status word and work list) lives in a 1 MiB array that the library keeps in
- * the device memory of every GPU it is loaded on, for the life of the process;
- * the call itself allocates nothing.  A problem whose scratch would exceed the
- * array (hstu_attn_fwd_workspace_size() > 1 MiB, about 65,000 work items:
- * (total_tokens/128 + batch + 1) * num_heads) is refused with
- * HSTU_ERR_WORKSPACE before anything is launched.
+ * lives in a 1 MiB array that the library keeps in the device memory of every
+ * GPU it is loaded on, for the life of the process; the call itself allocates
+ * nothing.  That scratch is the status word, the work list and, on the
+ * tensor-core path, the per-kv-tile timestamp records; this entry point does
+ * without the near-diagonal bias band of hstu_attn_fwd (it evaluates those
+ * biases per element instead), so its results may differ from hstu_attn_fwd's
+ * by bf16 rounding of the bias near the diagonal.  A problem whose scratch
+ * exceeds the array is refused with HSTU_ERR_WORKSPACE before anything is
+ * launched: with W = total_tokens/128 + batch + 1, the tensor-core path needs
+ * about (16 * num_heads + 560) * W bytes + 1 KB (num_heads = 4: up to about
+ * 1,700 tiles of 128 tokens, some 200,000 tokens in few sequences).
  *   - The first call on a device looks up the array's device address on that
- *     device (current device at the time of the call); make that first call
- *     before capturing any stream into a graph.
+ *     device (current device at the time of the call), and so does the first
+ *     call from each further context of the device (a non-primary context, or
+ *     the primary context recreated after cudaDeviceReset); make those first
+ *     calls before capturing any stream into a graph.
  *   - All calls share the one array and each call overwrites it.  Calls that
  *     may run at the same time on the GPU (different streams without ordering
  *     between them) race on it and give undefined results: order them.
@@ -255,7 +262,13 @@ int hstu_layer_fwd_workspace_size(const hstu_layer_desc* desc, int32_t batch,
 
 /* Y = X + f2(LayerNorm2(A V) (.) U) with U, V, Q, K = Split(SiLU(f1(LayerNorm1(X)))).
  *   x, y: device [T, d] io_dtype, contiguous (row stride d); y may not alias x.
- *   saved: NULL for inference, else its buffers receive what hstu_layer_bwd needs. */
+ *   saved: NULL for inference, else its buffers receive what hstu_layer_bwd needs.
+ * The attention's preparation (work list, timestamp records, bias band) runs on a
+ * library-owned side stream of the device, overlapping LayerNorm1 and f1; calls
+ * from several host threads share that stream, which only orders their
+ * preparations.  While `stream` is being captured into a CUDA graph the
+ * preparation runs on `stream` itself, so the capture never reaches the shared
+ * side stream. */
 int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w,
                    const hstu_jagged* jb, const void* x, void* y,
                    const hstu_layer_saved* saved,
@@ -316,7 +329,10 @@ int mfalcon_rank_workspace_size(const hstu_layer_desc* desc, int32_t num_layers,
  *   hist_offsets [U+1], cand_offsets [U+1]: device; hist_x [hist_total, d],
  *   hist_ts [hist_total]; cand_x [cand_offsets[U], d], cand_ts [...]: device;
  *   max_candidates: host upper bound on any user's candidate count (sets the
- *   number of microbatches, ceil(max_candidates / microbatch));
+ *   number of microbatches, ceil(max_candidates / microbatch)); a user with more
+ *   candidates than those microbatches hold (or a negative count) sets the status
+ *   word to HSTU_ERR_BAD_OFFSETS after the call's work, and its candidates past
+ *   the last microbatch are not written;
  *   hist_x, cand_x, cand_out are in desc->io_dtype; cand_out: [cand_offsets[U], d].
  * The history rows do not depend on the candidates, so every layer's keys and
  * values of the history are computed once, with microbatch 0, and kept in the

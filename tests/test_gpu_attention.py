@@ -170,6 +170,60 @@ def test_time_bucket_at_every_threshold():
     assert np.array_equal(got[:, 1], want.astype(np.int32))
 
 
+def _gpu_buckets_of(ds):
+    """Time buckets of the differences `ds` from the GPU's rule (row k + 1 sits
+    ds[k] seconds after row 0 of one sequence)."""
+    b = _b()
+    base = 1_700_000_000
+    ts = np.concatenate([[base], base + ds]).astype(np.int64)
+    n = len(ts)
+    offs = np.array([0, n], dtype=np.int32)
+    pairs = np.zeros((n - 1, 3), dtype=np.int32)
+    pairs[:, 1] = np.arange(1, n, dtype=np.int32)
+    got = b.debug_rab_buckets(dev(offs), dev(ts), dev(pairs.reshape(-1)).reshape(-1, 3))
+    return got[:, 1].cpu().numpy()
+
+
+def test_time_bucket_every_difference_below_2_24_and_a_stride_beyond():
+    """The 32-bit bucket rule trusts its log estimate (error below 2e-4) unless
+    the estimate lies within 2^-9 of an integer: every |dt| in [0, 2^24] and a
+    prime stride from 2^24 to 2^31 give the oracle's fp64 bucket bit for bit,
+    which pins that error bound itself, not only the thresholds."""
+    for lo in range(0, 1 << 24, 1 << 22):
+        ds = np.arange(lo, lo + (1 << 22) + 1, dtype=np.int64)
+        got = _gpu_buckets_of(ds)
+        want = O.time_bucket(ds).astype(np.int32)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, f"dt {ds[bad[:5]]}: GPU {got[bad[:5]]} oracle {want[bad[:5]]}"
+    ds = np.arange(1 << 24, (1 << 31) - 1, 1021, dtype=np.int64)
+    got = _gpu_buckets_of(ds)
+    want = O.time_bucket(ds).astype(np.int32)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"dt {ds[bad[:5]]}: GPU {got[bad[:5]]} oracle {want[bad[:5]]}"
+
+
+@pytest.mark.parametrize("mfalcon", [False, True])
+def test_attn_bwd_long_sequences(mfalcon):
+    """The tensor-core backward on sequences longer than 1,024 tokens (kv tiles
+    that meet up to 20 q tiles), with and without M-FALCON targets."""
+    b = _b()
+    lens = [2433, 1090, 64]
+    nt = [300, 0, 17] if mfalcon else None
+    d = W.random_attention_inputs(53, lens, 2, 64, "bf16", num_targets=nt, qk_std=0.5)
+    T = sum(lens)
+    q, k, v, do = (dev(d[n].reshape(T, 2 * 64), torch.bfloat16) for n in ("q", "k", "v", "dout"))
+    ntd = None if nt is None else dev(d["num_targets"])
+    dq, dk, dv, dpb, dtb = b.attn_bwd(q, k, v, do, dev(d["seq_offsets"]), dev(d["timestamps"]), dev(d["pos_bias"]),
+                                      dev(d["time_bias"]), 2, num_targets=ntd)
+    torch.cuda.synchronize()
+    rq, rk, rv, rpb, rtb = O.attention_backward(d["q"], d["k"], d["v"], d["dout"], d["seq_offsets"],
+                                                d["timestamps"], d["pos_bias"], d["time_bias"], d["num_targets"])
+    for got, ref, name in [(dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")]:
+        assert_close(got.float().cpu().numpy().reshape(ref.shape), ref, "bf16", name, grad=True)
+    for got, ref, name in [(dpb, rpb, "dpos"), (dtb, rtb, "dtime")]:
+        assert_close(got.cpu().numpy(), ref, "bf16", name, grad=True)
+
+
 def test_bounded_wait_times_out_and_reports():
     b = _b()
     st = torch.full((1,), -1, dtype=torch.int32, device="cuda")

@@ -186,12 +186,35 @@ def test_mfalcon_history_cache_ragged_users_two_layers():
 
 
 def test_mfalcon_user_without_history():
-    """A user with no history: its candidates attend only to themselves (N = 1).
-    One layer: with a single attended term the bf16 SiLU's rounding is not
-    averaged over a history, and a second layer amplifies it past the max-abs
-    bound for one of these candidates (a precision limit of the bf16 P)."""
-    got, ref = _mfalcon_ragged([64, 0, 37], [5, 9, 3], 1, 7)
-    assert_close(got, ref, "bf16", "mfalcon user without history")
+    """A user with no history: its candidates attend only to themselves (N = 1),
+    through two layers.  With a single attended term nothing averages the
+    rounding of P, and LayerNorm2 rescales the lone term: the attention's SiLU
+    must keep strongly negative scores accurate (fp32 tanh, one rounding)."""
+    got, ref = _mfalcon_ragged([64, 0, 37], [5, 9, 3], 2, 7)
+    assert_close(got, ref, "bf16", "mfalcon user without history, 2 layers")
+
+
+def test_mfalcon_too_few_microbatches_reported():
+    """max_candidates below a user's candidate count leaves that user's last
+    candidates unscored: the status word says so (HSTU_ERR_BAD_OFFSETS), and a
+    large enough bound leaves it clear."""
+    b = _b()
+    wl = W.make_workload(3, scale=1 / 32, batch=3, lengths=[40, 17, 64])
+    e = wl.extras
+    s = wl.spec
+    co = e["cand_offsets"]
+    counts = [5, 9, 3]
+    sel = np.concatenate([np.arange(co[u], co[u] + counts[u]) for u in range(3)]).astype(np.int64)
+    cand_offsets = dev(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32))
+    td = torch_dtype(s.dtype)
+    layers = _layers(wl)
+    args = (dev(wl.seq_offsets), dev(wl.x, td), dev(wl.timestamps), cand_offsets, dev(e["cand_x"][sel], td),
+            dev(e["cand_ts"][sel]))
+    for max_c, want in ((4, b.ERR_BAD_OFFSETS), (9, b.OK), (0, b.ERR_BAD_OFFSETS)):
+        ws = b.mfalcon_workspace(layers, 3, int(wl.seq_offsets[-1]), 4, "cuda")
+        b.mfalcon_rank(layers, *args, 4, max_c, workspace=ws)
+        torch.cuda.synchronize()
+        assert b.workspace_status(ws) == want, f"max_candidates {max_c}"
 
 
 def test_mfalcon_rank_config3_full_size_sampled():
@@ -314,60 +337,137 @@ def _layer_errors(r, gr, T, hv):
     return out
 
 
-def _check_train(run, wl, chained_rel_bound):
-    """Per layer, teacher-forced: the oracle's gradients of layer l at the GPU's
-    own layer input x_l and upstream gradient dy_l, at the specification's bf16
-    tolerance.  Chained: the oracle's whole-stack gradients from X and G, at
-    `chained_rel_bound` (bf16 operand rounding accumulates through the stack)."""
+def _gpu_layer_grads(wl, li, x, dy, offs, ts, residual_fp32=True):
+    """Layer li of the workload on the GPU: forward with saved activations from
+    the host input x, then backward from the host upstream gradient dy."""
+    b = _b()
+    s = wl.spec
+    td = torch.bfloat16
+    io = torch.float32 if residual_fp32 else td
+    T = int(offs[-1])
+    hv = s.num_heads * s.head_dim
+    ly = b.Layer(layer_to_dev(wl.layers[li], td), s.d_model, s.num_heads, s.head_dim, residual_fp32=residual_fp32)
+    sv = b.Saved.alloc(T, s.d_model, hv, td, "cuda")
+    offs_d, ts_d = dev(np.asarray(offs, np.int32)), dev(ts)
+    x_d = dev(np.asarray(x, np.float32), io)
+    ly.forward(x_d, offs_d, ts_d, saved=sv)
+    dx, gr = ly.backward(x_d, dev(np.asarray(dy, np.float32), io), sv, offs_d, ts_d)
+    torch.cuda.synchronize()
+    return dx.float().cpu().numpy().astype(np.float64), gr
+
+
+GRAD_KEYS = ["dU", "dV", "dQ", "dK", "pos_bias", "time_bias", "w1", "w2", "b1", "b2", "ln1_gamma", "ln1_beta",
+             "ln2_gamma", "ln2_beta"]
+
+
+def _check_layer_grads(got_grads, ref, T, hv, what):
+    """Every gradient of one layer at the specification's bf16 tolerance:
+    relative Frobenius <= 1e-2, max-abs <= 3e-2 * max(1, max|ref|)."""
+    for name, (got, want) in _layer_errors(ref, got_grads, T, hv).items():
+        ma, rel = errors(got, want)
+        print(f"{what} {name}: rel-fro {rel:.3e} max-abs {ma:.3e}")
+        assert_close(got, want, "bf16", f"{what} {name}", grad=True)
+
+
+def _oracle_chain(wl, x0, g0, offs, ts):
+    """The oracle's inputs x_l and upstream gradients dy_l of every layer of the
+    stack, and its per-layer gradients."""
+    s = wl.spec
+    xs = [np.asarray(x0, np.float64)]
+    for p in wl.layers[:-1]:
+        xs.append(O.layer_forward(xs[-1], p, offs, ts, s.num_heads, s.head_dim))
+    ref = O.stack_backward(x0, wl.layers, g0, offs, ts, s.num_heads, s.head_dim)
+    dys = [None] * len(wl.layers)
+    dys[-1] = np.asarray(g0, np.float64)
+    for li in range(len(wl.layers) - 1, 0, -1):
+        dys[li - 1] = ref[li]["dx"]
+    return xs, dys, ref
+
+
+def test_training_step_config4_per_layer():
+    """8-layer bf16 stack (fp32 residual stream) with Stochastic Length: each
+    layer's backward on the GPU, fed the oracle's own layer input x_l and
+    upstream gradient dy_l, against the oracle's gradients of that layer: dU,
+    dV, dQ, dK, both relative-bias tables and every weight, at relative
+    Frobenius <= 1e-2 and max-abs <= 3e-2 (times the gradient's scale)."""
+    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
+    g, offs = _sl_workload(wl)
+    e = wl.extras
+    x0, ts, g0 = wl.x[g].astype(np.float64), wl.timestamps[g], e["grad_out"][g].astype(np.float64)
+    xs, dys, ref = _oracle_chain(wl, x0, g0, offs, ts)
+    s = wl.spec
+    T, hv = int(offs[-1]), s.num_heads * s.head_dim
+    for li in range(len(wl.layers)):
+        dx, gr = _gpu_layer_grads(wl, li, xs[li], dys[li], offs, ts)
+        _check_layer_grads(gr, ref[li], T, hv, f"layer {li}")
+        assert_close(dx, ref[li]["dx"], "bf16", f"layer {li} dx", grad=True)
+
+
+def test_training_step_config4_chained_within_rounding_model():
+    """The whole 8-layer step from X and G (SL on the GPU, the stack's forward,
+    then its backward), against the oracle's whole-stack gradients.  Rounding
+    x-hat and U, V, Q, K to bf16 for the tensor cores alone moves these
+    gradients past 1e-2 (an exact fp64 computation with only those roundings,
+    tests/test_precision_model.py), so this check compares the GPU's error with
+    the error of the rounding model of the bf16 path on the same inputs: at
+    most 1.25 times the model's worst relative Frobenius error."""
+    import tests.precision_model as M
+    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
+    run = _train_step(wl, residual_fp32=True)
     s = wl.spec
     T, hv = run["T"], run["hv"]
     chained = O.stack_backward(run["x0"], wl.layers, run["g0"], run["offs"], run["ts"], s.num_heads, s.head_dim)
-    worst = 0.0
-    for li in range(len(wl.layers) - 1, -1, -1):
-        tf = O.layer_backward(run["xs"][li], wl.layers[li], run["dys"][li], run["offs"], run["ts"], s.num_heads,
-                              s.head_dim)
-        for name, (got, ref) in _layer_errors(tf, run["grads"][li], T, hv).items():
-            ma, rel = errors(got, ref)
-            print(f"layer {li} {name}: teacher-forced rel-fro {rel:.3e} max-abs {ma:.3e}")
-            if name in ("dU", "dV", "dQ", "dK"):
-                assert_close(got, ref, "bf16", f"L{li} {name} (teacher-forced)", grad=True)
-            elif name in ("pos_bias", "time_bias"):
-                # sums of dS over up to ~1e6 pairs, with heavy cancellation: even fed
-                # the GPU's own layer input, the oracle differs from the GPU by the
-                # bf16 rounding of the layer's internal operands (x-hat, U/V/Q/K,
-                # A V, the gate, dO).  An fp64 simulation of those roundings on this
-                # workload gives 3e-3 .. 8e-3 with exact upstream gradients, and the
-                # GPU's own upstream gradients have given up to 1.03e-2; the attention
-                # backward itself matches the oracle to ~1e-6 on identical inputs.
-                assert rel <= 2e-2, f"L{li} {name} (teacher-forced) rel-fro {rel:.3e}"
-            else:
-                assert rel <= 1e-2, f"L{li} {name} (teacher-forced) rel-fro {rel:.3e}"
+    M.set_rounding(M.ROUNDING_POINTS)
+    model = M.stack_backward(run["x0"], wl.layers, run["g0"], run["offs"], run["ts"], s.num_heads, s.head_dim,
+                             silu_p="f32", band=True)
+    worst_gpu = worst_model = 0.0
+    for li in range(len(wl.layers)):
         for name, (got, ref) in _layer_errors(chained[li], run["grads"][li], T, hv).items():
             _, rel = errors(got, ref)
-            worst = max(worst, rel)
-            assert rel <= chained_rel_bound, f"L{li} {name} (chained) rel-fro {rel:.3e}"
-    print(f"chained worst rel-fro {worst:.3e}")
-    tf0 = O.layer_backward(run["xs"][0], wl.layers[0], run["dys"][0], run["offs"], run["ts"], s.num_heads,
-                           s.head_dim)
-    assert_close(run["dx"], tf0["dx"], "bf16", "dx (teacher-forced)", grad=True)
+            worst_gpu = max(worst_gpu, rel)
+        for name in ("dU", "dV", "dQ", "dK", "dpos_bias", "dtime_bias", "dw1", "dw2", "db1", "dln1_g", "dln1_b",
+                     "dln2_g", "dln2_b"):
+            worst_model = max(worst_model, errors(model[li][name], chained[li][name])[1])
+    print(f"chained worst rel-fro: GPU {worst_gpu:.3e}, rounding model {worst_model:.3e}")
+    assert worst_gpu <= 1.25 * worst_model, f"chained {worst_gpu:.3e} > 1.25 x model {worst_model:.3e}"
 
 
-def test_training_step_config4_scaled():
-    """8-layer bf16 stack (fp32 residual stream) forward + backward with
-    Stochastic Length: dU, dV, dQ, dK, the rab gradients and the weight
-    gradients of every layer vs the oracle.  The chained bound 3e-2 comes from
-    an fp64 simulation of this workload that rounds to bf16 wherever the GPU
-    stores a bf16 value or feeds one to a tensor core (forward: x-hat, U/V/Q/K,
-    P with the bf16-pair SiLU, A V, the gate; backward: dY, dg, dO, dU, P and dS
-    as MMA operands, dQ/dK/dV, dz): it moves the chained gradients by up to
-    1.79e-2 (time-bias gradient, first layer) and 1.76e-2 (dK); the GPU, which
-    also sums in fp32 with atomics, has given up to 2.16e-2."""
-    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
-    _check_train(_train_step(wl, residual_fp32=True), wl, chained_rel_bound=3e-2)
+def test_training_config4_full_size_one_layer():
+    """The full training workload (64 sequences after Stochastic Length,
+    T = 27,037, lengths up to 2,433): the last layer's forward and backward on
+    the GPU from the generator's X and G against the oracle's gradients of the
+    same layer, element by element, at the specification's bf16 tolerance."""
+    wl = W.make_workload(4)
+    g, offs = _sl_workload(wl)
+    e = wl.extras
+    x0, ts, g0 = wl.x[g].astype(np.float64), wl.timestamps[g], e["grad_out"][g].astype(np.float64)
+    assert int(np.max(np.diff(offs))) > 2048
+    li = len(wl.layers) - 1
+    dx, gr = _gpu_layer_grads(wl, li, x0, g0, offs, ts)
+    s = wl.spec
+    ref = O.layer_backward(x0, wl.layers[li], g0, offs, ts, s.num_heads, s.head_dim)
+    _check_layer_grads(gr, ref, int(offs[-1]), s.num_heads * s.head_dim, "full size")
+    assert_close(dx, ref["dx"], "bf16", "full size dx", grad=True)
 
 
 def test_training_step_bf16_residual_two_layers():
-    """The same step with a bf16 residual stream, two layers deep."""
+    """A bf16 residual stream, two layers deep: each layer fed the oracle's own
+    input and upstream gradient (rounded to bf16, as such a stream holds them),
+    at the specification's bf16 tolerance."""
     wl = W.make_workload(4, batch=5, scale=1 / 8, random_affine=True)
     wl.layers = wl.layers[:2]
-    _check_train(_train_step(wl, residual_fp32=False), wl, chained_rel_bound=1e-2)
+    g, offs = _sl_workload(wl)
+    e = wl.extras
+    x0 = W.round_to_bf16(wl.x[g]).astype(np.float64)
+    ts, g0 = wl.timestamps[g], W.round_to_bf16(e["grad_out"][g]).astype(np.float64)
+    s = wl.spec
+    xs = [x0, W.round_to_bf16(O.layer_forward(x0, wl.layers[0], offs, ts, s.num_heads, s.head_dim)).astype(np.float64)]
+    dys = [None, g0]
+    ref = [None, O.layer_backward(xs[1], wl.layers[1], g0, offs, ts, s.num_heads, s.head_dim)]
+    dys[0] = W.round_to_bf16(ref[1]["dx"]).astype(np.float64)
+    ref[0] = O.layer_backward(xs[0], wl.layers[0], dys[0], offs, ts, s.num_heads, s.head_dim)
+    T, hv = int(offs[-1]), s.num_heads * s.head_dim
+    for li in range(2):
+        dx, gr = _gpu_layer_grads(wl, li, xs[li], dys[li], offs, ts, residual_fp32=False)
+        _check_layer_grads(gr, ref[li], T, hv, f"bf16 residual layer {li}")
+        assert_close(dx, ref[li]["dx"], "bf16", f"bf16 residual layer {li} dx", grad=True)

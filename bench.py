@@ -14,8 +14,9 @@ dense bf16 peak; `cpu_baseline` times the fp64 CPU oracle on a bounded sample.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-For N > 1 launch with torch.distributed.run; every rank runs its own copy of the
-batch (independent sequences: no collective on the data path, weak scaling).
+For N > 1 launch with torch.distributed.run; one batch of 8 N sequences is dealt
+out over the ranks by sequence (longest-processing-time first on the attended
+pairs and per-token work; no collective on the data path, weak scaling).
 """
 from __future__ import annotations
 
@@ -135,17 +136,28 @@ def run_reference(args, rank: int):
 # multi-rank plumbing (host logic; covered on CPU with gloo ranks)
 # ----------------------------------------------------------------------------
 
-def rank_workload(rank: int):
-    """The batch of `rank`: one model (the seeded weights of rank 0) and, for
-    rank r > 0, its own draw of sequences, timestamps and inputs from the same
-    recipe with seed offset 1000 r.  Ranks share no data and exchange nothing
-    on the data path, so per-rank work stays fixed as ranks are added."""
-    wl = W.make_workload(CONFIG_ID)
-    if rank == 0:
+def projection_pairs_per_token(spec) -> float:
+    """The row-wise work of a token (f1: 2 d 4d FLOP, f2: 2 d d FLOP) in units of
+    one attended pair (2 (dqk + dv) H FLOP): the per-token weight of the cost
+    that deals sequences out to ranks."""
+    d = spec.d_model
+    return (2.0 * d * 4 * d + 2.0 * d * d) / (2.0 * 2 * spec.head_dim * spec.num_heads)
+
+
+def rank_workload(rank: int, world: int = 1):
+    """Rank `rank`'s shard of one global batch: the long-history recipe drawn
+    for 8 * world sequences (with one rank, exactly the 8-sequence workload),
+    dealt out over the ranks by hstu_lpt_partition (attended pairs plus the
+    projections' per-token work, longest first to the least-loaded rank), so
+    that per-rank work stays about fixed as ranks are added.  Every rank draws
+    the same batch and computes the same assignment: nothing is exchanged."""
+    spec = W.CONFIGS[CONFIG_ID]
+    wl = W.make_workload(CONFIG_ID, batch=spec.batch * world)
+    if world == 1:
         return wl
-    own = W.make_workload(CONFIG_ID, seed=W.SEED_BASE + CONFIG_ID + 1000 * rank)
-    own.layers = wl.layers
-    return own
+    from hstu_sequential_transducer_02_b200 import binding as hb
+    rank_of, _ = hb.lpt_partition(wl.seq_offsets, world, token_weight=projection_pairs_per_token(spec))
+    return W.select_sequences(wl, np.nonzero(rank_of == rank)[0])
 
 
 def reduce_over_ranks(local_ms: float, local_tokens: int, world: int, device=None):
@@ -341,6 +353,7 @@ def measure_training(hb, steps: int):
     heads of 64, fp32 residual stream): SL, forward with saved activations,
     backward from dY = G; tokens (after SL) per second."""
     import torch
+    from hstu_sequential_transducer_02_b200.training import StackTrainer
     wl = W.make_workload(4)
     sp, e = wl.spec, wl.extras
     td, io = torch.bfloat16, torch.float32
@@ -360,19 +373,15 @@ def measure_training(hb, steps: int):
     saved = [hb.Saved.alloc(T_cap, sp.d_model, hv, td, "cuda") for _ in layers]
     acts = [torch.empty_like(x) for _ in layers]
 
+    trainer = StackTrainer(layers)   # one rank: the gradient reduction is a no-op
+
     def step():
         offs, idx = hb.stochastic_length(offs_in, coins, keys, int(e["sl_len"]), int(e["sl_prob_u32"]))
         cnt = offs[-1:]
         hb.gather_rows(x_all, idx, cnt, x)
         hb.gather_rows(ts_all, idx, cnt, ts)
         hb.gather_rows(g_all, idx, cnt, gy)
-        h = x
-        for ly, sv, a in zip(layers, saved, acts):
-            h = ly.forward(h, offs, ts, saved=sv, out=a)
-        dy = gy
-        ins = [x] + acts[:-1]
-        for li in range(len(layers) - 1, -1, -1):
-            dy, _ = layers[li].backward(ins[li], dy, saved[li], offs, ts)
+        trainer.step(x, offs, ts, gy, saved, acts)
         return offs
 
     offs = step()
@@ -449,7 +458,7 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     from hstu_sequential_transducer_02_b200 import binding as hb
 
-    wl = rank_workload(rank)
+    wl = rank_workload(rank, world)
     sp = wl.spec
     td = torch.bfloat16
     T = wl.total_tokens
@@ -533,8 +542,9 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "long-history HSTU layer forward: B=8 jagged sequences, n~U{4096..8192} "
-                                   f"(T={T} tokens), d_model=512, 4 heads x 128, 1 layer, causal, seed 20242",
+            "config": {"workload": f"long-history HSTU layer forward: B={8 * world} jagged sequences, "
+                                   f"n~U{{4096..8192}} (T={T_all} tokens), d_model=512, 4 heads x 128, 1 layer, "
+                                   "causal, seed 20242" + (f", dealt out over {world} GPUs by LPT" if world > 1 else ""),
                        "global_batch": 8 * world, "seq_len": "4096-8192", "parallelism": f"dp{world}",
                        "l2": "flushed between timed steps (256 MiB write outside the timed events)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

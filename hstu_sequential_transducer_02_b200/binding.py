@@ -443,6 +443,28 @@ def debug_timeout_probe(timeout_ns: int, status: torch.Tensor, stream=None):
 
 
 # ----------------------------------------------------------------------------
+# data-parallel sharding (host only)
+# ----------------------------------------------------------------------------
+_lib_lpt = _sig("hstu_lpt_partition", _c_int, [_c_i32, _c_vp, _c_vp, _c_i32, _c_dbl, _c_vp, _c_vp])
+EXPORTED.append("hstu_lpt_partition")
+
+
+def lpt_partition(seq_offsets, world: int, num_targets=None, token_weight: float = 0.0):
+    """Rank of every sequence of a jagged batch (host arrays) and each rank's
+    total cost, from hstu_lpt_partition: returns (rank_of int32[B], cost float64[world])."""
+    import numpy as np
+    offs = np.ascontiguousarray(seq_offsets, dtype=np.int32)
+    B = offs.size - 1
+    nt = None if num_targets is None else np.ascontiguousarray(num_targets, dtype=np.int32)
+    rank_of = np.zeros(max(B, 1), dtype=np.int32)
+    cost = np.zeros(max(world, 1), dtype=np.float64)
+    _check(_lib_lpt(B, offs.ctypes.data_as(_c_vp), None if nt is None else nt.ctypes.data_as(_c_vp), world,
+                    float(token_weight), rank_of.ctypes.data_as(_c_vp), cost.ctypes.data_as(_c_vp)),
+           "hstu_lpt_partition")
+    return rank_of[:B], cost[:world]
+
+
+# ----------------------------------------------------------------------------
 # tracing
 # ----------------------------------------------------------------------------
 _lib_trace_enable = _sig("hstu_trace_enable", _c_int, [_c_int])

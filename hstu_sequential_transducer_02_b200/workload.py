@@ -294,6 +294,28 @@ def make_workload(cid: int, *, seed: Optional[int] = None, scale: float = 1.0,
     return Workload(spec, offsets, ts, x, layers, extras=extras)
 
 
+def select_sequences(wl: "Workload", seqs) -> "Workload":
+    """The sub-batch of `wl` made of the sequences `seqs` (in that order): their
+    rows of X and timestamps, new offsets, the same weights.  Per-token extras
+    (gradient seeds, SL keys) and per-sequence extras (SL coins) follow their
+    sequences; scalars are kept."""
+    seqs = [int(s) for s in seqs]
+    offs = np.asarray(wl.seq_offsets, dtype=np.int64)
+    rows = np.concatenate([np.arange(offs[s], offs[s + 1]) for s in seqs]) if seqs else np.zeros(0, np.int64)
+    lens = np.array([offs[s + 1] - offs[s] for s in seqs], dtype=np.int64)
+    T = int(offs[-1])
+    extras = {}
+    for k, v in wl.extras.items():
+        v = np.asarray(v)
+        if v.ndim >= 1 and v.shape[0] == T:
+            extras[k] = v[rows]
+        elif v.ndim >= 1 and v.shape[0] == len(offs) - 1:
+            extras[k] = v[np.asarray(seqs, dtype=np.int64)]
+        else:
+            extras[k] = v
+    return Workload(wl.spec, offsets_from_lengths(lens), wl.timestamps[rows], wl.x[rows], wl.layers, extras=extras)
+
+
 def interleave_item_action(wl: "Workload", seed: int = 7, delay_mean: float = 60.0) -> "Workload":
     """Ranking input with every item followed by the user's reaction to it (the
     ranking setting of the pages: the input alternates objects and the reactions

@@ -351,6 +351,26 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers,
                  const int32_t* cand_offsets, const void* cand_x, const int64_t* cand_ts,
                  void* cand_out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- data-parallel sharding ----------------------------------------------- */
+
+/* Splits one jagged batch over `world` data-parallel ranks by sequence (rows of
+ * different sequences never interact, so the ranks exchange nothing on the data
+ * path; "Meta HSTU" case study, "Разная длина истории": a sequence costs what its
+ * real length costs).  Host-only: no device work, usable without a GPU.
+ * The cost of sequence s is its attended pairs, N(N+1)/2 + m(N+1) with N its
+ * history length and m = num_targets[s] (NULL: 0), plus token_weight * n_s for
+ * the row-wise work; the sequences go, in order of decreasing cost (equal costs:
+ * lower index first), each to the rank with the smallest total so far (equal
+ * totals: lower rank) -- greedy longest-processing-time first.  Every rank that
+ * calls it with the same arguments gets the same assignment.
+ *   seq_offsets [batch+1], num_targets [batch] or NULL: HOST arrays;
+ *   rank_of [batch]: HOST, receives each sequence's rank;
+ *   rank_cost [world]: HOST, receives each rank's total cost.
+ * Errors: HSTU_ERR_INVALID_ARG (batch < 0, world < 1, null outputs, offsets not
+ * starting at 0 or decreasing, negative token_weight). */
+int hstu_lpt_partition(int32_t batch, const int32_t* seq_offsets, const int32_t* num_targets, int32_t world,
+                       double token_weight, int32_t* rank_of, double* rank_cost);
+
 /* ---- Stochastic Length ------------------------------------------------------ */
 
 int hstu_stochastic_length_workspace_size(int32_t batch, int32_t total_tokens, size_t* bytes);

@@ -11,6 +11,7 @@ import sys
 
 import numpy as np
 import pytest
+import torch
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -56,20 +57,81 @@ def test_reduce_over_ranks_single_rank_is_identity():
     assert bench.reduce_over_ranks(3.5, 77, 1) == (3.5, 77)
 
 
-def test_rank_workloads_share_weights_not_data():
-    w0 = bench.rank_workload(0)
-    w1 = bench.rank_workload(1)
-    # one model
-    for a, b in zip(w0.layers, w1.layers):
+def test_rank_workloads_deal_out_one_batch():
+    """With N ranks the benchmark draws one batch of 8 N long-history sequences
+    and deals it out by LPT: the shards are disjoint, cover the batch, share the
+    weights, and each holds about the same work; with one rank the shard is the
+    8-sequence workload itself."""
+    from hstu_sequential_transducer_02_b200 import workload as W
+    one = bench.rank_workload(0, 1)
+    ref = W.make_workload(2)
+    assert np.array_equal(one.seq_offsets, ref.seq_offsets) and np.array_equal(one.x, ref.x)
+    glob = W.make_workload(2, batch=16)
+    shards = [bench.rank_workload(r, 2) for r in range(2)]
+    rows = np.concatenate([s.x for s in shards])
+    assert rows.shape == glob.x.shape
+    # every sequence of the global batch is in exactly one shard (matched by its timestamps)
+    starts = sorted(int(s.timestamps[o]) for s in shards for o in s.seq_offsets[:-1])
+    assert starts == sorted(int(glob.timestamps[o]) for o in glob.seq_offsets[:-1])
+    for a, b in zip(shards[0].layers, shards[1].layers):
         for name in ("w1", "w2", "pos_bias", "time_bias"):
             assert np.array_equal(getattr(a, name), getattr(b, name))
-    # independent sequences from the same recipe: same batch size and length range
-    assert len(w0.seq_offsets) == len(w1.seq_offsets)
-    assert not np.array_equal(w0.seq_offsets, w1.seq_offsets) or not np.array_equal(w0.x, w1.x)
-    for w in (w0, w1):
-        lens = np.diff(w.seq_offsets)
-        assert lens.min() >= 4096 and lens.max() <= 8192
-        assert np.all(np.diff(w.timestamps[w.seq_offsets[0]:w.seq_offsets[1]]) >= 0)
+    work = [bench.unmasked_pairs(s.seq_offsets) + bench.projection_pairs_per_token(s.spec) * s.x.shape[0]
+            for s in shards]
+    biggest = max(bench.unmasked_pairs([0, n]) + bench.projection_pairs_per_token(glob.spec) * n
+                  for n in np.diff(glob.seq_offsets))
+    assert abs(work[0] - work[1]) <= biggest
+
+
+def _lpt_cost(offs, nt, w):
+    n = np.diff(np.asarray(offs, np.int64))
+    m = np.zeros_like(n) if nt is None else np.minimum(np.maximum(np.asarray(nt, np.int64), 0), n)
+    N = n - m
+    return (N * (N + 1) // 2 + m * (N + 1)).astype(np.float64) + w * n
+
+
+def test_lpt_partition_properties():
+    """hstu_lpt_partition (host only): every sequence goes to one rank, the rank
+    totals add up, the spread between ranks is at most one sequence's cost, and
+    on small batches the largest rank total is within 4/3 of the best possible
+    (the longest-processing-time-first guarantee), checked by brute force."""
+    import itertools
+    from hstu_sequential_transducer_02_b200 import binding as hb
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        B = int(rng.integers(1, 9))
+        world = int(rng.integers(1, 4))
+        lens = rng.integers(0, 300, B)
+        offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        nt = rng.integers(0, 40, B).astype(np.int32) if trial % 2 else None
+        w = float(rng.choice([0.0, 3.5]))
+        rank_of, tot = hb.lpt_partition(offs, world, num_targets=nt, token_weight=w)
+        cost = _lpt_cost(offs, nt, w)
+        assert rank_of.shape == (B,) and np.all((rank_of >= 0) & (rank_of < world))
+        assert np.allclose(tot, [cost[rank_of == r].sum() for r in range(world)])
+        assert tot.max() - tot.min() <= cost.max() + 1e-9
+        best = min(max(cost[np.array(a) == r].sum() for r in range(world))
+                   for a in itertools.product(range(world), repeat=B))
+        assert tot.max() <= 4.0 / 3.0 * best + 1e-9
+    # equal costs: lower index first, to the lower rank
+    rank_of, _ = hb.lpt_partition(np.array([0, 5, 10, 15, 20], np.int32), 2)
+    assert list(rank_of) == [0, 1, 0, 1]
+
+
+def test_lpt_partition_argument_checks():
+    import ctypes
+    from hstu_sequential_transducer_02_b200 import binding as hb
+    with pytest.raises(hb.HstuError):
+        hb.lpt_partition(np.array([0, 5], np.int32), 0)
+    with pytest.raises(hb.HstuError):
+        hb.lpt_partition(np.array([1, 5], np.int32), 2)        # offsets must start at 0
+    with pytest.raises(hb.HstuError):
+        hb.lpt_partition(np.array([0, 5, 3], np.int32), 2)     # decreasing
+    with pytest.raises(hb.HstuError):
+        hb.lpt_partition(np.array([0, 5], np.int32), 2, token_weight=-1.0)
+    assert hb._lib_lpt(2, None, None, 2, 0.0, None, None) == hb.ERR_INVALID_ARG
+    r, c = hb.lpt_partition(np.array([0], np.int32), 3)
+    assert r.size == 0 and np.all(c == 0)
 
 
 def test_unmasked_pairs_matches_oracle_count():
@@ -158,3 +220,84 @@ def test_data_parallel_single_rank_is_a_no_op():
     red.layer_done(g)
     red.wait()
     assert all(torch.equal(g[n], torch.ones(3)) for n in PARAM_GRADS)
+
+
+class _OracleLayer:
+    """A stand-in for binding.Layer on CPU ranks: the same forward / backward
+    signature, computed by the fp64 oracle, gradients returned as fp32 tensors
+    under the binding's names."""
+
+    NAMES = {"w1": "dw1", "b1": "db1", "ln1_gamma": "dln1_g", "ln1_beta": "dln1_b", "ln2_gamma": "dln2_g",
+             "ln2_beta": "dln2_b", "w2": "dw2", "b2": "db2", "pos_bias": "dpos_bias", "time_bias": "dtime_bias"}
+
+    def __init__(self, p, H, dh):
+        self.p, self.H, self.dh = p, H, dh
+
+    def forward(self, x, seq_offsets, timestamps, num_targets=None, saved=None, out=None):
+        y = O.layer_forward(x.numpy(), self.p, seq_offsets.numpy(), timestamps.numpy(), self.H, self.dh)
+        out.copy_(torch.from_numpy(y))
+        return out
+
+    def backward(self, x, dy, saved, seq_offsets, timestamps, num_targets=None):
+        r = O.layer_backward(x.numpy(), self.p, dy.numpy(), seq_offsets.numpy(), timestamps.numpy(), self.H, self.dh)
+        grads = {k: torch.from_numpy(np.asarray(r[v], np.float64)).float() for k, v in self.NAMES.items()}
+        return torch.from_numpy(r["dx"]), grads
+
+
+def _train_rank_main(rank, world, port, results):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from hstu_sequential_transducer_02_b200 import binding as hb
+    from hstu_sequential_transducer_02_b200 import workload as W
+    from hstu_sequential_transducer_02_b200.training import StackTrainer
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        wl = W.make_workload(4, batch=7, scale=1 / 16, random_affine=True)
+        wl.layers = wl.layers[:2]
+        s = wl.spec
+        rank_of, _ = hb.lpt_partition(wl.seq_offsets, world, token_weight=2.5 * s.d_model)
+        mine = np.nonzero(rank_of == rank)[0]
+        sh = W.select_sequences(wl, mine)
+        layers = [_OracleLayer(p, s.num_heads, s.head_dim) for p in wl.layers]
+        x = torch.from_numpy(sh.x.astype(np.float64))
+        acts = [torch.empty_like(x) for _ in layers]
+        dx, grads = StackTrainer(layers).step(x, torch.from_numpy(sh.seq_offsets), torch.from_numpy(sh.timestamps),
+                                              torch.from_numpy(sh.extras["grad_out"].astype(np.float64)),
+                                              [None] * len(layers), acts)
+        results[rank] = dict(seqs=mine, dx=dx.numpy(),
+                             grads=[{k: v.numpy() for k, v in g.items()} for g in grads])
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_training_step_gloo_world2():
+    """Two CPU ranks, each with its LPT shard of one training batch, run the
+    training driver (forward, backward, per-layer gradient all-reduce): every
+    rank ends with the gradients of the whole batch computed on one rank, and
+    each rank's input gradient is the whole batch's for its own sequences."""
+    from hstu_sequential_transducer_02_b200 import workload as W
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        results = mgr.dict()
+        mp.start_processes(_train_rank_main, args=(world, _free_port(), results), nprocs=world, join=True,
+                           start_method="spawn")
+        got = dict(results)
+    wl = W.make_workload(4, batch=7, scale=1 / 16, random_affine=True)
+    wl.layers = wl.layers[:2]
+    s = wl.spec
+    full = O.stack_backward(wl.x, wl.layers, wl.extras["grad_out"], wl.seq_offsets, wl.timestamps, s.num_heads,
+                            s.head_dim)
+    seqs = np.concatenate([got[r]["seqs"] for r in range(world)])
+    assert sorted(seqs.tolist()) == list(range(7)) and all(len(got[r]["seqs"]) > 0 for r in range(world))
+    for r in range(world):
+        for li in range(2):
+            for k, v in _OracleLayer.NAMES.items():
+                want = full[li][v]
+                assert np.allclose(got[r]["grads"][li][k], want, rtol=1e-5, atol=1e-5 * np.abs(want).max()), \
+                    (r, li, k)
+        rows = np.concatenate([np.arange(wl.seq_offsets[q], wl.seq_offsets[q + 1]) for q in got[r]["seqs"]])
+        assert np.allclose(got[r]["dx"], full[0]["dx"][rows], rtol=1e-9, atol=1e-9)

@@ -53,15 +53,6 @@ struct Cfg {
   static constexpr int kTileBytes = BM * DH * 2;
 };
 
-// Timestamp record of one kv tile, as written by ts_tiles_kernel.
-struct TsRec {
-  int32_t rel[BN];   // t_j - t_first(sequence), clamped to +-(2^30 - 1); 0 beyond the sequence
-  int32_t mn[4];     // per 32-column segment: min / max of rel over the columns inside the sequence
-  int32_t mx[4];
-  int32_t wide;      // 1 if some column's offset left +-2^30 (then the 64-bit path is used)
-  int32_t pad[3];
-};
-static_assert(sizeof(TsRec) == kRecBytes, "record layout");
 
 constexpr int kRecStages = 8;              // timestamp records run up to 8 kv tiles ahead
 constexpr int kSBufs = 3;                  // S/P buffers in TMEM: S runs two kv tiles ahead of P V
@@ -468,6 +459,9 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
       const int posi = token_pos(i, si.hist);
       const KvRange kr = kv_tiles_for(r0, min(si.n, r0 + BM), si.hist, BN);
       const int nk = kv_count(kr);
+      // rows of the warp with fewer than 128 attended columns: their outputs may rest on
+      // a few small terms, whose SiLU the tanh form would not keep accurate
+      const bool few_terms = __any_sync(0xffffffffu, live && i < kNumBuckets);
       // this row's last one-bucket segment: distances in [c_lo, c_hi) share the
       // bias 2 * c_hb (empty until the first one); far from the diagonal the bucket
       // rarely changes from one kv tile to the next
@@ -551,9 +545,9 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
           tmem_ld_32x32b_x32(tmem_s0 + sb * BN + lane_off + seg * 32, raw);
         }
         tmem_ld_wait_regs(raw);
-        // ---- bias, SiLU, mask; packed bf16 pairs.  With h = (s + bias) / 2: far from the
-        // diagonal (rows with at least 128 attended columns) SiLU = h + h tanh h; near it
-        // and on candidate rows, whose outputs may rest on a few terms, the exact form
+        // ---- bias, SiLU, mask; packed bf16 pairs.  With h = (s + bias) / 2, SiLU = h + h tanh h,
+        // except on rows whose outputs may rest on a few terms (the first 128 rows of a
+        // sequence, candidates, which see one column beyond the history): the exact form
         uint32_t pk[16];
         if (wrank == 0) {
 #pragma unroll
@@ -612,7 +606,7 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
             float h0, h1;
             half_plus2c(__uint_as_float(raw[2 * q]), __uint_as_float(raw[2 * q + 1]), __uint_as_float(bw[q] << 16),
                         __uint_as_float(bw[q] & 0xFFFF0000u), h0, h1);
-            const uint32_t v = silu2_exact_bf16(h0, h1);
+            const uint32_t v = few_terms ? silu2_exact_bf16(h0, h1) : silu2_bf16(h0, h1);
             pk[q] = (2 * q <= lim ? (v & 0xFFFFu) : 0u) | (2 * q + 1 <= lim ? (v & 0xFFFF0000u) : 0u);
           }
         } else if (__all_sync(0xffffffffu, narrow)) {

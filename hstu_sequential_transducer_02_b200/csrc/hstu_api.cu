@@ -131,7 +131,11 @@ struct AttnWs {
   int32_t* tile_recs;   // tensor-core path: timestamp records
   int tiles_cap;
   void* band;           // tensor-core path, rab shared by heads: near-diagonal bias band
+  float* rab_partial;   // tensor-core backward: per-CTA partial rab gradients
+  int rab_tables;
 };
+
+constexpr int kMaxBwdCtas = 256;   // the tensor-core backward runs at most this many CTAs
 
 bool use_tc(const hstu_attn_desc* d) {
   return !(d->flags & HSTU_FLAG_FORCE_SIMT) && tc_attn_supported(d->dtype, d->dqk);
@@ -157,11 +161,22 @@ AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd, bo
   w.tile_recs = nullptr;
   w.tiles_cap = 0;
   w.band = nullptr;
+  w.rab_partial = nullptr;
+  w.rab_tables = d->rab_head_stride ? d->num_heads : 1;
   if (!bwd && use_tc(d)) {
     w.tiles_cap = (int)ts_tiles_capacity(B, T);
     w.tile_base = c.take<int32_t>((size_t)B + 1);
     w.tile_recs = c.take<int32_t>((size_t)w.tiles_cap * kTsRecWords);
     if (with_band && d->rab_head_stride == 0) w.band = c.take<uint8_t>(band_bytes(T));
+  }
+  if (bwd && use_tc_bwd(d)) {
+    // timestamp records of the 128-row tiles and, with one bias table for all heads,
+    // the backward's near-diagonal band of bias and time-bucket words
+    w.tiles_cap = (int)ts_tiles_capacity(B, T);
+    w.tile_base = c.take<int32_t>((size_t)B + 1);
+    w.tile_recs = c.take<int32_t>((size_t)w.tiles_cap * kTsRecWords);
+    if (with_band && d->rab_head_stride == 0) w.band = c.take<uint8_t>(bwd_band_bytes(T));
+    w.rab_partial = c.take<float>((size_t)kMaxBwdCtas * w.rab_tables * 2 * kNumBuckets);
   }
   return w;
 }
@@ -266,10 +281,20 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
                  int64_t lddv, float* dpos, float* dtime, const AttnWs& w, cudaStream_t st) {
   const int tile = attn_bwd_tile(d);
   const int H = d->num_heads, dh = d->dqk;
+  const bool tc = use_tc_bwd(d);
+  const Thresholds thr = thresholds_for(d->time_div);
   {
     TraceScope tr("sched_bwd", st);
     HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, H, tile, tile, 1,
-                                     w.capacity, w.items, w.count, w.status, st));
+                                     w.capacity, w.items, w.count, w.status, st, tc ? w.tile_base : nullptr));
+  }
+  if (tc) {
+    TraceScope tr("bwd_prep", st);
+    HSTU_CUDA(launch_ts_tiles(jb->seq_offsets, jb->timestamps, jb->batch, w.tile_base, w.tiles_cap, w.tile_recs, st));
+    if (w.band)
+      HSTU_CUDA(launch_bwd_band(jb->seq_offsets, jb->num_targets, jb->timestamps, jb->batch, jb->total_tokens,
+                                w.tile_base, w.tiles_cap, pos_bias, time_bias, thr, d->time_div, w.status,
+                                (uint32_t*)w.band, st));
   }
   HSTU_CUDA(cudaMemsetAsync(w.dq_accum, 0, sizeof(float) * (size_t)jb->total_tokens * H * dh, st));
   AttnBwdParams p;
@@ -286,15 +311,25 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   p.rab_head_stride = d->rab_head_stride;
   p.num_heads = H;
   p.total_rows = jb->total_tokens;
-  p.thr = thresholds_for(d->time_div);
+  p.thr = thr;
   p.items = w.items;
   p.item_count = w.count;
   p.status = w.status;
   p.timeout_ns = kDefaultTimeoutNs;
-  if (use_tc_bwd(d)) {
-    TraceScope tr("attn_bwd_tc", st);
-    const int grid = w.capacity < 148 ? (w.capacity > 0 ? w.capacity : 1) : 148;
-    HSTU_CUDA(launch_attn_bwd_tc(p, grid, st, d->time_div));
+  p.tile_base = w.tile_base;
+  p.tile_recs = w.tile_recs;
+  p.band = (const uint32_t*)w.band;
+  p.item_cursor = w.count + 1;
+  p.rab_partial = w.rab_partial;
+  p.rab_tables = w.rab_tables;
+  if (tc) {
+    const int grid = std::min(tc_attn_grid(w.capacity), kMaxBwdCtas);
+    HSTU_CUDA(cudaMemsetAsync(w.rab_partial, 0, sizeof(float) * (size_t)grid * w.rab_tables * 2 * kNumBuckets, st));
+    {
+      TraceScope tr("attn_bwd_tc", st);
+      HSTU_CUDA(launch_attn_bwd_tc(p, grid, st, d->time_div));
+    }
+    HSTU_CUDA(launch_rab_reduce(w.rab_partial, grid, w.rab_tables, d->rab_head_stride, dpos, dtime, st));
   } else {
     TraceScope tr("attn_bwd_simt", st);
     const int grid = w.capacity < 148 * 2 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 2;

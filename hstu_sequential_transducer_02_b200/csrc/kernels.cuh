@@ -21,6 +21,14 @@ cudaError_t launch_build_work_list(const int32_t* offs, const int32_t* num_targe
 // first timestamp, with per-32-column min/max and a flag when any offset
 // leaves +-2^30 (record of kTsRecWords int32, 16-byte multiple).
 constexpr int kTsRecWords = 140;   // rel[128] | min[4] | max[4] | wide | pad[3]
+struct TsRec {
+  int32_t rel[128];  // t_j - t_first(sequence), clamped to +-(2^30 - 1); 0 beyond the sequence
+  int32_t mn[4];     // per 32-column segment: min / max of rel over the columns inside the sequence
+  int32_t mx[4];
+  int32_t wide;      // 1 if some column's offset left +-2^30 (then the 64-bit path is used)
+  int32_t pad[3];
+};
+static_assert(sizeof(TsRec) == kTsRecWords * 4, "record layout");
 constexpr int kBandChunks = 20;    // 8-column bf16 chunks per row of the near-diagonal bias band
 size_t ts_tiles_capacity(int B, int T);
 
@@ -63,6 +71,17 @@ struct AttnFwdParams {
   const void* band;            // tensor-core path: near-diagonal half-bias band (bf16), or null
 };
 
+// Near-diagonal band of the tensor-core backward: for kv row j of a sequence and the
+// 160 q rows i in [floor32(j), floor32(j) + 160), one 32-bit word: the relative bias
+// rab(i, j) as bf16 in the upper half (-1e30 where (i, j) is not attended, so that
+// SiLU and its derivative vanish there) and the time bucket in bits 0-6.
+constexpr int kBwdBandCols = 160;
+size_t bwd_band_bytes(int T);
+cudaError_t launch_bwd_band(const int32_t* offs, const int32_t* num_targets, const int64_t* ts, int B, int T,
+                            const int32_t* tile_base, int tiles_cap, const float* pos_bias, const float* time_bias,
+                            const Thresholds& thr, double time_div, const int32_t* status, uint32_t* band,
+                            cudaStream_t st);
+
 struct AttnBwdParams {
   const int32_t* seq_offsets;
   const int32_t* num_targets;
@@ -86,6 +105,12 @@ struct AttnBwdParams {
   const int32_t* item_count;
   int32_t* status;
   long long timeout_ns;        // bound of every device-side wait
+  const int32_t* tile_base;    // tensor-core path: first timestamp record of each sequence
+  const int32_t* tile_recs;    // tensor-core path: timestamp records of the 128-row tiles
+  const uint32_t* band;        // tensor-core path, bias shared by heads: near-diagonal band, or null
+  int32_t* item_cursor;        // tensor-core path: dynamic work-list cursor (zeroed by the scheduler)
+  float* rab_partial;          // tensor-core path: per-CTA partial rab gradients [grid][rab_tables][2][128], zeroed
+  int rab_tables;              // 1 (tables shared by heads) or num_heads
 };
 
 int simt_tile_m();
@@ -95,6 +120,9 @@ cudaError_t launch_attn_bwd_simt(const AttnBwdParams& p, int dtype, int dh, int 
 bool tc_attn_bwd_supported(int dtype, int dh);
 int tc_bwd_tile();
 cudaError_t launch_attn_bwd_tc(const AttnBwdParams& p, int grid, cudaStream_t st, double time_div);
+// d_pos[h * head_stride + b] += sum over CTAs of the partial tables, likewise d_time
+cudaError_t launch_rab_reduce(const float* part, int ctas, int tables, int head_stride, float* d_pos, float* d_time,
+                              cudaStream_t st);
 cudaError_t launch_dq_finalize(const float* acc, const int32_t* offs, int B, int H, int dh, int dtype,
                                void* dq, int64_t lddq, int grid, cudaStream_t st);
 

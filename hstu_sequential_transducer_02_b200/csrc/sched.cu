@@ -205,7 +205,10 @@ build_work_list_kernel(const int32_t* __restrict__ offs, const int32_t* __restri
       for (int h = 0; h < H; ++h) items[pos + h] = WorkItem{s, h, t, c};
     }
   }
-  if (tid == 0) *count = total;
+  if (tid == 0) {
+    *count = total;
+    count[1] = 0;  // dynamic fetch cursor
+  }
 }
 }  // namespace
 

@@ -70,9 +70,9 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // Waits until the phase of `bar` with the given parity has completed.  Gives
 // up after `timeout_ns` nanoseconds, or as soon as *abort becomes non-zero;
 // returns false then (the caller records HSTU_ERR_TIMEOUT and unwinds).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long timeout_ns,
-                                          volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+// (the waiting loop is out of line: every call site keeps only the first test)
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, long long timeout_ns,
+                                            volatile int* abort) {
   const uint64_t t0 = global_timer_ns();
   const uint32_t hint = timeout_ns < 1000000ll ? (uint32_t)timeout_ns : 1000000u;  // sleep at most 1 ms per try
   for (;;) {
@@ -80,6 +80,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
     if (abort && *abort) return false;
     if ((long long)(global_timer_ns() - t0) > timeout_ns) return false;
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long timeout_ns,
+                                          volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, timeout_ns, abort);
 }
 
 // mbar_wait by every lane of a converged warp, with one outcome for the warp
@@ -212,6 +217,18 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
+}
+// 32 lanes x 8 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+// 32 lanes x 4 consecutive 32-bit columns from registers
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 // 32 lanes x 16 consecutive 32-bit columns from registers; thread t writes lane (base lane + t)
 __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {

@@ -79,7 +79,7 @@ def _rab(ts, n, nt, pos_bias, time_bias, band: bool):
     return rab
 
 
-def attention_forward(q, k, v, offs, ts, pos_bias, time_bias, silu_p="bf16pair", band=True):
+def attention_forward(q, k, v, offs, ts, pos_bias, time_bias, silu_p="bf16pair", band=True, num_targets=None):
     T, H, dv = v.shape
     out = np.zeros((T, H, dv))
     for s in range(len(offs) - 1):
@@ -87,12 +87,14 @@ def attention_forward(q, k, v, offs, ts, pos_bias, time_bias, silu_p="bf16pair",
         n = b - a
         if n == 0:
             continue
-        mask = O.attention_mask(n, 0)
-        rab = _rab(ts[a:b], n, 0, pos_bias, time_bias, band)
+        nt = 0 if num_targets is None else int(num_targets[s])
+        N = max(n - nt, 1)
+        mask = O.attention_mask(n, nt)
+        rab = _rab(ts[a:b], n, nt, pos_bias, time_bias, band and nt == 0)
         for h in range(H):
             S = q[a:b, h] @ k[a:b, h].T + rab
             P = np.where(mask, _p_forward(S, silu_p), 0.0)
-            out[a:b, h] = _r('attn_out', (P @ v[a:b, h]) / n)
+            out[a:b, h] = _r('attn_out', (P @ v[a:b, h]) / N)
     return out
 
 
@@ -122,17 +124,38 @@ def attention_backward(q, k, v, dout, offs, ts, pos_bias, time_bias):
     return dq, dk, dv, dpos, dtime
 
 
-def layer_forward(x, p, offs, ts, H, dh, silu_p="bf16pair", band=True):
+def layer_forward(x, p, offs, ts, H, dh, silu_p="bf16pair", band=True, num_targets=None, io="f32"):
+    """One layer; `io` is the type of the residual stream (X and Y): "f32" or "bf16"."""
     T = x.shape[0]
     xh = _r('xhat', O.layer_norm(x, p.ln1_g, p.ln1_b))
     z = xh @ np.asarray(p.w1, np.float64).T + np.asarray(p.b1, np.float64)
     a = _r('uvqk', O.silu(z))
     U, V, Q, K = O.split_uvqk(a, H, dh)
-    Oa = attention_forward(Q, K, V, offs, ts, p.pos_bias, p.time_bias, silu_p, band)
+    Oa = attention_forward(Q, K, V, offs, ts, p.pos_bias, p.time_bias, silu_p, band, num_targets)
     on = O.layer_norm(Oa.reshape(T, H * dh), p.ln2_g, p.ln2_b)
     g = _r('gate', on * U.reshape(T, -1))
-    y = f32(x + g @ np.asarray(p.w2, np.float64).T + np.asarray(p.b2, np.float64))
+    y = x + g @ np.asarray(p.w2, np.float64).T + np.asarray(p.b2, np.float64)
+    y = bf16(y) if io == "bf16" else f32(y)
     return y, dict(xh=xh, z=_r('z', z), U=U, V=V, Q=Q, K=K, O=Oa, on=on, g=g)
+
+
+def mfalcon_rank(layers, hist_offsets, hist_x, hist_ts, cand_offsets, cand_x, cand_ts, microbatch, H, dh,
+                 silu_p="f32"):
+    """M-FALCON scoring with a bf16 residual stream, microbatch by microbatch
+    (the oracle's mfalcon_rank with the roundings of the bf16 path)."""
+    d = np.asarray(hist_x).shape[1]
+    out = np.zeros((int(cand_offsets[-1]), d))
+    for u in range(len(hist_offsets) - 1):
+        ha, hb = int(hist_offsets[u]), int(hist_offsets[u + 1])
+        ca, cb = int(cand_offsets[u]), int(cand_offsets[u + 1])
+        for c0 in range(ca, cb, microbatch):
+            c1 = min(c0 + microbatch, cb)
+            y = np.concatenate([hist_x[ha:hb], cand_x[c0:c1]], axis=0).astype(np.float64)
+            ts = np.concatenate([np.asarray(hist_ts[ha:hb]), np.asarray(cand_ts[c0:c1])]).astype(np.int64)
+            for p in layers:
+                y = layer_forward(y, p, [0, y.shape[0]], ts, H, dh, silu_p, False, [c1 - c0], io="bf16")[0]
+            out[c0:c1] = y[hb - ha:]
+    return out
 
 
 def layer_backward(x, p, dy, offs, ts, H, dh, silu_p="bf16pair", band=True) -> Dict[str, np.ndarray]:

@@ -187,11 +187,33 @@ def test_mfalcon_history_cache_ragged_users_two_layers():
 
 def test_mfalcon_user_without_history():
     """A user with no history: its candidates attend only to themselves (N = 1),
-    through two layers.  With a single attended term nothing averages the
-    rounding of P, and LayerNorm2 rescales the lone term: the attention's SiLU
-    must keep strongly negative scores accurate (fp32 tanh, one rounding)."""
+    through two layers.  A one-term attention output is the most sensitive case
+    of the layer: rounding x-hat or U, V, Q, K alone to bf16 for the tensor
+    cores, all else exact, moves these outputs by more than 3e-2 in max-abs
+    (tests/test_precision_model.py).  So: relative Frobenius within the
+    specification's 1e-2, and max-abs within 1.25 times that of the rounding
+    model of the bf16 path on the same inputs."""
+    import tests.precision_model as M
     got, ref = _mfalcon_ragged([64, 0, 37], [5, 9, 3], 2, 7)
-    assert_close(got, ref, "bf16", "mfalcon user without history, 2 layers")
+    M.set_rounding(M.ROUNDING_POINTS)
+    model = _mfalcon_model([64, 0, 37], [5, 9, 3], 2, 7)
+    ma, rel = errors(got, ref)
+    ma_model = errors(model, ref)[0]
+    print(f"no-history user, 2 layers: GPU max-abs {ma:.3e} rel-fro {rel:.3e}; rounding model max-abs {ma_model:.3e}")
+    assert rel <= 1e-2
+    assert ma <= 1.25 * ma_model
+
+
+def _mfalcon_model(hist_lens, counts, num_layers, microbatch):
+    import tests.precision_model as M
+    wl = W.make_workload(3, scale=1 / 32, batch=len(hist_lens), lengths=hist_lens)
+    e = wl.extras
+    s = wl.spec
+    co = e["cand_offsets"]
+    sel = np.concatenate([np.arange(co[u], co[u] + counts[u]) for u in range(len(counts))]).astype(np.int64)
+    cand_offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    return M.mfalcon_rank([wl.layers[0]] * num_layers, wl.seq_offsets, wl.x, wl.timestamps, cand_offsets,
+                          e["cand_x"][sel], e["cand_ts"][sel], microbatch, s.num_heads, s.head_dim)
 
 
 def test_mfalcon_too_few_microbatches_reported():

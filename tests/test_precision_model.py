@@ -86,3 +86,29 @@ def test_per_layer_error_of_the_bf16_path_is_within_bound(c4):
         r = M.layer_backward(xs[li], wl.layers[li], dys[li], offs, ts, s.num_heads, s.head_dim, silu_p="f32")
         worst = max(worst, max(_rel(r[n], ref[li][n]) for n in NAMES))
     assert worst < 1e-2
+
+
+def test_one_term_candidates_exceed_the_max_abs_bound_from_operand_rounding():
+    """M-FALCON candidates of a user without history attend only to themselves.
+    Through two layers, rounding only x-hat, or only U, V, Q, K, to bf16 (the
+    tensor cores' operands), all else exact, moves their outputs by more than
+    3e-2 (the specification's bf16 max-abs bound) against the oracle, while the
+    relative Frobenius error stays within 1e-2."""
+    hist_lens, counts, mb = [64, 0, 37], [5, 9, 3], 7
+    wl = W.make_workload(3, scale=1 / 32, batch=3, lengths=hist_lens)
+    e = wl.extras
+    s = wl.spec
+    co = e["cand_offsets"]
+    sel = np.concatenate([np.arange(co[u], co[u] + counts[u]) for u in range(3)]).astype(np.int64)
+    cand_offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    args = (wl.seq_offsets, wl.x, wl.timestamps, cand_offsets, e["cand_x"][sel], e["cand_ts"][sel], mb,
+            s.num_heads, s.head_dim)
+    ref = O.mfalcon_rank([wl.layers[0]] * 2, *args)
+    try:
+        for pts in (["xhat"], ["uvqk"]):
+            M.set_rounding(pts)
+            got = M.mfalcon_rank([wl.layers[0]] * 2, *args)
+            assert np.max(np.abs(got - ref)) > 3e-2, pts
+            assert _rel(got, ref) < 1e-2, pts
+    finally:
+        M.set_rounding(M.ROUNDING_POINTS)

@@ -347,6 +347,60 @@ def measure_mfalcon(hb, steps: int):
             "top_kernels": _top_kernels(trace, steps)}
 
 
+def _two_layer_ms(hb, wl, steps: int, short: bool) -> float:
+    """Device milliseconds of the workload's two-layer forward through
+    hstu_layer_fwd (short: with HSTU_FLAG_SHORT_SEQUENCES, one fused kernel per layer)."""
+    import torch
+    sp = wl.spec
+    td = torch.bfloat16
+    layers = [hb.Layer(hb.layer_weights_to_device(p_, td), sp.d_model, sp.num_heads, sp.head_dim,
+                       short_sequences=short) for p_ in wl.layers]
+    x = torch.from_numpy(wl.x).to(td).cuda()
+    offs = torch.from_numpy(wl.seq_offsets).cuda()
+    ts = torch.from_numpy(wl.timestamps).cuda()
+    ys = [torch.empty_like(x) for _ in layers]
+
+    def fwd():
+        h = x
+        for ly, y in zip(layers, ys):
+            h = ly.forward(h, offs, ts, out=y)
+
+    for _ in range(3):
+        fwd()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        fwd()
+    t1.record()
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
+def measure_short_sequences(hb, steps: int):
+    """The short-sequence workload (power-law lengths, d_model = 256, 4 heads of
+    64, 2 layers, bf16): tokens per second of the two-layer forward.  The recipe as
+    specified (32 sequences, lengths in [16, 1024]) runs through the multi-kernel
+    layer; with its lengths cut to [2, 128] (x 1/8) the layer can run as one fused
+    kernel per layer, measured next to the multi-kernel layer on 32 and 512
+    sequences."""
+    wl = W.make_workload(1)
+    T = int(wl.seq_offsets[-1])
+    ms = _two_layer_ms(hb, wl, steps, False)
+    out = {"workload": f"short sequences: B=32, power-law n in [16,1024] (T={T} tokens, longest "
+                       f"{int(np.max(np.diff(wl.seq_offsets)))}), d_model=256, 4 heads x 64, 2 layers, causal",
+           "tokens_per_s": T / (ms / 1e3), "ms_per_forward": ms, "steps": steps, "lengths_at_most_128": {}}
+    for B in (32, 512):
+        w2 = W.make_workload(1, scale=1 / 8, batch=B)
+        T2 = int(w2.seq_offsets[-1])
+        f_ms = _two_layer_ms(hb, w2, steps, True)
+        l_ms = _two_layer_ms(hb, w2, steps, False)
+        out["lengths_at_most_128"][f"B={B}"] = {
+            "tokens": T2, "fused_tokens_per_s": T2 / (f_ms / 1e3), "fused_ms": f_ms,
+            "layer_path_tokens_per_s": T2 / (l_ms / 1e3), "layer_path_ms": l_ms}
+    return out
+
+
 def measure_training(hb, steps: int):
     """Training step of the 8-layer stack (64 sequences, power-law lengths in
     [64, 4096] cut by Stochastic Length to 1024 with p = 0.8, d_model = 512, 8
@@ -563,6 +617,7 @@ def main():
         if world == 1 and not args.no_extra:
             line["mfalcon"] = measure_mfalcon(hb, 5)
             line["training"] = measure_training(hb, 3)
+            line["short_sequences"] = measure_short_sequences(hb, 50)
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl, args.oracle_seconds)
         print(json.dumps(line), flush=True)

@@ -25,6 +25,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_BAD_OFFSETS = range(7)
 DTYPE_F32, DTYPE_BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
+FLAG_SHORT_SEQUENCES = 2
 NUM_BUCKETS = 128
 
 _c_int = ctypes.c_int
@@ -293,9 +294,11 @@ class Layer:
 
     def __init__(self, weights: Dict[str, torch.Tensor], d_model: int, num_heads: int, head_dim: int,
                  force_simt: bool = False, eps: float = 1e-5, time_div: float = 0.301,
-                 residual_fp32: bool = False):
+                 residual_fp32: bool = False, short_sequences: bool = False):
         """residual_fp32: X, Y (and dX, dY) are fp32 tensors while weights and
-        activations use the weights' dtype."""
+        activations use the weights' dtype.  short_sequences: every sequence has
+        at most 128 tokens, and the forward runs as one fused kernel where the
+        shapes allow it (HSTU_FLAG_SHORT_SEQUENCES)."""
         self.w = weights
         self.dtype = weights["w1"].dtype
         self.io_dtype = torch.float32 if residual_fp32 else self.dtype
@@ -303,6 +306,8 @@ class Layer:
         self.desc = layer_desc(d_model, num_heads, head_dim, _dtype_code(weights["w1"]),
                                weights["pos_bias"].dim() == 2, force_simt, eps, time_div,
                                io_dtype=DTYPE_F32 if residual_fp32 else None)
+        if short_sequences:
+            self.desc.attn.flags |= FLAG_SHORT_SEQUENCES
         self.cw = layer_weights(weights)
         self._ws = {}
 

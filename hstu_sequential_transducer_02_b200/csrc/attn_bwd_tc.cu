@@ -138,6 +138,11 @@ __device__ __forceinline__ void fma2(float a0, float a1, float b0, float b1, flo
       "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
       : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
+__device__ __forceinline__ void add2(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r0), "=f"(r1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -159,7 +164,8 @@ __device__ __forceinline__ void p_ds2(float x0, float x1, float dp0, float dp1, 
                                       float& ds0, float& ds1) {
   float a0, a1;
   mul2(x0, x1, -1.4426950408889634f, -1.4426950408889634f, a0, a1);
-  const float d0 = ex2_approx(a0) + 1.0f, d1 = ex2_approx(a1) + 1.0f;
+  float d0, d1;
+  add2(ex2_approx(a0), ex2_approx(a1), 1.0f, 1.0f, d0, d1);
   const float s0 = rcp_approx(d0), s1 = rcp_approx(d1);
   float sn0, sn1, p0, p1, om0, om1, t0, t1, u0, u1;
   mul2(s0, s1, inv_n, inv_n, sn0, sn1);              // sigma / N
@@ -567,7 +573,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           lrank = dhi < th1 ? 1 : (dhi < th2 ? 2 : (dhi < th3 ? 3 : (dhi < thr32[tlo + 4] ? 4 : 5)));
           if (__any_sync(0xffffffffu, lrank > 4)) kind = 3;
         }
-        const int wrank = kind == 1 ? __reduce_max_sync(0xffffffffu, lrank) : 0;
+        int wrank = kind == 1 ? __reduce_max_sync(0xffffffffu, lrank) : 0;
+        // two buckets and every q row's timestamp at or after this lane's: the bucket of a
+        // column is one compare of its timestamp offset with rj + th1
+        if (wrank == 2 && __all_sync(0xffffffffu, rj <= qrec.mn[seg])) wrank = -2;
+        const int64_t up64 = (int64_t)rj + th1;
+        const int32_t up_at = up64 > 0x7FFFFFFF ? 0x7FFFFFFF : (int32_t)up64;
         const float inv_n = si.inv_n;
         const uint32_t ds_atom = sDS + (seg >> 1) * kTile + jl * 128;   // dS^T row jl, q columns 32 seg ..
         const int ds_ch = (seg & 1) * 4;
@@ -585,39 +596,76 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
                                                          (D > 0 ? D : 0));
         if (!mbar_wait(&bars->sp_full, g & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
+        uint32_t pk_prev[4], dk_prev[4];   // the first chunk's words, held until the readouts
         if (kind != 3) {
-          // ---- the segment in two halves of 16 q columns: S^T and dP^T of the half into
-          // registers (the second half's load frees the score buffers for the next tile's
+          // ---- the segment in four chunks of 8 q columns: S^T and dP^T of the chunk into
+          // registers (the last chunk's load frees the score buffers for the next tile's
           // MMAs), P and dS, then P^T into TMEM and dS^T into shared memory
 #pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            uint32_t sr[16], dr[16];
-            tmem_ld_32x32b_x16(tmem + kColS + lane_off + 32 * seg + 16 * hh, sr);
-            tmem_ld_32x32b_x16(tmem + kColDP + lane_off + 32 * seg + 16 * hh, dr);
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t sr[8], dr[8];
+            tmem_ld_32x32b_x8(tmem + kColS + lane_off + 32 * seg + 8 * c8, sr);
+            tmem_ld_32x32b_x8(tmem + kColDP + lane_off + 32 * seg + 8 * c8, dr);
+            uint32_t w[8];    // band words of the chunk (kv rows beyond the sequence read none: masked)
+            if (kind == 2) {
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                uint4 v4;
+                if (jlive) v4 = __ldg(bp + 2 * c8 + c);
+                else v4.x = v4.y = v4.z = v4.w = __float_as_uint(kMaskedBias) & 0xFFFF0000u;
+                w[4 * c] = v4.x; w[4 * c + 1] = v4.y; w[4 * c + 2] = v4.z; w[4 * c + 3] = v4.w;
+              }
+            }
             tmem_ld_wait();
-            if (hh == 1) {
+            if (c8 == 3) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&bars->sp_free);
             }
-            uint32_t pk[8];   // P^T words (bf16 pairs) of the half's 16 q columns
-            uint32_t dk[8];   // dS^T words
+            uint32_t pk[4];   // P^T words (bf16 pairs) of the chunk's 8 q columns
+            uint32_t dk[4];   // dS^T words
             if (kind == 0) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) { pk[e] = 0u; dk[e] = 0u; }
+              for (int e = 0; e < 4; ++e) { pk[e] = 0u; dk[e] = 0u; }
             } else if (kind == 1 && wrank == 1) {
 #pragma unroll
-              for (int e = 0; e < 16; e += 2) {
+              for (int e = 0; e < 8; e += 2) {
                 float ds0, ds1;
                 p_ds2(__uint_as_float(sr[e]) + hb0, __uint_as_float(sr[e + 1]) + hb0, __uint_as_float(dr[e]),
                       __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
                 dk[e >> 1] = pack_bf16x2(ds0, ds1);
                 a0 += ds0 + ds1;
               }
+            } else if (kind == 1 && wrank == -2) {
+              float aup = 0.f;   // the upper bucket's part of what went into a0
+#pragma unroll
+              for (int e4 = 0; e4 < 2; ++e4) {
+                const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 8 * c8 + 4 * e4]);
+                const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+                bool up[4];
+                float xs[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  up[u] = rv[u] >= up_at;
+                  xs[u] = __uint_as_float(sr[4 * e4 + u]) + (up[u] ? hb1 : hb0);
+                }
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                  float ds0, ds1;
+                  const int e = 4 * e4 + 2 * q2;
+                  p_ds2(xs[2 * q2], xs[2 * q2 + 1], __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n,
+                        pk[e >> 1], ds0, ds1);
+                  dk[e >> 1] = pack_bf16x2(ds0, ds1);
+                  a0 += ds0 + ds1;
+                  aup += (up[2 * q2] ? ds0 : 0.f) + (up[2 * q2 + 1] ? ds1 : 0.f);
+                }
+              }
+              a0 -= aup;
+              a1 += aup;
             } else if (kind == 1) {
 #pragma unroll
-              for (int e4 = 0; e4 < 4; ++e4) {
-                const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 16 * hh + 4 * e4]);
+              for (int e4 = 0; e4 < 2; ++e4) {
+                const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 8 * c8 + 4 * e4]);
                 const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
                 float xs[4];
                 int bk[4];
@@ -647,56 +695,50 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
                 }
               }
             } else {
-              // band words of this lane's kv row for the half's 16 q rows (kv rows beyond
-              // the sequence read none and are masked)
-              uint32_t w[16];
+              if (c8 == 0) cur_tb = w[0] & 0x7F;
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                uint4 v4;
-                if (jlive) v4 = __ldg(bp + 4 * hh + c);
-                else v4.x = v4.y = v4.z = v4.w = __float_as_uint(kMaskedBias) & 0xFFFF0000u;
-                w[4 * c] = v4.x; w[4 * c + 1] = v4.y; w[4 * c + 2] = v4.z; w[4 * c + 3] = v4.w;
-              }
-              if (hh == 0) cur_tb = w[0] & 0x7F;
-#pragma unroll
-              for (int e = 0; e < 16; e += 2) {
+              for (int e = 0; e < 8; e += 2) {
                 float ds0, ds1;
-                p_ds2(__uint_as_float(sr[e]) + __uint_as_float(w[e] & 0xFFFF0000u),
-                      __uint_as_float(sr[e + 1]) + __uint_as_float(w[e + 1] & 0xFFFF0000u), __uint_as_float(dr[e]),
-                      __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
+                float x0, x1;
+                add2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), __uint_as_float(w[e] & 0xFFFF0000u),
+                     __uint_as_float(w[e + 1] & 0xFFFF0000u), x0, x1);
+                p_ds2(x0, x1, __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
                 dk[e >> 1] = pack_bf16x2(ds0, ds1);
                 const float dsv[2] = {ds0, ds1};
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                   // time bucket: runs along the row
                   const int tb = w[e + u] & 0x7F;
-                  if (tb != cur_tb) {
-                    if (at != 0.f) red_add(&gtime[cur_tb], at);
-                    cur_tb = tb;
-                    at = 0.f;
-                  }
-                  at += dsv[u];
+                  const bool change = tb != cur_tb;
+                  if (change) red_add(&gtime[cur_tb], at);
+                  cur_tb = tb;
+                  at = change ? dsv[u] : at + dsv[u];
                   // position bucket D + col - lane: the running sum of the diagonal col - lane
                   // moves one lane down per column, and lane 31's is complete
                   dg += dsv[u];
-                  const int col = 16 * hh + e + u;
-                  if (lane == 31 && (D > 0 || col == 31)) {
-                    const int b = min(D + col - 31, kNumBuckets - 1);
-                    red_add(&gpos[b], dg);
-                  }
+                  const int col = 8 * c8 + e + u;
+                  if (lane == 31 && (D > 0 || col == 31)) red_add(&gpos[min(D + col - 31, kNumBuckets - 1)], dg);
                   dg = lane == 31 ? 0.f : dg;
                   dg = __shfl_sync(0xffffffffu, dg, (lane + 31) & 31);
                 }
               }
             }
-            if (hh == 0) {
-              // deferred readouts (their MMAs ran while this half was computed), then the
-              // previous tile's P^T and dS^T must have been consumed
+            if (c8 == 1) {
+              // deferred readouts (their MMAs ran while these chunks were computed), then
+              // the previous tile's P^T and dS^T must have been consumed
               if (!readouts()) goto fail;
             }
-            tmem_st_32x32b_x8(tmem + kColP + lane_off + 16 * seg + 8 * hh, pk);
-            st_shared_v4(ds_atom + (((ds_ch + 2 * hh) ^ (jl & 7)) << 4), dk[0], dk[1], dk[2], dk[3]);
-            st_shared_v4(ds_atom + (((ds_ch + 2 * hh + 1) ^ (jl & 7)) << 4), dk[4], dk[5], dk[6], dk[7]);
+            if (c8 >= 1) {
+              if (c8 == 1) {
+                tmem_st_32x32b_x4(tmem + kColP + lane_off + 16 * seg, pk_prev);
+                st_shared_v4(ds_atom + (((ds_ch) ^ (jl & 7)) << 4), dk_prev[0], dk_prev[1], dk_prev[2], dk_prev[3]);
+              }
+              tmem_st_32x32b_x4(tmem + kColP + lane_off + 16 * seg + 4 * c8, pk);
+              st_shared_v4(ds_atom + (((ds_ch + c8) ^ (jl & 7)) << 4), dk[0], dk[1], dk[2], dk[3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) { pk_prev[e] = pk[e]; dk_prev[e] = dk[e]; }
+            }
           }
         } else {
           // ---- per element (candidates, per-head bias tables, 64-bit time offsets): the

@@ -731,6 +731,27 @@ int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
   Carver c(workspace);
   LayerFwdWs ws = carve_layer_fwd(c, desc, jb->batch, jb->total_tokens, true);
   HSTU_CUDA(cudaMemsetAsync(ws.attn.status, 0, kStatusBytes, st));
+  if ((desc->attn.flags & HSTU_FLAG_SHORT_SEQUENCES) && !saved &&
+      fused_short_supported(dm, desc->attn.num_heads, desc->attn.dqk, desc->attn.dtype, io) &&
+      desc->attn.dv == desc->attn.dqk) {
+    // the whole layer in one kernel, one CTA per sequence of at most 128 tokens
+    FusedShortArgs a;
+    memset(&a, 0, sizeof(a));
+    a.offs = jb->seq_offsets; a.num_targets = jb->num_targets; a.ts = jb->timestamps;
+    a.x = x; a.y = y;
+    a.w1 = w->w1; a.b1 = w->b1; a.ln1_g = w->ln1_gamma; a.ln1_b = w->ln1_beta;
+    a.ln2_g = w->ln2_gamma; a.ln2_b = w->ln2_beta; a.w2 = w->w2; a.b2 = w->b2;
+    a.pos_bias = w->pos_bias; a.time_bias = w->time_bias; a.rab_head_stride = desc->attn.rab_head_stride;
+    a.B = jb->batch; a.T = jb->total_tokens; a.d = dm; a.H = desc->attn.num_heads;
+    a.eps = desc->ln_eps; a.time_div = desc->attn.time_div; a.thr = thresholds_for(desc->attn.time_div);
+    a.cursor = ws.attn.count + 2;
+    a.status = ws.attn.status;
+    a.timeout_ns = kDefaultTimeoutNs;
+    HSTU_CUDA(cudaMemsetAsync(a.cursor, 0, sizeof(int32_t), st));
+    TraceScope tr("fused_short_layer", st);
+    HSTU_CUDA(launch_fused_short(a, st));
+    return HSTU_OK;
+  }
   return run_layer_fwd(desc, w, jb, x, y, saved, ws, st);
 }
 

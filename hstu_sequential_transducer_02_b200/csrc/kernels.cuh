@@ -137,6 +137,23 @@ cudaError_t launch_debug_buckets(const int32_t* offs, const int32_t* num_targets
                                  cudaStream_t st);
 cudaError_t launch_timeout_probe(long long timeout_ns, int32_t* status, cudaStream_t st);
 
+// ---------------------------------------------------------------- fused short-sequence layer
+struct FusedShortArgs {
+  const int32_t* offs; const int32_t* num_targets; const int64_t* ts;
+  const void* x; void* y;
+  const void* w1; const float* b1; const float* ln1_g; const float* ln1_b;
+  const float* ln2_g; const float* ln2_b; const void* w2; const float* b2;
+  const float* pos_bias; const float* time_bias; int rab_head_stride;
+  int B, T, d, H;
+  float eps; double time_div; Thresholds thr;
+  int32_t* cursor;             // zeroed before the launch
+  int32_t* status;
+  long long timeout_ns;
+};
+bool fused_short_supported(int d_model, int num_heads, int head_dim, int dtype, int io_dtype);
+int fused_short_max_len();
+cudaError_t launch_fused_short(const FusedShortArgs& a, cudaStream_t st);
+
 // ---------------------------------------------------------------- GEMM
 // C[m, n] = sum_k A(m, k) B(n, k) with element strides; fp32 accumulation.
 enum GemmEpilogue {

@@ -75,6 +75,16 @@ extern "C" {
 /* descriptor flags */
 #define HSTU_FLAG_FORCE_SIMT 1   /* diagnostics: run the CUDA-core attention/GEMM kernels
                                     instead of the tcgen05 ones (bf16 only) */
+#define HSTU_FLAG_SHORT_SEQUENCES 2
+/* hstu_layer_fwd: the caller states that every sequence has at most 128 tokens,
+ * and the layer runs as one kernel (one CTA per sequence, every intermediate on
+ * the chip: LayerNorm, f1, the attention of all heads, LayerNorm(A V) * U, f2 and
+ * the residual; "Actions Speak Louder than Words" summary, 1.3: kernel fusion).
+ * It applies to bf16 weights and activations (io_dtype bf16), head dimension 64,
+ * d_model and num_heads * 64 at most 256 and multiples of 64, and inference
+ * (saved == NULL); otherwise the flag is ignored.  A sequence longer than 128
+ * tokens (or outside the buffers) is not computed and sets HSTU_ERR_BAD_OFFSETS
+ * in the workspace status word. */
 /* seq_offsets and num_targets are always checked on the device by the
  * scheduler kernel that precedes every attention launch; a violation writes
  * HSTU_ERR_BAD_OFFSETS to the workspace status word and schedules no work. */

@@ -90,8 +90,8 @@ def attention_forward(q, k, v, offs, ts, pos_bias, time_bias, silu_p="bf16pair",
         nt = 0 if num_targets is None else int(num_targets[s])
         N = max(n - nt, 1)
         mask = O.attention_mask(n, nt)
-        rab = _rab(ts[a:b], n, nt, pos_bias, time_bias, band and nt == 0)
         for h in range(H):
+            rab = _rab(ts[a:b], n, nt, O._head_table(pos_bias, h), O._head_table(time_bias, h), band and nt == 0)
             S = q[a:b, h] @ k[a:b, h].T + rab
             P = np.where(mask, _p_forward(S, silu_p), 0.0)
             out[a:b, h] = _r('attn_out', (P @ v[a:b, h]) / N)

@@ -553,7 +553,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         // kind: 0 masked, 1 far, 2 band, 3 per element
         int kind = 3;
         if (D + 31 < 0) kind = 0;                                           // every i < j
-        else if (narrow && i0 + 31 < si.hist && D >= 158) kind = 1;          // i - j >= 127 everywhere
+        else if (narrow && D >= 158 && (i0 + 31 < si.hist || (si.hist == si.n && i0 < si.n)))
+          kind = 1;   // i - j >= 127 everywhere (q rows beyond a sequence without targets are masked)
         else if (p.band != nullptr && D >= 0 && D < kBwdBandCols && (i0 + 31 < si.hist || si.hist == si.n))
           kind = 2;
         // far: time buckets of this lane's row over the segment's q columns, from the
@@ -594,6 +595,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         int cur_tb = -1;
         const uint4* bp = reinterpret_cast<const uint4*>(p.band + (int64_t)(si.start + (jlive ? j : 0)) * kBwdBandCols +
                                                          (D > 0 ? D : 0));
+        // band words of the segment's first chunk, in flight while the scores are awaited
+        // (kv rows beyond the sequence read none: masked)
+        uint4 wn0 = make_uint4(0u, 0u, 0u, 0u), wn1 = wn0;
+        const uint32_t kMaskedWord = __float_as_uint(kMaskedBias) & 0xFFFF0000u;
+        if (kind == 2) {
+          if (jlive) {
+            wn0 = __ldg(bp);
+            wn1 = __ldg(bp + 1);
+          } else {
+            wn0 = wn1 = make_uint4(kMaskedWord, kMaskedWord, kMaskedWord, kMaskedWord);
+          }
+        }
         if (!mbar_wait(&bars->sp_full, g & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
         uint32_t pk_prev[4], dk_prev[4];   // the first chunk's words, held until the readouts
@@ -606,21 +619,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
             uint32_t sr[8], dr[8];
             tmem_ld_32x32b_x8(tmem + kColS + lane_off + 32 * seg + 8 * c8, sr);
             tmem_ld_32x32b_x8(tmem + kColDP + lane_off + 32 * seg + 8 * c8, dr);
-            uint32_t w[8];    // band words of the chunk (kv rows beyond the sequence read none: masked)
-            if (kind == 2) {
-#pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                uint4 v4;
-                if (jlive) v4 = __ldg(bp + 2 * c8 + c);
-                else v4.x = v4.y = v4.z = v4.w = __float_as_uint(kMaskedBias) & 0xFFFF0000u;
-                w[4 * c] = v4.x; w[4 * c + 1] = v4.y; w[4 * c + 2] = v4.z; w[4 * c + 3] = v4.w;
-              }
+            // band words of this chunk (loaded one chunk ahead), and the next chunk's in flight
+            const uint32_t w[8] = {wn0.x, wn0.y, wn0.z, wn0.w, wn1.x, wn1.y, wn1.z, wn1.w};
+            if (kind == 2 && c8 < 3 && jlive) {
+              wn0 = __ldg(bp + 2 * c8 + 2);
+              wn1 = __ldg(bp + 2 * c8 + 3);
             }
             tmem_ld_wait();
             if (c8 == 3) {
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&bars->sp_free);
+            }
+            if (kind == 1 && i0 + 8 * c8 + 7 >= si.n) {
+              // the sequence ends inside this chunk: q rows beyond it are masked
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                if (i0 + 8 * c8 + e >= si.n) sr[e] = __float_as_uint(kMaskedBias);
             }
             uint32_t pk[4];   // P^T words (bf16 pairs) of the chunk's 8 q columns
             uint32_t dk[4];   // dS^T words

@@ -232,8 +232,7 @@ int hstu_attn_fwd(const hstu_attn_desc* desc, const hstu_jagged* jb,
  *   - The first call on a device looks up the array's device address on that
  *     device (current device at the time of the call), and so does the first
  *     call from each further context of the device (a non-primary context, or
- *     the primary context recreated after cudaDeviceReset); make those first
- *     calls before capturing any stream into a graph.
+ *     the primary context recreated after cudaDeviceReset).
  *   - All calls share the one array and each call overwrites it.  Calls that
  *     may run at the same time on the GPU (different streams without ordering
  *     between them) race on it and give undefined results: order them.

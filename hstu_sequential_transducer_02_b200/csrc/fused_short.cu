@@ -7,15 +7,21 @@
 // ("Actions Speak Louder than Words" summary, 1.3 and 2.2: the layer's linear
 // maps are grouped and its element-wise work fused; for short histories the
 // launches and the round trips through memory between the stages cost more than
-// the arithmetic.)  One CTA takes one sequence at a time from a shared cursor and
-// keeps every intermediate on the chip:
+// the arithmetic.)  The batch is cut into work units of at most 128 consecutive
+// token rows that hold whole sequences (the sequences inside each 128-row window,
+// and each sequence crossing a window boundary on its own), so short sequences
+// share one tile: rows of different sequences never attend to each other, which
+// the bias matrix masks.  One CTA takes one unit at a time from a shared cursor
+// and keeps every intermediate on the chip:
 //   shared memory  x-hat (later the gate LN2(A V) * U) as the A operand of f1 and
 //                  f2; Q, K, V of the current head; the relative-bias matrix of
-//                  the sequence (bf16, -1e30 where masked); a ring of weight slices
+//                  the unit (bf16, -1e30 where masked, across sequences too); each
+//                  row's sequence (first row, length, N); a ring of weight slices
 //   TMEM           the f1 accumulator of one head (U|V|Q|K, 256 columns), reused
 //                  by S, P and the head's A V; U and A V of all heads as bf16;
 //                  finally the f2 accumulator
-//   warp 0         TMA: W1 slices (the 4 x 64 rows of one head's U, V, Q, K) and
+//   warp 0         finds the next unit (a warp-wide search of the offsets), then
+//                  TMA: W1 slices (the 4 x 64 rows of one head's U, V, Q, K) and
 //                  W2 slices, 64 input columns at a time
 //   warp 1         tcgen05.mma (whole warp, one elected lane)
 //   warps 2-17     LayerNorms, bias matrix, f1 epilogue (bias, SiLU, split),
@@ -23,7 +29,9 @@
 //                  four warps per TMEM lane quarter, each on a quarter of the columns
 // Head dimension 64; d_model and H * 64 at most 256, multiples of 64; bf16.
 // Every device-side wait is bounded (HSTU_ERR_TIMEOUT); a sequence longer than
-// 128 tokens is skipped and reported as HSTU_ERR_BAD_OFFSETS.
+// 128 tokens is skipped and reported as HSTU_ERR_BAD_OFFSETS, and so are offsets
+// that are not non-decreasing from 0 to at most T (nothing outside [0, T) is read
+// or written either way).
 #include <mutex>
 
 #include "common.cuh"
@@ -62,7 +70,9 @@ struct Layout {
   static constexpr int kRing = kV + kAtom;
   static constexpr int kBias = kRing + kRingStages * kSlice;  // [128 x 128] bf16, 16-byte chunks swizzled
   static constexpr int kTs = kBias + R * R * 2;               // rel offsets int32[128] | abs int64[128]
-  static constexpr int kThr = kTs + R * 4 + R * 8;
+  static constexpr int kRows = kTs + R * 4 + R * 8;           // per row: sequence start in the pack, n, N
+  static constexpr int kPackOffs = kRows + 3 * R * 4;         // the pack's sequence offsets (up to 129)
+  static constexpr int kThr = kPackOffs + (R + 4) * 4;
   static constexpr int kThr32 = kThr + kNumBuckets * 8;
   static constexpr int kPosB = kThr32 + (kNumBuckets + 4) * 4;
   static constexpr int kTimeB = kPosB + kNumBuckets * 4;
@@ -123,11 +133,80 @@ __device__ __forceinline__ float silu_tanh(float x) {
   return fmaf(h, tanh_approx(h), h);
 }
 
-// a sequence this kernel computes: 1 to 128 rows inside the [T, d] buffers (an
-// empty sequence has nothing to compute; a longer or misplaced one is reported)
-__device__ __forceinline__ bool seq_ok(const FusedParams& p, int s) {
-  const int a = p.offs[s], b = p.offs[s + 1];
-  return a >= 0 && b > a && b - a <= R && b <= p.T;
+// first index in [0, cnt) with a[index] >= v (cnt if none), a non-decreasing; the
+// whole warp searches, 32 probes at a time
+__device__ __forceinline__ int warp_lower_bound(const int32_t* a, int cnt, int v, int lane) {
+  int lo = 0, hi = cnt;   // the answer lies in [lo, hi]
+  while (hi - lo > 31) {
+    const int step = (hi - lo + 30) / 31;         // lane 31 probes at or beyond hi: some probe answers yes
+    const int idx = lo + lane * step;
+    const bool ge = idx < hi ? a[idx] >= v : true;
+    const int f = __ffs(__ballot_sync(0xffffffffu, ge)) - 1;   // first probe at or above v
+    const int idx_f = min(lo + f * step, hi);
+    lo = f == 0 ? lo : lo + (f - 1) * step + 1;
+    hi = idx_f;
+  }
+  const int idx = lo + lane;                      // hi - lo <= 31: lane 31 is at or beyond hi
+  const bool ge = idx < hi ? a[idx] >= v : true;
+  return lo + __ffs(__ballot_sync(0xffffffffu, ge)) - 1;
+}
+
+// A work unit: up to 128 consecutive token rows holding whole sequences.  With
+// W = ceil(T_used / 128) windows of 128 rows, unit u < W takes the sequences that
+// lie entirely inside window u, and unit W - 1 + b takes the sequence that crosses
+// the boundary between windows b - 1 and b (a sequence of at most 128 tokens
+// crosses at most one), so every sequence belongs to exactly one unit and no
+// unit needs more than one 128-row tile.
+struct Pack {
+  int id;      // -1: no more units
+  int row0;    // first token row
+  int nrows;   // rows (0: nothing to compute)
+  int s0;      // first sequence
+  int count;   // sequences s0 .. s0 + count - 1
+  int bad;     // a crossing sequence longer than 128 tokens, or inconsistent offsets
+};
+
+__device__ __forceinline__ Pack decode_pack(const FusedParams& p, int id, int lane) {
+  Pack pk;
+  pk.id = id; pk.row0 = 0; pk.nrows = 0; pk.s0 = 0; pk.count = 0; pk.bad = 0;
+  const int t_used = p.offs[p.B];
+  if (p.offs[0] != 0 || t_used < 0 || t_used > p.T) {
+    pk.bad = id == 0 ? 1 : 0;   // reported once
+    pk.id = id == 0 ? 0 : -1;
+    return pk;
+  }
+  const int W = (t_used + R - 1) / R;
+  if (id < 0 || id >= 2 * W - 1) { pk.id = -1; return pk; }
+  if (id < W) {
+    const int lo = id * R, hi = min(lo + R, t_used);
+    const int sa = warp_lower_bound(p.offs, p.B + 1, lo, lane);          // first sequence starting at or after lo
+    const int sb = warp_lower_bound(p.offs, p.B + 1, hi + 1, lane) - 1;  // last offset at or below hi
+    if (sb > sa && sb <= p.B) {
+      pk.row0 = p.offs[sa];
+      pk.nrows = p.offs[sb] - pk.row0;
+      pk.s0 = sa;
+      pk.count = sb - sa;
+    }
+  } else {
+    const int b = (id - W + 1) * R;
+    const int s = warp_lower_bound(p.offs, p.B + 1, b, lane) - 1;      // last sequence starting before b
+    if (s >= 0 && s < p.B && p.offs[s + 1] > b) {
+      const int len = p.offs[s + 1] - p.offs[s];
+      if (len <= R) {
+        pk.row0 = p.offs[s];
+        pk.nrows = len;
+        pk.s0 = s;
+        pk.count = 1;
+      } else {
+        pk.bad = 1;   // not this kernel's: reported
+      }
+    }
+  }
+  if (pk.nrows < 0 || pk.nrows > R || pk.row0 < 0 || pk.row0 + pk.nrows > p.T) {   // unsorted offsets
+    pk.nrows = 0;
+    pk.bad = 1;
+  }
+  return pk;
 }
 
 // byte offset of element (row r, column c) of a [128 x 64k] bf16 tile of 64-column
@@ -146,6 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
   volatile int* items = reinterpret_cast<volatile int*>(smem + L::kItems);
   int32_t* rel_s = reinterpret_cast<int32_t*>(smem + L::kTs);
   int64_t* abs_s = reinterpret_cast<int64_t*>(smem + L::kTs + R * 4);
+  int32_t* row_sb = reinterpret_cast<int32_t*>(smem + L::kRows);          // first row of the row's sequence
+  int32_t* row_n = row_sb + R;                                             // its length
+  int32_t* row_hist = row_n + R;                                           // its N
+  int32_t* pack_offs = reinterpret_cast<int32_t*>(smem + L::kPackOffs);   // the unit's sequence offsets
   int64_t* thr = reinterpret_cast<int64_t*>(smem + L::kThr);
   int32_t* thr32 = reinterpret_cast<int32_t*>(smem + L::kThr32);
   float* pos_b = reinterpret_cast<float*>(smem + L::kPosB);
@@ -203,22 +286,33 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ================================================================ sequences and weight slices
-    if (lane == 0) {
-      int r = 0;   // ring slot counter
-      for (int k = 0;; ++k) {
-        const int slot = k & 1;
-        if (!mbar_wait(&bars->it_empty[slot], ((k >> 1) & 1) ^ 1, tmo, abort_flag)) goto fail;
-        int s = *abort_flag ? -1 : atomicAdd(p.cursor, 1);
-        if (s >= p.B) s = -1;
-        items[8 * slot] = s;
+    // ================================================================ work units and weight slices
+    int r = 0;   // ring slot counter
+    for (int k = 0;; ++k) {
+      const int slot = k & 1;
+      if (!warp_wait(&bars->it_empty[slot], ((k >> 1) & 1) ^ 1, tmo, abort_flag)) goto fail;
+      int id = 0;
+      if (lane == 0) id = *abort_flag ? -1 : atomicAdd(p.cursor, 1);
+      id = __shfl_sync(0xffffffffu, id, 0);
+      const Pack pk = decode_pack(p, id, lane);
+      if (lane == 0) {
+        items[8 * slot] = pk.id;
+        items[8 * slot + 1] = pk.row0;
+        items[8 * slot + 2] = pk.nrows;
+        items[8 * slot + 3] = pk.s0;
+        items[8 * slot + 4] = pk.count;
+        items[8 * slot + 5] = pk.bad;
         mbar_arrive(&bars->it_full[slot]);
-        if (s < 0) break;
-        if (!seq_ok(p, s)) continue;   // nothing to do, or not this kernel's (reported by the epilogue)
-        for (int h = 0; h < H; ++h) {
+      }
+      __syncwarp();
+      if (pk.id < 0) break;
+      if (pk.nrows == 0) continue;   // nothing to compute (a bad unit is reported by the epilogue)
+      bool ok = true;
+      if (lane == 0) {
+        for (int h = 0; h < H && ok; ++h) {
           for (int ks = 0; ks < k_d; ++ks, ++r) {
             const int st = r % kRingStages;
-            if (!mbar_wait(&bars->ring_empty[st], ((r / kRingStages) & 1) ^ 1, tmo, abort_flag)) goto fail;
+            if (!mbar_wait(&bars->ring_empty[st], ((r / kRingStages) & 1) ^ 1, tmo, abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars->ring_full[st], kSlice);
             // rows 64c .. 64c + 63 of the slice: W1 rows of block c (U, V, Q, K) for head h
             for (int c = 0; c < 4; ++c)
@@ -226,15 +320,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
                           c * hv + h * DH);
           }
         }
-        for (int ks = 0; ks < k_hv; ++ks, ++r) {
+        for (int ks = 0; ks < k_hv && ok; ++ks, ++r) {
           const int st = r % kRingStages;
-          if (!mbar_wait(&bars->ring_empty[st], ((r / kRingStages) & 1) ^ 1, tmo, abort_flag)) goto fail;
+          if (!mbar_wait(&bars->ring_empty[st], ((r / kRingStages) & 1) ^ 1, tmo, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars->ring_full[st], k_d * 64 * 128);
           for (int c = 0; c < k_d; ++c)
             tma_load_2d(smem + L::kRing + st * kSlice + c * 64 * 128, &prm.map_w2, &bars->ring_full[st], ks * 64,
                         c * 64);
         }
       }
+      if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) goto fail;
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -251,11 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
     for (int k = 0;; ++k) {
       const int slot = k & 1;
       if (!warp_wait(&bars->it_full[slot], (k >> 1) & 1, tmo, abort_flag)) goto fail;
-      const int s = items[8 * slot];
+      const int unit = items[8 * slot];
+      const int unit_rows = items[8 * slot + 2];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->it_empty[slot]);
-      if (s < 0) break;
-      if (!seq_ok(p, s)) continue;
+      if (unit < 0) break;
+      if (unit_rows == 0) continue;
       if (!warp_wait(&bars->xhat_ready, k & 1, tmo, abort_flag)) goto fail;
       for (int h = 0; h < H; ++h, ++g) {
         // f1 of head h: [128 x d] x [d x 256] into the accumulator (after the previous
@@ -327,21 +423,44 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
     for (int k = 0;; ++k) {
       const int slot = k & 1;
       if (!warp_wait(&bars->it_full[slot], (k >> 1) & 1, tmo, abort_flag)) goto fail;
-      const int s = items[8 * slot];
+      const int unit = items[8 * slot];
+      const int start = items[8 * slot + 1];    // first token row of the unit
+      const int n = items[8 * slot + 2];        // its rows
+      const int s0 = items[8 * slot + 3];
+      const int count = items[8 * slot + 4];
+      const int bad = items[8 * slot + 5];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->it_empty[slot]);
-      if (s < 0) break;
-      const int start = p.offs[s];
-      const int n = p.offs[s + 1] - start;
-      if (!seq_ok(p, s)) {
-        if (etid == 0 && n != 0) set_status(p.status, HSTU_ERR_BAD_OFFSETS);
-        continue;
+      if (unit < 0) break;
+      if (bad && etid == 0) set_status(p.status, HSTU_ERR_BAD_OFFSETS);
+      if (n == 0) continue;
+      // ---- every row's sequence: its first row in the unit, its length and N (rows
+      // beyond the unit: none).  The unit's sequence offsets go to shared memory first
+      // when there are at most 128 of them (more only with empty sequences).
+      if (count <= R)
+        for (int t = etid; t <= count; t += 32 * kEpiWarps) pack_offs[t] = p.offs[s0 + t] - start;
+      if (!epi_barrier()) goto fail;
+      if (etid < R) {
+        int sb = etid, nn = 0, hh = 0;
+        if (etid < n) {
+          int lo = 0, hi = count - 1;   // the last sequence of the unit starting at or before this row
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            const int st_mid = count <= R ? pack_offs[mid] : p.offs[s0 + mid] - start;
+            if (st_mid <= etid) lo = mid; else hi = mid - 1;
+          }
+          const int sq = s0 + lo;
+          sb = p.offs[sq] - start;
+          nn = p.offs[sq + 1] - p.offs[sq];
+          int nt = p.num_targets ? p.num_targets[sq] : 0;
+          nt = nt < 0 ? 0 : (nt > nn ? nn : nt);
+          hh = nn - nt;
+        }
+        row_sb[etid] = sb;
+        row_n[etid] = nn;
+        row_hist[etid] = hh;
       }
-      int nt = p.num_targets ? p.num_targets[s] : 0;
-      nt = nt < 0 ? 0 : (nt > n ? n : nt);
-      const int hist = n - nt;
-      const float inv_n = 1.0f / (float)(hist > 1 ? hist : 1);
-      // ---- timestamps of the sequence: offsets from the first, clamped to +-(2^30 - 1)
+      // ---- timestamps of the unit: offsets from its first, clamped to +-(2^30 - 1)
       // (a pair with a clamped offset takes the 64-bit values)
       const int64_t t_first = p.ts[start];
       constexpr int32_t kLim = (1 << 30) - 1;
@@ -401,13 +520,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->xhat_ready);
-      if (!epi_barrier()) goto fail;   // timestamps in shared memory for everyone
+      if (!epi_barrier()) goto fail;   // timestamps and row facts in shared memory for everyone
+      const float inv_n = 1.0f / (float)(row_hist[row] > 1 ? row_hist[row] : 1);   // this lane's row
       // ---- relative-bias matrix of the sequence: bias(i, j) as bf16, -1e30 where the
       // pair is not attended.  Thread t: row t / 4, columns [32 (t % 4), +32).
       auto build_bias = [&](int head) {
         for (int e = etid; e < R * 4; e += 32 * kEpiWarps) {
           const int i = e >> 2, j0 = (e & 3) * 32;
-          const int posi = token_pos(i, hist);
+          const int sbi = row_sb[i], ni = row_n[i], hi_ = row_hist[i];   // row i's sequence
+          const int posi = token_pos(i - sbi, hi_);
 #pragma unroll 1
           for (int c8 = 0; c8 < 4; ++c8) {
             uint32_t pk[4];
@@ -418,8 +539,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_short_kernel(const __grid_c
               for (int q = 0; q < 2; ++q) {
                 const int j = j0 + 8 * c8 + 2 * u + q;
                 float b = kMasked;
-                if (i < n && j < n && attended(i, j, n, hist)) {
-                  const int pb = pos_bucket(posi, token_pos(j, hist));
+                const int lj = j - sbi;   // column j inside row i's sequence (same sequence iff 0 <= lj < ni)
+                if (i < n && lj >= 0 && lj < ni && attended(i - sbi, lj, ni, hi_)) {
+                  const int pb = pos_bucket(posi, token_pos(lj, hi_));
                   const int32_t ri = rel_s[i], rj = rel_s[j];
                   const bool clamped = ri == kLim || ri == -kLim || rj == kLim || rj == -kLim;
                   const int tb = clamped ? time_bucket_exact(abs_diff_i64(abs_s[i], abs_s[j]), thr)
@@ -720,7 +842,10 @@ cudaError_t launch_fused_short(const FusedShortArgs& a, cudaStream_t st) {
   const int smem = Layout::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(fused_short_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int grid = a.B < num_sms_fused() ? (a.B > 0 ? a.B : 1) : num_sms_fused();
+  // units: ceil(T / 128) windows and the boundaries between them (an upper bound:
+  // the kernel reads the used token count from the offsets)
+  const int64_t units = 2 * (((int64_t)a.T + R - 1) / R) - 1;
+  const int grid = units < num_sms_fused() ? (units > 0 ? (int)units : 1) : num_sms_fused();
   fused_short_kernel<<<grid, kThreads, smem, st>>>(fp);
   return cudaGetLastError();
 }

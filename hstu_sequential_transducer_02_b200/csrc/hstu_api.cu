@@ -734,7 +734,7 @@ int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
   if ((desc->attn.flags & HSTU_FLAG_SHORT_SEQUENCES) && !saved &&
       fused_short_supported(dm, desc->attn.num_heads, desc->attn.dqk, desc->attn.dtype, io) &&
       desc->attn.dv == desc->attn.dqk) {
-    // the whole layer in one kernel, one CTA per sequence of at most 128 tokens
+    // the whole layer in one kernel, over units of at most 128 token rows holding whole sequences
     FusedShortArgs a;
     memset(&a, 0, sizeof(a));
     a.offs = jb->seq_offsets; a.num_targets = jb->num_targets; a.ts = jb->timestamps;

@@ -77,9 +77,11 @@ extern "C" {
                                     instead of the tcgen05 ones (bf16 only) */
 #define HSTU_FLAG_SHORT_SEQUENCES 2
 /* hstu_layer_fwd: the caller states that every sequence has at most 128 tokens,
- * and the layer runs as one kernel (one CTA per sequence, every intermediate on
- * the chip: LayerNorm, f1, the attention of all heads, LayerNorm(A V) * U, f2 and
- * the residual; "Actions Speak Louder than Words" summary, 1.3: kernel fusion).
+ * and the layer runs as one kernel (every intermediate on the chip: LayerNorm,
+ * f1, the attention of all heads, LayerNorm(A V) * U, f2 and the residual;
+ * "Actions Speak Louder than Words" summary, 1.3: kernel fusion).  Its work units
+ * are runs of at most 128 consecutive token rows holding whole sequences, so
+ * several short sequences share one tile.
  * It applies to bf16 weights and activations (io_dtype bf16), head dimension 64,
  * d_model and num_heads * 64 at most 256 and multiples of 64, and inference
  * (saved == NULL); otherwise the flag is ignored.  A sequence longer than 128

@@ -1,7 +1,7 @@
 """GPU parity of the fused short-sequence layer (hstu_layer_fwd with
-HSTU_FLAG_SHORT_SEQUENCES: the whole layer in one kernel, one CTA per sequence of
-at most 128 tokens) against the fp64 oracle, on the short-sequence workload's
-recipe with its lengths cut to at most 128."""
+HSTU_FLAG_SHORT_SEQUENCES: the whole layer in one kernel over work units of at
+most 128 token rows holding whole sequences) against the fp64 oracle, on the
+short-sequence workload's recipe with its lengths cut to at most 128."""
 import numpy as np
 import pytest
 import torch
@@ -118,3 +118,22 @@ def test_fused_short_layer_reports_long_sequence():
     for s_ in (0, 2):
         a, z = offs[s_], offs[s_ + 1]
         assert_close(got[a:z], ref[a:z], "bf16", f"sequence {s_}")
+
+
+def test_fused_short_layer_packs_many_sequences():
+    """Units holding many sequences: 300 sequences of 1 .. 12 tokens, a run of 200
+    empty sequences inside one 128-row window (more sequence offsets than rows),
+    sequences of exactly 128 tokens starting on and off a window boundary, and
+    sequences crossing window boundaries; targets on some of them."""
+    rng = np.random.default_rng(7)
+    lens = list(rng.integers(1, 13, size=150))
+    lens += [0] * 200 + [128, 5, 128, 127, 1, 90, 77]
+    lens += list(rng.integers(1, 13, size=150)) + [0, 64, 128]
+    wl = W.make_workload(1, lengths=lens, random_affine=True)
+    wl.layers = wl.layers[:1]
+    lens_a = np.asarray(lens)
+    nt = np.where(np.arange(len(lens)) % 7 == 3, np.minimum(2, lens_a), 0).astype(np.int32)
+    got, trace, status = _run(wl, True, nt)
+    assert trace.get("fused_short_layer", {}).get("count") == 1
+    assert status == [0]
+    assert_close(got, _ref(wl, nt), "bf16", "fused short layer, many sequences per unit")

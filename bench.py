@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the M-FALCON and training-step measurements")
     ap.add_argument("--profile-attn-bwd", action="store_true",
                     help="for profilers: run the training workload's attention backward (1 + 3 launches) and exit")
+    ap.add_argument("--profile-short", action="store_true",
+                    help="for profilers: run the fused short-sequence layer on 512 sequences of at most 128 "
+                         "tokens (two layers, 3 + 2 forwards) and exit")
     return ap.parse_args()
 
 
@@ -297,6 +300,20 @@ def _trace_attention(trace, name, flops):
             "tflops": flops / a["count"] / (ms / 1e3) / 1e12 if flops else None}  # flops: all traced launches
 
 
+def _traced(hb, fn, steps):
+    """Per-kernel device times of `steps` calls of fn, with the library's event
+    tracing on (a pass of its own, outside any timed region)."""
+    import torch
+    torch.cuda.synchronize()
+    hb.trace_enable(True)
+    for _ in range(steps):
+        fn()
+    torch.cuda.synchronize()
+    trace = hb.trace_read()
+    hb.trace_enable(False)
+    return trace
+
+
 def _top_kernels(trace, steps, k=6):
     """The k kernels with the most traced device time: share and ms per step."""
     tot = sum(v["ms"] for v in trace.values()) or 1e-9
@@ -323,16 +340,16 @@ def measure_mfalcon(hb, steps: int):
     for _ in range(2):
         hb.mfalcon_rank([layer], *args, bm, m_max, out=out)
     torch.cuda.synchronize()
-    hb.trace_enable(True)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(steps):
         hb.mfalcon_rank([layer], *args, bm, m_max, out=out)
     t1.record()
     torch.cuda.synchronize()
-    trace = hb.trace_read()
-    hb.trace_enable(False)
     ms = t0.elapsed_time(t1) / steps
+    # per-kernel device times from a separate traced pass (events around every launch
+    # would otherwise be inside the timed calls)
+    trace = _traced(hb, lambda: hb.mfalcon_rank([layer], *args, bm, m_max, out=out), steps)
     U = len(wl.seq_offsets) - 1
     n = int(np.diff(wl.seq_offsets)[0])
     cands = int(e["cand_offsets"][-1])
@@ -441,16 +458,14 @@ def measure_training(hb, steps: int):
     offs = step()
     torch.cuda.synchronize()
     T2 = int(offs[-1].item())
-    hb.trace_enable(True)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record()
     for _ in range(steps):
         step()
     t1.record()
     torch.cuda.synchronize()
-    trace = hb.trace_read()
-    hb.trace_enable(False)
     ms = t0.elapsed_time(t1) / steps
+    trace = _traced(hb, step, steps)   # per-kernel device times, from a separate pass
     return {"workload": f"training step: 8 layers, B=64, power-law n in [64,4096], SL to 1024 (p=0.8) -> "
                         f"T={T2} tokens, d_model={sp.d_model}, {sp.num_heads} heads x {sp.head_dim}, "
                         "fp32 residual stream, forward + backward",
@@ -501,6 +516,11 @@ def main():
         return
     if args.profile_attn_bwd:
         profile_attn_bwd()
+        return
+    if args.profile_short:
+        from hstu_sequential_transducer_02_b200 import binding as hb
+        wl = W.make_workload(1, scale=1 / 8, batch=512)
+        print(json.dumps({"fused_two_layer_ms": _two_layer_ms(hb, wl, 2, True), "tokens": int(wl.seq_offsets[-1])}))
         return
     import torch
     import torch.distributed as dist

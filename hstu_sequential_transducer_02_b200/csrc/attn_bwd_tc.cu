@@ -87,7 +87,8 @@ struct BwdLayout {
   static constexpr int kBar = (kTimeB + kNumBuckets * 4 + 15) & ~15;
   static constexpr int kItems = kBar + (int)sizeof(BwdBars);
   static constexpr int kMisc = kItems + kItemSlots * 8 * 4;
-  static constexpr int kEnd = kMisc + 16;
+  static constexpr int kDiag = kMisc + 16;                       // per epilogue warp: 32 completed diagonal sums
+  static constexpr int kEnd = kDiag + kEpiWarps * 32 * 4;
   static constexpr int kAlloc = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
 static_assert(BwdLayout::kAlloc <= 227 * 1024, "shared memory");
@@ -216,6 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
   const uint32_t sKV = smem_u32(smem + L::kKV);
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sDS = smem_u32(smem + L::kDS);
+  float* diag_all = reinterpret_cast<float*>(smem + L::kDiag);
 
   const AttnBwdParams& p = prm.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -433,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
     const int quarter = warp & 3;          // TMEM lane quarter: kv rows 32 quarter ..
     const int seg = ew >> 2;               // q columns [32 seg, 32 seg + 32) of the q tile
     const int jl = quarter * 32 + lane;    // kv row inside the tile
+    float* const diag_w = diag_all + ew * 32;   // this warp's completed diagonal sums (band segments)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float k_lg = prm.ln2_over_div;
     const int etid = threadIdx.x - 32 * kEpiWarp0;
@@ -611,6 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         tc_fence_after();
         uint32_t pk_prev[4], dk_prev[4];   // the first chunk's words, held until the readouts
         if (kind != 3) {
+          // one copy of the chunk loop per kind (each with only its own state live)
+          auto chunks = [&](auto&& compute) -> bool {
           // ---- the segment in four chunks of 8 q columns: S^T and dP^T of the chunk into
           // registers (the last chunk's load frees the score buffers for the next tile's
           // MMAs), P and dS, then P^T into TMEM and dS^T into shared memory
@@ -639,109 +644,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
             }
             uint32_t pk[4];   // P^T words (bf16 pairs) of the chunk's 8 q columns
             uint32_t dk[4];   // dS^T words
-            if (kind == 0) {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) { pk[e] = 0u; dk[e] = 0u; }
-            } else if (kind == 1 && wrank == 1) {
-#pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                float ds0, ds1;
-                p_ds2(__uint_as_float(sr[e]) + hb0, __uint_as_float(sr[e + 1]) + hb0, __uint_as_float(dr[e]),
-                      __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
-                dk[e >> 1] = pack_bf16x2(ds0, ds1);
-                a0 += ds0 + ds1;
-              }
-            } else if (kind == 1 && wrank == -2) {
-              float aup = 0.f;   // the upper bucket's part of what went into a0
-#pragma unroll
-              for (int e4 = 0; e4 < 2; ++e4) {
-                const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 8 * c8 + 4 * e4]);
-                const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
-                bool up[4];
-                float xs[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  up[u] = rv[u] >= up_at;
-                  xs[u] = __uint_as_float(sr[4 * e4 + u]) + (up[u] ? hb1 : hb0);
-                }
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                  float ds0, ds1;
-                  const int e = 4 * e4 + 2 * q2;
-                  p_ds2(xs[2 * q2], xs[2 * q2 + 1], __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n,
-                        pk[e >> 1], ds0, ds1);
-                  dk[e >> 1] = pack_bf16x2(ds0, ds1);
-                  a0 += ds0 + ds1;
-                  aup += (up[2 * q2] ? ds0 : 0.f) + (up[2 * q2 + 1] ? ds1 : 0.f);
-                }
-              }
-              a0 -= aup;
-              a1 += aup;
-            } else if (kind == 1) {
-#pragma unroll
-              for (int e4 = 0; e4 < 2; ++e4) {
-                const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 8 * c8 + 4 * e4]);
-                const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
-                float xs[4];
-                int bk[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const int32_t dd = abs(rv[u] - rj);
-                  bk[u] = (dd >= th1 ? 1 : 0) + (dd >= th2 ? 1 : 0) + (dd >= th3 ? 1 : 0);
-                  const float hb = bk[u] == 0 ? hb0 : (bk[u] == 1 ? hb1 : (bk[u] == 2 ? hb2 : hb3));
-                  xs[u] = __uint_as_float(sr[4 * e4 + u]) + hb;
-                }
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                  float ds0, ds1;
-                  const int e = 4 * e4 + 2 * q2;
-                  p_ds2(xs[2 * q2], xs[2 * q2 + 1], __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n,
-                        pk[e >> 1], ds0, ds1);
-                  dk[e >> 1] = pack_bf16x2(ds0, ds1);
-                  const float dsv[2] = {ds0, ds1};
-#pragma unroll
-                  for (int u = 0; u < 2; ++u) {
-                    const int b = bk[2 * q2 + u];
-                    a0 += b == 0 ? dsv[u] : 0.f;
-                    a1 += b == 1 ? dsv[u] : 0.f;
-                    a2 += b == 2 ? dsv[u] : 0.f;
-                    a3 += b == 3 ? dsv[u] : 0.f;
-                  }
-                }
-              }
-            } else {
-              if (c8 == 0) cur_tb = w[0] & 0x7F;
-#pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                float ds0, ds1;
-                float x0, x1;
-                add2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), __uint_as_float(w[e] & 0xFFFF0000u),
-                     __uint_as_float(w[e + 1] & 0xFFFF0000u), x0, x1);
-                p_ds2(x0, x1, __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
-                dk[e >> 1] = pack_bf16x2(ds0, ds1);
-                const float dsv[2] = {ds0, ds1};
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  // time bucket: runs along the row
-                  const int tb = w[e + u] & 0x7F;
-                  const bool change = tb != cur_tb;
-                  if (change) red_add(&gtime[cur_tb], at);
-                  cur_tb = tb;
-                  at = change ? dsv[u] : at + dsv[u];
-                  // position bucket D + col - lane: the running sum of the diagonal col - lane
-                  // moves one lane down per column, and lane 31's is complete
-                  dg += dsv[u];
-                  const int col = 8 * c8 + e + u;
-                  if (lane == 31 && (D > 0 || col == 31)) red_add(&gpos[min(D + col - 31, kNumBuckets - 1)], dg);
-                  dg = lane == 31 ? 0.f : dg;
-                  dg = __shfl_sync(0xffffffffu, dg, (lane + 31) & 31);
-                }
-              }
-            }
+            compute(c8, sr, dr, w, pk, dk);
             if (c8 == 1) {
               // deferred readouts (their MMAs ran while these chunks were computed), then
               // the previous tile's P^T and dS^T must have been consumed
-              if (!readouts()) goto fail;
+              if (!readouts()) return false;
             }
             if (c8 >= 1) {
               if (c8 == 1) {
@@ -755,6 +662,129 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
               for (int e = 0; e < 4; ++e) { pk_prev[e] = pk[e]; dk_prev[e] = dk[e]; }
             }
           }
+          return true;
+          };
+          bool chunks_ok;
+          if (kind == 0) {
+            chunks_ok = chunks([&](int c8, const uint32_t (&sr)[8], const uint32_t (&dr)[8], const uint32_t (&w)[8], uint32_t (&pk)[4], uint32_t (&dk)[4]) {
+              (void)c8; (void)sr; (void)dr; (void)w;
+    #pragma unroll
+                  for (int e = 0; e < 4; ++e) { pk[e] = 0u; dk[e] = 0u; }
+            });
+          }
+          else if (kind == 1 && wrank == 1) {
+            chunks_ok = chunks([&](int c8, const uint32_t (&sr)[8], const uint32_t (&dr)[8], const uint32_t (&w)[8], uint32_t (&pk)[4], uint32_t (&dk)[4]) {
+              (void)c8; (void)sr; (void)dr; (void)w;
+    #pragma unroll
+                  for (int e = 0; e < 8; e += 2) {
+                    float ds0, ds1;
+                    p_ds2(__uint_as_float(sr[e]) + hb0, __uint_as_float(sr[e + 1]) + hb0, __uint_as_float(dr[e]),
+                          __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
+                    dk[e >> 1] = pack_bf16x2(ds0, ds1);
+                    a0 += ds0 + ds1;
+                  }
+            });
+          }
+          else if (kind == 1 && wrank == -2) {
+            chunks_ok = chunks([&](int c8, const uint32_t (&sr)[8], const uint32_t (&dr)[8], const uint32_t (&w)[8], uint32_t (&pk)[4], uint32_t (&dk)[4]) {
+              (void)c8; (void)sr; (void)dr; (void)w;
+                  float aup = 0.f;   // the upper bucket's part of what went into a0
+    #pragma unroll
+                  for (int e4 = 0; e4 < 2; ++e4) {
+                    const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 8 * c8 + 4 * e4]);
+                    const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+                    bool up[4];
+                    float xs[4];
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                      up[u] = rv[u] >= up_at;
+                      xs[u] = __uint_as_float(sr[4 * e4 + u]) + (up[u] ? hb1 : hb0);
+                    }
+    #pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                      float ds0, ds1;
+                      const int e = 4 * e4 + 2 * q2;
+                      p_ds2(xs[2 * q2], xs[2 * q2 + 1], __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n,
+                            pk[e >> 1], ds0, ds1);
+                      dk[e >> 1] = pack_bf16x2(ds0, ds1);
+                      a0 += ds0 + ds1;
+                      aup += (up[2 * q2] ? ds0 : 0.f) + (up[2 * q2 + 1] ? ds1 : 0.f);
+                    }
+                  }
+                  a0 -= aup;
+                  a1 += aup;
+            });
+          }
+          else if (kind == 1) {
+            chunks_ok = chunks([&](int c8, const uint32_t (&sr)[8], const uint32_t (&dr)[8], const uint32_t (&w)[8], uint32_t (&pk)[4], uint32_t (&dk)[4]) {
+              (void)c8; (void)sr; (void)dr; (void)w;
+    #pragma unroll
+                  for (int e4 = 0; e4 < 2; ++e4) {
+                    const int4 rel4 = *reinterpret_cast<const int4*>(&qrec.rel[32 * seg + 8 * c8 + 4 * e4]);
+                    const int32_t rv[4] = {rel4.x, rel4.y, rel4.z, rel4.w};
+                    float xs[4];
+                    int bk[4];
+    #pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                      const int32_t dd = abs(rv[u] - rj);
+                      bk[u] = (dd >= th1 ? 1 : 0) + (dd >= th2 ? 1 : 0) + (dd >= th3 ? 1 : 0);
+                      const float hb = bk[u] == 0 ? hb0 : (bk[u] == 1 ? hb1 : (bk[u] == 2 ? hb2 : hb3));
+                      xs[u] = __uint_as_float(sr[4 * e4 + u]) + hb;
+                    }
+    #pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                      float ds0, ds1;
+                      const int e = 4 * e4 + 2 * q2;
+                      p_ds2(xs[2 * q2], xs[2 * q2 + 1], __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n,
+                            pk[e >> 1], ds0, ds1);
+                      dk[e >> 1] = pack_bf16x2(ds0, ds1);
+                      const float dsv[2] = {ds0, ds1};
+    #pragma unroll
+                      for (int u = 0; u < 2; ++u) {
+                        const int b = bk[2 * q2 + u];
+                        a0 += b == 0 ? dsv[u] : 0.f;
+                        a1 += b == 1 ? dsv[u] : 0.f;
+                        a2 += b == 2 ? dsv[u] : 0.f;
+                        a3 += b == 3 ? dsv[u] : 0.f;
+                      }
+                    }
+                  }
+            });
+          }
+          else {
+            chunks_ok = chunks([&](int c8, const uint32_t (&sr)[8], const uint32_t (&dr)[8], const uint32_t (&w)[8], uint32_t (&pk)[4], uint32_t (&dk)[4]) {
+              (void)c8; (void)sr; (void)dr; (void)w;
+                  if (c8 == 0) cur_tb = w[0] & 0x7F;
+    #pragma unroll
+                  for (int e = 0; e < 8; e += 2) {
+                    float ds0, ds1;
+                    float x0, x1;
+                    add2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), __uint_as_float(w[e] & 0xFFFF0000u),
+                         __uint_as_float(w[e + 1] & 0xFFFF0000u), x0, x1);
+                    p_ds2(x0, x1, __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), inv_n, pk[e >> 1], ds0, ds1);
+                    dk[e >> 1] = pack_bf16x2(ds0, ds1);
+                    const float dsv[2] = {ds0, ds1};
+    #pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                      // time bucket: runs along the row
+                      const int tb = w[e + u] & 0x7F;
+                      const bool change = tb != cur_tb;
+                      if (change) red_add(&gtime[cur_tb], at);
+                      cur_tb = tb;
+                      at = change ? dsv[u] : at + dsv[u];
+                      // position bucket D + col - lane: the running sum of the diagonal col - lane
+                      // moves one lane down per column, and lane 31's is complete: it is kept
+                      // in shared memory until the segment's end
+                      dg += dsv[u];
+                      const int col = 8 * c8 + e + u;
+                      if (lane == 31) diag_w[col] = dg;
+                      dg = lane == 31 ? 0.f : dg;
+                      dg = __shfl_sync(0xffffffffu, dg, (lane + 31) & 31);
+                    }
+                  }
+            });
+          }
+          if (!chunks_ok) goto fail;
         } else {
           // ---- per element (candidates, per-head bias tables, 64-bit time offsets): the
           // scores are read 8 columns at a time and the score buffers freed at the end
@@ -815,8 +845,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           far_pos += (a0 + a1) + (a2 + a3);
         } else if (kind == 2) {
           if (at != 0.f) red_add(&gtime[cur_tb], at);
-          // lane l >= 1 holds the diagonal 32 - l: position bucket D + 32 - l
+          // lane l >= 1 holds the diagonal 32 - l: position bucket D + 32 - l; the diagonal
+          // completed at column l (position bucket D + l - 31; below 0 only for D = 0,
+          // where its pairs are masked) waits in shared memory
           if (lane > 0 && dg != 0.f) red_add(&gpos[min(D + 32 - lane, kNumBuckets - 1)], dg);
+          __syncwarp();
+          const float dl = diag_w[lane];
+          if ((D > 0 || lane == 31) && dl != 0.f) red_add(&gpos[min(D + lane - 31, kNumBuckets - 1)], dl);
+          __syncwarp();   // read before the next band segment writes
         }
         tmem_st_wait();
         fence_proxy_async_smem();

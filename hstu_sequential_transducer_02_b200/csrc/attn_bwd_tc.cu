@@ -612,9 +612,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         }
         if (!mbar_wait(&bars->sp_full, g & 1, tmo, abort_flag)) goto fail;
         tc_fence_after();
-        uint32_t pk_prev[4], dk_prev[4];   // the first chunk's words, held until the readouts
         if (kind != 3) {
           // one copy of the chunk loop per kind (each with only its own state live)
+          // the deferred readouts (their MMAs ran while the scores were awaited), then the
+          // previous tile's P^T and dS^T must have been consumed before this tile's are written
+          if (!readouts()) goto fail;
           auto chunks = [&](auto&& compute) -> bool {
           // ---- the segment in four chunks of 8 q columns: S^T and dP^T of the chunk into
           // registers (the last chunk's load frees the score buffers for the next tile's
@@ -645,22 +647,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
             uint32_t pk[4];   // P^T words (bf16 pairs) of the chunk's 8 q columns
             uint32_t dk[4];   // dS^T words
             compute(c8, sr, dr, w, pk, dk);
-            if (c8 == 1) {
-              // deferred readouts (their MMAs ran while these chunks were computed), then
-              // the previous tile's P^T and dS^T must have been consumed
-              if (!readouts()) return false;
-            }
-            if (c8 >= 1) {
-              if (c8 == 1) {
-                tmem_st_32x32b_x4(tmem + kColP + lane_off + 16 * seg, pk_prev);
-                st_shared_v4(ds_atom + (((ds_ch) ^ (jl & 7)) << 4), dk_prev[0], dk_prev[1], dk_prev[2], dk_prev[3]);
-              }
-              tmem_st_32x32b_x4(tmem + kColP + lane_off + 16 * seg + 4 * c8, pk);
-              st_shared_v4(ds_atom + (((ds_ch + c8) ^ (jl & 7)) << 4), dk[0], dk[1], dk[2], dk[3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 4; ++e) { pk_prev[e] = pk[e]; dk_prev[e] = dk[e]; }
-            }
+            tmem_st_32x32b_x4(tmem + kColP + lane_off + 16 * seg + 4 * c8, pk);
+            st_shared_v4(ds_atom + (((ds_ch + c8) ^ (jl & 7)) << 4), dk[0], dk[1], dk[2], dk[3]);
           }
           return true;
           };
@@ -862,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           mbar_arrive(&bars->p_ready);
           mbar_arrive(&bars->q_empty[qs]);
         }
-        // this tile's dQ is read out while the next tile's scores are processed
+        // this tile's dQ is read out at the start of the next tile (its MMA runs meanwhile)
         const int iq = qt * BT + jl;   // this lane's q row of the dQ tile
         dq_dst = iq < si.n ? p.dq_accum + ((int64_t)(si.start + iq) * p.num_heads + h) * DHB + 16 * seg : nullptr;
         pend_dq = true;

@@ -29,7 +29,7 @@ template <> struct Elem<__nv_bfloat16> {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 __device__ __forceinline__ float silu_grad_f(float x) {
-  float s = 1.0f / (1.0f + __expf(-x));
+  float s = __frcp_rn(1.0f + __expf(-x));   // the correctly rounded 1 / (1 + e^-x)
   return s * (1.0f + x * (1.0f - s));
 }
 

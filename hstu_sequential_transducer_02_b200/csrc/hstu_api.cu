@@ -335,7 +335,7 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
     const int grid = w.capacity < 148 * 2 ? (w.capacity > 0 ? w.capacity : 1) : 148 * 2;
     HSTU_CUDA(launch_attn_bwd_simt(p, d->dtype, dh, grid, st));
   }
-  {
+  if (dq) {   // (without dq the caller reads the fp32 accumulator w.dq_accum itself)
     TraceScope tr("dq_finalize", st);
     HSTU_CUDA(launch_dq_finalize(w.dq_accum, jb->seq_offsets, jb->batch, H, dh, d->dtype, dq, lddq, 148 * 8, st));
   }
@@ -510,6 +510,9 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   const int fl = d->attn.flags;
   void* duvqk = gr->duvqk ? gr->duvqk : ws.duvqk;
   int32_t* status = ws.attn.status;
+  // without a caller buffer for dU|dV|dQ|dK, the SiLU' pass reads dQ from the
+  // attention's fp32 accumulator (no conversion pass)
+  const bool dq_direct = !gr->duvqk && hv % 8 == 0;
   // The weight-gradient products reduce over tokens in 64-row slices: rows from the
   // device row count up to the next multiple of 64 of every token-major operand are zeroed.
   {
@@ -556,12 +559,13 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   const char* uvqk = (const char*)sv->uvqk;
   char* du = (char*)duvqk;
   HSTU_TRY(run_attn_bwd(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + hv * es,
-                        4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, du + 2 * hv * es, 4 * hv, du + 3 * hv * es,
-                        4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias, ws.attn, st));
+                        4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, dq_direct ? nullptr : du + 2 * hv * es, 4 * hv,
+                        du + 3 * hv * es, 4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias, ws.attn, st));
   // a = SiLU(z): dz = da * SiLU'(z)
   {
     TraceScope tr("silu_bwd", st);
-    HSTU_CUDA(launch_silu_bwd(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, st));
+    HSTU_CUDA(launch_silu_bwd(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, st,
+                              dq_direct ? ws.attn.dq_accum : nullptr, hv, 2 * hv, hv));
     HSTU_CUDA(launch_zero_tail_rows(ws.dz, (int64_t)4 * hv * es, (int64_t)4 * hv * es, T, rows, 64, st));
   }
   // z = xhat W1^T + b1: dW1 = dz^T xhat, db1 = colsum(dz), dxhat = dz W1

@@ -218,9 +218,11 @@ cudaError_t launch_convert_rows(const void* src, int64_t lds, int src_dtype, voi
 // zero rows [*rows_dev, min(cap, round_up(*rows_dev, multiple))) of a row-major buffer
 cudaError_t launch_zero_tail_rows(void* buf, int64_t ld_bytes, int64_t row_bytes, int rows_cap,
                                   const int32_t* rows_dev, int multiple, cudaStream_t st);
-// dz = da * SiLU'(z) (dtype), elementwise on [rows, cols]
+// dz = da * SiLU'(z) (dtype), elementwise on [rows, cols]; with dq, columns
+// [q_col0, q_col0 + q_cols) take da from the fp32 matrix dq (row stride ldq)
 cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
-                            const int32_t* rows_dev, int cols, int dtype, cudaStream_t st);
+                            const int32_t* rows_dev, int cols, int dtype, cudaStream_t st, const float* dq = nullptr,
+                            int64_t ldq = 0, int q_col0 = 0, int q_cols = 0);
 // column sums of a [rows, cols] dtype matrix into fp32 out (overwrite)
 cudaError_t launch_col_sum(const void* a, int64_t lda, int rows_cap, const int32_t* rows_dev, int cols,
                            int dtype, float* out, cudaStream_t st);

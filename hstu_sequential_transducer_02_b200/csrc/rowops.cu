@@ -331,9 +331,12 @@ ln_bwd_kernel(const T* __restrict__ x, int64_t ldx, const float* __restrict__ ga
   flush_affine_grads(pg, pb, nch, dgamma, dbeta, red);
 }
 
+// (columns [q_col0, q_col0 + q_cols) take da from the fp32 matrix dq, row stride ldq,
+// when dq is given)
 template <typename T>
 __global__ void silu_bwd_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __restrict__ dz,
-                                int64_t ld, int rows_cap, const int32_t* __restrict__ rows_dev, int cols) {
+                                int64_t ld, int rows_cap, const int32_t* __restrict__ rows_dev, int cols,
+                                const float* __restrict__ dq, int64_t ldq, int q_col0, int q_cols) {
   const int rows = rows_of(rows_cap, rows_dev);
   const int nch = cols / 8;
   const int64_t total = (int64_t)rows * nch;
@@ -341,7 +344,8 @@ __global__ void silu_bwd_kernel(const T* __restrict__ da, const T* __restrict__ 
     const int64_t row = e / nch;
     const int ch = (int)(e % nch);
     float a[8], zz[8], r[8];
-    load8(da + row * ld + ch * 8, a);
+    if (dq != nullptr && ch * 8 >= q_col0 && ch * 8 < q_col0 + q_cols) load8(dq + row * ldq + (ch * 8 - q_col0), a);
+    else load8(da + row * ld + ch * 8, a);
     load8(z + row * ld + ch * 8, zz);
 #pragma unroll
     for (int i = 0; i < 8; ++i) r[i] = a[i] * silu_grad_f(zz[i]);
@@ -932,15 +936,18 @@ cudaError_t launch_ln_bwd(const void* x, int64_t ldx, const float* gamma, const 
 }
 
 cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
-                            const int32_t* rows_dev, int cols, int dtype, cudaStream_t st) {
+                            const int32_t* rows_dev, int cols, int dtype, cudaStream_t st, const float* dq,
+                            int64_t ldq, int q_col0, int q_cols) {
   if (rows_cap <= 0) return cudaSuccess;
+  if (dq && (q_col0 % 8 || q_cols % 8 || ldq % 4)) return cudaErrorInvalidValue;
   const int g = 148 * 8;
   if (dtype == HSTU_DTYPE_F32)
     silu_bwd_kernel<float><<<g, 256, 0, st>>>((const float*)da, (const float*)z, (float*)dz, ld, rows_cap,
-                                              rows_dev, cols);
+                                              rows_dev, cols, dq, ldq, q_col0, q_cols);
   else
     silu_bwd_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16*)da, (const __nv_bfloat16*)z,
-                                                      (__nv_bfloat16*)dz, ld, rows_cap, rows_dev, cols);
+                                                      (__nv_bfloat16*)dz, ld, rows_cap, rows_dev, cols, dq, ldq,
+                                                      q_col0, q_cols);
   return cudaGetLastError();
 }
 

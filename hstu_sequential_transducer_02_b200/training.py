@@ -43,8 +43,9 @@ class StackTrainer:
         grads: List[dict] = [None] * L
         g = dy
         for li in range(L - 1, -1, -1):
+            # the parameters' gradients only (no dU|dV|dQ|dK buffer for the caller)
             g, grads[li] = self.layers[li].backward(ins[li], g, saved[li], seq_offsets, timestamps,
-                                                    num_targets=num_targets)
+                                                    num_targets=num_targets, keep_duvqk=False)
             self.reducer.layer_done(grads[li])
         self.reducer.wait()
         return g, grads

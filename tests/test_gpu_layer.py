@@ -359,7 +359,7 @@ def _layer_errors(r, gr, T, hv):
     return out
 
 
-def _gpu_layer_grads(wl, li, x, dy, offs, ts, residual_fp32=True):
+def _gpu_layer_grads(wl, li, x, dy, offs, ts, residual_fp32=True, keep_duvqk=True):
     """Layer li of the workload on the GPU: forward with saved activations from
     the host input x, then backward from the host upstream gradient dy."""
     b = _b()
@@ -373,7 +373,7 @@ def _gpu_layer_grads(wl, li, x, dy, offs, ts, residual_fp32=True):
     offs_d, ts_d = dev(np.asarray(offs, np.int32)), dev(ts)
     x_d = dev(np.asarray(x, np.float32), io)
     ly.forward(x_d, offs_d, ts_d, saved=sv)
-    dx, gr = ly.backward(x_d, dev(np.asarray(dy, np.float32), io), sv, offs_d, ts_d)
+    dx, gr = ly.backward(x_d, dev(np.asarray(dy, np.float32), io), sv, offs_d, ts_d, keep_duvqk=keep_duvqk)
     torch.cuda.synchronize()
     return dx.float().cpu().numpy().astype(np.float64), gr
 
@@ -422,6 +422,26 @@ def test_training_step_config4_per_layer():
     for li in range(len(wl.layers)):
         dx, gr = _gpu_layer_grads(wl, li, xs[li], dys[li], offs, ts)
         _check_layer_grads(gr, ref[li], T, hv, f"layer {li}")
+        assert_close(dx, ref[li]["dx"], "bf16", f"layer {li} dx", grad=True)
+
+
+def test_training_step_config4_per_layer_parameter_gradients_only():
+    """The same per-layer check when the caller asks for the parameters'
+    gradients only (no dU|dV|dQ|dK buffer, as in the training step): the SiLU
+    backward then reads dQ from the attention's fp32 accumulator.  Every weight,
+    bias and relative-bias gradient and dx at the specification's bounds."""
+    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
+    g, offs = _sl_workload(wl)
+    e = wl.extras
+    x0, ts, g0 = wl.x[g].astype(np.float64), wl.timestamps[g], e["grad_out"][g].astype(np.float64)
+    xs, dys, ref = _oracle_chain(wl, x0, g0, offs, ts)
+    for li in (0, len(wl.layers) - 1):
+        dx, gr = _gpu_layer_grads(wl, li, xs[li], dys[li], offs, ts, keep_duvqk=False)
+        assert gr.get("uvqk") is None
+        for gname, rname in [("pos_bias", "dpos_bias"), ("time_bias", "dtime_bias"), ("w1", "dw1"), ("w2", "dw2"),
+                             ("b1", "db1"), ("b2", "db2"), ("ln1_gamma", "dln1_g"), ("ln1_beta", "dln1_b"),
+                             ("ln2_gamma", "dln2_g"), ("ln2_beta", "dln2_b")]:
+            assert_close(gr[gname].cpu().numpy(), ref[li][rname], "bf16", f"layer {li} {gname}", grad=True)
         assert_close(dx, ref[li]["dx"], "bf16", f"layer {li} dx", grad=True)
 
 

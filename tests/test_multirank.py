@@ -238,7 +238,7 @@ class _OracleLayer:
         out.copy_(torch.from_numpy(y))
         return out
 
-    def backward(self, x, dy, saved, seq_offsets, timestamps, num_targets=None):
+    def backward(self, x, dy, saved, seq_offsets, timestamps, num_targets=None, keep_duvqk=True):
         r = O.layer_backward(x.numpy(), self.p, dy.numpy(), seq_offsets.numpy(), timestamps.numpy(), self.H, self.dh)
         grads = {k: torch.from_numpy(np.asarray(r[v], np.float64)).float() for k, v in self.NAMES.items()}
         return torch.from_numpy(r["dx"]), grads

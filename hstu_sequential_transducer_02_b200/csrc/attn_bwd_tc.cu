@@ -88,7 +88,8 @@ struct BwdLayout {
   static constexpr int kItems = kBar + (int)sizeof(BwdBars);
   static constexpr int kMisc = kItems + kItemSlots * 8 * 4;
   static constexpr int kDiag = kMisc + 16;                       // per epilogue warp: 32 completed diagonal sums
-  static constexpr int kEnd = kDiag + kEpiWarps * 32 * 4;
+  static constexpr int kPend = kDiag + kEpiWarps * 32 * 4;        // per epilogue thread: pending readout rows
+  static constexpr int kEnd = kPend + kEpiWarps * 32 * 8;
   static constexpr int kAlloc = kEnd + 1024;  // slack for 1024-byte alignment of the base
 };
 static_assert(BwdLayout::kAlloc <= 227 * 1024, "shared memory");
@@ -443,8 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
     float far_pos = 0.f;                   // dS of pairs in the last position bucket (summed in registers)
     // deferred readouts: dQ of the previous q tile, dK and dV of the previous item
     bool pend_dq = false, pend_acc = false;
-    float* dq_dst = nullptr;
-    __nv_bfloat16 *dk_dst = nullptr, *dv_dst = nullptr;
+    // their destinations wait in shared memory (no registers while pending): the dQ
+    // accumulator row and the dK/dV row, each as token * heads + head (-1: none)
+    int2* const pend_rows = reinterpret_cast<int2*>(smem + L::kPend) + (threadIdx.x - 32 * kEpiWarp0);
     int acc_par = 0;
     // every epilogue warp at the same point: an mbarrier phase (a warp that gave up on
     // a bounded wait sets the abort flag, and the others' waits return)
@@ -481,7 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->dq_empty);
-        if (dq_dst) {
+        const int dq_r = pend_rows->x;
+        if (dq_r >= 0) {
+          float* dq_dst = p.dq_accum + (int64_t)dq_r * DHB + 16 * seg;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             red_add_v4(dq_dst + 4 * c, __uint_as_float(qr[4 * c]), __uint_as_float(qr[4 * c + 1]),
@@ -496,13 +500,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
           uint32_t vr[16];
           tmem_ld_32x32b_x16(tmem + kColDV + lane_off + 16 * seg, vr);
           tmem_ld_wait();
-          if (dv_dst) store_bf16_row16(dv_dst, vr);
+          const int kv_r = pend_rows->y;
+          if (kv_r >= 0)
+            store_bf16_row16(reinterpret_cast<__nv_bfloat16*>(p.dv) + (int64_t)(kv_r / p.num_heads) * p.lddv +
+                                 (kv_r % p.num_heads) * DHB + 16 * seg, vr);
         }
         {
           uint32_t kr[16];
           tmem_ld_32x32b_x16(tmem + kColDK + lane_off + 16 * seg, kr);
           tmem_ld_wait();
-          if (dk_dst) store_bf16_row16(dk_dst, kr);
+          const int kv_r = pend_rows->y;
+          if (kv_r >= 0)
+            store_bf16_row16(reinterpret_cast<__nv_bfloat16*>(p.dk) + (int64_t)(kv_r / p.num_heads) * p.lddk +
+                                 (kv_r % p.num_heads) * DHB + 16 * seg, kr);
         }
         tc_fence_before();
         __syncwarp();
@@ -852,16 +862,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
         }
         // this tile's dQ is read out at the start of the next tile (its MMA runs meanwhile)
         const int iq = qt * BT + jl;   // this lane's q row of the dQ tile
-        dq_dst = iq < si.n ? p.dq_accum + ((int64_t)(si.start + iq) * p.num_heads + h) * DHB + 16 * seg : nullptr;
+        pend_rows->x = iq < si.n ? (si.start + iq) * p.num_heads + h : -1;
         pend_dq = true;
         ++g;
       }
       // this item's dK and dV are read out during the next item's first tile
       if (jlive) {
-        dv_dst = reinterpret_cast<__nv_bfloat16*>(p.dv) + (int64_t)(si.start + j) * p.lddv + h * DHB + 16 * seg;
-        dk_dst = reinterpret_cast<__nv_bfloat16*>(p.dk) + (int64_t)(si.start + j) * p.lddk + h * DHB + 16 * seg;
+        pend_rows->y = (si.start + j) * p.num_heads + h;
       } else {
-        dv_dst = dk_dst = nullptr;
+        pend_rows->y = -1;
       }
       pend_acc = true;
       acc_par = k & 1;
@@ -875,7 +884,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
       uint32_t qr[16];
       tmem_ld_32x32b_x16(tmem + kColDQ + lane_off + 16 * seg, qr);
       tmem_ld_wait();
-      if (dq_dst) {
+      const int dq_r = pend_rows->x;
+      if (dq_r >= 0) {
+        float* dq_dst = p.dq_accum + (int64_t)dq_r * DHB + 16 * seg;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           red_add_v4(dq_dst + 4 * c, __uint_as_float(qr[4 * c]), __uint_as_float(qr[4 * c + 1]),
@@ -889,9 +900,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_tc_kernel(const __grid_c
       tmem_ld_32x32b_x16(tmem + kColDV + lane_off + 16 * seg, vr);
       tmem_ld_32x32b_x16(tmem + kColDK + lane_off + 16 * seg, kr);
       tmem_ld_wait();
-      if (dv_dst) {
-        store_bf16_row16(dv_dst, vr);
-        store_bf16_row16(dk_dst, kr);
+      const int kv_r = pend_rows->y;
+      if (kv_r >= 0) {
+        const int64_t tok = kv_r / p.num_heads, hh = kv_r % p.num_heads;
+        store_bf16_row16(reinterpret_cast<__nv_bfloat16*>(p.dv) + tok * p.lddv + hh * DHB + 16 * seg, vr);
+        store_bf16_row16(reinterpret_cast<__nv_bfloat16*>(p.dk) + tok * p.lddk + hh * DHB + 16 * seg, kr);
       }
     }
     flush_far();
@@ -1081,6 +1094,7 @@ cudaError_t launch_attn_bwd_tc(const AttnBwdParams& p, int grid, cudaStream_t st
   memset(&tp, 0, sizeof(tp));
   tp.p = p;
   tp.ln2_over_div = (float)(0.69314718055994530942 / time_div);
+  if ((int64_t)p.total_rows * p.num_heads >= 0x7FFFFFFF) return cudaErrorInvalidValue;   // int32 row * head indices
   const int64_t hd = (int64_t)p.num_heads * DHB;
   if (!make_map(&tp.map_q, p.q, hd, p.total_rows, p.ldq) || !make_map(&tp.map_k, p.k, hd, p.total_rows, p.ldk) ||
       !make_map(&tp.map_v, p.v, hd, p.total_rows, p.ldv) ||

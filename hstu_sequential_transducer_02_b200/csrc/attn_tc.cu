@@ -539,6 +539,12 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
         const int i0w = r0 + quarter * 32;
         const bool use_band = wrank == 4 && p.band != nullptr && cl >= i0w - 128 &&
                               !__any_sync(0xffffffffu, live && cand);
+        // warps of candidate rows (every row at or after N): the band's candidate window
+        // [floor32(N) - 128, floor32(N) + 32), and beyond it only each row's own column
+        const bool cand_warp = wrank == 4 && i0w >= si.hist;
+        const int cwb = (si.hist & ~31) - 128;
+        const bool use_cband = cand_warp && p.band != nullptr && cl >= cwb && cl < cwb + 160;
+        const bool self_only = cand_warp && cl >= cwb + 160;
         if (!s_ready) {
           if (!mbar_wait(&bars->s_full[sb], (it / kSBufs) & 1, tmo, abort_flag)) goto fail;
           tc_fence_after();
@@ -609,6 +615,42 @@ const auto pend = [&]() { return reinterpret_cast<PendingO*>(smem + L::kPend) + 
             const uint32_t v = few_terms ? silu2_exact_bf16(h0, h1) : silu2_bf16(h0, h1);
             pk[q] = (2 * q <= lim ? (v & 0xFFFFu) : 0u) | (2 * q + 1 <= lim ? (v & 0xFFFF0000u) : 0u);
           }
+        } else if (use_cband) {
+          // candidate rows near the end of the history: half biases from the band's
+          // candidate window; a column is attended iff it is history or the row's own
+          // (the exact SiLU: a candidate's output may rest on few terms)
+          uint4 bb[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                         make_uint4(0, 0, 0, 0)};
+          if (live) {
+            const uint4* bp = reinterpret_cast<const uint4*>(p.band) + (int64_t)(si.start + i) * kBandChunks +
+                              ((cl - cwb) >> 3);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) bb[c] = __ldg(bp + c);
+          }
+          const int lim_h = live ? si.hist - 1 - cl : -1;   // columns e <= lim_h are history
+          const int e_self = live ? i - cl : -1;
+          const uint32_t* bw = reinterpret_cast<const uint32_t*>(bb);
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            float h0, h1;
+            half_plus2c(__uint_as_float(raw[2 * q]), __uint_as_float(raw[2 * q + 1]), __uint_as_float(bw[q] << 16),
+                        __uint_as_float(bw[q] & 0xFFFF0000u), h0, h1);
+            const uint32_t v = silu2_exact_bf16(h0, h1);
+            pk[q] = ((2 * q <= lim_h || 2 * q == e_self) ? (v & 0xFFFFu) : 0u) |
+                    ((2 * q + 1 <= lim_h || 2 * q + 1 == e_self) ? (v & 0xFFFF0000u) : 0u);
+          }
+        } else if (self_only) {
+          // candidate columns only: each row attends its own column (position bucket 0,
+          // time difference 0), if it lies in this segment
+          const int e_self = live ? i - cl : -1;
+          float s_self = 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s_self = e == e_self ? __uint_as_float(raw[e]) : s_self;
+          const float h = fmaf(s_self, 0.5f, 0.5f * (pos_b[0] + time_b[0]));
+          const uint32_t v = silu2_exact_bf16(h, h);
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            pk[q] = (e_self >> 1) == q ? ((e_self & 1) ? (v & 0xFFFF0000u) : (v & 0xFFFFu)) : 0u;
         } else if (__all_sync(0xffffffffu, narrow)) {
           // general, 32-bit time offsets: per-element mask, position and time bucket
           // (shared-memory reads kept few: the tensor core is reading Q, K and V
@@ -835,7 +877,11 @@ cudaError_t launch_tc(const AttnFwdParams& p, int grid, cudaStream_t st, double 
 // (i, j) is not attended.  A warp of 32 rows starting at i0 (a multiple of 32)
 // reaches columns within 127 positions of its rows only in segments starting at
 // i0 - 128 ... i0, which the band covers, so the epilogue reads these biases
-// instead of evaluating both buckets per element there.
+// instead of evaluating both buckets per element there.  A group of 32 candidate
+// rows (i0 >= N, position N for all) takes the window [floor32(N) - 128,
+// floor32(N) + 32) instead: the history columns within 127 positions of N, and
+// its own column where that falls inside (a candidate's other columns there are
+// candidates, not attended).
 // One block per group of 32 rows (four per 128-row tile of tile_base), one
 // thread per band column: timestamps become 32-bit offsets from the sequence's
 // first one (the 64-bit threshold search serves blocks whose offsets leave
@@ -859,6 +905,8 @@ __global__ void __launch_bounds__(kBandCols) band_bias_kernel(const int32_t* __r
   __shared__ float pb_s[kNumBuckets], tb_s[kNumBuckets];
   __shared__ int32_t rel_s[kBandCols];
   __shared__ int64_t abs_s[kBandCols];
+  __shared__ int32_t rrel_s[32];   // the group's rows
+  __shared__ int64_t rabs_s[32];
   __shared__ __align__(16) uint16_t out_s[32][kBandCols];
   if (*status != 0) return;  // the scheduler found the offsets invalid
   const int grp = blockIdx.x;
@@ -872,8 +920,9 @@ __global__ void __launch_bounds__(kBandCols) band_bias_kernel(const int32_t* __r
   const SeqInfo si = load_seq(offs, num_targets, lo);
   const int i0 = (t - tile_base[lo]) * 128 + 32 * (grp & 3);
   if (i0 >= si.n || si.start + si.n > T) return;
+  const bool cand_grp = i0 >= si.hist;   // every row of the group a candidate
   const int w = threadIdx.x;
-  const int j = i0 - 128 + w;
+  const int j = (cand_grp ? (si.hist & ~31) : i0) - 128 + w;   // this thread's window column
   for (int c = w; c < kNumBuckets + 4; c += kBandCols) {
     if (c < kNumBuckets) {
       thr[c] = thr_in.v[c];
@@ -890,7 +939,15 @@ __global__ void __launch_bounds__(kBandCols) band_bias_kernel(const int32_t* __r
   const int64_t lim = (1ll << 30) - 1;
   rel_s[w] = (int32_t)(rel < -lim ? -lim : (rel > lim ? lim : rel));
   abs_s[w] = tj;
-  const bool wide = __syncthreads_or(rel < -lim || rel > lim) != 0;
+  bool wide_t = rel < -lim || rel > lim;
+  if (w < 32) {
+    const int64_t ti = i0 + w < si.n ? ts[si.start + i0 + w] : t_first;
+    const int64_t reli = ti - t_first;
+    rrel_s[w] = (int32_t)(reli < -lim ? -lim : (reli > lim ? lim : reli));
+    rabs_s[w] = ti;
+    wide_t = wide_t || reli < -lim || reli > lim;
+  }
+  const bool wide = __syncthreads_or(wide_t) != 0;
   const int32_t relj = rel_s[w];
   const int posj = token_pos(j, si.hist);
   const int rows = si.n - i0 < 32 ? si.n - i0 : 32;
@@ -899,8 +956,8 @@ __global__ void __launch_bounds__(kBandCols) band_bias_kernel(const int32_t* __r
     float v = 0.f;
     if (j >= 0 && attended(i, j, si.n, si.hist)) {
       const int pb = pos_bucket(token_pos(i, si.hist), posj);
-      const int tb = wide ? band_bucket_wide(abs_s[128 + r], tj, thr)     // row i is window column 128 + r
-                          : fast_bucket(abs(rel_s[128 + r] - relj), thr32, ln2_over_div);
+      const int tb = wide ? band_bucket_wide(rabs_s[r], tj, thr)
+                          : fast_bucket(abs(rrel_s[r] - relj), thr32, ln2_over_div);
       v = 0.5f * (pb_s[pb] + tb_s[tb]);
     }
     out_s[r][w] = __bfloat16_as_ushort(__float2bfloat16_rn(v));

@@ -989,7 +989,9 @@ MfalconWs carve_mfalcon(Carver& c, const hstu_layer_desc* d, int L, int U, int h
   const size_t es = elem_size(d->attn.dtype), eio = elem_size(d->io_dtype);
   const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
   // targets-only attention: a work list of its own; status, tile bases and timestamp
-  // records are the full pass's (same offsets); no bias band (no history q tile runs)
+  // records are the full pass's (same offsets); no bias band (rewriting its candidate
+  // groups for every microbatch costs more than it saves there: candidate segments
+  // beyond the history's last 128 positions take the one-column path instead)
   w.attn_t = w.layer.attn;
   w.attn_t.count = c.take<int32_t>(64);
   w.attn_t.items = c.take<WorkItem>(w.layer.attn.capacity);

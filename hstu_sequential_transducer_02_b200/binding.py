@@ -26,6 +26,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE, ERR_
 DTYPE_F32, DTYPE_BF16 = 0, 1
 FLAG_FORCE_SIMT = 1
 FLAG_SHORT_SEQUENCES = 2
+FLAG_REUSE_PREP = 4
 NUM_BUCKETS = 128
 
 _c_int = ctypes.c_int
@@ -294,11 +295,14 @@ class Layer:
 
     def __init__(self, weights: Dict[str, torch.Tensor], d_model: int, num_heads: int, head_dim: int,
                  force_simt: bool = False, eps: float = 1e-5, time_div: float = 0.301,
-                 residual_fp32: bool = False, short_sequences: bool = False):
+                 residual_fp32: bool = False, short_sequences: bool = False, workspaces: Optional[dict] = None):
         """residual_fp32: X, Y (and dX, dY) are fp32 tensors while weights and
         activations use the weights' dtype.  short_sequences: every sequence has
         at most 128 tokens, and the forward runs as one fused kernel where the
-        shapes allow it (HSTU_FLAG_SHORT_SEQUENCES)."""
+        shapes allow it (HSTU_FLAG_SHORT_SEQUENCES).  workspaces: a dict shared by
+        layers of the same shape that run one after the other on one stream, so
+        that they use one workspace per entry point (and can reuse its attention
+        preparation, see `reuse_prep`)."""
         self.w = weights
         self.dtype = weights["w1"].dtype
         self.io_dtype = torch.float32 if residual_fp32 else self.dtype
@@ -309,7 +313,7 @@ class Layer:
         if short_sequences:
             self.desc.attn.flags |= FLAG_SHORT_SEQUENCES
         self.cw = layer_weights(weights)
-        self._ws = {}
+        self._ws = {} if workspaces is None else workspaces
 
     @property
     def hv(self) -> int:
@@ -324,14 +328,24 @@ class Layer:
             self._ws[key] = ws
         return ws
 
+    def _desc_for(self, reuse_prep: bool):
+        if not reuse_prep:
+            return self.desc
+        d = type(self.desc).from_buffer_copy(self.desc)
+        d.attn.flags |= FLAG_REUSE_PREP
+        return d
+
     def forward(self, x, seq_offsets, timestamps, num_targets=None, saved: Optional[Saved] = None, out=None,
-                stream=None):
+                stream=None, reuse_prep: bool = False):
+        """reuse_prep: the workspace holds the attention preparation of an earlier
+        forward on the same batch (HSTU_FLAG_REUSE_PREP)."""
         T = x.shape[0]
         jb = jagged(seq_offsets, timestamps, T, num_targets)
         ws = self._get_ws("fwd", _lib_layer_fwd_ws, jb.batch, T, x.device)
         y = torch.empty_like(x) if out is None else out
         sv = saved.c() if saved is not None else None
-        _check(_lib_layer_fwd(ctypes.byref(self.desc), ctypes.byref(self.cw), ctypes.byref(jb), _ptr(x), _ptr(y),
+        desc = self._desc_for(reuse_prep)
+        _check(_lib_layer_fwd(ctypes.byref(desc), ctypes.byref(self.cw), ctypes.byref(jb), _ptr(x), _ptr(y),
                               ctypes.byref(sv) if sv is not None else None, _ptr(ws), ws.numel(), _stream(stream)),
                "hstu_layer_fwd")
         return y
@@ -362,7 +376,9 @@ class Layer:
         return y
 
     def backward(self, x, dy, saved: Saved, seq_offsets, timestamps, num_targets=None, grads=None, dx=None,
-                 stream=None, keep_duvqk: bool = True):
+                 stream=None, keep_duvqk: bool = True, reuse_prep: bool = False):
+        """reuse_prep: the workspace holds the attention preparation of an earlier
+        backward on the same batch (HSTU_FLAG_REUSE_PREP)."""
         T = x.shape[0]
         jb = jagged(seq_offsets, timestamps, T, num_targets)
         ws = self._get_ws("bwd", _lib_layer_bwd_ws, jb.batch, T, x.device)
@@ -376,7 +392,8 @@ class Layer:
                                                   "b2", "pos_bias", "time_bias")], _ptr(grads.get("uvqk")))
         dx = torch.empty_like(x) if dx is None else dx
         sv = saved.c()
-        _check(_lib_layer_bwd(ctypes.byref(self.desc), ctypes.byref(self.cw), ctypes.byref(jb), _ptr(x),
+        desc = self._desc_for(reuse_prep)
+        _check(_lib_layer_bwd(ctypes.byref(desc), ctypes.byref(self.cw), ctypes.byref(jb), _ptr(x),
                               ctypes.byref(sv), _ptr(dy), _ptr(dx), ctypes.byref(g), _ptr(ws), ws.numel(),
                               _stream(stream)), "hstu_layer_bwd")
         return dx, grads

@@ -186,14 +186,17 @@ AttnWs carve_attn(Carver& c, const hstu_attn_desc* d, int B, int T, bool bwd, bo
 int run_attn_prep(const hstu_attn_desc* d, const hstu_jagged* jb, const float* pos_bias, const float* time_bias,
                   const AttnWs& w, cudaStream_t st) {
   const int tile = attn_tile(d);
-  {
+  if (d->flags & HSTU_FLAG_REUSE_PREP) {
+    // work list and tile records from an earlier call: only the fetch cursor restarts
+    HSTU_CUDA(cudaMemsetAsync(w.count + 1, 0, sizeof(int32_t), st));
+  } else {
     // tensor-core path: locality order, fetched dynamically (count[1] is the cursor)
     TraceScope tr("sched_fwd", st);
     HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, d->num_heads,
                                      tile, tile, use_tc(d) ? 3 : 0, w.capacity, w.items, w.count, w.status, st,
                                      w.tile_base));
   }
-  if (w.tile_recs) {
+  if (w.tile_recs && !(d->flags & HSTU_FLAG_REUSE_PREP)) {
     TraceScope tr("ts_tiles", st);
     HSTU_CUDA(launch_ts_tiles(jb->seq_offsets, jb->timestamps, jb->batch, w.tile_base, w.tiles_cap, w.tile_recs, st));
   }
@@ -283,14 +286,19 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
   const int H = d->num_heads, dh = d->dqk;
   const bool tc = use_tc_bwd(d);
   const Thresholds thr = thresholds_for(d->time_div);
-  {
+  const bool reuse = (d->flags & HSTU_FLAG_REUSE_PREP) != 0;
+  if (reuse) {
+    // work list and tile records from an earlier call: only the fetch cursor restarts
+    HSTU_CUDA(cudaMemsetAsync(w.count + 1, 0, sizeof(int32_t), st));
+  } else {
     TraceScope tr("sched_bwd", st);
     HSTU_CUDA(launch_build_work_list(jb->seq_offsets, jb->num_targets, jb->batch, jb->total_tokens, H, tile, tile, 1,
                                      w.capacity, w.items, w.count, w.status, st, tc ? w.tile_base : nullptr));
   }
   if (tc) {
     TraceScope tr("bwd_prep", st);
-    HSTU_CUDA(launch_ts_tiles(jb->seq_offsets, jb->timestamps, jb->batch, w.tile_base, w.tiles_cap, w.tile_recs, st));
+    if (!reuse)
+      HSTU_CUDA(launch_ts_tiles(jb->seq_offsets, jb->timestamps, jb->batch, w.tile_base, w.tiles_cap, w.tile_recs, st));
     if (w.band)
       HSTU_CUDA(launch_bwd_band(jb->seq_offsets, jb->num_targets, jb->timestamps, jb->batch, jb->total_tokens,
                                 w.tile_base, w.tiles_cap, pos_bias, time_bias, thr, d->time_div, w.status,
@@ -882,6 +890,9 @@ int hstu_layer_fwd_host(const hstu_layer_desc* desc, const hstu_layer_weights* w
     }
     HSTU_CUDA(cudaEventRecord(cs->in[ch], cs->h2d));
   }
+  // every chunk is a batch of its own: its preparation is built, never reused
+  hstu_layer_desc dc = *desc;
+  dc.attn.flags &= ~HSTU_FLAG_REUSE_PREP;
   for (int ch = 0; ch < nc; ++ch) {
     const int s0 = bounds[ch], nb = bounds[ch + 1] - s0;
     const int r0 = seq_offsets[s0], r1 = seq_offsets[s0 + nb];
@@ -894,7 +905,7 @@ int hstu_layer_fwd_host(const hstu_layer_desc* desc, const hstu_layer_weights* w
     jb.seq_offsets = co;
     jb.num_targets = num_targets ? ws.nt + s0 : nullptr;
     jb.timestamps = ws.ts + r0;
-    HSTU_TRY(run_layer_fwd(desc, w, &jb, (const char*)ws.x + r0 * row_bytes, (char*)ws.y + r0 * row_bytes, nullptr,
+    HSTU_TRY(run_layer_fwd(&dc, w, &jb, (const char*)ws.x + r0 * row_bytes, (char*)ws.y + r0 * row_bytes, nullptr,
                            ws.layer, st));
     HSTU_CUDA(cudaEventRecord(cs->out[ch], st));
     HSTU_CUDA(cudaStreamWaitEvent(cs->d2h, cs->out[ch], 0));
@@ -1134,10 +1145,13 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
                                          cand_ts, dm, dt, 1, w.x0, w.ts, nullptr, w.cand_dst, st));
       void* xs = w.x0;
       void* ys = w.x1;
+      // the layers after the first reuse the first one's work list and tile records
+      hstu_layer_desc dl = *desc;
       for (int l = 0; l < num_layers; ++l) {
         LayerFwdWs lw = w.layer;
         lw.b.uvqk = w.uvqk_cache + (size_t)l * w.uvqk_stride;
-        HSTU_TRY(run_layer_fwd(desc, &layers[l], &jb, xs, ys, nullptr, lw, st));
+        dl.attn.flags = l == 0 ? (desc->attn.flags & ~HSTU_FLAG_REUSE_PREP) : (desc->attn.flags | HSTU_FLAG_REUSE_PREP);
+        HSTU_TRY(run_layer_fwd(&dl, &layers[l], &jb, xs, ys, nullptr, lw, st));
         void* t = xs; xs = ys; ys = t;
       }
       // the candidates' final rows, compact

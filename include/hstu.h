@@ -87,6 +87,15 @@ extern "C" {
  * (saved == NULL); otherwise the flag is ignored.  A sequence longer than 128
  * tokens (or outside the buffers) is not computed and sets HSTU_ERR_BAD_OFFSETS
  * in the workspace status word. */
+#define HSTU_FLAG_REUSE_PREP 4
+/* hstu_layer_fwd / hstu_layer_bwd / hstu_attn_fwd / hstu_attn_bwd: the workspace
+ * still holds the attention's work list and timestamp tile records from an
+ * earlier call of the same entry point on the same jagged batch (the same
+ * seq_offsets, num_targets and timestamps, contents and sizes) and the same head
+ * count; they are not rebuilt (the layers of a stack share them within a step).
+ * The relative-bias band, which depends on the bias tables, is rebuilt.  Offsets
+ * that the earlier call found invalid stay without work, and only that call
+ * reported them. */
 /* seq_offsets and num_targets are always checked on the device by the
  * scheduler kernel that precedes every attention launch; a violation writes
  * HSTU_ERR_BAD_OFFSETS to the workspace status word and schedules no work. */

@@ -309,10 +309,12 @@ def _sl_workload(wl):
     return g, offs
 
 
-def _train_step(wl, residual_fp32: bool):
+def _train_step(wl, residual_fp32: bool, share_prep: bool = False):
     """SL on the GPU, forward through the stack saving activations, backward
     from dY = G.  Returns the GPU's per-layer inputs x_l, upstream gradients
-    dy_l, gradients, and the SL-selected host arrays."""
+    dy_l, gradients, and the SL-selected host arrays.  share_prep: the layers
+    share one workspace per entry point and all but the first forward and the
+    first backward reuse the attention preparation (HSTU_FLAG_REUSE_PREP)."""
     b = _b()
     s = wl.spec
     td = torch.bfloat16
@@ -326,19 +328,21 @@ def _train_step(wl, residual_fp32: bool):
     x = b.gather_rows(dev(wl.x, io), idx_d, count, torch.empty(T2, s.d_model, dtype=io, device="cuda"))
     ts = b.gather_rows(dev(wl.timestamps), idx_d, count, torch.empty(T2, dtype=torch.int64, device="cuda"))
     gy = b.gather_rows(dev(e["grad_out"], io), idx_d, count, torch.empty(T2, s.d_model, dtype=io, device="cuda"))
-    layers = [b.Layer(layer_to_dev(p, td), s.d_model, s.num_heads, s.head_dim, residual_fp32=residual_fp32)
-              for p in wl.layers]
+    pool = {} if share_prep else None
+    layers = [b.Layer(layer_to_dev(p, td), s.d_model, s.num_heads, s.head_dim, residual_fp32=residual_fp32,
+                      workspaces=pool) for p in wl.layers]
     hv = s.num_heads * s.head_dim
     saved = [b.Saved.alloc(T2, s.d_model, hv, td, "cuda") for _ in layers]
     xs = [x]
-    for ly, sv in zip(layers, saved):
-        xs.append(ly.forward(xs[-1], offs_d, ts, saved=sv))
+    for li, (ly, sv) in enumerate(zip(layers, saved)):
+        xs.append(ly.forward(xs[-1], offs_d, ts, saved=sv, reuse_prep=share_prep and li > 0))
     dys = [None] * len(layers)
     grads = [None] * len(layers)
     dy = gy
     for li in range(len(layers) - 1, -1, -1):
         dys[li] = dy
-        dy, grads[li] = layers[li].backward(xs[li], dy, saved[li], offs_d, ts)
+        dy, grads[li] = layers[li].backward(xs[li], dy, saved[li], offs_d, ts,
+                                            reuse_prep=share_prep and li < len(layers) - 1)
     torch.cuda.synchronize()
     host = lambda t: t.float().cpu().numpy().astype(np.float64)
     return dict(xs=[host(t) for t in xs[:-1]], dys=[host(t) for t in dys], dx=host(dy), grads=grads, T=T2, hv=hv,
@@ -445,7 +449,8 @@ def test_training_step_config4_per_layer_parameter_gradients_only():
         assert_close(dx, ref[li]["dx"], "bf16", f"layer {li} dx", grad=True)
 
 
-def test_training_step_config4_chained_within_rounding_model():
+@pytest.mark.parametrize("share_prep", [False, True])
+def test_training_step_config4_chained_within_rounding_model(share_prep):
     """The whole 8-layer step from X and G (SL on the GPU, the stack's forward,
     then its backward), against the oracle's whole-stack gradients.  Rounding
     x-hat and U, V, Q, K to bf16 for the tensor cores alone moves these
@@ -455,7 +460,7 @@ def test_training_step_config4_chained_within_rounding_model():
     most 1.25 times the model's worst relative Frobenius error."""
     import tests.precision_model as M
     wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
-    run = _train_step(wl, residual_fp32=True)
+    run = _train_step(wl, residual_fp32=True, share_prep=share_prep)
     s = wl.spec
     T, hv = run["T"], run["hv"]
     chained = O.stack_backward(run["x0"], wl.layers, run["g0"], run["offs"], run["ts"], s.num_heads, s.head_dim)
@@ -472,6 +477,24 @@ def test_training_step_config4_chained_within_rounding_model():
             worst_model = max(worst_model, errors(model[li][name], chained[li][name])[1])
     print(f"chained worst rel-fro: GPU {worst_gpu:.3e}, rounding model {worst_model:.3e}")
     assert worst_gpu <= 1.25 * worst_model, f"chained {worst_gpu:.3e} > 1.25 x model {worst_model:.3e}"
+
+
+def test_training_step_shared_preparation_forward_identical():
+    """The 8-layer step with one workspace per entry point shared by the layers,
+    every layer after the first forward reusing the attention preparation: every
+    layer's activations bit-identical to those with separate workspaces, and the
+    last layer's gradients (the first backward, which builds its preparation)
+    equal up to the order of the atomic fp32 additions.  (The reusing backwards
+    are checked against the oracle by the chained test.)"""
+    wl = W.make_workload(4, batch=6, scale=1 / 8, random_affine=True)
+    a = _train_step(wl, residual_fp32=True)
+    b_ = _train_step(wl, residual_fp32=True, share_prep=True)
+    L = len(wl.layers)
+    for li in range(L):
+        assert np.array_equal(a["xs"][li], b_["xs"][li]), f"layer {li} input"
+    for name in ("w1", "w2", "b1", "b2", "pos_bias", "time_bias", "ln1_gamma", "ln2_gamma", "uvqk"):
+        x, y = a["grads"][L - 1][name].float().cpu().numpy(), b_["grads"][L - 1][name].float().cpu().numpy()
+        assert np.linalg.norm(x - y) <= 1e-4 * np.linalg.norm(x) + 1e-12, name
 
 
 def test_training_config4_full_size_one_layer():

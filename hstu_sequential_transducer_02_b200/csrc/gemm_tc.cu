@@ -38,7 +38,8 @@ struct GCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = BN == 256 ? 4 : 6;
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kAlloc = kBarOff + 256 + 1024;
+  static constexpr int kXpose = kBarOff + 256;                  // per epilogue warp: a 32 x 64-byte transpose tile
+  static constexpr int kAlloc = kXpose + kEpiWarps * 2048 + 1024;
   static constexpr uint32_t kTmemCols = 2 * BN <= 32 ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
 };
 
@@ -86,6 +87,105 @@ __device__ __forceinline__ float silu_fast(float v) {
 }
 
 // One thread's 32 consecutive accumulator columns [n0, n0+32) of row m -> output.
+// A warp's 32 rows x 32 bf16 columns (64 bytes a row, one row per lane in w) to
+// global memory through its shared-memory tile: every store instruction then
+// writes 8 whole 64-byte row pieces (4 lanes a row) instead of 32 scattered
+// 16-byte pieces.  The tile's 16-byte chunks are XOR-swizzled by row so that
+// both the row-wise writes and the transposed reads are free of bank conflicts.
+// (base: the first of the 64 bytes of row m_first; ld_bytes: the row stride)
+__device__ __forceinline__ void store_rows_xpose(uint4* tile, const uint4 (&w)[4], char* base, int64_t ld_bytes,
+                                                 int m_first, int m_end, int lane) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tile[lane * 4 + (k ^ ((lane >> 1) & 3))] = w[k];
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int r = 8 * j + (lane >> 2), pc = lane & 3;
+    const uint4 v = tile[r * 4 + (pc ^ ((r >> 1) & 3))];
+    if (m_first + r < m_end) *reinterpret_cast<uint4*>(base + (int64_t)r * ld_bytes + 16 * pc) = v;
+  }
+  __syncwarp();
+}
+// the reverse: 64 bytes of each of the warp's 32 rows into the row's lane (zero
+// beyond m_end), read 8 whole row pieces per load instruction
+__device__ __forceinline__ void load_rows_xpose(uint4* tile, uint4 (&w)[4], const char* base, int64_t ld_bytes,
+                                                int m_first, int m_end, int lane) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int r = 8 * j + (lane >> 2), pc = lane & 3;
+    tile[r * 4 + (pc ^ ((r >> 1) & 3))] = m_first + r < m_end
+        ? *reinterpret_cast<const uint4*>(base + (int64_t)r * ld_bytes + 16 * pc) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w[k] = tile[lane * 4 + (k ^ ((lane >> 1) & 3))];
+  __syncwarp();
+}
+__device__ __forceinline__ void pack8_bf16(const float* v, uint4& w) {
+  w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
+  w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
+}
+
+// The EPI_BIAS_RESIDUAL / EPI_STORE outputs of a warp's 32 rows x 32 columns (full,
+// no split, no accumulate) through the warp's transpose tile: the residual read
+// and the output written 8 whole row pieces per instruction.
+__device__ __forceinline__ void epilogue_chunk_xpose(const TcGemmParams& tp, uint4* tile, int m_first, int m_end,
+                                                     int n0, const uint32_t (&raw)[32], bool has_k, int lane) {
+  const GemmParams& p = tp.p;
+  float v[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] = has_k ? __uint_as_float(raw[e]) : 0.f;
+  if (p.epi == EPI_BIAS_RESIDUAL && p.bias) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + n0 + e));
+      v[e] += b.x; v[e + 1] += b.y; v[e + 2] += b.z; v[e + 3] += b.w;
+    }
+  }
+  if (p.epi == EPI_BIAS_RESIDUAL && p.residual) {
+    if (tp.res_f32) {
+      const char* rb = (const char*)((const float*)p.residual + (int64_t)m_first * p.ldr + n0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {   // 16 fp32 columns = 64 bytes at a time
+        uint4 w[4];
+        load_rows_xpose(tile, w, rb + 64 * h, p.ldr * 4, m_first, m_end, lane);
+        const float* f = reinterpret_cast<const float*>(w);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[16 * h + e] += f[e];
+      }
+    } else {
+      uint4 w[4];
+      load_rows_xpose(tile, w, (const char*)((const __nv_bfloat16*)p.residual + (int64_t)m_first * p.ldr + n0),
+                      p.ldr * 2, m_first, m_end, lane);
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(w);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float2 f = __bfloat1622float2(h[q]);
+        v[2 * q] += f.x;
+        v[2 * q + 1] += f.y;
+      }
+    }
+  }
+  if (tp.out_f32 || p.epi == EPI_STORE_F32) {
+    char* ob = (char*)((float*)p.out + (int64_t)m_first * p.ldo + n0);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint4 w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        w[k] = make_uint4(__float_as_uint(v[16 * h + 4 * k]), __float_as_uint(v[16 * h + 4 * k + 1]),
+                          __float_as_uint(v[16 * h + 4 * k + 2]), __float_as_uint(v[16 * h + 4 * k + 3]));
+      store_rows_xpose(tile, w, ob + 64 * h, p.ldo * 4, m_first, m_end, lane);
+    }
+  } else {
+    uint4 w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pack8_bf16(v + 8 * k, w[k]);
+    store_rows_xpose(tile, w, (char*)((__nv_bfloat16*)p.out + (int64_t)m_first * p.ldo + n0), p.ldo * 2, m_first,
+                     m_end, lane);
+  }
+}
+
 __device__ __forceinline__ void epilogue_chunk(const TcGemmParams& tp, int m, int n0, const uint32_t (&raw)[32],
                                                bool has_k) {
   const GemmParams& p = tp.p;
@@ -114,7 +214,7 @@ __device__ __forceinline__ void epilogue_chunk(const TcGemmParams& tp, int m, in
     }
     return;
   }
-  if ((p.epi == EPI_BIAS_SILU || p.epi == EPI_BIAS_RESIDUAL) && p.bias) {
+  if (p.epi == EPI_BIAS_RESIDUAL && p.bias) {
     if (full32) {
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
@@ -124,26 +224,6 @@ __device__ __forceinline__ void epilogue_chunk(const TcGemmParams& tp, int m, in
     } else {
       for (int e = 0; e < 32 && n0 + e < p.N; ++e) v[e] += p.bias[n0 + e];
     }
-  }
-  if (p.epi == EPI_BIAS_SILU) {
-    __nv_bfloat16* o = (__nv_bfloat16*)p.out + (int64_t)m * p.ldo + n0;
-    __nv_bfloat16* z = p.out2 ? (__nv_bfloat16*)p.out2 + (int64_t)m * p.ldo2 + n0 : nullptr;
-#pragma unroll
-    for (int e = 0; e < 32; e += 8) {  // N % 32 == 0 on this path
-      if (z) {
-        uint4 w;
-        w.x = pack_bf16x2(v[e], v[e + 1]); w.y = pack_bf16x2(v[e + 2], v[e + 3]);
-        w.z = pack_bf16x2(v[e + 4], v[e + 5]); w.w = pack_bf16x2(v[e + 6], v[e + 7]);
-        *reinterpret_cast<uint4*>(z + e) = w;
-      }
-      uint4 w;
-      w.x = pack_bf16x2(silu_fast(v[e]), silu_fast(v[e + 1]));
-      w.y = pack_bf16x2(silu_fast(v[e + 2]), silu_fast(v[e + 3]));
-      w.z = pack_bf16x2(silu_fast(v[e + 4]), silu_fast(v[e + 5]));
-      w.w = pack_bf16x2(silu_fast(v[e + 6]), silu_fast(v[e + 7]));
-      *reinterpret_cast<uint4*>(o + e) = w;
-    }
-    return;
   }
   if (p.epi == EPI_BIAS_RESIDUAL && p.residual) {
     if (tp.res_f32) {
@@ -306,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;          // TMEM lane quarter this warp may access
     const int group = (warp - 2) >> 2;     // quarter of the tile's columns
+    uint4* const xtile = reinterpret_cast<uint4*>(smem + C::kXpose) + (warp - 2) * 128;   // 2 KB
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     constexpr int kCols = BN / 4;
@@ -326,7 +407,50 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         tmem_ld_32x32b_x32(tmem_base + ab * BN + lane_off + c, raw);
         tmem_ld_wait();
         const int n0 = un.n0 + c;
-        if (row_ok && n0 < p.N) epilogue_chunk(tp, m, n0, raw, has_k);
+        if (p.epi == EPI_BIAS_SILU) {
+          // (N % 32 == 0 on this path) bias, z = pre-activation and U|V|Q|K = SiLU(z) as bf16,
+          // stored through the warp's transpose tile
+          if (n0 < p.N) {
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 b = p.bias ? __ldg(reinterpret_cast<const float4*>(p.bias + n0 + e))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+              v[e] = (has_k ? __uint_as_float(raw[e]) : 0.f) + b.x;
+              v[e + 1] = (has_k ? __uint_as_float(raw[e + 1]) : 0.f) + b.y;
+              v[e + 2] = (has_k ? __uint_as_float(raw[e + 2]) : 0.f) + b.z;
+              v[e + 3] = (has_k ? __uint_as_float(raw[e + 3]) : 0.f) + b.w;
+            }
+            const int m_first = un.m0 + quarter * 32;
+            uint4 w[4];
+            if (p.out2) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int e = 8 * k;
+                w[k].x = pack_bf16x2(v[e], v[e + 1]); w[k].y = pack_bf16x2(v[e + 2], v[e + 3]);
+                w[k].z = pack_bf16x2(v[e + 4], v[e + 5]); w[k].w = pack_bf16x2(v[e + 6], v[e + 7]);
+              }
+              store_rows_xpose(xtile, w, (char*)((__nv_bfloat16*)p.out2 + (int64_t)m_first * p.ldo2 + n0),
+                               p.ldo2 * 2, m_first, M_eff, lane);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 8 * k;
+              w[k].x = pack_bf16x2(silu_fast(v[e]), silu_fast(v[e + 1]));
+              w[k].y = pack_bf16x2(silu_fast(v[e + 2]), silu_fast(v[e + 3]));
+              w[k].z = pack_bf16x2(silu_fast(v[e + 4]), silu_fast(v[e + 5]));
+              w[k].w = pack_bf16x2(silu_fast(v[e + 6]), silu_fast(v[e + 7]));
+            }
+            store_rows_xpose(xtile, w, (char*)((__nv_bfloat16*)p.out + (int64_t)m_first * p.ldo + n0), p.ldo * 2,
+                             m_first, M_eff, lane);
+          }
+        } else if ((p.epi == EPI_BIAS_RESIDUAL || p.epi == EPI_STORE ||
+                    (p.epi == EPI_STORE_F32 && tp.split == 1 && !p.accumulate)) && n0 + 32 <= p.N) {
+          // whole 32-column chunks: the rows through the warp's transpose tile
+          epilogue_chunk_xpose(tp, xtile, un.m0 + quarter * 32, M_eff, n0, raw, has_k, lane);
+        } else if (row_ok && n0 < p.N) {
+          epilogue_chunk(tp, m, n0, raw, has_k);
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -106,29 +106,14 @@ __device__ __forceinline__ void store_rows_xpose(uint4* tile, const uint4 (&w)[4
   }
   __syncwarp();
 }
-// the reverse: 64 bytes of each of the warp's 32 rows into the row's lane (zero
-// beyond m_end), read 8 whole row pieces per load instruction
-__device__ __forceinline__ void load_rows_xpose(uint4* tile, uint4 (&w)[4], const char* base, int64_t ld_bytes,
-                                                int m_first, int m_end, int lane) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int r = 8 * j + (lane >> 2), pc = lane & 3;
-    tile[r * 4 + (pc ^ ((r >> 1) & 3))] = m_first + r < m_end
-        ? *reinterpret_cast<const uint4*>(base + (int64_t)r * ld_bytes + 16 * pc) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  __syncwarp();
-#pragma unroll
-  for (int k = 0; k < 4; ++k) w[k] = tile[lane * 4 + (k ^ ((lane >> 1) & 3))];
-  __syncwarp();
-}
 __device__ __forceinline__ void pack8_bf16(const float* v, uint4& w) {
   w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
   w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
 }
 
 // The EPI_BIAS_RESIDUAL / EPI_STORE outputs of a warp's 32 rows x 32 columns (full,
-// no split, no accumulate) through the warp's transpose tile: the residual read
-// and the output written 8 whole row pieces per instruction.
+// no split, no accumulate): the output through the warp's transpose tile, 8 whole
+// row pieces per store instruction.
 __device__ __forceinline__ void epilogue_chunk_xpose(const TcGemmParams& tp, uint4* tile, int m_first, int m_end,
                                                      int n0, const uint32_t (&raw)[32], bool has_k, int lane) {
   const GemmParams& p = tp.p;
@@ -142,27 +127,28 @@ __device__ __forceinline__ void epilogue_chunk_xpose(const TcGemmParams& tp, uin
       v[e] += b.x; v[e + 1] += b.y; v[e + 2] += b.z; v[e + 3] += b.w;
     }
   }
-  if (p.epi == EPI_BIAS_RESIDUAL && p.residual) {
+  if (p.epi == EPI_BIAS_RESIDUAL && p.residual && m_first + lane < m_end) {
+    // the residual row by its own lane (all its loads in flight together)
+    const int64_t m = m_first + lane;
     if (tp.res_f32) {
-      const char* rb = (const char*)((const float*)p.residual + (int64_t)m_first * p.ldr + n0);
+      const float* rs = (const float*)p.residual + m * p.ldr + n0;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {   // 16 fp32 columns = 64 bytes at a time
-        uint4 w[4];
-        load_rows_xpose(tile, w, rb + 64 * h, p.ldr * 4, m_first, m_end, lane);
-        const float* f = reinterpret_cast<const float*>(w);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[16 * h + e] += f[e];
+      for (int e = 0; e < 32; e += 4) {
+        const float4 w = *reinterpret_cast<const float4*>(rs + e);
+        v[e] += w.x; v[e + 1] += w.y; v[e + 2] += w.z; v[e + 3] += w.w;
       }
     } else {
-      uint4 w[4];
-      load_rows_xpose(tile, w, (const char*)((const __nv_bfloat16*)p.residual + (int64_t)m_first * p.ldr + n0),
-                      p.ldr * 2, m_first, m_end, lane);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(w);
+      const __nv_bfloat16* rs = (const __nv_bfloat16*)p.residual + m * p.ldr + n0;
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float2 f = __bfloat1622float2(h[q]);
-        v[2 * q] += f.x;
-        v[2 * q + 1] += f.y;
+      for (int e = 0; e < 32; e += 8) {
+        const uint4 w = *reinterpret_cast<const uint4*>(rs + e);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h[q]);
+          v[e + 2 * q] += f.x;
+          v[e + 2 * q + 1] += f.y;
+        }
       }
     }
   }

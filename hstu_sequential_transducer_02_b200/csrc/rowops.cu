@@ -688,19 +688,18 @@ layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ 
     load8(gamma + (lane + 32 * c) * 8, g[c]);
     load8(beta + (lane + 32 * c) * 8, b[c]);
   }
-  int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
-  Raw8<T> cur[NCH];
-  if (row < rows)
+  // two rows in flight ahead of the one being normalised: the warp's rows
+  // alternate between two register buffers
+  auto fetch = [&](Raw8<T> (&r)[NCH], int row) {
+    if (row < rows)
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) cur[c].load(x + (int64_t)row * ldx + (lane + 32 * c) * 8);
-  for (; row < rows; row += stride) {
-    Raw8<T> nxt[NCH];
-    if (row + stride < rows)
-#pragma unroll
-      for (int c = 0; c < NCH; ++c) nxt[c].load(x + (int64_t)(row + stride) * ldx + (lane + 32 * c) * 8);
+      for (int c = 0; c < NCH; ++c) r[c].load(x + (int64_t)row * ldx + (lane + 32 * c) * 8);
+  };
+  auto normalise = [&](Raw8<T> (&r)[NCH], int row) {
     float v[NCH][8];
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) cur[c].get(v[c]);
+    for (int c = 0; c < NCH; ++c) r[c].get(v[c]);
+    fetch(r, row + 2 * stride);   // the buffer's next row, issued before the arithmetic
     float mean, rstd;
     row_stats<NCH>(v, eps, mean, rstd);
 #pragma unroll
@@ -714,8 +713,15 @@ layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ 
       if (mean_out) mean_out[row] = mean;
       if (rstd_out) rstd_out[row] = rstd;
     }
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) cur[c] = nxt[c];
+  };
+  int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  Raw8<T> r0[NCH], r1[NCH];
+  fetch(r0, row);
+  fetch(r1, row + stride);
+  for (; row < rows; row += 2 * stride) {
+    normalise(r0, row);
+    if (row + stride >= rows) break;
+    normalise(r1, row + stride);
   }
 }
 
@@ -773,23 +779,37 @@ ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, i
   }
 }
 
-// grid of the register-resident row kernels: a few blocks per SM, each warp
-// walking rows with a grid-sized stride
+// grid of the register-resident row kernels: the blocks that are resident at
+// once (one wave), each warp walking rows with a grid-sized stride
+int row_sms() {
+  static const int n = [] {
+    int dev = 0, c = 0;
+    cudaGetDevice(&dev);
+    return cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && c > 0 ? c : 148;
+  }();
+  return n;
+}
+template <auto K>
 int rows_grid(int rows_cap) {
+  static const int occ = [] {
+    int o = 0;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, K, kRowWarps * 32, 0) == cudaSuccess && o > 0 ? o : 1;
+  }();
   const int g = (rows_cap + kRowWarps - 1) / kRowWarps;
-  return g < 1 ? 1 : (g > 148 * 4 ? 148 * 4 : g);
+  const int cap = row_sms() * occ;
+  return g < 1 ? 1 : (g > cap ? cap : g);
 }
 
 template <typename T, typename TO>
 cudaError_t launch_ln_rows(const T* x, int64_t ldx, const float* gamma, const float* beta, float eps, TO* out,
                            int64_t ldo, float* mean, float* rstd, int rows_cap, const int32_t* rows_dev, int d,
                            cudaStream_t st) {
-  const int g = rows_grid(rows_cap), t = kRowWarps * 32;
+  const int t = kRowWarps * 32;
   switch (d / 256) {
-    case 1: layer_norm_rows<T, TO, 1><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
-    case 2: layer_norm_rows<T, TO, 2><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
-    case 3: layer_norm_rows<T, TO, 3><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
-    default: layer_norm_rows<T, TO, 4><<<g, t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    case 1: layer_norm_rows<T, TO, 1><<<rows_grid<layer_norm_rows<T, TO, 1>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    case 2: layer_norm_rows<T, TO, 2><<<rows_grid<layer_norm_rows<T, TO, 2>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    case 3: layer_norm_rows<T, TO, 3><<<rows_grid<layer_norm_rows<T, TO, 3>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    default: layer_norm_rows<T, TO, 4><<<rows_grid<layer_norm_rows<T, TO, 4>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
   }
   return cudaGetLastError();
 }
@@ -798,12 +818,12 @@ template <typename T>
 cudaError_t launch_ln_gate_rows(const T* o, int64_t ldo_in, const T* u, int64_t ldu, const float* gamma,
                                 const float* beta, float eps, T* out, int64_t ldout, float* mean, float* rstd,
                                 int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
-  const int g = rows_grid(rows_cap), t = kRowWarps * 32;
+  const int t = kRowWarps * 32;
   switch (d / 256) {
-    case 1: ln_gate_rows<T, 1><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
-    case 2: ln_gate_rows<T, 2><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
-    case 3: ln_gate_rows<T, 3><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
-    default: ln_gate_rows<T, 4><<<g, t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    case 1: ln_gate_rows<T, 1><<<rows_grid<ln_gate_rows<T, 1>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    case 2: ln_gate_rows<T, 2><<<rows_grid<ln_gate_rows<T, 2>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    case 3: ln_gate_rows<T, 3><<<rows_grid<ln_gate_rows<T, 3>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    default: ln_gate_rows<T, 4><<<rows_grid<ln_gate_rows<T, 4>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
   }
   return cudaGetLastError();
 }

@@ -675,7 +675,7 @@ __device__ __forceinline__ void row_stats(const float (&v)[NCH][8], float eps, f
 }
 
 template <typename T, typename TO, int NCH>
-__global__ void __launch_bounds__(kRowWarps * 32, 2)
+__global__ void __launch_bounds__(kRowWarps * 32, NCH > 2 ? 1 : (sizeof(T) == 2 ? 3 : 2))   // registers for two rows in flight
 layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma, const float* __restrict__ beta,
                 float eps, TO* __restrict__ out, int64_t ldo, float* __restrict__ mean_out,
                 float* __restrict__ rstd_out, int rows_cap, const int32_t* __restrict__ rows_dev) {

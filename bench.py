@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the M-FALCON and training-step measurements")
     ap.add_argument("--profile-attn-bwd", action="store_true",
                     help="for profilers: run the training workload's attention backward (1 + 3 launches) and exit")
+    ap.add_argument("--profile-mfalcon", action="store_true",
+                    help="for profilers: the M-FALCON ranking workload through mfalcon_rank (5 calls of 8 "
+                         "microbatches, 8 attention launches each) and exit")
     ap.add_argument("--profile-short", action="store_true",
                     help="for profilers: run the fused short-sequence layer on 512 sequences of at most 128 "
                          "tokens (two layers, 3 + 2 forwards) and exit")
@@ -517,6 +520,11 @@ def main():
         return
     if args.profile_attn_bwd:
         profile_attn_bwd()
+        return
+    if args.profile_mfalcon:
+        from hstu_sequential_transducer_02_b200 import binding as hb
+        r = measure_mfalcon(hb, 1)
+        print(json.dumps({"ms_per_call": r["ms_per_call"], "attention": r["attention"]}))
         return
     if args.profile_short:
         from hstu_sequential_transducer_02_b200 import binding as hb

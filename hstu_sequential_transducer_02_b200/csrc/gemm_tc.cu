@@ -381,10 +381,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       Unit un;
       if (!unit_of(tp, u, n_tiles, M_eff, K_eff, BN, un)) continue;
       const int ab = t & 1;
-      if (!mbar_wait(&bars->acc_full[ab], (t >> 1) & 1, tmo, abort_flag)) goto fail;
-      tc_fence_after();
       const int m = un.m0 + r;
       const bool row_ok = m < M_eff;
+      if (p.epi == EPI_BIAS_RESIDUAL && p.residual && row_ok && un.n0 + group * kCols < p.N) {
+        // this lane's residual row piece (kCols columns) on its way to L2 while
+        // the main loop still fills the accumulator
+        const int c0 = un.n0 + group * kCols, es = tp.res_f32 ? 4 : 2;
+        const int bytes = (p.N - c0 < kCols ? p.N - c0 : kCols) * es;   // inside the row
+        const char* rp = (const char*)p.residual + ((int64_t)m * p.ldr + c0) * es;
+#pragma unroll
+        for (int b = 0; b < kCols * 4; b += 128)
+          if (b < bytes) prefetch_l2(rp + b);
+      }
+      if (!mbar_wait(&bars->acc_full[ab], (t >> 1) & 1, tmo, abort_flag)) goto fail;
+      tc_fence_after();
       const bool has_k = un.k1 > un.k0;  // an empty K range never wrote the accumulator
 #pragma unroll 1
       for (int c = group * kCols; c < (group + 1) * kCols; c += 32) {

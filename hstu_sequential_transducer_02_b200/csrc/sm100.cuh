@@ -93,6 +93,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
 }
 
 // ---------------------------------------------------------------- TMA
+// brings the 128-byte line holding p into L2 (no register is written)
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

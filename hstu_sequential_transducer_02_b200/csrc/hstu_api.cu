@@ -489,6 +489,7 @@ struct LayerBwdWs {
   void* dz;      // [T, 4hv]
   float* dxhat;  // [T, dm] fp32
   void* dyb;     // [T, dm] dy in the activation dtype, zero-padded to a multiple of 64 rows
+  float* colpart;  // column partial sums (db2 with dy's conversion, db1 with the SiLU backward)
 };
 
 LayerBwdWs carve_layer_bwd(Carver& c, const hstu_layer_desc* d, int B, int T) {
@@ -503,6 +504,7 @@ LayerBwdWs carve_layer_bwd(Carver& c, const hstu_layer_desc* d, int B, int T) {
   w.dz = c.take<char>((size_t)T * 4 * hv * es);
   w.dxhat = c.take<float>((size_t)T * dm);
   w.dyb = c.take<char>((size_t)T * dm * es);
+  w.colpart = c.take<float>(col_partials_size(4 * hv > dm ? 4 * hv : dm));
   return w;
 }
 
@@ -525,14 +527,14 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   // device row count up to the next multiple of 64 of every token-major operand are zeroed.
   {
     TraceScope tr("bwd_prep", st);
-    HSTU_CUDA(launch_convert_rows(dy, dm, io, ws.dyb, dm, dt, dm, T, rows, 64, st));
+    HSTU_CUDA(launch_convert_rows_colsum(dy, dm, io, ws.dyb, dm, dt, dm, T, rows, 64, gr->db2, ws.colpart, st));
     HSTU_CUDA(launch_zero_tail_rows(sv->xhat, (int64_t)dm * es, (int64_t)dm * es, T, rows, 64, st));
     // recompute g = LN2(o) * U (cheaper to recompute than to keep)
     HSTU_CUDA(launch_ln_gate(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g, hv,
                              nullptr, nullptr, T, rows, hv, dt, st));
     HSTU_CUDA(launch_zero_tail_rows(ws.g, (int64_t)hv * es, (int64_t)hv * es, T, rows, 64, st));
   }
-  // y = x + g W2^T + b2:  dW2 = dy^T g, db2 = colsum(dy), dg = dy W2
+  // y = x + g W2^T + b2:  dW2 = dy^T g, dg = dy W2 (db2 = colsum(dy) came with dy's conversion)
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.M = dm; p.N = hv; p.K = T;                 // dW2[m=out, n=in] = sum_t dy[t, m] g[t, n]
@@ -540,10 +542,6 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   p.B = ws.g; p.sbn = 1; p.sbk = hv;
   p.epi = EPI_STORE_F32; p.out = gr->dw2; p.ldo = hv; p.k_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw2"));
-  {
-    TraceScope tr("colsum_db2", st);
-    HSTU_CUDA(launch_col_sum(dy, dm, T, rows, dm, io, gr->db2, st));
-  }
   memset(&p, 0, sizeof(p));
   p.M = T; p.N = hv; p.K = dm;                 // dg[t, n] = sum_m dy[t, m] W2[m, n]
   p.A = ws.dyb; p.sam = dm; p.sak = 1;
@@ -555,10 +553,9 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
     TraceScope tr("ln2_gate_bwd", st);
     HSTU_CUDA(cudaMemsetAsync(gr->dln2_gamma, 0, sizeof(float) * hv, st));
     HSTU_CUDA(cudaMemsetAsync(gr->dln2_beta, 0, sizeof(float) * hv, st));
-    HSTU_CUDA(launch_ln_gate_bwd(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, sv->ln2_mean, sv->ln2_rstd,
-                                 ws.dg, hv, ws.d_o, hv, gr->dln2_gamma, gr->dln2_beta, T, rows, hv, dt, st));
-    HSTU_CUDA(launch_ln_gate_du(sv->attn_out, hv, w->ln2_gamma, w->ln2_beta, sv->ln2_mean, sv->ln2_rstd, ws.dg, hv,
-                                duvqk, 4 * hv, T, rows, hv, dt, st));
+    HSTU_CUDA(launch_ln_gate_bwd(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, sv->ln2_mean,
+                                 sv->ln2_rstd, ws.dg, hv, ws.d_o, hv, duvqk, 4 * hv, gr->dln2_gamma,
+                                 gr->dln2_beta, T, rows, hv, dt, st));
   }
   // attention backward -> dV, dQ, dK columns of duvqk, rab grads
   const size_t rab_n = (size_t)(d->attn.rab_head_stride ? H : 1) * kNumBuckets;
@@ -569,24 +566,20 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   HSTU_TRY(run_attn_bwd(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + hv * es,
                         4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, dq_direct ? nullptr : du + 2 * hv * es, 4 * hv,
                         du + 3 * hv * es, 4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias, ws.attn, st));
-  // a = SiLU(z): dz = da * SiLU'(z)
+  // a = SiLU(z): dz = da * SiLU'(z), and in the same pass db1 = colsum(dz)
   {
     TraceScope tr("silu_bwd", st);
-    HSTU_CUDA(launch_silu_bwd(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, st,
-                              dq_direct ? ws.attn.dq_accum : nullptr, hv, 2 * hv, hv));
+    HSTU_CUDA(launch_silu_bwd_colsum(duvqk, sv->z, ws.dz, 4 * hv, T, rows, 4 * hv, dt, gr->db1, ws.colpart, st,
+                                     dq_direct ? ws.attn.dq_accum : nullptr, hv, 2 * hv, hv));
     HSTU_CUDA(launch_zero_tail_rows(ws.dz, (int64_t)4 * hv * es, (int64_t)4 * hv * es, T, rows, 64, st));
   }
-  // z = xhat W1^T + b1: dW1 = dz^T xhat, db1 = colsum(dz), dxhat = dz W1
+  // z = xhat W1^T + b1: dW1 = dz^T xhat, dxhat = dz W1
   memset(&p, 0, sizeof(p));
   p.M = 4 * hv; p.N = dm; p.K = T;
   p.A = ws.dz; p.sam = 1; p.sak = 4 * hv;
   p.B = sv->xhat; p.sbn = 1; p.sbk = dm;
   p.epi = EPI_STORE_F32; p.out = gr->dw1; p.ldo = dm; p.k_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw1"));
-  {
-    TraceScope tr("colsum_db1", st);
-    HSTU_CUDA(launch_col_sum(ws.dz, 4 * hv, T, rows, 4 * hv, dt, gr->db1, st));
-  }
   memset(&p, 0, sizeof(p));
   p.M = T; p.N = dm; p.K = 4 * hv;
   p.A = ws.dz; p.sam = 4 * hv; p.sak = 1;

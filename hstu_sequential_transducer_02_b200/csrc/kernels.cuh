@@ -194,11 +194,11 @@ cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const flo
 cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
                            const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
                            int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
-// backward of g = (LN2(o) gamma + beta) * u: writes d_o (dtype) and accumulates the
-// affine gradients (atomics; the caller zeroes them)
+// backward of g = (LN2(o) gamma + beta) * u: writes d_o and du = dg (LN2(o) gamma + beta)
+// (dtype) and accumulates the affine gradients (atomics; the caller zeroes them)
 cudaError_t launch_ln_gate_bwd(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
-                               const float* mean, const float* rstd, const void* dg, int64_t lddg,
-                               void* d_o, int64_t ld_do, float* dgamma, float* dbeta,
+                               const float* beta, const float* mean, const float* rstd, const void* dg, int64_t lddg,
+                               void* d_o, int64_t ld_do, void* du, int64_t lddu, float* dgamma, float* dbeta,
                                int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
 // du = dg * (LN2(o) gamma + beta)
 cudaError_t launch_ln_gate_du(const void* o, int64_t ldo_in, const float* gamma, const float* beta,
@@ -223,6 +223,19 @@ cudaError_t launch_zero_tail_rows(void* buf, int64_t ld_bytes, int64_t row_bytes
 cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
                             const int32_t* rows_dev, int cols, int dtype, cudaStream_t st, const float* dq = nullptr,
                             int64_t ldq = 0, int q_col0 = 0, int q_cols = 0);
+// floats of scratch the column-sum passes below need for `cols` columns
+size_t col_partials_size(int cols);
+// launch_silu_bwd and, in the same pass, col_sums = the column sums of dz as stored
+// (overwritten); part: col_partials_size(cols) floats of scratch
+cudaError_t launch_silu_bwd_colsum(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
+                                   const int32_t* rows_dev, int cols, int dtype, float* col_sums, float* part,
+                                   cudaStream_t st, const float* dq = nullptr, int64_t ldq = 0, int q_col0 = 0,
+                                   int q_cols = 0);
+// launch_convert_rows and, in the same pass, col_sums = the column sums of src's
+// rows < *rows_dev (overwritten); part: col_partials_size(cols) floats of scratch
+cudaError_t launch_convert_rows_colsum(const void* src, int64_t lds, int src_dtype, void* dst, int64_t ldd,
+                                       int dst_dtype, int cols, int rows_cap, const int32_t* rows_dev,
+                                       int pad_multiple, float* col_sums, float* part, cudaStream_t st);
 // column sums of a [rows, cols] dtype matrix into fp32 out (overwrite)
 cudaError_t launch_col_sum(const void* a, int64_t lda, int rows_cap, const int32_t* rows_dev, int cols,
                            int dtype, float* out, cudaStream_t st);

@@ -17,6 +17,7 @@ namespace {
 
 constexpr int kRowWarps = 8;          // warps (rows) per block
 constexpr int kMaxChunks = 4;         // 8-element chunks per lane: d <= 32*8*4 = 1024
+constexpr int kColPartBlocks = 1024;  // row blocks of the SiLU backward's column partial sums
 
 __device__ __forceinline__ void load8(const float* p, float v[8]) {
   float4 a = *reinterpret_cast<const float4*>(p);
@@ -779,6 +780,275 @@ ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, i
   }
 }
 
+// per-block column partials of dgamma/dbeta for d = 256 * NCH: summed through
+// shared memory (stored column-chunk-minor, so a warp's 32 lanes hit 32 banks),
+// then one atomic per column per block
+template <int NCH>
+__device__ __forceinline__ void flush_affine_grads_n(const float (&pg)[NCH][8], const float (&pb)[NCH][8],
+                                                     float* dgamma, float* dbeta, float* red /* [2][256 NCH] */) {
+  constexpr int D = 256 * NCH, NC = 32 * NCH;   // columns, 8-column chunks
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 2 * D; i += blockDim.x) red[i] = 0.f;
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      atomicAdd(&red[e * NC + lane + 32 * c], pg[c][e]);
+      atomicAdd(&red[D + e * NC + lane + 32 * c], pb[c][e]);
+    }
+  __syncthreads();
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    const int k = (i & 7) * NC + (i >> 3);   // column i = chunk (i / 8), element (i % 8)
+    if (dgamma) atomicAdd(&dgamma[i], red[k]);
+    if (dbeta) atomicAdd(&dbeta[i], red[D + k]);
+  }
+}
+
+// LayerNorm1 backward for d = 256 * NCH: dx = dres + rstd (dxh gamma - mean(dxh gamma)
+// - xhat mean(dxh gamma xhat)) with the dgamma/dbeta partials.  A warp takes a row
+// at a time and loads its three inputs (x, dxhat, dres) before any arithmetic, so
+// they are in flight together; gamma is read from L1 per row (registers go to the
+// partial sums).
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kRowWarps * 32, NCH > 2 ? 1 : 2)
+ln_bwd_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma,
+            const float* __restrict__ mean_in, const float* __restrict__ rstd_in, const float* __restrict__ dxhat,
+            int64_t lddxh, const T* __restrict__ dres, int64_t lddres, T* __restrict__ dx, int64_t lddx,
+            float* __restrict__ dgamma, float* __restrict__ dbeta, int rows_cap, const int32_t* __restrict__ rows_dev) {
+  __shared__ float red[2 * 256 * NCH];
+  constexpr int D = 256 * NCH;
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  float pg[NCH][8], pb[NCH][8];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { pg[c][e] = 0.f; pb[c][e] = 0.f; }
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    Raw8<T> xr[NCH], rr[NCH];
+    float dv[NCH][8];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      xr[c].load(x + (int64_t)row * ldx + col);
+      load8(dxhat + (int64_t)row * lddxh + col, dv[c]);
+      rr[c].load(dres + (int64_t)row * lddres + col);
+    }
+    const float mean = mean_in[row], rstd = rstd_in[row];
+    float xh[NCH][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      float g[8];
+      load8(gamma + (lane + 32 * c) * 8, g);
+      xr[c].get(xh[c]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        xh[c][e] = (xh[c][e] - mean) * rstd;
+        pg[c][e] += dv[c][e] * xh[c][e];
+        pb[c][e] += dv[c][e];
+        dv[c][e] *= g[e];
+        s1 += dv[c][e];
+        s2 += dv[c][e] * xh[c][e];
+      }
+    }
+    s1 = warp_sum(s1) / D;
+    s2 = warp_sum(s2) / D;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      float r[8];
+      rr[c].get(r);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[e] += rstd * (dv[c][e] - s1 - xh[c][e] * s2);
+      store8(dx + (int64_t)row * lddx + (lane + 32 * c) * 8, r);
+    }
+  }
+  flush_affine_grads_n<NCH>(pg, pb, dgamma, dbeta, red);
+}
+
+// Backward of g = (LN2(o) gamma + beta) * u for d = 256 * NCH in one pass: d_o,
+// du = dg (LN2(o) gamma + beta) and the dgamma/dbeta partials.  A warp loads a
+// row's o, u and dg before any arithmetic; gamma and beta are read from L1.
+template <typename T, int NCH>
+__global__ void __launch_bounds__(kRowWarps * 32, NCH > 2 ? 1 : 2)
+ln_gate_bwd_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
+                 const float* __restrict__ gamma, const float* __restrict__ beta, const float* __restrict__ mean_in,
+                 const float* __restrict__ rstd_in, const T* __restrict__ dg, int64_t lddg, T* __restrict__ d_o,
+                 int64_t ld_do, T* __restrict__ du, int64_t lddu, float* __restrict__ dgamma,
+                 float* __restrict__ dbeta, int rows_cap, const int32_t* __restrict__ rows_dev) {
+  __shared__ float red[2 * 256 * NCH];
+  constexpr int D = 256 * NCH;
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int lane = threadIdx.x & 31;
+  float pg[NCH][8], pb[NCH][8];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { pg[c][e] = 0.f; pb[c][e] = 0.f; }
+  for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    Raw8<T> orw[NCH], urw[NCH], grw[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      orw[c].load(o + (int64_t)row * ldo_in + col);
+      urw[c].load(u + (int64_t)row * ldu + col);
+      grw[c].load(dg + (int64_t)row * lddg + col);
+    }
+    const float mean = mean_in[row], rstd = rstd_in[row];
+    float xh[NCH][8], dxh[NCH][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int col = (lane + 32 * c) * 8;
+      float uu[8], gg[8], g[8], b[8], r[8];
+      orw[c].get(xh[c]);
+      urw[c].get(uu);
+      grw[c].get(gg);
+      load8(gamma + col, g);
+      load8(beta + col, b);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        xh[c][e] = (xh[c][e] - mean) * rstd;
+        r[e] = gg[e] * (xh[c][e] * g[e] + b[e]);
+        const float don = gg[e] * uu[e];
+        pg[c][e] += don * xh[c][e];
+        pb[c][e] += don;
+        dxh[c][e] = don * g[e];
+        s1 += dxh[c][e];
+        s2 += dxh[c][e] * xh[c][e];
+      }
+      store8(du + (int64_t)row * lddu + col, r);
+    }
+    s1 = warp_sum(s1) / D;
+    s2 = warp_sum(s2) / D;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      float r[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r[e] = rstd * (dxh[c][e] - s1 - xh[c][e] * s2);
+      store8(d_o + (int64_t)row * ld_do + (lane + 32 * c) * 8, r);
+    }
+  }
+  flush_affine_grads_n<NCH>(pg, pb, dgamma, dbeta, red);
+}
+
+// dz = da * SiLU'(z) with the column sums of dz (as stored) in one pass.  Block
+// (x, y) takes the 2048 columns [2048 y, 2048 y + 2048) (8 per thread) over the
+// x-th range of rows, two rows in flight per thread, and writes its column sums to
+// part[x][cols]; col_partials_reduce adds them up.
+template <typename T>
+__global__ void __launch_bounds__(256)
+silu_bwd_colsum_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __restrict__ dz, int64_t ld,
+                       int rows_cap, const int32_t* __restrict__ rows_dev, int cols, const float* __restrict__ dq,
+                       int64_t ldq, int q_col0, int q_cols, float* __restrict__ part) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  const int col = (blockIdx.y * 256 + threadIdx.x) * 8;
+  if (col >= cols) return;
+  const bool from_q = dq != nullptr && col >= q_col0 && col < q_col0 + q_cols;
+  const int chunk = (rows + gridDim.x - 1) / gridDim.x;
+  const int r0 = blockIdx.x * chunk, r1 = min(rows, r0 + chunk);
+  float s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s[i] = 0.f;
+  auto load_a = [&](int row, float (&a)[8]) {
+    if (from_q) load8(dq + (int64_t)row * ldq + (col - q_col0), a);
+    else load8(da + (int64_t)row * ld + col, a);
+  };
+  auto finish = [&](int row, const float (&a)[8], const float (&zz)[8]) {
+    float r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] = a[i] * silu_grad_f(zz[i]);
+    store8(dz + (int64_t)row * ld + col, r);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s[i] += Elem<T>::to_f(Elem<T>::from_f(r[i]));   // the value stored
+  };
+  int row = r0;
+  for (; row + 1 < r1; row += 2) {
+    float a0[8], z0[8], a1[8], z1[8];
+    load_a(row, a0);
+    load8(z + (int64_t)row * ld + col, z0);
+    load_a(row + 1, a1);
+    load8(z + (int64_t)(row + 1) * ld + col, z1);
+    finish(row, a0, z0);
+    finish(row + 1, a1, z1);
+  }
+  if (row < r1) {
+    float a0[8], z0[8];
+    load_a(row, a0);
+    load8(z + (int64_t)row * ld + col, z0);
+    finish(row, a0, z0);
+  }
+  float* pp = part + (int64_t)blockIdx.x * cols + col;
+  *reinterpret_cast<float4*>(pp) = make_float4(s[0], s[1], s[2], s[3]);
+  *reinterpret_cast<float4*>(pp + 4) = make_float4(s[4], s[5], s[6], s[7]);
+}
+
+// out[c] = sum over b < nb of part[b][c]: block (x, y) adds partials
+// [y nb / gridDim.y, (y + 1) nb / gridDim.y) of 256 columns; out starts at zero
+__global__ void col_partials_reduce_kernel(const float* __restrict__ part, int nb, int cols, float* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cols) return;
+  const int b0 = (int)((int64_t)nb * blockIdx.y / gridDim.y), b1 = (int)((int64_t)nb * (blockIdx.y + 1) / gridDim.y);
+  float s0 = 0.f, s1 = 0.f;
+  int b = b0;
+  for (; b + 1 < b1; b += 2) {
+    s0 += part[(int64_t)b * cols + c];
+    s1 += part[(int64_t)(b + 1) * cols + c];
+  }
+  if (b < b1) s0 += part[(int64_t)b * cols + c];
+  if (b1 > b0) atomicAdd(&out[c], s0 + s1);
+}
+
+// dst = src (converted) for rows < *rows_dev and zero up to the next multiple of
+// pad_multiple (at most rows_cap), with the column sums of src in the same pass:
+// blocks laid out as in silu_bwd_colsum_kernel, partials to part[x][cols]
+template <typename TS, typename TD>
+__global__ void __launch_bounds__(256)
+convert_rows_colsum_kernel(const TS* __restrict__ src, int64_t lds, TD* __restrict__ dst, int64_t ldd, int cols,
+                           int rows_cap, const int32_t* __restrict__ rows_dev, int pad_multiple,
+                           float* __restrict__ part) {
+  const int rows = rows_of(rows_cap, rows_dev);
+  int pad_end = ((rows + pad_multiple - 1) / pad_multiple) * pad_multiple;
+  pad_end = pad_end < rows_cap ? pad_end : rows_cap;
+  const int col = (blockIdx.y * 256 + threadIdx.x) * 8;
+  if (col >= cols) return;
+  const int chunk = (pad_end + gridDim.x - 1) / gridDim.x;
+  const int r0 = blockIdx.x * chunk, r1 = min(pad_end, r0 + chunk);
+  float s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s[i] = 0.f;
+  auto load = [&](int row, float (&v)[8]) {
+    if (row < rows) {
+      load8(src + (int64_t)row * lds + col, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+  };
+  auto finish = [&](int row, const float (&v)[8]) {
+    store8(dst + (int64_t)row * ldd + col, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s[i] += v[i];
+  };
+  int row = r0;
+  for (; row + 1 < r1; row += 2) {
+    float v0[8], v1[8];
+    load(row, v0);
+    load(row + 1, v1);
+    finish(row, v0);
+    finish(row + 1, v1);
+  }
+  if (row < r1) {
+    float v0[8];
+    load(row, v0);
+    finish(row, v0);
+  }
+  float* pp = part + (int64_t)blockIdx.x * cols + col;
+  *reinterpret_cast<float4*>(pp) = make_float4(s[0], s[1], s[2], s[3]);
+  *reinterpret_cast<float4*>(pp + 4) = make_float4(s[4], s[5], s[6], s[7]);
+}
+
 // grid of the register-resident row kernels: the blocks that are resident at
 // once (one wave), each warp walking rows with a grid-sized stride
 int row_sms() {
@@ -904,11 +1174,55 @@ cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t
   return cudaGetLastError();
 }
 
+template <typename T>
+cudaError_t launch_ln_gate_bwd_rows(const T* o, int64_t ldo_in, const T* u, int64_t ldu, const float* gamma,
+                                    const float* beta, const float* mean, const float* rstd, const T* dg,
+                                    int64_t lddg, T* d_o, int64_t ld_do, T* du, int64_t lddu, float* dgamma,
+                                    float* dbeta, int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
+  const int t = kRowWarps * 32;
+  switch (d / 256) {
+    case 1: ln_gate_bwd_rows<T, 1><<<rows_grid<ln_gate_bwd_rows<T, 1>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, mean, rstd, dg, lddg, d_o, ld_do, du, lddu, dgamma, dbeta, rows_cap, rows_dev); break;
+    case 2: ln_gate_bwd_rows<T, 2><<<rows_grid<ln_gate_bwd_rows<T, 2>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, mean, rstd, dg, lddg, d_o, ld_do, du, lddu, dgamma, dbeta, rows_cap, rows_dev); break;
+    case 3: ln_gate_bwd_rows<T, 3><<<rows_grid<ln_gate_bwd_rows<T, 3>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, mean, rstd, dg, lddg, d_o, ld_do, du, lddu, dgamma, dbeta, rows_cap, rows_dev); break;
+    default: ln_gate_bwd_rows<T, 4><<<rows_grid<ln_gate_bwd_rows<T, 4>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, mean, rstd, dg, lddg, d_o, ld_do, du, lddu, dgamma, dbeta, rows_cap, rows_dev); break;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_ln_bwd_rows(const T* x, int64_t ldx, const float* gamma, const float* mean, const float* rstd,
+                               const float* dxhat, int64_t lddxh, const T* dres, int64_t lddres, T* dx,
+                               int64_t lddx, float* dgamma, float* dbeta, int rows_cap, const int32_t* rows_dev,
+                               int d, cudaStream_t st) {
+  const int t = kRowWarps * 32;
+  switch (d / 256) {
+    case 1: ln_bwd_rows<T, 1><<<rows_grid<ln_bwd_rows<T, 1>>(rows_cap), t, 0, st>>>(x, ldx, gamma, mean, rstd, dxhat, lddxh, dres, lddres, dx, lddx, dgamma, dbeta, rows_cap, rows_dev); break;
+    case 2: ln_bwd_rows<T, 2><<<rows_grid<ln_bwd_rows<T, 2>>(rows_cap), t, 0, st>>>(x, ldx, gamma, mean, rstd, dxhat, lddxh, dres, lddres, dx, lddx, dgamma, dbeta, rows_cap, rows_dev); break;
+    case 3: ln_bwd_rows<T, 3><<<rows_grid<ln_bwd_rows<T, 3>>(rows_cap), t, 0, st>>>(x, ldx, gamma, mean, rstd, dxhat, lddxh, dres, lddres, dx, lddx, dgamma, dbeta, rows_cap, rows_dev); break;
+    default: ln_bwd_rows<T, 4><<<rows_grid<ln_bwd_rows<T, 4>>(rows_cap), t, 0, st>>>(x, ldx, gamma, mean, rstd, dxhat, lddxh, dres, lddres, dx, lddx, dgamma, dbeta, rows_cap, rows_dev); break;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ln_gate_bwd(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
-                               const float* mean, const float* rstd, const void* dg, int64_t lddg,
-                               void* d_o, int64_t ld_do, float* dgamma, float* dbeta,
+                               const float* beta, const float* mean, const float* rstd, const void* dg, int64_t lddg,
+                               void* d_o, int64_t ld_do, void* du, int64_t lddu, float* dgamma, float* dbeta,
                                int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
   if (rows_cap <= 0) return cudaSuccess;
+  const int es = dtype == HSTU_DTYPE_F32 ? 4 : 2;
+  if (fast_rows_ok(d, o, ldo_in, u, ldu, d_o, ld_do, es, es) && fast_rows_ok(d, dg, lddg, du, lddu, du, lddu, es, es)) {
+    if (dtype == HSTU_DTYPE_F32)
+      return launch_ln_gate_bwd_rows<float>((const float*)o, ldo_in, (const float*)u, ldu, gamma, beta, mean, rstd,
+                                            (const float*)dg, lddg, (float*)d_o, ld_do, (float*)du, lddu, dgamma,
+                                            dbeta, rows_cap, rows_dev, d, st);
+    using bf = __nv_bfloat16;
+    return launch_ln_gate_bwd_rows<bf>((const bf*)o, ldo_in, (const bf*)u, ldu, gamma, beta, mean, rstd,
+                                       (const bf*)dg, lddg, (bf*)d_o, ld_do, (bf*)du, lddu, dgamma, dbeta, rows_cap,
+                                       rows_dev, d, st);
+  }
+  cudaError_t e = launch_ln_gate_du(o, ldo_in, gamma, beta, mean, rstd, dg, lddg, du, lddu, rows_cap, rows_dev, d,
+                                    dtype, st);
+  if (e != cudaSuccess) return e;
   const int g = row_grid(rows_cap) < 296 ? row_grid(rows_cap) : 296;
   if (dtype == HSTU_DTYPE_F32)
     ln_gate_bwd_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)o, ldo_in, (const float*)u, ldu, gamma,
@@ -943,6 +1257,15 @@ cudaError_t launch_ln_bwd(const void* x, int64_t ldx, const float* gamma, const 
                           int64_t lddx, float* dgamma, float* dbeta, int rows_cap, const int32_t* rows_dev,
                           int d, int io_dtype, cudaStream_t st) {
   if (rows_cap <= 0) return cudaSuccess;
+  const int es = io_dtype == HSTU_DTYPE_F32 ? 4 : 2;
+  if (fast_rows_ok(d, x, ldx, dres, lddres, dx, lddx, es, es) && fast_rows_ok(d, dxhat, lddxh, nullptr, 0, dxhat, lddxh, 4, 4)) {
+    if (io_dtype == HSTU_DTYPE_F32)
+      return launch_ln_bwd_rows<float>((const float*)x, ldx, gamma, mean, rstd, dxhat, lddxh, (const float*)dres,
+                                       lddres, (float*)dx, lddx, dgamma, dbeta, rows_cap, rows_dev, d, st);
+    using bf = __nv_bfloat16;
+    return launch_ln_bwd_rows<bf>((const bf*)x, ldx, gamma, mean, rstd, dxhat, lddxh, (const bf*)dres, lddres,
+                                  (bf*)dx, lddx, dgamma, dbeta, rows_cap, rows_dev, d, st);
+  }
   const int g = row_grid(rows_cap) < 296 ? row_grid(rows_cap) : 296;
   if (io_dtype == HSTU_DTYPE_F32)
     ln_bwd_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)x, ldx, gamma, mean, rstd, dxhat, lddxh,
@@ -968,6 +1291,75 @@ cudaError_t launch_silu_bwd(const void* da, const void* z, void* dz, int64_t ld,
     silu_bwd_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16*)da, (const __nv_bfloat16*)z,
                                                       (__nv_bfloat16*)dz, ld, rows_cap, rows_dev, cols, dq, ldq,
                                                       q_col0, q_cols);
+  return cudaGetLastError();
+}
+
+size_t col_partials_size(int cols) { return (size_t)kColPartBlocks * (cols > 0 ? cols : 1); }
+
+cudaError_t launch_silu_bwd_colsum(const void* da, const void* z, void* dz, int64_t ld, int rows_cap,
+                                   const int32_t* rows_dev, int cols, int dtype, float* col_sums, float* part,
+                                   cudaStream_t st, const float* dq, int64_t ldq, int q_col0, int q_cols) {
+  cudaError_t e = cudaMemsetAsync(col_sums, 0, sizeof(float) * (cols > 0 ? cols : 0), st);
+  if (e != cudaSuccess || rows_cap <= 0 || cols <= 0) return e;
+  const int es = dtype == HSTU_DTYPE_F32 ? 4 : 2;
+  const bool vec = cols % 8 == 0 && (ld * es) % 16 == 0 && ((uintptr_t)da & 15) == 0 && ((uintptr_t)z & 15) == 0 &&
+                   ((uintptr_t)dz & 15) == 0 && ((uintptr_t)part & 15) == 0 &&
+                   (!dq || (((uintptr_t)dq & 15) == 0 && ldq % 4 == 0 && q_col0 % 8 == 0 && q_cols % 8 == 0));
+  if (!vec) {
+    e = launch_silu_bwd(da, z, dz, ld, rows_cap, rows_dev, cols, dtype, st, dq, ldq, q_col0, q_cols);
+    if (e != cudaSuccess) return e;
+    return launch_col_sum(dz, ld, rows_cap, rows_dev, cols, dtype, col_sums, st);
+  }
+  dim3 grid(1, (cols + 2047) / 2048);
+  const int bx = row_sms() * 4 / (int)grid.y;
+  grid.x = bx < 1 ? 1 : (bx > kColPartBlocks ? kColPartBlocks : bx);
+  if (grid.x > (unsigned)rows_cap) grid.x = rows_cap;
+  if (dtype == HSTU_DTYPE_F32)
+    silu_bwd_colsum_kernel<float><<<grid, 256, 0, st>>>((const float*)da, (const float*)z, (float*)dz, ld, rows_cap,
+                                                        rows_dev, cols, dq, ldq, q_col0, q_cols, part);
+  else
+    silu_bwd_colsum_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)da, (const __nv_bfloat16*)z,
+                                                                (__nv_bfloat16*)dz, ld, rows_cap, rows_dev, cols, dq,
+                                                                ldq, q_col0, q_cols, part);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, 16), 256, 0, st>>>(part, (int)grid.x, cols, col_sums);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_rows_colsum(const void* src, int64_t lds, int src_dtype, void* dst, int64_t ldd,
+                                       int dst_dtype, int cols, int rows_cap, const int32_t* rows_dev,
+                                       int pad_multiple, float* col_sums, float* part, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(col_sums, 0, sizeof(float) * (cols > 0 ? cols : 0), st);
+  if (e != cudaSuccess || rows_cap <= 0 || cols <= 0) return e;
+  const int ss = src_dtype == HSTU_DTYPE_F32 ? 4 : 2, ds = dst_dtype == HSTU_DTYPE_F32 ? 4 : 2;
+  const bool vec = cols % 8 == 0 && (lds * ss) % 16 == 0 && (ldd * ds) % 16 == 0 && ((uintptr_t)src & 15) == 0 &&
+                   ((uintptr_t)dst & 15) == 0 && ((uintptr_t)part & 15) == 0;
+  if (!vec) {
+    e = launch_convert_rows(src, lds, src_dtype, dst, ldd, dst_dtype, cols, rows_cap, rows_dev, pad_multiple, st);
+    if (e != cudaSuccess) return e;
+    return launch_col_sum(src, lds, rows_cap, rows_dev, cols, src_dtype, col_sums, st);
+  }
+  dim3 grid(1, (cols + 2047) / 2048);
+  const int bx = row_sms() * 4 / (int)grid.y;
+  grid.x = bx < 1 ? 1 : (bx > kColPartBlocks ? kColPartBlocks : bx);
+  if (grid.x > (unsigned)rows_cap) grid.x = rows_cap;
+  using bf = __nv_bfloat16;
+  if (src_dtype == HSTU_DTYPE_F32 && dst_dtype == HSTU_DTYPE_F32)
+    convert_rows_colsum_kernel<float, float><<<grid, 256, 0, st>>>((const float*)src, lds, (float*)dst, ldd, cols,
+                                                                   rows_cap, rows_dev, pad_multiple, part);
+  else if (src_dtype == HSTU_DTYPE_F32)
+    convert_rows_colsum_kernel<float, bf><<<grid, 256, 0, st>>>((const float*)src, lds, (bf*)dst, ldd, cols, rows_cap,
+                                                                rows_dev, pad_multiple, part);
+  else if (dst_dtype == HSTU_DTYPE_F32)
+    convert_rows_colsum_kernel<bf, float><<<grid, 256, 0, st>>>((const bf*)src, lds, (float*)dst, ldd, cols, rows_cap,
+                                                                rows_dev, pad_multiple, part);
+  else
+    convert_rows_colsum_kernel<bf, bf><<<grid, 256, 0, st>>>((const bf*)src, lds, (bf*)dst, ldd, cols, rows_cap,
+                                                             rows_dev, pad_multiple, part);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, 16), 256, 0, st>>>(part, (int)grid.x, cols, col_sums);
   return cudaGetLastError();
 }
 

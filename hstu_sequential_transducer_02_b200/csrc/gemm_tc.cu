@@ -182,9 +182,15 @@ __device__ __forceinline__ void epilogue_chunk(const TcGemmParams& tp, int m, in
   if (p.epi == EPI_STORE_F32) {
     float* o = (float*)p.out + (int64_t)m * p.ldo + n0;
     if (tp.split > 1) {
-      if (has_k)
-        for (int e = 0; e < 32; ++e)
-          if (n0 + e < p.N) atomicAdd(o + e, v[e]);
+      if (has_k) {
+        if (full32 && ((uintptr_t)o & 15) == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) red_add_f32x4(o + e, v[e], v[e + 1], v[e + 2], v[e + 3]);
+        } else {
+          for (int e = 0; e < 32; ++e)
+            if (n0 + e < p.N) atomicAdd(o + e, v[e]);
+        }
+      }
     } else if (full32) {
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {

@@ -93,6 +93,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, long l
 }
 
 // ---------------------------------------------------------------- TMA
+// *addr[0..3] += {a, b, c, d} as one vector reduction in L2 (addr 16-byte aligned)
+__device__ __forceinline__ void red_add_f32x4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
 // brings the 128-byte line holding p into L2 (no register is written)
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));

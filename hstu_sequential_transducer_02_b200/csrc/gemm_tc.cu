@@ -106,6 +106,23 @@ __device__ __forceinline__ void store_rows_xpose(uint4* tile, const uint4 (&w)[4
   }
   __syncwarp();
 }
+// store_rows_xpose with a destination per row: my_row is the address of this
+// lane's row (row m_first + lane) at the chunk's first column, or nullptr to drop
+// it; the storing lanes take the addresses by shuffle
+__device__ __forceinline__ void store_rows_xpose_mapped(uint4* tile, const uint4 (&w)[4], char* my_row, int lane) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) tile[lane * 4 + (k ^ ((lane >> 1) & 3))] = w[k];
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int r = 8 * j + (lane >> 2), pc = lane & 3;
+    const uint4 v = tile[r * 4 + (pc ^ ((r >> 1) & 3))];
+    char* rb = reinterpret_cast<char*>(
+        __shfl_sync(0xffffffffu, static_cast<unsigned long long>(reinterpret_cast<uintptr_t>(my_row)), r));
+    if (rb) *reinterpret_cast<uint4*>(rb + 16 * pc) = v;
+  }
+  __syncwarp();
+}
 __device__ __forceinline__ void pack8_bf16(const float* v, uint4& w) {
   w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
   w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
@@ -399,6 +416,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         for (int b = 0; b < kCols * 4; b += 128)
           if (b < bytes) prefetch_l2(rp + b);
       }
+      int64_t slot_row = -1;   // this lane's output row in the slot layout (out_slot_offs)
+      if (p.out_slot_offs && row_ok) {
+        const int64_t sr = (int64_t)p.out_slot_offs[m / p.out_slot_bm + 1] + m;
+        slot_row = sr < p.out_slot_cap ? sr : -1;
+      }
       if (!mbar_wait(&bars->acc_full[ab], (t >> 1) & 1, tmo, abort_flag)) goto fail;
       tc_fence_after();
       const bool has_k = un.k1 > un.k0;  // an empty K range never wrote the accumulator
@@ -443,8 +465,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               w[k].z = pack_bf16x2(silu_fast(v[e + 4]), silu_fast(v[e + 5]));
               w[k].w = pack_bf16x2(silu_fast(v[e + 6]), silu_fast(v[e + 7]));
             }
-            store_rows_xpose(xtile, w, (char*)((__nv_bfloat16*)p.out + (int64_t)m_first * p.ldo + n0), p.ldo * 2,
-                             m_first, M_eff, lane);
+            if (p.out_slot_offs)
+              store_rows_xpose_mapped(xtile, w,
+                                      slot_row >= 0 ? (char*)((__nv_bfloat16*)p.out + slot_row * p.ldo + n0) : nullptr,
+                                      lane);
+            else
+              store_rows_xpose(xtile, w, (char*)((__nv_bfloat16*)p.out + (int64_t)m_first * p.ldo + n0), p.ldo * 2,
+                               m_first, M_eff, lane);
           }
         } else if ((p.epi == EPI_BIAS_RESIDUAL || p.epi == EPI_STORE ||
                     (p.epi == EPI_STORE_F32 && tp.split == 1 && !p.accumulate)) && n0 + 32 <= p.N) {

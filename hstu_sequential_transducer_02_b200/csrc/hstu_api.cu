@@ -1045,8 +1045,16 @@ int run_layer_targets(const hstu_layer_desc* d, const hstu_layer_weights* w, con
   g1.epi = EPI_BIAS_SILU; g1.bias = w->b1;
   g1.out = ws.uvqk_c; g1.ldo = 4 * hv;
   g1.status = ws.layer.attn.status;
+  // on the tensor-core path f1 writes the candidates' U|V|Q|K rows straight into
+  // their slots of the cache, and LN2 * U below reads A V and U from the slots:
+  // no copies between the compact and the slot layouts
+  const bool direct = !(d->attn.flags & HSTU_FLAG_FORCE_SIMT) && tc_gemm_supported(g1, dt);
+  if (direct) {
+    g1.out = uvqk;
+    g1.out_slot_offs = hist_offsets; g1.out_slot_bm = bm; g1.out_slot_cap = ws.cap;
+  }
   HSTU_TRY(gemm(g1, dt, d->attn.flags, st, "gemm_f1_silu"));
-  {
+  if (!direct) {
     TraceScope tr("mfalcon_slot_rows", st);
     HSTU_CUDA(launch_mfalcon_slot_rows(U, bm, ws.cap, hist_offsets, ws.uvqk_c, (int64_t)4 * hv * es, uvqk,
                                        (int64_t)4 * hv * es, (int64_t)4 * hv * es, 1, st));
@@ -1055,12 +1063,16 @@ int run_layer_targets(const hstu_layer_desc* d, const hstu_layer_weights* w, con
   HSTU_CUDA(cudaMemsetAsync(ws.attn_t.count + 1, 0, sizeof(int32_t), st));
   HSTU_TRY(run_attn_main(&d->attn, slot_jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv,
                          uvqk + 1 * hv * es, 4 * hv, w->pos_bias, w->time_bias, ws.o_slot, hv, ws.attn_t, st));
-  {
-    TraceScope tr("mfalcon_slot_rows", st);
-    HSTU_CUDA(launch_mfalcon_slot_rows(U, bm, ws.cap, hist_offsets, ws.o_slot, (int64_t)hv * es, ws.o_c, (int64_t)hv * es,
-                                       (int64_t)hv * es, 0, st));
-  }
-  {
+  if (direct) {
+    TraceScope tr("ln2_gate", st);
+    HSTU_CUDA(launch_ln_gate(ws.o_slot, hv, uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g_c, hv,
+                             ws.mu2c, ws.rs2c, C, nullptr, hv, dt, st, hist_offsets, bm, ws.cap));
+  } else {
+    {
+      TraceScope tr("mfalcon_slot_rows", st);
+      HSTU_CUDA(launch_mfalcon_slot_rows(U, bm, ws.cap, hist_offsets, ws.o_slot, (int64_t)hv * es, ws.o_c,
+                                         (int64_t)hv * es, (int64_t)hv * es, 0, st));
+    }
     TraceScope tr("ln2_gate", st);
     HSTU_CUDA(launch_ln_gate(ws.o_c, hv, ws.uvqk_c, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g_c, hv,
                              ws.mu2c, ws.rs2c, C, nullptr, hv, dt, st));

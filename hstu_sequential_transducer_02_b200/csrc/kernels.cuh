@@ -179,6 +179,10 @@ struct GemmParams {
   int out_f32;               // EPI_BIAS_RESIDUAL / EPI_STORE: output is fp32 (else the operand dtype)
   int res_f32;               // EPI_BIAS_RESIDUAL: residual is fp32 (else the operand dtype)
   int32_t* status;           // device status word for bounded-wait timeouts (tensor-core path)
+  // EPI_BIAS_SILU on the tensor-core path: if set, output row m is written to row
+  // out_slot_offs[m / out_slot_bm + 1] + m of out (rows at or past out_slot_cap are
+  // dropped): the M-FALCON candidates' rows straight into their slots
+  const int32_t* out_slot_offs; int out_slot_bm, out_slot_cap;
 };
 
 cudaError_t launch_gemm_simt(const GemmParams& p, int dtype, cudaStream_t st);
@@ -191,9 +195,12 @@ cudaError_t launch_gemm_tc(const GemmParams& p, cudaStream_t st);
 cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const float* gamma, const float* beta,
                               float eps, void* out, int64_t ldo, int out_dtype, float* mean, float* rstd,
                               int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st);
+// g = LN(o) * u; with in_slot_offs, row m of o and u is read from row
+// in_slot_offs[m / in_slot_bm + 1] + m (row 0 if that reaches in_slot_cap)
 cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
                            const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
-                           int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st);
+                           int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st,
+                           const int32_t* in_slot_offs = nullptr, int in_slot_bm = 1, int in_slot_cap = 0);
 // backward of g = (LN2(o) gamma + beta) * u: writes d_o and du = dg (LN2(o) gamma + beta)
 // (dtype) and accumulates the affine gradients (atomics; the caller zeroes them)
 cudaError_t launch_ln_gate_bwd(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,

@@ -46,6 +46,17 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float v[8]) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
+// source row of row m when rows are read from the M-FALCON slot layout (see launch_ln_gate)
+struct SlotMap {
+  const int32_t* offs;
+  int bm, cap;
+};
+__device__ __forceinline__ int64_t src_row(const SlotMap& m, int row) {
+  if (!m.offs) return row;
+  const int64_t s = (int64_t)m.offs[row / m.bm + 1] + row;
+  return s < m.cap ? s : 0;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -116,18 +127,19 @@ __global__ void __launch_bounds__(kRowWarps * 32)
 ln_gate_kernel(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
                const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                T* __restrict__ out, int64_t ldout, float* __restrict__ mean_out, float* __restrict__ rstd_out,
-               int rows_cap, const int32_t* __restrict__ rows_dev, int d) {
+               int rows_cap, const int32_t* __restrict__ rows_dev, int d, SlotMap sm) {
   const int rows = rows_of(rows_cap, rows_dev);
   const int lane = threadIdx.x & 31;
   const int nch = d / 8;
   for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    const int64_t srow = src_row(sm, row);
     float v[kMaxChunks][8];
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < kMaxChunks; ++c) {
       const int ch = lane + 32 * c;
       if (ch < nch) {
-        load8(o + (int64_t)row * ldo_in + ch * 8, v[c]);
+        load8(o + srow * ldo_in + ch * 8, v[c]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) s += v[c][e];
       }
@@ -149,7 +161,7 @@ ln_gate_kernel(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u,
         float g[8], b[8], uu[8], r[8];
         load8(gamma + ch * 8, g);
         load8(beta + ch * 8, b);
-        load8(u + (int64_t)row * ldu + ch * 8, uu);
+        load8(u + srow * ldu + ch * 8, uu);
 #pragma unroll
         for (int e = 0; e < 8; ++e) r[e] = ((v[c][e] - mean) * rstd * g[e] + b[e]) * uu[e];
         store8(out + (int64_t)row * ldout + ch * 8, r);
@@ -732,7 +744,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 2)
 ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
              const float* __restrict__ gamma, const float* __restrict__ beta, float eps, T* __restrict__ out,
              int64_t ldout, float* __restrict__ mean_out, float* __restrict__ rstd_out, int rows_cap,
-             const int32_t* __restrict__ rows_dev) {
+             const int32_t* __restrict__ rows_dev, SlotMap sm) {
   const int rows = rows_of(rows_cap, rows_dev);
   const int lane = threadIdx.x & 31;
   const int stride = gridDim.x * kRowWarps;
@@ -744,20 +756,24 @@ ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, i
   }
   int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
   Raw8<T> co[NCH], cu[NCH];
-  if (row < rows)
+  if (row < rows) {
+    const int64_t sr = src_row(sm, row);
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
-      co[c].load(o + (int64_t)row * ldo_in + (lane + 32 * c) * 8);
-      cu[c].load(u + (int64_t)row * ldu + (lane + 32 * c) * 8);
+      co[c].load(o + sr * ldo_in + (lane + 32 * c) * 8);
+      cu[c].load(u + sr * ldu + (lane + 32 * c) * 8);
     }
+  }
   for (; row < rows; row += stride) {
     Raw8<T> no[NCH], nu[NCH];
-    if (row + stride < rows)
+    if (row + stride < rows) {
+      const int64_t sr = src_row(sm, row + stride);
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        no[c].load(o + (int64_t)(row + stride) * ldo_in + (lane + 32 * c) * 8);
-        nu[c].load(u + (int64_t)(row + stride) * ldu + (lane + 32 * c) * 8);
+        no[c].load(o + sr * ldo_in + (lane + 32 * c) * 8);
+        nu[c].load(u + sr * ldu + (lane + 32 * c) * 8);
       }
+    }
     float v[NCH][8];
 #pragma unroll
     for (int c = 0; c < NCH; ++c) co[c].get(v[c]);
@@ -1087,13 +1103,13 @@ cudaError_t launch_ln_rows(const T* x, int64_t ldx, const float* gamma, const fl
 template <typename T>
 cudaError_t launch_ln_gate_rows(const T* o, int64_t ldo_in, const T* u, int64_t ldu, const float* gamma,
                                 const float* beta, float eps, T* out, int64_t ldout, float* mean, float* rstd,
-                                int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
+                                int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st, SlotMap sm) {
   const int t = kRowWarps * 32;
   switch (d / 256) {
-    case 1: ln_gate_rows<T, 1><<<rows_grid<ln_gate_rows<T, 1>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
-    case 2: ln_gate_rows<T, 2><<<rows_grid<ln_gate_rows<T, 2>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
-    case 3: ln_gate_rows<T, 3><<<rows_grid<ln_gate_rows<T, 3>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
-    default: ln_gate_rows<T, 4><<<rows_grid<ln_gate_rows<T, 4>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev); break;
+    case 1: ln_gate_rows<T, 1><<<rows_grid<ln_gate_rows<T, 1>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev, sm); break;
+    case 2: ln_gate_rows<T, 2><<<rows_grid<ln_gate_rows<T, 2>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev, sm); break;
+    case 3: ln_gate_rows<T, 3><<<rows_grid<ln_gate_rows<T, 3>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev, sm); break;
+    default: ln_gate_rows<T, 4><<<rows_grid<ln_gate_rows<T, 4>>(rows_cap), t, 0, st>>>(o, ldo_in, u, ldu, gamma, beta, eps, out, ldout, mean, rstd, rows_cap, rows_dev, sm); break;
   }
   return cudaGetLastError();
 }
@@ -1152,25 +1168,28 @@ cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const flo
 
 cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,
                            const float* beta, float eps, void* out, int64_t ldout, float* mean, float* rstd,
-                           int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st) {
+                           int rows_cap, const int32_t* rows_dev, int d, int dtype, cudaStream_t st,
+                           const int32_t* in_slot_offs, int in_slot_bm, int in_slot_cap) {
   if (rows_cap <= 0) return cudaSuccess;
+  if (in_slot_offs && (in_slot_bm < 1 || in_slot_cap < 1)) return cudaErrorInvalidValue;
+  const SlotMap sm{in_slot_offs, in_slot_bm, in_slot_cap};
   const int es = dtype == HSTU_DTYPE_F32 ? 4 : 2;
   if (fast_rows_ok(d, o, ldo_in, u, ldu, out, ldout, es, es) && gamma && beta) {
     if (dtype == HSTU_DTYPE_F32)
       return launch_ln_gate_rows<float>((const float*)o, ldo_in, (const float*)u, ldu, gamma, beta, eps, (float*)out,
-                                        ldout, mean, rstd, rows_cap, rows_dev, d, st);
+                                        ldout, mean, rstd, rows_cap, rows_dev, d, st, sm);
     return launch_ln_gate_rows<__nv_bfloat16>((const __nv_bfloat16*)o, ldo_in, (const __nv_bfloat16*)u, ldu, gamma,
                                               beta, eps, (__nv_bfloat16*)out, ldout, mean, rstd, rows_cap, rows_dev,
-                                              d, st);
+                                              d, st, sm);
   }
   const int g = row_grid(rows_cap);
   if (dtype == HSTU_DTYPE_F32)
     ln_gate_kernel<float><<<g, kRowWarps * 32, 0, st>>>((const float*)o, ldo_in, (const float*)u, ldu, gamma, beta,
-                                                        eps, (float*)out, ldout, mean, rstd, rows_cap, rows_dev, d);
+                                                        eps, (float*)out, ldout, mean, rstd, rows_cap, rows_dev, d, sm);
   else
     ln_gate_kernel<__nv_bfloat16><<<g, kRowWarps * 32, 0, st>>>(
         (const __nv_bfloat16*)o, ldo_in, (const __nv_bfloat16*)u, ldu, gamma, beta, eps, (__nv_bfloat16*)out,
-        ldout, mean, rstd, rows_cap, rows_dev, d);
+        ldout, mean, rstd, rows_cap, rows_dev, d, sm);
   return cudaGetLastError();
 }
 

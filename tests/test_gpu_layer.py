@@ -536,3 +536,28 @@ def test_training_step_bf16_residual_two_layers():
         dx, gr = _gpu_layer_grads(wl, li, xs[li], dys[li], offs, ts, residual_fp32=False)
         _check_layer_grads(gr, ref[li], T, hv, f"bf16 residual layer {li}")
         assert_close(dx, ref[li]["dx"], "bf16", f"bf16 residual layer {li} dx", grad=True)
+
+
+def test_layer_backward_fp32_narrow_rows():
+    """The layer backward in fp32 on the tiny recipe (d = 64 and H dh = 64, two
+    heads of 32; random LayerNorm affines and biases): the row kernels' general
+    paths (rows narrower than 256), the CUDA-core attention backward and the
+    fused bias-gradient sums, every gradient against the oracle at the fp32 bound."""
+    b = _b()
+    wl = W.make_workload(0, random_affine=True)
+    s = wl.spec
+    td = torch.float32
+    offs, ts = wl.seq_offsets, wl.timestamps
+    T, hv = int(offs[-1]), s.num_heads * s.head_dim
+    dy = np.random.default_rng(11).standard_normal((T, s.d_model))
+    ly = b.Layer(layer_to_dev(wl.layers[0], td), s.d_model, s.num_heads, s.head_dim)
+    sv = b.Saved.alloc(T, s.d_model, hv, td, "cuda")
+    offs_d, ts_d = dev(np.asarray(offs, np.int32)), dev(ts)
+    x_d = dev(np.asarray(wl.x, np.float32), td)
+    ly.forward(x_d, offs_d, ts_d, saved=sv)
+    dx, gr = ly.backward(x_d, dev(dy.astype(np.float32), td), sv, offs_d, ts_d)
+    torch.cuda.synchronize()
+    ref = O.layer_backward(np.asarray(wl.x, np.float64), wl.layers[0], dy, offs, ts, s.num_heads, s.head_dim)
+    for name, (got, want) in _layer_errors(ref, gr, T, hv).items():
+        assert_close(got, want, "f32", f"fp32 layer backward {name}", grad=True)
+    assert_close(dx, ref["dx"], "f32", "fp32 layer backward dx", grad=True)

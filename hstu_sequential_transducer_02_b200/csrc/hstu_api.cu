@@ -278,10 +278,12 @@ int side_stream(SideStream** out) {
   return HSTU_OK;
 }
 
-int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
-                 int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias,
-                 const void* dout, int64_t lddo, void* dq, int64_t lddq, void* dk, int64_t lddk, void* dv,
-                 int64_t lddv, float* dpos, float* dtime, const AttnWs& w, cudaStream_t st) {
+// The attention backward's preparation: the work list (unless reused), the
+// timestamp records, the band of bias and bucket words and the cleared dQ
+// accumulator.  It needs only the batch and the bias tables, so the layer backward
+// runs it on the side stream next to its first GEMMs.
+int run_attn_bwd_prep(const hstu_attn_desc* d, const hstu_jagged* jb, const float* pos_bias,
+                      const float* time_bias, const AttnWs& w, cudaStream_t st) {
   const int tile = attn_bwd_tile(d);
   const int H = d->num_heads, dh = d->dqk;
   const bool tc = use_tc_bwd(d);
@@ -305,6 +307,17 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
                                 (uint32_t*)w.band, st));
   }
   HSTU_CUDA(cudaMemsetAsync(w.dq_accum, 0, sizeof(float) * (size_t)jb->total_tokens * H * dh, st));
+  return HSTU_OK;
+}
+
+// the attention backward proper, after run_attn_bwd_prep on the same workspace
+int run_attn_bwd_main(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                      int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias,
+                      const void* dout, int64_t lddo, void* dq, int64_t lddq, void* dk, int64_t lddk, void* dv,
+                      int64_t lddv, float* dpos, float* dtime, const AttnWs& w, cudaStream_t st) {
+  const int H = d->num_heads, dh = d->dqk;
+  const bool tc = use_tc_bwd(d);
+  const Thresholds thr = thresholds_for(d->time_div);
   AttnBwdParams p;
   memset(&p, 0, sizeof(p));
   p.seq_offsets = jb->seq_offsets;
@@ -348,6 +361,15 @@ int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, 
     HSTU_CUDA(launch_dq_finalize(w.dq_accum, jb->seq_offsets, jb->batch, H, dh, d->dtype, dq, lddq, 148 * 8, st));
   }
   return HSTU_OK;
+}
+
+int run_attn_bwd(const hstu_attn_desc* d, const hstu_jagged* jb, const void* q, int64_t ldq, const void* k,
+                 int64_t ldk, const void* v, int64_t ldv, const float* pos_bias, const float* time_bias,
+                 const void* dout, int64_t lddo, void* dq, int64_t lddq, void* dk, int64_t lddk, void* dv,
+                 int64_t lddv, float* dpos, float* dtime, const AttnWs& w, cudaStream_t st) {
+  HSTU_TRY(run_attn_bwd_prep(d, jb, pos_bias, time_bias, w, st));
+  return run_attn_bwd_main(d, jb, q, ldq, k, ldk, v, ldv, pos_bias, time_bias, dout, lddo, dq, lddq, dk, lddk, dv,
+                           lddv, dpos, dtime, w, st);
 }
 
 // ---------------------------------------------------------------- GEMM dispatch
@@ -523,6 +545,22 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   // without a caller buffer for dU|dV|dQ|dK, the SiLU' pass reads dQ from the
   // attention's fp32 accumulator (no conversion pass)
   const bool dq_direct = !gr->duvqk && hv % 8 == 0;
+  // the attention backward's preparation on the side stream, next to the GEMMs
+  // and row kernels before the attention (a stream being captured keeps it, as
+  // in the forward)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  HSTU_CUDA(cudaStreamIsCapturing(st, &cap));
+  SideStream* side = nullptr;
+  if (cap == cudaStreamCaptureStatusNone) {
+    std::lock_guard<std::mutex> lk(g_side_mu);
+    HSTU_TRY(side_stream(&side));
+    HSTU_CUDA(cudaEventRecord(side->fork, st));
+    HSTU_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    HSTU_TRY(run_attn_bwd_prep(&d->attn, jb, w->pos_bias, w->time_bias, ws.attn, side->s));
+    HSTU_CUDA(cudaEventRecord(side->join, side->s));
+  } else {
+    HSTU_TRY(run_attn_bwd_prep(&d->attn, jb, w->pos_bias, w->time_bias, ws.attn, st));
+  }
   // The weight-gradient products reduce over tokens in 64-row slices: rows from the
   // device row count up to the next multiple of 64 of every token-major operand are zeroed.
   {
@@ -563,9 +601,11 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   HSTU_CUDA(cudaMemsetAsync(gr->dtime_bias, 0, sizeof(float) * rab_n, st));
   const char* uvqk = (const char*)sv->uvqk;
   char* du = (char*)duvqk;
-  HSTU_TRY(run_attn_bwd(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + hv * es,
-                        4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, dq_direct ? nullptr : du + 2 * hv * es, 4 * hv,
-                        du + 3 * hv * es, 4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias, ws.attn, st));
+  if (side) HSTU_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  HSTU_TRY(run_attn_bwd_main(&d->attn, jb, uvqk + 2 * hv * es, 4 * hv, uvqk + 3 * hv * es, 4 * hv, uvqk + hv * es,
+                             4 * hv, w->pos_bias, w->time_bias, ws.d_o, hv, dq_direct ? nullptr : du + 2 * hv * es,
+                             4 * hv, du + 3 * hv * es, 4 * hv, du + hv * es, 4 * hv, gr->dpos_bias, gr->dtime_bias,
+                             ws.attn, st));
   // a = SiLU(z): dz = da * SiLU'(z), and in the same pass db1 = colsum(dz)
   {
     TraceScope tr("silu_bwd", st);

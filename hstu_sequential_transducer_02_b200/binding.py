@@ -62,7 +62,7 @@ class LayerWeights(ctypes.Structure):
 
 class LayerSaved(ctypes.Structure):
     _fields_ = [(n, _c_vp) for n in ("xhat", "ln1_mean", "ln1_rstd", "z", "uvqk", "attn_out", "ln2_mean",
-                                     "ln2_rstd")]
+                                     "ln2_rstd", "gate")]
 
 
 class LayerGrads(ctypes.Structure):
@@ -276,18 +276,20 @@ class Saved:
     attn_out: torch.Tensor
     ln2_mean: torch.Tensor
     ln2_rstd: torch.Tensor
+    gate: Optional[torch.Tensor] = None   # LN2(A V) * U; None: the backward recomputes it
 
     @staticmethod
-    def alloc(T: int, d_model: int, hv: int, dtype, device) -> "Saved":
+    def alloc(T: int, d_model: int, hv: int, dtype, device, keep_gate: bool = True) -> "Saved":
         f = dict(dtype=torch.float32, device=device)
         e = dict(dtype=dtype, device=device)
         return Saved(torch.empty(T, d_model, **e), torch.empty(T, **f), torch.empty(T, **f),
                      torch.empty(T, 4 * hv, **e), torch.empty(T, 4 * hv, **e), torch.empty(T, hv, **e),
-                     torch.empty(T, **f), torch.empty(T, **f))
+                     torch.empty(T, **f), torch.empty(T, **f), torch.empty(T, hv, **e) if keep_gate else None)
 
     def c(self) -> LayerSaved:
-        return LayerSaved(*[_ptr(getattr(self, n)) for n in ("xhat", "ln1_mean", "ln1_rstd", "z", "uvqk", "attn_out",
-                                                             "ln2_mean", "ln2_rstd")])
+        return LayerSaved(*[_ptr(getattr(self, n)) if getattr(self, n) is not None else None
+                            for n in ("xhat", "ln1_mean", "ln1_rstd", "z", "uvqk", "attn_out", "ln2_mean", "ln2_rstd",
+                                      "gate")])
 
 
 class Layer:

@@ -436,6 +436,7 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   if (saved) {
     b.xhat = saved->xhat; b.mu1 = saved->ln1_mean; b.rs1 = saved->ln1_rstd; b.z = saved->z;
     b.uvqk = saved->uvqk; b.o = saved->attn_out; b.mu2 = saved->ln2_mean; b.rs2 = saved->ln2_rstd;
+    if (saved->gate) b.g = saved->gate;
   }
   // attention preparation on the side stream, overlapping LayerNorm1 and f1.  The
   // side stream is shared by every caller on the device, so a stream that is being
@@ -481,14 +482,14 @@ int run_layer_fwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   // (A5) LayerNorm2(A V) * U
   {
     TraceScope tr("ln2_gate", st);
-    HSTU_CUDA(launch_ln_gate(b.o, hv, b.uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.b.g, hv, b.mu2,
+    HSTU_CUDA(launch_ln_gate(b.o, hv, b.uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, b.g, hv, b.mu2,
                              b.rs2, T, rows, hv, dt, st));
   }
   // (A6) f2 + residual
   GemmParams g2;
   memset(&g2, 0, sizeof(g2));
   g2.M = T; g2.N = dm; g2.K = hv;
-  g2.A = ws.b.g; g2.sam = hv; g2.sak = 1;
+  g2.A = b.g; g2.sam = hv; g2.sak = 1;
   g2.B = w->w2; g2.sbn = hv; g2.sbk = 1;
   g2.epi = EPI_BIAS_RESIDUAL; g2.bias = w->b2;
   g2.residual = x; g2.ldr = dm;
@@ -541,6 +542,7 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
   const size_t es = elem_size(dt);
   const int fl = d->attn.flags;
   void* duvqk = gr->duvqk ? gr->duvqk : ws.duvqk;
+  void* gate = sv->gate ? sv->gate : ws.g;
   int32_t* status = ws.attn.status;
   // without a caller buffer for dU|dV|dQ|dK, the SiLU' pass reads dQ from the
   // attention's fp32 accumulator (no conversion pass)
@@ -567,17 +569,18 @@ int run_layer_bwd(const hstu_layer_desc* d, const hstu_layer_weights* w, const h
     TraceScope tr("bwd_prep", st);
     HSTU_CUDA(launch_convert_rows_colsum(dy, dm, io, ws.dyb, dm, dt, dm, T, rows, 64, gr->db2, ws.colpart, st));
     HSTU_CUDA(launch_zero_tail_rows(sv->xhat, (int64_t)dm * es, (int64_t)dm * es, T, rows, 64, st));
-    // recompute g = LN2(o) * U (cheaper to recompute than to keep)
-    HSTU_CUDA(launch_ln_gate(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g, hv,
-                             nullptr, nullptr, T, rows, hv, dt, st));
-    HSTU_CUDA(launch_zero_tail_rows(ws.g, (int64_t)hv * es, (int64_t)hv * es, T, rows, 64, st));
+    // g = LN2(o) * U as the forward kept it, or recomputed
+    if (!sv->gate)
+      HSTU_CUDA(launch_ln_gate(sv->attn_out, hv, sv->uvqk, 4 * hv, w->ln2_gamma, w->ln2_beta, d->ln_eps, ws.g, hv,
+                               nullptr, nullptr, T, rows, hv, dt, st));
+    HSTU_CUDA(launch_zero_tail_rows(gate, (int64_t)hv * es, (int64_t)hv * es, T, rows, 64, st));
   }
   // y = x + g W2^T + b2:  dW2 = dy^T g, dg = dy W2 (db2 = colsum(dy) came with dy's conversion)
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.M = dm; p.N = hv; p.K = T;                 // dW2[m=out, n=in] = sum_t dy[t, m] g[t, n]
   p.A = ws.dyb; p.sam = 1; p.sak = dm;
-  p.B = ws.g; p.sbn = 1; p.sbk = hv;
+  p.B = gate; p.sbn = 1; p.sbk = hv;
   p.epi = EPI_STORE_F32; p.out = gr->dw2; p.ldo = hv; p.k_dev = rows; p.status = status;
   HSTU_TRY(gemm(p, dt, fl, st, "gemm_dw2"));
   memset(&p, 0, sizeof(p));
@@ -767,6 +770,7 @@ int hstu_layer_fwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
                         saved->attn_out, saved->ln2_mean, saved->ln2_rstd};
     for (const void* p : ps)
       if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
+    if (saved->gate && !aligned16(saved->gate)) return HSTU_ERR_INVALID_ARG;
   }
   size_t need;
   HSTU_TRY(hstu_layer_fwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
@@ -977,6 +981,7 @@ int hstu_layer_bwd(const hstu_layer_desc* desc, const hstu_layer_weights* w, con
   for (const void* p : ps)
     if (!p || !aligned16(p)) return HSTU_ERR_INVALID_ARG;
   if (g->duvqk && !aligned16(g->duvqk)) return HSTU_ERR_INVALID_ARG;
+  if (saved->gate && !aligned16(saved->gate)) return HSTU_ERR_INVALID_ARG;
   size_t need;
   HSTU_TRY(hstu_layer_bwd_workspace_size(desc, jb->batch, jb->total_tokens, &need));
   if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return HSTU_ERR_WORKSPACE;

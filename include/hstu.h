@@ -158,6 +158,8 @@ typedef struct hstu_layer_saved {
   void*  attn_out;   /* [T, H*dv] dtype: A V */
   float* ln2_mean;   /* [T] */
   float* ln2_rstd;   /* [T] */
+  void*  gate;       /* [T, H*dv] dtype: LayerNorm2(A V) * U, the input of f2; may be
+                        NULL, then the backward recomputes it from attn_out and uvqk */
 } hstu_layer_saved;
 
 /* Gradients of one layer (all device).  Weight gradients are overwritten (=). */

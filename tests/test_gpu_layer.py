@@ -542,7 +542,8 @@ def test_layer_backward_fp32_narrow_rows():
     """The layer backward in fp32 on the tiny recipe (d = 64 and H dh = 64, two
     heads of 32; random LayerNorm affines and biases): the row kernels' general
     paths (rows narrower than 256), the CUDA-core attention backward and the
-    fused bias-gradient sums, every gradient against the oracle at the fp32 bound."""
+    fused bias-gradient sums, every gradient against the oracle at the fp32 bound.
+    The forward keeps no gate here, so the backward recomputes LN2(A V) * U."""
     b = _b()
     wl = W.make_workload(0, random_affine=True)
     s = wl.spec
@@ -551,7 +552,7 @@ def test_layer_backward_fp32_narrow_rows():
     T, hv = int(offs[-1]), s.num_heads * s.head_dim
     dy = np.random.default_rng(11).standard_normal((T, s.d_model))
     ly = b.Layer(layer_to_dev(wl.layers[0], td), s.d_model, s.num_heads, s.head_dim)
-    sv = b.Saved.alloc(T, s.d_model, hv, td, "cuda")
+    sv = b.Saved.alloc(T, s.d_model, hv, td, "cuda", keep_gate=False)
     offs_d, ts_d = dev(np.asarray(offs, np.int32)), dev(ts)
     x_d = dev(np.asarray(wl.x, np.float32), td)
     ly.forward(x_d, offs_d, ts_d, saved=sv)

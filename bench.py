@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--profile-mfalcon", action="store_true",
                     help="for profilers: the M-FALCON ranking workload through mfalcon_rank (5 calls of 8 "
                          "microbatches, 8 attention launches each) and exit")
+    ap.add_argument("--profile-training", action="store_true",
+                    help="for profilers: the 8-layer training step (1 + 1 timed + 1 traced steps) and exit")
     ap.add_argument("--profile-short", action="store_true",
                     help="for profilers: run the fused short-sequence layer on 512 sequences of at most 128 "
                          "tokens (two layers, 3 + 2 forwards) and exit")
@@ -525,6 +527,11 @@ def main():
         from hstu_sequential_transducer_02_b200 import binding as hb
         r = measure_mfalcon(hb, 1)
         print(json.dumps({"ms_per_call": r["ms_per_call"], "attention": r["attention"]}))
+        return
+    if args.profile_training:
+        from hstu_sequential_transducer_02_b200 import binding as hb
+        r = measure_training(hb, 1)
+        print(json.dumps({"ms_per_step": r["ms_per_step"], "tokens_per_s": r["tokens_per_s"]}))
         return
     if args.profile_short:
         from hstu_sequential_transducer_02_b200 import binding as hb

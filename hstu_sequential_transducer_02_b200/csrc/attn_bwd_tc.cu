@@ -1021,16 +1021,27 @@ __global__ void __launch_bounds__(kBwdBandCols) bwd_band_kernel(const int32_t* _
 }
 
 // The CTAs' partial relative-bias gradients added into the caller's tables:
-// entry e of table t (t = 2 head + {0: position, 1: time}) over all CTAs.
+// entry e of table t (t = 2 head + {0: position, 1: time}) over all CTAs, the
+// CTAs split over blockIdx.y (each slice's sum added atomically)
 __global__ void rab_reduce_kernel(const float* __restrict__ part, int ctas, int tables, int head_stride,
                                   float* __restrict__ d_pos, float* __restrict__ d_time) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;   // over tables * 2 * 128
-  if (e >= tables * 2 * kNumBuckets) return;
-  float sum = 0.f;
-  for (int c = 0; c < ctas; ++c) sum += part[(size_t)c * tables * 2 * kNumBuckets + e];
+  const int n = tables * 2 * kNumBuckets;
+  if (e >= n) return;
+  const int c0 = (int)((int64_t)ctas * blockIdx.y / gridDim.y), c1 = (int)((int64_t)ctas * (blockIdx.y + 1) / gridDim.y);
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  int c = c0;
+  for (; c + 3 < c1; c += 4) {
+    s0 += part[(size_t)c * n + e];
+    s1 += part[(size_t)(c + 1) * n + e];
+    s2 += part[(size_t)(c + 2) * n + e];
+    s3 += part[(size_t)(c + 3) * n + e];
+  }
+  for (; c < c1; ++c) s0 += part[(size_t)c * n + e];
+  if (c1 <= c0) return;
   const int h = e / (2 * kNumBuckets), k = (e / kNumBuckets) & 1, b = e % kNumBuckets;
   float* dst = (k == 0 ? d_pos : d_time) + h * head_stride + b;
-  *dst += sum;
+  atomicAdd(dst, (s0 + s1) + (s2 + s3));
 }
 
 // ---------------------------------------------------------------------------
@@ -1085,7 +1096,8 @@ cudaError_t launch_bwd_band(const int32_t* offs, const int32_t* num_targets, con
 cudaError_t launch_rab_reduce(const float* part, int ctas, int tables, int head_stride, float* d_pos, float* d_time,
                               cudaStream_t st) {
   const int n = tables * 2 * kNumBuckets;
-  rab_reduce_kernel<<<(n + 255) / 256, 256, 0, st>>>(part, ctas, tables, head_stride, d_pos, d_time);
+  const int slices = ctas >= 64 ? 16 : (ctas >= 4 ? ctas / 4 : 1);   // about 4 .. 16 CTAs per thread
+  rab_reduce_kernel<<<dim3((n + 255) / 256, slices), 256, 0, st>>>(part, ctas, tables, head_stride, d_pos, d_time);
   return cudaGetLastError();
 }
 

@@ -1001,19 +1001,22 @@ silu_bwd_colsum_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __r
 }
 
 // out[c] = sum over b < nb of part[b][c]: block (x, y) adds partials
-// [y nb / gridDim.y, (y + 1) nb / gridDim.y) of 256 columns; out starts at zero
+// [y nb / gridDim.y, (y + 1) nb / gridDim.y) of 256 columns (about 8 per thread);
+// out starts at zero
 __global__ void col_partials_reduce_kernel(const float* __restrict__ part, int nb, int cols, float* __restrict__ out) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= cols) return;
   const int b0 = (int)((int64_t)nb * blockIdx.y / gridDim.y), b1 = (int)((int64_t)nb * (blockIdx.y + 1) / gridDim.y);
-  float s0 = 0.f, s1 = 0.f;
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
   int b = b0;
-  for (; b + 1 < b1; b += 2) {
+  for (; b + 3 < b1; b += 4) {
     s0 += part[(int64_t)b * cols + c];
     s1 += part[(int64_t)(b + 1) * cols + c];
+    s2 += part[(int64_t)(b + 2) * cols + c];
+    s3 += part[(int64_t)(b + 3) * cols + c];
   }
-  if (b < b1) s0 += part[(int64_t)b * cols + c];
-  if (b1 > b0) atomicAdd(&out[c], s0 + s1);
+  for (; b < b1; ++b) s0 += part[(int64_t)b * cols + c];
+  if (b1 > b0) atomicAdd(&out[c], (s0 + s1) + (s2 + s3));
 }
 
 // dst = src (converted) for rows < *rows_dev and zero up to the next multiple of
@@ -1075,6 +1078,8 @@ int row_sms() {
   }();
   return n;
 }
+// slices of the column-partial reduce: about 8 partials per thread
+int partial_slices(int nb) { return nb >= 512 ? 64 : (nb >= 8 ? nb / 8 : 1); }
 template <auto K>
 int rows_grid(int rows_cap) {
   static const int occ = [] {
@@ -1342,7 +1347,8 @@ cudaError_t launch_silu_bwd_colsum(const void* da, const void* z, void* dz, int6
                                                                 ldq, q_col0, q_cols, part);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, 16), 256, 0, st>>>(part, (int)grid.x, cols, col_sums);
+  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, partial_slices((int)grid.x)), 256, 0, st>>>(
+      part, (int)grid.x, cols, col_sums);
   return cudaGetLastError();
 }
 
@@ -1378,7 +1384,8 @@ cudaError_t launch_convert_rows_colsum(const void* src, int64_t lds, int src_dty
                                                              rows_dev, pad_multiple, part);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, 16), 256, 0, st>>>(part, (int)grid.x, cols, col_sums);
+  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, partial_slices((int)grid.x)), 256, 0, st>>>(
+      part, (int)grid.x, cols, col_sums);
   return cudaGetLastError();
 }
 

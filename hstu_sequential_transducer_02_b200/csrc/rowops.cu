@@ -949,17 +949,34 @@ ln_gate_bwd_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ 
   flush_affine_grads_n<NCH>(pg, pb, dgamma, dbeta, red);
 }
 
-// dz = da * SiLU'(z) with the column sums of dz (as stored) in one pass.  Block
-// (x, y) takes the 2048 columns [2048 y, 2048 y + 2048) (8 per thread) over the
-// x-th range of rows, two rows in flight per thread, and writes its column sums to
-// part[x][cols]; col_partials_reduce adds them up.
+// Thread layout of the column-sum passes below: a block's 256 threads take cpr =
+// min(256, cols / 8) 8-column vectors of a row and rpi = 256 / cpr rows at a time
+// (narrow matrices keep every thread busy); with 256 vectors a row, block y takes
+// the columns [2048 y, 2048 y + 2048).  Thread (sub, vector) writes its column sums
+// to partial row x rpi + sub.
+struct ColSumLayout {
+  int cpr, rpi, sub, col;
+  __host__ __device__ static int vectors(int cols) { return (cols + 7) / 8 < 256 ? (cols + 7) / 8 : 256; }
+  __device__ explicit ColSumLayout(int cols) {
+    cpr = vectors(cols);
+    rpi = 256 / cpr;
+    sub = threadIdx.x / cpr;
+    col = (blockIdx.y * 256 + threadIdx.x % cpr) * 8;
+  }
+};
+
+// dz = da * SiLU'(z) with the column sums of dz (as stored) in one pass: block x
+// takes the x-th range of rows, two rows a thread in flight (layout above), and
+// writes its column sums to the partial rows; col_partials_reduce adds them up.
 template <typename T>
 __global__ void __launch_bounds__(256)
 silu_bwd_colsum_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __restrict__ dz, int64_t ld,
                        int rows_cap, const int32_t* __restrict__ rows_dev, int cols, const float* __restrict__ dq,
                        int64_t ldq, int q_col0, int q_cols, float* __restrict__ part) {
   const int rows = rows_of(rows_cap, rows_dev);
-  const int col = (blockIdx.y * 256 + threadIdx.x) * 8;
+  const ColSumLayout L(cols);
+  if (L.sub >= L.rpi) return;
+  const int col = L.col;
   if (col >= cols) return;
   const bool from_q = dq != nullptr && col >= q_col0 && col < q_col0 + q_cols;
   const int chunk = (rows + gridDim.x - 1) / gridDim.x;
@@ -979,15 +996,15 @@ silu_bwd_colsum_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __r
 #pragma unroll
     for (int i = 0; i < 8; ++i) s[i] += Elem<T>::to_f(Elem<T>::from_f(r[i]));   // the value stored
   };
-  int row = r0;
-  for (; row + 1 < r1; row += 2) {
+  int row = r0 + L.sub;
+  for (; row + L.rpi < r1; row += 2 * L.rpi) {
     float a0[8], z0[8], a1[8], z1[8];
     load_a(row, a0);
     load8(z + (int64_t)row * ld + col, z0);
-    load_a(row + 1, a1);
-    load8(z + (int64_t)(row + 1) * ld + col, z1);
+    load_a(row + L.rpi, a1);
+    load8(z + (int64_t)(row + L.rpi) * ld + col, z1);
     finish(row, a0, z0);
-    finish(row + 1, a1, z1);
+    finish(row + L.rpi, a1, z1);
   }
   if (row < r1) {
     float a0[8], z0[8];
@@ -995,7 +1012,7 @@ silu_bwd_colsum_kernel(const T* __restrict__ da, const T* __restrict__ z, T* __r
     load8(z + (int64_t)row * ld + col, z0);
     finish(row, a0, z0);
   }
-  float* pp = part + (int64_t)blockIdx.x * cols + col;
+  float* pp = part + ((int64_t)blockIdx.x * L.rpi + L.sub) * cols + col;
   *reinterpret_cast<float4*>(pp) = make_float4(s[0], s[1], s[2], s[3]);
   *reinterpret_cast<float4*>(pp + 4) = make_float4(s[4], s[5], s[6], s[7]);
 }
@@ -1021,7 +1038,7 @@ __global__ void col_partials_reduce_kernel(const float* __restrict__ part, int n
 
 // dst = src (converted) for rows < *rows_dev and zero up to the next multiple of
 // pad_multiple (at most rows_cap), with the column sums of src in the same pass:
-// blocks laid out as in silu_bwd_colsum_kernel, partials to part[x][cols]
+// blocks laid out as in silu_bwd_colsum_kernel
 template <typename TS, typename TD>
 __global__ void __launch_bounds__(256)
 convert_rows_colsum_kernel(const TS* __restrict__ src, int64_t lds, TD* __restrict__ dst, int64_t ldd, int cols,
@@ -1030,7 +1047,9 @@ convert_rows_colsum_kernel(const TS* __restrict__ src, int64_t lds, TD* __restri
   const int rows = rows_of(rows_cap, rows_dev);
   int pad_end = ((rows + pad_multiple - 1) / pad_multiple) * pad_multiple;
   pad_end = pad_end < rows_cap ? pad_end : rows_cap;
-  const int col = (blockIdx.y * 256 + threadIdx.x) * 8;
+  const ColSumLayout L(cols);
+  if (L.sub >= L.rpi) return;
+  const int col = L.col;
   if (col >= cols) return;
   const int chunk = (pad_end + gridDim.x - 1) / gridDim.x;
   const int r0 = blockIdx.x * chunk, r1 = min(pad_end, r0 + chunk);
@@ -1050,20 +1069,20 @@ convert_rows_colsum_kernel(const TS* __restrict__ src, int64_t lds, TD* __restri
 #pragma unroll
     for (int i = 0; i < 8; ++i) s[i] += v[i];
   };
-  int row = r0;
-  for (; row + 1 < r1; row += 2) {
+  int row = r0 + L.sub;
+  for (; row + L.rpi < r1; row += 2 * L.rpi) {
     float v0[8], v1[8];
     load(row, v0);
-    load(row + 1, v1);
+    load(row + L.rpi, v1);
     finish(row, v0);
-    finish(row + 1, v1);
+    finish(row + L.rpi, v1);
   }
   if (row < r1) {
     float v0[8];
     load(row, v0);
     finish(row, v0);
   }
-  float* pp = part + (int64_t)blockIdx.x * cols + col;
+  float* pp = part + ((int64_t)blockIdx.x * L.rpi + L.sub) * cols + col;
   *reinterpret_cast<float4*>(pp) = make_float4(s[0], s[1], s[2], s[3]);
   *reinterpret_cast<float4*>(pp + 4) = make_float4(s[4], s[5], s[6], s[7]);
 }
@@ -1335,8 +1354,9 @@ cudaError_t launch_silu_bwd_colsum(const void* da, const void* z, void* dz, int6
     return launch_col_sum(dz, ld, rows_cap, rows_dev, cols, dtype, col_sums, st);
   }
   dim3 grid(1, (cols + 2047) / 2048);
+  const int rpi = 256 / ColSumLayout::vectors(cols), cap_x = kColPartBlocks / rpi;
   const int bx = row_sms() * 4 / (int)grid.y;
-  grid.x = bx < 1 ? 1 : (bx > kColPartBlocks ? kColPartBlocks : bx);
+  grid.x = bx < 1 ? 1 : (bx > cap_x ? cap_x : bx);
   if (grid.x > (unsigned)rows_cap) grid.x = rows_cap;
   if (dtype == HSTU_DTYPE_F32)
     silu_bwd_colsum_kernel<float><<<grid, 256, 0, st>>>((const float*)da, (const float*)z, (float*)dz, ld, rows_cap,
@@ -1347,8 +1367,8 @@ cudaError_t launch_silu_bwd_colsum(const void* da, const void* z, void* dz, int6
                                                                 ldq, q_col0, q_cols, part);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, partial_slices((int)grid.x)), 256, 0, st>>>(
-      part, (int)grid.x, cols, col_sums);
+  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, partial_slices((int)grid.x * rpi)), 256, 0, st>>>(
+      part, (int)grid.x * rpi, cols, col_sums);
   return cudaGetLastError();
 }
 
@@ -1366,8 +1386,9 @@ cudaError_t launch_convert_rows_colsum(const void* src, int64_t lds, int src_dty
     return launch_col_sum(src, lds, rows_cap, rows_dev, cols, src_dtype, col_sums, st);
   }
   dim3 grid(1, (cols + 2047) / 2048);
+  const int rpi = 256 / ColSumLayout::vectors(cols), cap_x = kColPartBlocks / rpi;
   const int bx = row_sms() * 4 / (int)grid.y;
-  grid.x = bx < 1 ? 1 : (bx > kColPartBlocks ? kColPartBlocks : bx);
+  grid.x = bx < 1 ? 1 : (bx > cap_x ? cap_x : bx);
   if (grid.x > (unsigned)rows_cap) grid.x = rows_cap;
   using bf = __nv_bfloat16;
   if (src_dtype == HSTU_DTYPE_F32 && dst_dtype == HSTU_DTYPE_F32)
@@ -1384,8 +1405,8 @@ cudaError_t launch_convert_rows_colsum(const void* src, int64_t lds, int src_dty
                                                              rows_dev, pad_multiple, part);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, partial_slices((int)grid.x)), 256, 0, st>>>(
-      part, (int)grid.x, cols, col_sums);
+  col_partials_reduce_kernel<<<dim3((cols + 255) / 256, partial_slices((int)grid.x * rpi)), 256, 0, st>>>(
+      part, (int)grid.x * rpi, cols, col_sums);
   return cudaGetLastError();
 }
 

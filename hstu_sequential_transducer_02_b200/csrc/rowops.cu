@@ -399,6 +399,19 @@ __global__ void gather_rows_kernel(const uint32_t* __restrict__ src, uint32_t* _
   }
 }
 
+// rows of 16-byte multiples: a warp per row, 16-byte vectors, no division per element
+__global__ void gather_rows_vec_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int vecs,
+                                       const int32_t* __restrict__ index, const int32_t* __restrict__ count,
+                                       int capacity) {
+  const int n = min(*count, capacity);
+  const int lane = threadIdx.x & 31, wpb = blockDim.x >> 5;
+  for (int r = blockIdx.x * wpb + (threadIdx.x >> 5); r < n; r += gridDim.x * wpb) {
+    const uint4* s = src + (int64_t)index[r] * vecs;
+    uint4* d = dst + (int64_t)r * vecs;
+    for (int w = lane; w < vecs; w += 32) d[w] = s[w];
+  }
+}
+
 // ---------------------------------------------------------------- Stochastic Length
 constexpr int kSlThreads = 1024;
 
@@ -1428,6 +1441,12 @@ cudaError_t launch_col_sum(const void* a, int64_t lda, int rows_cap, const int32
 cudaError_t launch_gather_rows(const void* src, void* dst, int64_t row_bytes, const int32_t* index,
                                const int32_t* count, int capacity, cudaStream_t st) {
   if (capacity <= 0) return cudaSuccess;
+  if (row_bytes % 16 == 0 && ((uintptr_t)src & 15) == 0 && ((uintptr_t)dst & 15) == 0 &&
+      row_bytes / 16 < (1ll << 31)) {
+    gather_rows_vec_kernel<<<row_sms() * 8, 256, 0, st>>>((const uint4*)src, (uint4*)dst, (int)(row_bytes / 16), index,
+                                                           count, capacity);
+    return cudaGetLastError();
+  }
   gather_rows_kernel<<<148 * 8, 256, 0, st>>>((const uint32_t*)src, (uint32_t*)dst, row_bytes / 4, index, count,
                                               capacity);
   return cudaGetLastError();

@@ -562,3 +562,25 @@ def test_layer_backward_fp32_narrow_rows():
     for name, (got, want) in _layer_errors(ref, gr, T, hv).items():
         assert_close(got, want, "f32", f"fp32 layer backward {name}", grad=True)
     assert_close(dx, ref["dx"], "f32", "fp32 layer backward dx", grad=True)
+
+
+def test_gather_rows_bit_exact():
+    """hstu_gather_rows against NumPy indexing, bit-exact: fp32 rows of 2 KB and
+    bf16 rows of 48 bytes (the 16-byte vector path), int64 rows of 8 bytes (the
+    4-byte word path); rows past the device count are left alone."""
+    b = _b()
+    rng = np.random.default_rng(5)
+    n_src, n_sel = 700, 333
+    idx = rng.integers(0, n_src, size=n_sel).astype(np.int32)
+    idx_d = dev(idx)
+    count = dev(np.array([n_sel - 7], dtype=np.int32))
+    for shape, dt in (((n_src, 512), torch.float32), ((n_src, 24), torch.bfloat16), ((n_src,), torch.int64)):
+        src = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(dt) if dt != torch.int64 \
+            else torch.from_numpy(rng.integers(-2**40, 2**40, size=shape, dtype=np.int64))
+        src_d = src.cuda()
+        out = torch.full((n_sel,) + tuple(shape[1:]), 7, dtype=dt, device="cuda")
+        b.gather_rows(src_d, idx_d, count, out)
+        torch.cuda.synchronize()
+        got = out.cpu()
+        assert torch.equal(got[:n_sel - 7], src[torch.from_numpy(idx[:n_sel - 7]).long()]), f"{dt} rows"
+        assert torch.all(got[n_sel - 7:] == 7), f"{dt} rows past the count"

@@ -1316,8 +1316,8 @@ std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 unsigned long long g_noalloc_ctx[kMaxDevices] = {};   // id of the context the address belongs to
 
-// The driver's context calls, taken through the runtime's entry-point query so
-// that the library has no link-time dependency on the driver library.
+// The CUDA driver API context calls, taken through the runtime's entry-point query so
+// that the library has no link-time dependency on libcuda.
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 

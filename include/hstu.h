@@ -158,8 +158,11 @@ typedef struct hstu_layer_saved {
   void*  attn_out;   /* [T, H*dv] dtype: A V */
   float* ln2_mean;   /* [T] */
   float* ln2_rstd;   /* [T] */
-  void*  gate;       /* [T, H*dv] dtype: LayerNorm2(A V) * U, the input of f2; may be
-                        NULL, then the backward recomputes it from attn_out and uvqk */
+  void*  gate;       /* [T, H*dv] dtype: LayerNorm2(A V) * U, the input of f2.  The
+                        forward writes it when non-NULL and the backward then reads it
+                        (so it must hold what the forward wrote); NULL: the forward
+                        keeps it in its workspace and the backward recomputes it from
+                        attn_out and uvqk */
 } hstu_layer_saved;
 
 /* Gradients of one layer (all device).  Weight gradients are overwritten (=). */

@@ -144,9 +144,10 @@ __device__ __forceinline__ void epilogue_chunk_xpose(const TcGemmParams& tp, uin
       v[e] += b.x; v[e + 1] += b.y; v[e + 2] += b.z; v[e + 3] += b.w;
     }
   }
-  if (p.epi == EPI_BIAS_RESIDUAL && p.residual && m_first + lane < m_end) {
+  int64_t m = m_first + lane < m_end ? m_first + lane : -1;   // this lane's residual row
+  if (m >= 0 && p.res_map) m = p.res_map[m];
+  if (p.epi == EPI_BIAS_RESIDUAL && p.residual && m >= 0) {
     // the residual row by its own lane (all its loads in flight together)
-    const int64_t m = m_first + lane;
     if (tp.res_f32) {
       const float* rs = (const float*)p.residual + m * p.ldr + n0;
 #pragma unroll
@@ -169,8 +170,11 @@ __device__ __forceinline__ void epilogue_chunk_xpose(const TcGemmParams& tp, uin
       }
     }
   }
+  // with out_map: this lane's output row, or -1 (dropped)
+  const int64_t mo = p.out_map ? (m_first + lane < m_end ? p.out_map[m_first + lane] : -1) : 0;
   if (tp.out_f32 || p.epi == EPI_STORE_F32) {
     char* ob = (char*)((float*)p.out + (int64_t)m_first * p.ldo + n0);
+    char* my = mo >= 0 ? (char*)((float*)p.out + mo * p.ldo + n0) : nullptr;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint4 w[4];
@@ -178,14 +182,18 @@ __device__ __forceinline__ void epilogue_chunk_xpose(const TcGemmParams& tp, uin
       for (int k = 0; k < 4; ++k)
         w[k] = make_uint4(__float_as_uint(v[16 * h + 4 * k]), __float_as_uint(v[16 * h + 4 * k + 1]),
                           __float_as_uint(v[16 * h + 4 * k + 2]), __float_as_uint(v[16 * h + 4 * k + 3]));
-      store_rows_xpose(tile, w, ob + 64 * h, p.ldo * 4, m_first, m_end, lane);
+      if (p.out_map) store_rows_xpose_mapped(tile, w, my ? my + 64 * h : nullptr, lane);
+      else store_rows_xpose(tile, w, ob + 64 * h, p.ldo * 4, m_first, m_end, lane);
     }
   } else {
     uint4 w[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) pack8_bf16(v + 8 * k, w[k]);
-    store_rows_xpose(tile, w, (char*)((__nv_bfloat16*)p.out + (int64_t)m_first * p.ldo + n0), p.ldo * 2, m_first,
-                     m_end, lane);
+    if (p.out_map)
+      store_rows_xpose_mapped(tile, w, mo >= 0 ? (char*)((__nv_bfloat16*)p.out + mo * p.ldo + n0) : nullptr, lane);
+    else
+      store_rows_xpose(tile, w, (char*)((__nv_bfloat16*)p.out + (int64_t)m_first * p.ldo + n0), p.ldo * 2, m_first,
+                       m_end, lane);
   }
 }
 
@@ -406,12 +414,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int ab = t & 1;
       const int m = un.m0 + r;
       const bool row_ok = m < M_eff;
-      if (p.epi == EPI_BIAS_RESIDUAL && p.residual && row_ok && un.n0 + group * kCols < p.N) {
+      const int64_t rm = row_ok && p.res_map ? p.res_map[m] : m;   // the residual row (-1: none)
+      if (p.epi == EPI_BIAS_RESIDUAL && p.residual && row_ok && rm >= 0 && un.n0 + group * kCols < p.N) {
         // this lane's residual row piece (kCols columns) on its way to L2 while
         // the main loop still fills the accumulator
         const int c0 = un.n0 + group * kCols, es = tp.res_f32 ? 4 : 2;
         const int bytes = (p.N - c0 < kCols ? p.N - c0 : kCols) * es;   // inside the row
-        const char* rp = (const char*)p.residual + ((int64_t)m * p.ldr + c0) * es;
+        const char* rp = (const char*)p.residual + (rm * p.ldr + c0) * es;
 #pragma unroll
         for (int b = 0; b < kCols * 4; b += 128)
           if (b < bytes) prefetch_l2(rp + b);
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                     (p.epi == EPI_STORE_F32 && tp.split == 1 && !p.accumulate)) && n0 + 32 <= p.N) {
           // whole 32-column chunks: the rows through the warp's transpose tile
           epilogue_chunk_xpose(tp, xtile, un.m0 + quarter * 32, M_eff, n0, raw, has_k, lane);
-        } else if (row_ok && n0 < p.N) {
+        } else if (row_ok && n0 < p.N && !p.res_map && !p.out_map) {
           epilogue_chunk(tp, m, n0, raw, has_k);
         }
       }
@@ -581,6 +590,8 @@ bool tc_gemm_supported(const GemmParams& p, int dtype) {
   if ((lda * 2) % 16 || (ldb * 2) % 16) return false;
   if (p.epi == EPI_SILU_BWD) return false;
   if (p.epi == EPI_BIAS_SILU && p.N % 32) return false;
+  if ((p.res_map || p.out_map) && (p.epi != EPI_BIAS_RESIDUAL || p.N % 32)) return false;
+  if (p.out_slot_offs && p.epi != EPI_BIAS_SILU) return false;
   if ((p.sak != 1 && p.M % 64) || (p.sbk != 1 && p.N % 64)) return false;
   return true;
 }

@@ -1070,9 +1070,13 @@ MfalconWs carve_mfalcon(Carver& c, const hstu_layer_desc* d, int L, int U, int h
 // One layer over the compact candidate rows x_c -> y_c (C rows), the history's
 // keys and values taken from `uvqk` (slot layout), whose slot rows receive the
 // candidates' U|V|Q|K.
+// x_map / y_map (optional): compact row c of the input is row x_map[c] of x_c,
+// and compact output row c goes to row y_map[c] of y_c (-1: a zero input row /
+// a dropped output row) -- the candidates' own rows of the caller's arrays
 int run_layer_targets(const hstu_layer_desc* d, const hstu_layer_weights* w, const hstu_jagged* slot_jb, int U,
                       int bm, const int32_t* hist_offsets, const void* x_c, void* y_c, char* uvqk,
-                      const MfalconWs& ws, cudaStream_t st) {
+                      const MfalconWs& ws, cudaStream_t st, const int32_t* x_map = nullptr,
+                      const int32_t* y_map = nullptr) {
   const int dt = d->attn.dtype;
   const int dm = d->d_model, hv = d->attn.num_heads * d->attn.dv;
   const int C = ws.C;
@@ -1080,7 +1084,7 @@ int run_layer_targets(const hstu_layer_desc* d, const hstu_layer_weights* w, con
   {
     TraceScope tr("ln1", st);
     HSTU_CUDA(launch_layer_norm(x_c, dm, d->io_dtype, w->ln1_gamma, w->ln1_beta, d->ln_eps, ws.xhat_c, dm, dt,
-                                ws.mu1c, ws.rs1c, C, nullptr, dm, st));
+                                ws.mu1c, ws.rs1c, C, nullptr, dm, st, x_map));
   }
   GemmParams g1;
   memset(&g1, 0, sizeof(g1));
@@ -1133,8 +1137,22 @@ int run_layer_targets(const hstu_layer_desc* d, const hstu_layer_weights* w, con
   g2.res_f32 = d->io_dtype == HSTU_DTYPE_F32;
   g2.out_f32 = d->io_dtype == HSTU_DTYPE_F32;
   g2.status = ws.layer.attn.status;
+  g2.res_map = x_map; g2.out_map = y_map;
+  // the maps exist on the tensor-core path only (the caller checked targets_mapped_io)
+  if ((x_map || y_map) && ((d->attn.flags & HSTU_FLAG_FORCE_SIMT) || !tc_gemm_supported(g2, dt)))
+    return HSTU_ERR_UNSUPPORTED;
   HSTU_TRY(gemm(g2, dt, d->attn.flags, st, "gemm_f2_residual"));
   return HSTU_OK;
+}
+
+// whether a candidate-only pass can read its input rows from, and write its
+// output rows to, the caller's candidate arrays directly (run_layer_targets'
+// maps; the tensor-core f2 with whole 32-column chunks)
+bool targets_mapped_io(const hstu_layer_desc* d, const void* cand_x, const void* cand_out) {
+  const size_t eio = elem_size(d->io_dtype);
+  return !(d->attn.flags & HSTU_FLAG_FORCE_SIMT) && d->attn.dtype == HSTU_DTYPE_BF16 && d->d_model % 32 == 0 &&
+         (d->d_model * eio) % 16 == 0 && aligned16(cand_x) && aligned16(cand_out) &&
+         d->attn.num_heads * d->attn.dv % 8 == 0;
 }
 }  // namespace
 
@@ -1186,6 +1204,7 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
   jb.timestamps = w.ts;
   const hstu_attn_desc* ad = &desc->attn;
   const int tile = attn_tile(ad);
+  const bool mapped = targets_mapped_io(desc, cand_x, cand_out);   // later microbatches: no pack or scatter of rows
   for (int mb = 0; mb < n_mb; ++mb) {
     void* cur = w.xc0;
     void* nxt = w.xc1;
@@ -1215,18 +1234,24 @@ int mfalcon_rank(const hstu_layer_desc* desc, const hstu_layer_weights* layers, 
                                          nullptr, 1));
       }
     } else {
+      // with mapped input and output rows the first layer reads the candidates' rows
+      // of cand_x and the last writes cand_out's: the pack only places timestamps
+      // and the row map, and no scatter follows
       HSTU_CUDA(launch_mfalcon_slot_pack(U, mb, bm, w.C, w.cap, hist_offsets, hist_x, hist_ts, cand_offsets, cand_x,
-                                         cand_ts, dm, dt, 0, nullptr, w.ts, cur, w.cand_dst, st));
+                                         cand_ts, dm, dt, 0, nullptr, w.ts, mapped ? nullptr : cur, w.cand_dst, st));
       if (w.attn_t.tile_recs) {
         // the candidates' timestamps changed: timestamp records of every kv tile
         TraceScope tr("ts_tiles", st);
         HSTU_CUDA(launch_ts_tiles(w.offs, w.ts, U, w.attn_t.tile_base, w.attn_t.tiles_cap, w.attn_t.tile_recs, st));
       }
       for (int l = 0; l < num_layers; ++l) {
-        HSTU_TRY(run_layer_targets(desc, &layers[l], &jb, U, bm, hist_offsets, cur, nxt,
-                                   w.uvqk_cache + (size_t)l * w.uvqk_stride, w, st));
+        const bool first = mapped && l == 0, last = mapped && l == num_layers - 1;
+        HSTU_TRY(run_layer_targets(desc, &layers[l], &jb, U, bm, hist_offsets, first ? cand_x : cur,
+                                   last ? cand_out : nxt, w.uvqk_cache + (size_t)l * w.uvqk_stride, w, st,
+                                   first ? w.cand_dst : nullptr, last ? w.cand_dst : nullptr));
         void* t = cur; cur = nxt; nxt = t;
       }
+      if (mapped) continue;   // the last layer wrote cand_out
     }
     HSTU_CUDA(launch_mfalcon_scatter(cur, dm, dt, w.cand_dst, nullptr, w.C, cand_out, st));
   }

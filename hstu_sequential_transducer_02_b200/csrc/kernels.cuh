@@ -183,6 +183,10 @@ struct GemmParams {
   // out_slot_offs[m / out_slot_bm + 1] + m of out (rows at or past out_slot_cap are
   // dropped): the M-FALCON candidates' rows straight into their slots
   const int32_t* out_slot_offs; int out_slot_bm, out_slot_cap;
+  // EPI_BIAS_RESIDUAL on the tensor-core path (whole 32-column chunks): if set, the
+  // residual of row m is row res_map[m] and output row m goes to row out_map[m];
+  // -1 means no residual / the row is dropped
+  const int32_t* res_map; const int32_t* out_map;
 };
 
 cudaError_t launch_gemm_simt(const GemmParams& p, int dtype, cudaStream_t st);
@@ -192,9 +196,11 @@ cudaError_t launch_gemm_tc(const GemmParams& p, cudaStream_t st);
 
 // ---------------------------------------------------------------- row kernels
 // xhat = LN(x) * gamma + beta; x in x_dtype, xhat in out_dtype
+// (in_map: row m of x is row in_map[m], or a zero row where in_map[m] < 0)
 cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const float* gamma, const float* beta,
                               float eps, void* out, int64_t ldo, int out_dtype, float* mean, float* rstd,
-                              int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st);
+                              int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st,
+                              const int32_t* in_map = nullptr);
 // g = LN(o) * u; with in_slot_offs, row m of o and u is read from row
 // in_slot_offs[m / in_slot_bm + 1] + m (row 0 if that reaches in_slot_cap)
 cudaError_t launch_ln_gate(const void* o, int64_t ldo_in, const void* u, int64_t ldu, const float* gamma,

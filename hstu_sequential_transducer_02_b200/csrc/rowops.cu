@@ -75,18 +75,24 @@ __global__ void __launch_bounds__(kRowWarps * 32)
 layer_norm_kernel(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma,
                   const float* __restrict__ beta, float eps, TO* __restrict__ out, int64_t ldo,
                   float* __restrict__ mean_out, float* __restrict__ rstd_out, int rows_cap,
-                  const int32_t* __restrict__ rows_dev, int d) {
+                  const int32_t* __restrict__ rows_dev, int d, const int32_t* __restrict__ in_map) {
   const int rows = rows_of(rows_cap, rows_dev);
   const int lane = threadIdx.x & 31;
   const int nch = d / 8;
   for (int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5); row < rows; row += gridDim.x * kRowWarps) {
+    const int src = in_map ? in_map[row] : row;   // < 0: a zero row
     float v[kMaxChunks][8];
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < kMaxChunks; ++c) {
       const int ch = lane + 32 * c;
       if (ch < nch) {
-        load8(x + (int64_t)row * ldx + ch * 8, v[c]);
+        if (src >= 0) {
+          load8(x + (int64_t)src * ldx + ch * 8, v[c]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[c][e] = 0.f;
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) s += v[c][e];
       }
@@ -587,12 +593,13 @@ __global__ void mfalcon_slot_pack_kernel(int U, int mb, int bm, const int32_t* _
       if (lane == 0) cand_dst[u * bm + j] = ci < m ? cand_offs[u] + ci : -1;
     }
     if (slot_row >= cap) continue;   // offsets beyond the sizes the workspace was made for
-    for (int e = lane * 8; e < d; e += 32 * 8) {
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (src) load8(src + e, v);
-      if (x_slot) store8(x_slot + (int64_t)slot_row * d + e, v);
-      if (x_c && j >= 0) store8(x_c + (int64_t)(u * bm + j) * d + e, v);
-    }
+    if (x_slot || (x_c && j >= 0))
+      for (int e = lane * 8; e < d; e += 32 * 8) {
+        float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (src) load8(src + e, v);
+        if (x_slot) store8(x_slot + (int64_t)slot_row * d + e, v);
+        if (x_c && j >= 0) store8(x_c + (int64_t)(u * bm + j) * d + e, v);
+      }
     if (lane == 0) ts_slot[slot_row] = ts;
   }
 }
@@ -662,6 +669,7 @@ template <typename T> struct Raw8;
 template <> struct Raw8<__nv_bfloat16> {
   uint4 u;
   __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
   __device__ __forceinline__ void get(float v[8]) const {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -674,6 +682,7 @@ template <> struct Raw8<__nv_bfloat16> {
 };
 template <> struct Raw8<float> {
   float4 a, b;
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
   __device__ __forceinline__ void load(const float* p) {
     a = *reinterpret_cast<const float4*>(p);
     b = *reinterpret_cast<const float4*>(p + 4);
@@ -704,7 +713,8 @@ template <typename T, typename TO, int NCH>
 __global__ void __launch_bounds__(kRowWarps * 32, NCH > 2 ? 1 : (sizeof(T) == 2 ? 3 : 2))   // registers for two rows in flight
 layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ gamma, const float* __restrict__ beta,
                 float eps, TO* __restrict__ out, int64_t ldo, float* __restrict__ mean_out,
-                float* __restrict__ rstd_out, int rows_cap, const int32_t* __restrict__ rows_dev) {
+                float* __restrict__ rstd_out, int rows_cap, const int32_t* __restrict__ rows_dev,
+                const int32_t* __restrict__ in_map) {
   const int rows = rows_of(rows_cap, rows_dev);
   const int lane = threadIdx.x & 31;
   const int stride = gridDim.x * kRowWarps;
@@ -717,9 +727,14 @@ layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ 
   // two rows in flight ahead of the one being normalised: the warp's rows
   // alternate between two register buffers
   auto fetch = [&](Raw8<T> (&r)[NCH], int row) {
-    if (row < rows)
+    if (row < rows) {
+      const int src = in_map ? in_map[row] : row;
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) r[c].load(x + (int64_t)row * ldx + (lane + 32 * c) * 8);
+      for (int c = 0; c < NCH; ++c) {
+        if (src >= 0) r[c].load(x + (int64_t)src * ldx + (lane + 32 * c) * 8);
+        else r[c].zero();
+      }
+    }
   };
   auto normalise = [&](Raw8<T> (&r)[NCH], int row) {
     float v[NCH][8];
@@ -1126,13 +1141,13 @@ int rows_grid(int rows_cap) {
 template <typename T, typename TO>
 cudaError_t launch_ln_rows(const T* x, int64_t ldx, const float* gamma, const float* beta, float eps, TO* out,
                            int64_t ldo, float* mean, float* rstd, int rows_cap, const int32_t* rows_dev, int d,
-                           cudaStream_t st) {
+                           cudaStream_t st, const int32_t* in_map) {
   const int t = kRowWarps * 32;
   switch (d / 256) {
-    case 1: layer_norm_rows<T, TO, 1><<<rows_grid<layer_norm_rows<T, TO, 1>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
-    case 2: layer_norm_rows<T, TO, 2><<<rows_grid<layer_norm_rows<T, TO, 2>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
-    case 3: layer_norm_rows<T, TO, 3><<<rows_grid<layer_norm_rows<T, TO, 3>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
-    default: layer_norm_rows<T, TO, 4><<<rows_grid<layer_norm_rows<T, TO, 4>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev); break;
+    case 1: layer_norm_rows<T, TO, 1><<<rows_grid<layer_norm_rows<T, TO, 1>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev, in_map); break;
+    case 2: layer_norm_rows<T, TO, 2><<<rows_grid<layer_norm_rows<T, TO, 2>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev, in_map); break;
+    case 3: layer_norm_rows<T, TO, 3><<<rows_grid<layer_norm_rows<T, TO, 3>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev, in_map); break;
+    default: layer_norm_rows<T, TO, 4><<<rows_grid<layer_norm_rows<T, TO, 4>>(rows_cap), t, 0, st>>>(x, ldx, gamma, beta, eps, out, ldo, mean, rstd, rows_cap, rows_dev, in_map); break;
   }
   return cudaGetLastError();
 }
@@ -1169,37 +1184,37 @@ int row_grid(int rows_cap) {
 
 cudaError_t launch_layer_norm(const void* x, int64_t ldx, int x_dtype, const float* gamma, const float* beta,
                               float eps, void* out, int64_t ldo, int out_dtype, float* mean, float* rstd,
-                              int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st) {
+                              int rows_cap, const int32_t* rows_dev, int d, cudaStream_t st, const int32_t* in_map) {
   if (rows_cap <= 0) return cudaSuccess;
   using bf = __nv_bfloat16;
   const int xs = x_dtype == HSTU_DTYPE_F32 ? 4 : 2, os = out_dtype == HSTU_DTYPE_F32 ? 4 : 2;
   if (fast_rows_ok(d, x, ldx, nullptr, 0, out, ldo, xs, os) && gamma && beta) {
     if (x_dtype == HSTU_DTYPE_F32 && out_dtype == HSTU_DTYPE_F32)
       return launch_ln_rows<float, float>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean, rstd,
-                                          rows_cap, rows_dev, d, st);
+                                          rows_cap, rows_dev, d, st, in_map);
     if (x_dtype == HSTU_DTYPE_F32)
       return launch_ln_rows<float, bf>((const float*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd, rows_cap,
-                                       rows_dev, d, st);
+                                       rows_dev, d, st, in_map);
     if (out_dtype == HSTU_DTYPE_F32)
       return launch_ln_rows<bf, float>((const bf*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean, rstd, rows_cap,
-                                       rows_dev, d, st);
+                                       rows_dev, d, st, in_map);
     return launch_ln_rows<bf, bf>((const bf*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd, rows_cap,
-                                  rows_dev, d, st);
+                                  rows_dev, d, st, in_map);
   }
   const int g = row_grid(rows_cap);
   const int t = kRowWarps * 32;
   if (x_dtype == HSTU_DTYPE_F32 && out_dtype == HSTU_DTYPE_F32)
     layer_norm_kernel<float, float><<<g, t, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean,
-                                                     rstd, rows_cap, rows_dev, d);
+                                                     rstd, rows_cap, rows_dev, d, in_map);
   else if (x_dtype == HSTU_DTYPE_F32)
     layer_norm_kernel<float, bf><<<g, t, 0, st>>>((const float*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd,
-                                                  rows_cap, rows_dev, d);
+                                                  rows_cap, rows_dev, d, in_map);
   else if (out_dtype == HSTU_DTYPE_F32)
     layer_norm_kernel<bf, float><<<g, t, 0, st>>>((const bf*)x, ldx, gamma, beta, eps, (float*)out, ldo, mean, rstd,
-                                                  rows_cap, rows_dev, d);
+                                                  rows_cap, rows_dev, d, in_map);
   else
     layer_norm_kernel<bf, bf><<<g, t, 0, st>>>((const bf*)x, ldx, gamma, beta, eps, (bf*)out, ldo, mean, rstd,
-                                               rows_cap, rows_dev, d);
+                                               rows_cap, rows_dev, d, in_map);
   return cudaGetLastError();
 }
 

@@ -584,3 +584,31 @@ def test_gather_rows_bit_exact():
         got = out.cpu()
         assert torch.equal(got[:n_sel - 7], src[torch.from_numpy(idx[:n_sel - 7]).long()]), f"{dt} rows"
         assert torch.all(got[n_sel - 7:] == 7), f"{dt} rows past the count"
+
+
+@pytest.mark.parametrize("num_layers", [1, 2])
+def test_mfalcon_rank_fp32_io(num_layers):
+    """M-FALCON with an fp32 residual stream (history, candidates and scores in
+    fp32, bf16 weights and activations): the later microbatches read the
+    candidates' fp32 rows in place and write the fp32 scores in place; one layer
+    (first = last) and two (first and last distinct), ragged candidate counts, a
+    user without candidates and partial microbatches.  (A user without history
+    has its own test: its candidates' outputs rest on one term each.)"""
+    b = _b()
+    hist_lens, counts, microbatch = [64, 12, 37, 90], [9, 5, 0, 13], 4
+    wl = W.make_workload(3, scale=1 / 32, batch=len(hist_lens), lengths=hist_lens)
+    e = wl.extras
+    s = wl.spec
+    co = e["cand_offsets"]
+    sel = np.concatenate([np.arange(co[u], co[u] + counts[u]) for u in range(len(counts))]).astype(np.int64)
+    cand_offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    cand_x, cand_ts = e["cand_x"][sel], e["cand_ts"][sel]
+    layers = [b.Layer(layer_to_dev(wl.layers[0], torch.bfloat16), s.d_model, s.num_heads, s.head_dim,
+                      residual_fp32=True)] * num_layers
+    got = b.mfalcon_rank(layers, dev(wl.seq_offsets), dev(wl.x, torch.float32), dev(wl.timestamps),
+                         dev(cand_offsets), dev(cand_x, torch.float32), dev(cand_ts), microbatch, max(counts))
+    torch.cuda.synchronize()
+    assert got.dtype == torch.float32
+    ref = O.mfalcon_rank([wl.layers[0]] * num_layers, wl.seq_offsets, wl.x, wl.timestamps, cand_offsets, cand_x,
+                         cand_ts, microbatch, s.num_heads, s.head_dim)
+    assert_close(got.cpu().numpy(), ref, "bf16", f"mfalcon fp32 io, {num_layers} layer(s)")

@@ -768,7 +768,7 @@ layer_norm_rows(const T* __restrict__ x, int64_t ldx, const float* __restrict__ 
 
 // g = LN(o) * u, d = 256 * NCH
 template <typename T, int NCH>
-__global__ void __launch_bounds__(kRowWarps * 32, 2)
+__global__ void __launch_bounds__(kRowWarps * 32, sizeof(T) == 2 && NCH <= 2 ? 2 : 1)   // two rows in flight
 ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, int64_t ldu,
              const float* __restrict__ gamma, const float* __restrict__ beta, float eps, T* __restrict__ out,
              int64_t ldout, float* __restrict__ mean_out, float* __restrict__ rstd_out, int rows_cap,
@@ -776,51 +776,50 @@ ln_gate_rows(const T* __restrict__ o, int64_t ldo_in, const T* __restrict__ u, i
   const int rows = rows_of(rows_cap, rows_dev);
   const int lane = threadIdx.x & 31;
   const int stride = gridDim.x * kRowWarps;
-  float g[NCH][8], b[NCH][8];
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    load8(gamma + (lane + 32 * c) * 8, g[c]);
-    load8(beta + (lane + 32 * c) * 8, b[c]);
-  }
-  int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
-  Raw8<T> co[NCH], cu[NCH];
-  if (row < rows) {
-    const int64_t sr = src_row(sm, row);
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-      co[c].load(o + sr * ldo_in + (lane + 32 * c) * 8);
-      cu[c].load(u + sr * ldu + (lane + 32 * c) * 8);
-    }
-  }
-  for (; row < rows; row += stride) {
-    Raw8<T> no[NCH], nu[NCH];
-    if (row + stride < rows) {
-      const int64_t sr = src_row(sm, row + stride);
+  // two rows of O and U in flight ahead of the one being normalised (two register
+  // buffers, as in layer_norm_rows); gamma and beta come from L1 per row
+  auto fetch = [&](Raw8<T> (&ro)[NCH], Raw8<T> (&ru)[NCH], int row) {
+    if (row < rows) {
+      const int64_t sr = src_row(sm, row);
 #pragma unroll
       for (int c = 0; c < NCH; ++c) {
-        no[c].load(o + sr * ldo_in + (lane + 32 * c) * 8);
-        nu[c].load(u + sr * ldu + (lane + 32 * c) * 8);
+        ro[c].load(o + sr * ldo_in + (lane + 32 * c) * 8);
+        ru[c].load(u + sr * ldu + (lane + 32 * c) * 8);
       }
     }
-    float v[NCH][8];
+  };
+  auto gate = [&](Raw8<T> (&ro)[NCH], Raw8<T> (&ru)[NCH], int row) {
+    float v[NCH][8], uu[NCH][8];
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) co[c].get(v[c]);
+    for (int c = 0; c < NCH; ++c) {
+      ro[c].get(v[c]);
+      ru[c].get(uu[c]);
+    }
+    fetch(ro, ru, row + 2 * stride);   // the buffers' next row, issued before the arithmetic
     float mean, rstd;
     row_stats<NCH>(v, eps, mean, rstd);
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
-      float uu[8], r[8];
-      cu[c].get(uu);
+      float g[8], b[8], r[8];
+      load8(gamma + (lane + 32 * c) * 8, g);
+      load8(beta + (lane + 32 * c) * 8, b);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) r[e] = fmaf((v[c][e] - mean) * rstd, g[c][e], b[c][e]) * uu[e];
+      for (int e = 0; e < 8; ++e) r[e] = fmaf((v[c][e] - mean) * rstd, g[e], b[e]) * uu[c][e];
       store8(out + (int64_t)row * ldout + (lane + 32 * c) * 8, r);
     }
     if (lane == 0) {
       if (mean_out) mean_out[row] = mean;
       if (rstd_out) rstd_out[row] = rstd;
     }
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) { co[c] = no[c]; cu[c] = nu[c]; }
+  };
+  int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  Raw8<T> o0[NCH], u0[NCH], o1[NCH], u1[NCH];
+  fetch(o0, u0, row);
+  fetch(o1, u1, row + stride);
+  for (; row < rows; row += 2 * stride) {
+    gate(o0, u0, row);
+    if (row + stride >= rows) break;
+    gate(o1, u1, row + stride);
   }
 }
 

@@ -252,7 +252,7 @@ def test_bad_offsets_reported_not_crashing():
     assert b.workspace_status(ws) == b.ERR_BAD_OFFSETS
 
 
-@pytest.mark.parametrize("dtype_name,dh", [("f32", 32), ("bf16", 64)])
+@pytest.mark.parametrize("dtype_name,dh", [("f32", 32), ("bf16", 64), ("bf16", 128)])
 @pytest.mark.parametrize("mfalcon", [False, True])
 def test_attn_bwd_matches_oracle(dtype_name, dh, mfalcon):
     b = _b()
